@@ -1,0 +1,470 @@
+"""Pins for the CPU oracle: every routine is checked against something other
+than itself -- a library routine on a special case, a closed form, an
+invariant, brute force on tiny inputs, or the numbers the pages print.
+
+Sources: "SVG-EAR measured error" (frontier-cs.org blog) worked example and
+probe paragraph; SVG2 summary (paper-graph) section 3.4 on clustering,
+permutation validity and k-means++; the SVG-EAR review (pith.science) on greedy
+error-to-cost routing under a density budget.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import softmax
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# Philox4x64-10 and the uniform draws
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("key,counter", [(0, (0, 0, 0, 0)), (5, (0, 0, 0, 0)),
+                                         (2**64 - 1, (7, 3, 0, 0)),
+                                         (123456789, (41, 9, 2, 5))])
+def test_philox_matches_numpy_bit_generator(key, counter):
+    # numpy's Philox increments its 256-bit counter before each block.
+    bg = np.random.Philox(key=key, counter=np.array(counter, dtype=np.uint64))
+    ref = bg.random_raw(4)
+    ctr = list(counter)
+    ctr[0] = (ctr[0] + 1) % 2**64
+    got = oracle.philox4x64_10(ctr, [key % 2**64, key >> 64])
+    assert [int(x) for x in got] == [int(x) for x in ref]
+
+
+def test_uniform_is_top53_bits_of_first_word():
+    for j in range(5):
+        ctr = np.array([(j - 1) % 2**64, 3 if j else 2, 0, 0], dtype=np.uint64)
+        bg = np.random.Philox(key=77, counter=ctr)
+        w0 = int(bg.random_raw(1)[0])
+        assert oracle.uniform(77, 3, j) == (w0 >> 11) * 2.0**-53
+    u = [oracle.uniform(1, 0, j) for j in range(2000)]
+    assert min(u) >= 0.0 and max(u) < 1.0
+    assert abs(np.mean(u) - 0.5) < 0.03
+
+
+# --------------------------------------------------------------------------
+# k-means++ seeding
+# --------------------------------------------------------------------------
+def _kpp_numpy(X, C, seed, stream):
+    N = X.shape[0]
+    idx = [int(math.floor(oracle.uniform(seed, stream, 0) * N))]
+    for j in range(1, C):
+        D2 = np.min(((X[:, None, :] - X[idx][None]) ** 2).sum(-1), axis=1)
+        cs = np.cumsum(D2)
+        target = oracle.uniform(seed, stream, j) * cs[-1]
+        idx.append(int(np.searchsorted(cs, target, side="right")))
+    return np.array(idx)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 99])
+def test_kmeanspp_matches_cumsum_searchsorted(seed):
+    g = np.random.default_rng(seed)
+    X = g.standard_normal((64, 4))
+    idx, margin = oracle.kmeanspp(X, 12, seed, 5)
+    ref = _kpp_numpy(X, 12, seed, 5)
+    ok = margin[1:] > 1e-12
+    assert np.array_equal(idx[0], ref[0])
+    assert np.array_equal(idx[1:][ok], ref[1:][ok])
+    assert len(set(idx.tolist())) == 12
+
+
+def test_kmeanspp_d2_sampling_finds_every_separated_blob():
+    # 10 tight blobs 1000 apart: D^2 sampling puts one seed in each blob
+    # (uniform sampling would collide with probability ~ 1 - 10!/10^10).
+    g = np.random.default_rng(3)
+    centres = g.standard_normal((10, 8)) * 1000.0
+    blob = np.repeat(np.arange(10), 50)
+    X = centres[blob] + g.standard_normal((500, 8))
+    for seed in range(5):
+        idx, _ = oracle.kmeanspp(X, 10, seed, 0)
+        assert sorted(blob[idx].tolist()) == list(range(10))
+
+
+def test_kmeanspp_follow_reproduces_own_choices():
+    g = np.random.default_rng(4)
+    X = g.standard_normal((300, 6))
+    own, _ = oracle.kmeanspp(X, 20, 11, 2)
+    chk, margin = oracle.kmeanspp(X, 20, 11, 2, follow=own)
+    assert np.array_equal(own, chk)
+    assert np.all(margin[1:] >= 0)
+
+
+def test_kmeanspp_all_identical_takes_lowest_unchosen():
+    X = np.ones((8, 3))
+    idx, _ = oracle.kmeanspp(X, 4, 0, 0)
+    first = int(idx[0])
+    rest = [t for t in range(8) if t != first][:3]
+    assert idx[1:].tolist() == rest
+
+
+# --------------------------------------------------------------------------
+# assign / update / sort / segment mean
+# --------------------------------------------------------------------------
+def test_assign_matches_numpy_argmin_bruteforce():
+    g = np.random.default_rng(0)
+    X = g.standard_normal((500, 16))
+    cent = g.standard_normal((23, 16))
+    labels, second, best, gap = oracle.assign(X, cent)
+    D = ((X[:, None, :] - cent[None]) ** 2).sum(-1)
+    assert np.array_equal(labels, np.argmin(D, axis=1))
+    assert np.allclose(best, D.min(1))
+    Ds = np.sort(D, axis=1)
+    assert np.allclose(gap, Ds[:, 1] - Ds[:, 0])
+    assert np.all(second != labels)
+
+
+def test_assign_exact_tie_goes_to_lowest_index():
+    X = np.array([[0.0, 0.0], [1.0, 1.0]])
+    cent = np.array([[1.0, 0.0], [0.0, 1.0], [-1.0, 0.0], [5.0, 5.0]])
+    labels, second, _, gap = oracle.assign(X, cent)
+    assert labels[0] == 0 and second[0] == 1 and gap[0] == 0.0
+    assert labels[1] == 0 and second[1] == 1
+
+
+def test_update_means_and_empty_cluster_keeps_previous():
+    g = np.random.default_rng(1)
+    X = g.standard_normal((200, 5))
+    labels = g.integers(0, 6, 200)
+    labels[labels == 4] = 5           # cluster 4 is empty
+    prev = g.standard_normal((6, 5))
+    out = oracle.update(X, labels, prev)
+    cnt = np.bincount(labels, minlength=6)
+    for c in range(6):
+        if cnt[c]:
+            assert np.allclose(out[c], X[labels == c].mean(0))
+    assert np.array_equal(out[4], prev[4])
+    assert np.allclose((out * cnt[:, None]).sum(0), X.sum(0))
+
+
+def test_stable_sort_matches_numpy_stable_argsort():
+    g = np.random.default_rng(2)
+    for C in (1, 7, 50):
+        labels = g.integers(0, C, 1000).astype(np.int32)
+        perm, off = oracle.stable_sort(labels, C)
+        assert np.array_equal(perm, np.argsort(labels, kind="stable"))
+        assert np.array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(labels, minlength=C))]))
+        assert np.array_equal(np.sort(perm), np.arange(1000))
+
+
+def test_segment_mean_matches_reduceat_singletons_and_empties():
+    g = np.random.default_rng(5)
+    sizes = np.array([3, 1, 0, 7, 1, 0, 4])
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Xp = g.standard_normal((sizes.sum(), 9))
+    out = oracle.segment_mean(Xp, off)
+    nz = sizes > 0
+    ref = np.add.reduceat(Xp, off[:-1][nz], axis=0) / sizes[nz][:, None]
+    assert np.allclose(out[nz], ref)
+    assert np.array_equal(out[1], Xp[3]) and np.array_equal(out[4], Xp[11])
+    assert np.all(out[2] == 0) and np.all(out[5] == 0)
+    prev = np.full((7, 9), 3.5)
+    assert np.all(oracle.segment_mean(Xp, off, prev)[5] == 3.5)
+
+
+def test_cluster_recovers_separated_blobs_and_centroids_are_member_means():
+    g = np.random.default_rng(6)
+    centres = g.standard_normal((8, 16)) * 50
+    truth = g.integers(0, 8, 2000)
+    X = centres[truth] + g.standard_normal((2000, 16))
+    out = oracle.cluster(X, 8, 10, seed=3, stream=0)
+    # a bijection between found and true clusters
+    pairs = set(zip(out["labels"].tolist(), truth.tolist()))
+    assert len(pairs) == 8
+    for c in range(8):
+        members = X[out["labels"] == c]
+        assert np.allclose(out["centroids"][c], members.mean(0))
+    assert np.array_equal(out["Xp"], X[out["perm"]])
+
+
+# --------------------------------------------------------------------------
+# The worked toy example (golden numbers printed on the blog page)
+# --------------------------------------------------------------------------
+def _toy(vA=(1.0,), vB=((1.0,), (3.0,)), d=64):
+    """q = 8 e1 so that q.k/sqrt(64) = k_1: keys score 1, 1 (A) and 0, 2 (B)."""
+    q = np.zeros((1, d)); q[0, 0] = 8.0
+    K = np.zeros((4, d)); K[:, 0] = [1.0, 1.0, 0.0, 2.0]
+    V = np.zeros((4, d))
+    V[0, 1] = V[1, 1] = vA[0]
+    V[2, 1], V[3, 1] = vB[0][0], vB[1][0]
+    k_off = np.array([0, 2, 4], dtype=np.int32)
+    q_off = np.array([0, 1], dtype=np.int32)
+    kbar = oracle.segment_mean(K, k_off)
+    vbar = oracle.segment_mean(V, k_off)
+    return q, K, V, q_off, k_off, kbar, vbar
+
+
+def test_toy_example_weights_match_the_page():
+    gold = json.load(open(os.path.join(GOLDEN, "toy_example.json")))["printed"]
+    q, K, V, q_off, k_off, kbar, vbar = _toy()
+    scale = 1.0 / 8.0
+    perm = np.zeros(1, dtype=np.int32)
+    # exact (both clusters computed): weight = e^lse
+    _, lse_all = oracle.attend(q, K, V, q_off, k_off, np.array([0, 2], np.int32),
+                               np.array([0, 1], np.int32), kbar, vbar, perm, scale)
+    # A computed, B compensated / B computed, A compensated / both compensated
+    _, lse_a = oracle.attend(q, K, V, q_off, k_off, np.array([0, 1], np.int32),
+                             np.array([0], np.int32), kbar, vbar, perm, scale)
+    _, lse_b = oracle.attend(q, K, V, q_off, k_off, np.array([0, 1], np.int32),
+                             np.array([1], np.int32), kbar, vbar, perm, scale)
+    _, lse_0 = oracle.attend(q, K, V, q_off, k_off, np.array([0, 0], np.int32),
+                             np.zeros(0, np.int32), kbar, vbar, perm, scale)
+    total = math.exp(lse_all[0])
+    est_a = est_b = math.exp(lse_0[0]) / 2.0
+    true_b = math.exp(lse_a[0]) - est_b       # A exact + B estimated
+    true_a = total - (math.exp(lse_b[0]) - est_a)
+    assert abs(total - gold["weight_total"]) < 0.05
+    assert abs(true_a - gold["weight_A"]) < 0.05
+    assert abs((total - true_a) - gold["weight_B"]) < 0.05
+    assert abs(est_a - gold["centroid_estimate_A"]) < 0.05
+    assert abs(est_b - gold["centroid_estimate_B"]) < 0.05
+    assert abs((total - true_a) - est_b - gold["shortfall_B"]) < 0.1
+    # "For A that is exact": computing B alone already gives the exact weight
+    assert math.isclose(math.exp(lse_b[0]), total, rel_tol=1e-12)
+    del true_b
+
+
+def test_toy_example_error_aware_routing_picks_b_and_is_exact():
+    q, K, V, q_off, k_off, kbar, vbar = _toy()
+    scale = 1.0 / 8.0
+    E = oracle.probe(q, K, V, kbar, vbar, k_off, scale)
+    assert E[0, 0] == 0.0 and E[0, 1] > 0.0
+    # room for one cluster: density 0.5 of Nk=4 keys = 2 keys
+    pair_off, pair_kc = oracle.route(E.astype(np.float32), q_off, k_off, 4, 0.5)
+    assert pair_kc.tolist() == [1]
+    O, _ = oracle.attend(q, K, V, q_off, k_off, pair_off, pair_kc, kbar, vbar,
+                         np.zeros(1, np.int32), scale)
+    dense = softmax(q @ K.T * scale, axis=-1) @ V
+    assert np.allclose(O, dense, rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Probe closed forms
+# --------------------------------------------------------------------------
+def test_probe_identical_keys_is_shifted_value_variance():
+    # keys identical inside each cluster: e^{s_t} = e^{sbar}, so
+    # E_ic = e^{2(s_c - m)} * sum_t |v_t - vbar_c|^2 = e^{2(s_c-m)} n_c sum var.
+    g = np.random.default_rng(7)
+    d, sizes = 8, [5, 3, 9, 1]
+    kc = g.standard_normal((4, d))
+    K = np.repeat(kc, sizes, axis=0)
+    V = g.standard_normal((sum(sizes), d))
+    k_off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    qbar = g.standard_normal((3, d))
+    scale = 0.7
+    E = oracle.probe(qbar, K, V, kc, oracle.segment_mean(V, k_off), k_off, scale)
+    for i in range(3):
+        s = scale * kc @ qbar[i]
+        m = s.max()
+        for c in range(4):
+            Vc = V[k_off[c]:k_off[c + 1]]
+            ref = math.exp(2 * (s[c] - m)) * sizes[c] * np.var(Vc, axis=0).sum()
+            assert math.isclose(E[i, c], ref, rel_tol=1e-10, abs_tol=1e-300)
+    assert np.all(E[:, 3] == 0.0)          # a singleton is exact
+
+
+def test_probe_scales_with_value_square_and_ignores_key_order():
+    g = np.random.default_rng(8)
+    d = 6
+    K = g.standard_normal((20, d)); V = g.standard_normal((20, d))
+    k_off = np.array([0, 4, 11, 20], dtype=np.int32)
+    kbar = oracle.segment_mean(K, k_off); vbar = oracle.segment_mean(V, k_off)
+    qbar = g.standard_normal((2, d))
+    E = oracle.probe(qbar, K, V, kbar, vbar, k_off, 0.5)
+    E3 = oracle.probe(qbar, K, 3 * V, kbar, 3 * vbar, k_off, 0.5)
+    assert np.allclose(E3, 9 * E, rtol=1e-12)
+    p = np.concatenate([g.permutation(np.arange(a, b)) for a, b in zip(k_off[:-1], k_off[1:])])
+    Ep = oracle.probe(qbar, K[p], V[p], kbar, vbar, k_off, 0.5)
+    assert np.allclose(Ep, E, rtol=1e-12)
+
+
+def test_probe_shift_is_the_global_row_max():
+    # Two identical-key clusters: the ratio E_1/E_0 must carry e^{2(s1-s0)};
+    # a per-cluster shift would cancel it.
+    d = 2
+    K = np.array([[0.0, 0.0]] * 2 + [[1.0, 0.0]] * 2)
+    V = np.array([[1.0, 0.0], [-1.0, 0.0], [1.0, 0.0], [-1.0, 0.0]])
+    k_off = np.array([0, 2, 4], dtype=np.int32)
+    qbar = np.array([[2.0, 0.0]])
+    E = oracle.probe(qbar, K, V, oracle.segment_mean(K, k_off),
+                     oracle.segment_mean(V, k_off), k_off, 1.0)
+    assert math.isclose(E[0, 1] / E[0, 0], math.exp(4.0), rel_tol=1e-12)
+    assert math.isclose(E[0, 1], 2.0, rel_tol=1e-12)   # m = s_1 = 2: e^0 * 2 * 1
+
+
+# --------------------------------------------------------------------------
+# Greedy routing
+# --------------------------------------------------------------------------
+def _best_subset(E_row, sizes, budget):
+    best = 0.0
+    idx = [c for c in range(len(sizes)) if sizes[c] > 0]
+    for r in range(len(idx) + 1):
+        for S in itertools.combinations(idx, r):
+            if sum(sizes[c] for c in S) <= budget:
+                best = max(best, float(sum(E_row[c] for c in S)))
+    return best
+
+
+def test_route_equal_sizes_equals_exhaustive_optimum():
+    g = np.random.default_rng(9)
+    for trial in range(20):
+        Ck, n = 10, 4
+        k_off = np.arange(0, (Ck + 1) * n, n, dtype=np.int32)
+        E = g.random((1, Ck)).astype(np.float32)
+        density = g.random()
+        po, pk = oracle.route(E, np.array([0, 3], np.int32), k_off, Ck * n, density)
+        budget = math.floor(density * Ck * n)
+        got = float(E[0, pk].astype(np.float64).sum())
+        assert math.isclose(got, _best_subset(E[0].astype(np.float64), [n] * Ck, budget), rel_tol=1e-6)
+
+
+def test_route_unequal_sizes_within_fractional_knapsack_bound():
+    g = np.random.default_rng(10)
+    for trial in range(30):
+        Ck = 9
+        sizes = g.integers(0, 8, Ck)
+        k_off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+        Nk = int(sizes.sum())
+        E = g.random((1, Ck)).astype(np.float32) * 10
+        density = g.random()
+        po, pk = oracle.route(E, np.array([0, 5], np.int32), k_off, Nk, density)
+        budget = math.floor(density * Nk)
+        assert sizes[pk].sum() <= budget
+        assert np.all(sizes[pk] > 0) and np.all(np.diff(pk) > 0)
+        got = float(E[0, pk].astype(np.float64).sum())
+        opt = _best_subset(E[0].astype(np.float64), sizes.tolist(), budget)
+        assert got >= opt - float(E[0][sizes > 0].max()) - 1e-6
+        assert got <= opt + 1e-6
+
+
+def test_route_skips_a_misfit_and_continues():
+    # ratios: c1 = 9/2, c0 = 10/3, c2 = 1/1; budget 4 keys: take c1, c0 does
+    # not fit (5 > 4) and is skipped, c2 still fits.
+    E = np.array([[10.0, 9.0, 1.0]], dtype=np.float32)
+    k_off = np.array([0, 3, 5, 6], dtype=np.int32)
+    po, pk = oracle.route(E, np.array([0, 2], np.int32), k_off, 8, 0.5)
+    assert pk.tolist() == [1, 2]
+
+
+def test_route_density_one_takes_everything_and_ties_go_low():
+    k_off = np.array([0, 2, 2, 5, 6], dtype=np.int32)         # cluster 1 empty
+    q_off = np.array([0, 3, 3, 4], dtype=np.int32)            # query cluster 1 empty
+    E = np.ones((3, 4), dtype=np.float32)
+    po, pk = oracle.route(E, q_off, k_off, 6, 1.0)
+    assert po.tolist() == [0, 3, 3, 6]
+    assert pk.tolist() == [0, 2, 3, 0, 2, 3]
+    # equal ratio everywhere, room for two of three size-2 clusters -> 0 and 1
+    k2 = np.array([0, 2, 4, 6], dtype=np.int32)
+    po, pk = oracle.route(np.ones((1, 3), np.float32) * 2, np.array([0, 1], np.int32), k2, 6, 0.7)
+    assert pk.tolist() == [0, 1]
+
+
+# --------------------------------------------------------------------------
+# Attention with compensation
+# --------------------------------------------------------------------------
+def _random_clustered_head(g, Nq=40, Nk=50, d=8, Cq=5, Ck=7):
+    Q = g.standard_normal((Nq, d)); K = g.standard_normal((Nk, d)); V = g.standard_normal((Nk, d))
+    lq = g.integers(0, Cq, Nq); lk = g.integers(0, Ck, Nk)
+    pq, oq = oracle.stable_sort(lq, Cq)
+    pk, ok = oracle.stable_sort(lk, Ck)
+    return Q, K, V, pq, oq, pk, ok
+
+
+def _all_pairs(q_off, k_off):
+    Cq, Ck = len(q_off) - 1, len(k_off) - 1
+    po, pk = [0], []
+    for i in range(Cq):
+        if q_off[i + 1] > q_off[i]:
+            pk += [c for c in range(Ck) if k_off[c + 1] > k_off[c]]
+        po.append(len(pk))
+    return np.array(po, np.int32), np.array(pk, np.int32)
+
+
+def test_density_one_is_dense_softmax_attention_in_original_order():
+    g = np.random.default_rng(11)
+    Q, K, V, pq, oq, pk, ok = _random_clustered_head(g)
+    Kp, Vp = K[pk], V[pk]
+    kbar, vbar = oracle.segment_mean(Kp, ok), oracle.segment_mean(Vp, ok)
+    po, pkc = _all_pairs(oq, ok)
+    scale = 0.35
+    O, lse = oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, scale)
+    S = Q @ K.T * scale
+    assert np.allclose(O, softmax(S, axis=-1) @ V, rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse, np.log(np.exp(S).sum(-1)), rtol=1e-12)
+
+
+def test_identical_keys_or_singletons_make_compensation_exact():
+    g = np.random.default_rng(12)
+    d, Ck = 8, 6
+    sizes = np.array([4, 1, 6, 1, 3, 5])
+    kc = g.standard_normal((Ck, d))
+    Kp = np.repeat(kc, sizes, axis=0)
+    Vp = g.standard_normal((sizes.sum(), d))
+    ok = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Q = g.standard_normal((30, d))
+    oq = np.array([0, 10, 30], np.int32)
+    pq = g.permutation(30).astype(np.int32)
+    kbar, vbar = oracle.segment_mean(Kp, ok), oracle.segment_mean(Vp, ok)
+    po = np.array([0, 2, 3], np.int32); pkc = np.array([1, 4, 2], np.int32)
+    O, _ = oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, 0.5)
+    dense = softmax(Q @ Kp.T * 0.5, axis=-1) @ Vp
+    assert np.allclose(O, dense, rtol=1e-11, atol=1e-12)
+
+
+def test_output_is_invariant_under_token_relabelling():
+    g = np.random.default_rng(13)
+    Q, K, V, pq, oq, pk, ok = _random_clustered_head(g)
+    lq = np.repeat(np.arange(len(oq) - 1), np.diff(oq))[np.argsort(pq)]
+    lk = np.repeat(np.arange(len(ok) - 1), np.diff(ok))[np.argsort(pk)]
+    po, pkc = np.array([0, 2, 3, 3, 5, 6], np.int32), np.array([0, 3, 6, 1, 5, 2], np.int32)
+
+    def run(Q, K, V, lq, lk):
+        pq, oq = oracle.stable_sort(lq, 5)
+        pk, ok = oracle.stable_sort(lk, 7)
+        Kp, Vp = K[pk], V[pk]
+        kbar, vbar = oracle.segment_mean(Kp, ok), oracle.segment_mean(Vp, ok)
+        return oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, 0.4)[0]
+
+    O = run(Q, K, V, lq, lk)
+    sq, sk = g.permutation(len(Q)), g.permutation(len(K))
+    O2 = run(Q[sq], K[sk], V[sk], lq[sq], lk[sk])
+    assert np.allclose(O2, O[sq], rtol=1e-11, atol=1e-12)
+
+
+def test_centroid_estimate_never_exceeds_true_weight():
+    # mean(e^s) >= e^{mean s} (Jensen): compensated denominators under-count.
+    g = np.random.default_rng(14)
+    Q, K, V, pq, oq, pk, ok = _random_clustered_head(g, d=16)
+    Kp, Vp = K[pk], V[pk]
+    kbar, vbar = oracle.segment_mean(Kp, ok), oracle.segment_mean(Vp, ok)
+    po_all, pk_all = _all_pairs(oq, ok)
+    _, lse_dense = oracle.attend(Q[pq], Kp, Vp, oq, ok, po_all, pk_all, kbar, vbar, pq, 0.5)
+    po = np.array([0, 1, 1, 3, 3, 4], np.int32); pkc = np.array([2, 0, 6, 4], np.int32)
+    _, lse = oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, 0.5)
+    assert np.all(lse <= lse_dense + 1e-12)
+    assert np.any(lse < lse_dense - 1e-3)
+
+
+def test_row_subset_matches_full_output():
+    g = np.random.default_rng(15)
+    Q, K, V, pq, oq, pk, ok = _random_clustered_head(g)
+    Kp, Vp = K[pk], V[pk]
+    kbar, vbar = oracle.segment_mean(Kp, ok), oracle.segment_mean(Vp, ok)
+    po = np.array([0, 2, 3, 3, 5, 6], np.int32); pkc = np.array([0, 3, 6, 1, 5, 2], np.int32)
+    O, lse = oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, 0.4)
+    rows = np.array([39, 0, 17, 5])
+    Or, lr = oracle.attend(Q[pq], Kp, Vp, oq, ok, po, pkc, kbar, vbar, pq, 0.4, rows=rows)
+    assert np.array_equal(Or, O[pq[rows]]) and np.array_equal(lr, lse[pq[rows]])
+
+
+def test_layer_at_density_one_equals_dense_attention():
+    g = np.random.default_rng(16)
+    Q = g.standard_normal((96, 8)); K = g.standard_normal((80, 8)); V = g.standard_normal((80, 8))
+    out = oracle.layer(Q, K, V, Cq=4, Ck=6, iters=3, density=1.0, scale=0.3,
+                       seed_q=1, seed_k=2, stream=0)
+    assert np.allclose(out["O"], softmax(Q @ K.T * 0.3, axis=-1) @ V, rtol=1e-11, atol=1e-12)
