@@ -1,0 +1,16 @@
+"""B200-native clustered sparse attention (SVG-EAR on SVG2's permutation).
+
+The compute path lives in libsvgear.so (CUDA, sm_100a) behind the C ABI of
+include/svgear.h; ``_lib`` is its thin ctypes binding.  Import of the
+package does not load the library; the first call does, and raises if the
+library is missing -- there is no CPU path.
+"""
+from ._lib import (Clustering, SvgearError, kernel_launches, layer, lib, svgear_attend, svgear_centroids,
+                   svgear_cluster, svgear_kmeans_assign, svgear_kmeans_update,
+                   svgear_kmeanspp_init, svgear_label_sort, svgear_permute, svgear_probe,
+                   svgear_route, svgear_route_select, workspace_bytes)
+
+__all__ = ["Clustering", "SvgearError", "kernel_launches", "layer", "lib", "svgear_attend", "svgear_centroids",
+           "svgear_cluster", "svgear_kmeans_assign", "svgear_kmeans_update",
+           "svgear_kmeanspp_init", "svgear_label_sort", "svgear_permute", "svgear_probe",
+           "svgear_route", "svgear_route_select", "workspace_bytes"]

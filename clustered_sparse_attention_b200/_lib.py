@@ -1,0 +1,302 @@
+"""ctypes binding of libsvgear.so (include/svgear.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels on
+torch's current stream.  Output and workspace buffers are allocated with
+torch (device memory plumbing); the library itself never allocates.  There
+is no CPU path: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libsvgear.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+F32, BF16 = 0, 1
+OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
+MAX_CLUSTERS = 4096
+
+EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
+            "svgear_label_sort", "svgear_kmeans_update", "svgear_permute",
+            "svgear_centroids", "svgear_probe", "svgear_route_select", "svgear_route",
+            "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
+            "svgear_version", "svgear_kernel_launches")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class SvgearError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__("%s failed: %s (%d)" % (fn, msg, status))
+        self.status = status
+
+
+_L = None
+
+
+def lib():
+    """Load libsvgear.so; raises if it has not been built."""
+    global _L
+    if _L is not None:
+        return _L
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libsvgear.so is not built (run clustered_sparse_attention_b200/build.py"
+                           " or __graft_entry__.build()); there is no fallback path")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, U64, F, SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_float,
+                          ctypes.c_size_t)
+    sig = {
+        "svgear_cluster": [P, Dims, I32, I32, P, U64, P, P, P, P, P, P, SZ, P],
+        "svgear_kmeanspp_init": [P, Dims, I32, U64, P, P, P, SZ, P],
+        "svgear_kmeans_assign": [P, Dims, P, I32, P, P],
+        "svgear_label_sort": [P, Dims, I32, P, P, P, SZ, P],
+        "svgear_kmeans_update": [P, Dims, P, I32, P, P, SZ, P],
+        "svgear_permute": [P, P, Dims, P, P],
+        "svgear_centroids": [P, P, I32, Dims, P, P],
+        "svgear_probe": [P, I32, P, P, P, P, P, I32, Dims, F, P, P, SZ, P],
+        "svgear_route_select": [P, P, I32, P, I32, I32, I32, I32, F, P, P, P, SZ, P],
+        "svgear_route": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, SZ, P],
+        "svgear_attend": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, P, SZ, P],
+        "svgear_workspace_bytes": [I32, Dims, I32, I32],
+        "svgear_status_string": [ctypes.c_int],
+        "svgear_version": [],
+        "svgear_kernel_launches": [],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    L.svgear_workspace_bytes.restype = SZ
+    L.svgear_status_string.restype = ctypes.c_char_p
+    L.svgear_kernel_launches.restype = ctypes.c_uint64
+    _L = L
+    return L
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(lib().svgear_kernel_launches())
+
+
+def _check(fn, status):
+    if status != OK:
+        raise SvgearError(fn, status, lib().svgear_status_string(status).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("token tensors must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _tokens(t, name):
+    if not (t.is_cuda and t.dim() == 4 and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous CUDA tensor [B, H, N, d]" % name)
+    B, H, N, d = t.shape
+    return Dims(B, H, N, d, _dtype_code(t))
+
+
+def _cuda(t, name, dtype):
+    if not (t.is_cuda and t.is_contiguous() and t.dtype == dtype):
+        raise ValueError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
+    return t
+
+
+def workspace_bytes(op, dims, c1, c2=0):
+    return int(lib().svgear_workspace_bytes(op, dims, c1, c2))
+
+
+def _workspace(op, dims, c1, c2, device):
+    # A zero answer means the sizes are invalid: pass a token buffer and let
+    # the entry point report the precise status.
+    n = max(workspace_bytes(op, dims, c1, c2), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device), n
+
+
+@dataclass
+class Clustering:
+    labels: torch.Tensor      # int32 [B, H, N]
+    perm: torch.Tensor        # int32 [B, H, N]
+    offsets: torch.Tensor     # int32 [B, H, C+1]
+    centroids: torch.Tensor   # float32 [B, H, C, d]
+    Xp: torch.Tensor | None   # [B, H, N, d] permuted copy
+
+
+def svgear_cluster(X, C, iters, warm_centroids=None, seed=0, permuted=True, out=None):
+    dims = _tokens(X, "X")
+    B, H, N, d = X.shape
+    dev = X.device
+    if out is None:
+        out = Clustering(
+            torch.empty((B, H, N), dtype=torch.int32, device=dev),
+            torch.empty((B, H, N), dtype=torch.int32, device=dev),
+            torch.empty((B, H, C + 1), dtype=torch.int32, device=dev),
+            torch.empty((B, H, C, d), dtype=torch.float32, device=dev),
+            torch.empty_like(X) if permuted else None)
+    if warm_centroids is not None:
+        _cuda(warm_centroids, "warm_centroids", torch.float32)
+    ws, n = _workspace(OP_CLUSTER, dims, C, 0, dev)
+    _check("svgear_cluster", lib().svgear_cluster(
+        _ptr(X), dims, C, iters, _ptr(warm_centroids), seed, _ptr(out.labels), _ptr(out.perm),
+        _ptr(out.offsets), _ptr(out.centroids), _ptr(out.Xp), _ptr(ws), n, _stream()))
+    return out
+
+
+def svgear_kmeanspp_init(X, C, seed=0):
+    dims = _tokens(X, "X")
+    B, H, N, d = X.shape
+    cent = torch.empty((B, H, C, d), dtype=torch.float32, device=X.device)
+    idx = torch.empty((B, H, C), dtype=torch.int32, device=X.device)
+    ws, n = _workspace(OP_KMEANSPP, dims, C, 0, X.device)
+    _check("svgear_kmeanspp_init", lib().svgear_kmeanspp_init(
+        _ptr(X), dims, C, seed, _ptr(cent), _ptr(idx), _ptr(ws), n, _stream()))
+    return cent, idx
+
+
+def svgear_kmeans_assign(X, centroids):
+    dims = _tokens(X, "X")
+    _cuda(centroids, "centroids", torch.float32)
+    B, H, N, d = X.shape
+    C = centroids.shape[2]
+    labels = torch.empty((B, H, N), dtype=torch.int32, device=X.device)
+    _check("svgear_kmeans_assign", lib().svgear_kmeans_assign(
+        _ptr(X), dims, _ptr(centroids), C, _ptr(labels), _stream()))
+    return labels
+
+
+def svgear_label_sort(labels, C):
+    _cuda(labels, "labels", torch.int32)
+    B, H, N = labels.shape
+    dims = Dims(B, H, N, 64, F32)
+    perm = torch.empty_like(labels)
+    off = torch.empty((B, H, C + 1), dtype=torch.int32, device=labels.device)
+    ws, n = _workspace(OP_LABEL_SORT, dims, C, 0, labels.device)
+    _check("svgear_label_sort", lib().svgear_label_sort(
+        _ptr(labels), dims, C, _ptr(perm), _ptr(off), _ptr(ws), n, _stream()))
+    return perm, off
+
+
+def svgear_kmeans_update(X, labels, centroids):
+    """Returns a new tensor: member means, previous rows for empty clusters."""
+    dims = _tokens(X, "X")
+    _cuda(labels, "labels", torch.int32)
+    out = _cuda(centroids, "centroids", torch.float32).clone()
+    C = centroids.shape[2]
+    ws, n = _workspace(OP_KMEANS_UPDATE, dims, C, 0, X.device)
+    _check("svgear_kmeans_update", lib().svgear_kmeans_update(
+        _ptr(X), dims, _ptr(labels), C, _ptr(out), _ptr(ws), n, _stream()))
+    return out
+
+
+def svgear_permute(X, perm):
+    dims = _tokens(X, "X")
+    _cuda(perm, "perm", torch.int32)
+    Xp = torch.empty_like(X)
+    _check("svgear_permute", lib().svgear_permute(_ptr(X), _ptr(perm), dims, _ptr(Xp), _stream()))
+    return Xp
+
+
+def svgear_centroids(Xp, offsets, C=None):
+    dims = _tokens(Xp, "Xp")
+    _cuda(offsets, "offsets", torch.int32)
+    C = offsets.shape[-1] - 1 if C is None else C
+    B, H, N, d = Xp.shape
+    out = torch.empty((B, H, C, d), dtype=torch.float32, device=Xp.device)
+    _check("svgear_centroids", lib().svgear_centroids(
+        _ptr(Xp), _ptr(offsets), C, dims, _ptr(out), _stream()))
+    return out
+
+
+def svgear_probe(qbar, Kp, Vp, kbar, vbar, k_off, scale):
+    kd = _tokens(Kp, "Kp")
+    _tokens(Vp, "Vp")
+    B, H, Cq, d = qbar.shape
+    Ck = kbar.shape[2]
+    E = torch.empty((B, H, Cq, Ck), dtype=torch.float32, device=Kp.device)
+    ws, n = _workspace(OP_ROUTE, kd, Cq, Ck, Kp.device)
+    _check("svgear_probe", lib().svgear_probe(
+        _ptr(qbar), Cq, _ptr(Kp), _ptr(Vp), _ptr(kbar), _ptr(vbar), _ptr(k_off), Ck, kd,
+        float(scale), _ptr(E), _ptr(ws), n, _stream()))
+    return E
+
+
+def svgear_route_select(E, q_off, k_off, Nk, density):
+    _cuda(E, "E", torch.float32)
+    B, H, Cq, Ck = E.shape
+    pair_off = torch.empty((B, H, Cq + 1), dtype=torch.int32, device=E.device)
+    pair_kc = torch.empty((B, H, Cq * Ck), dtype=torch.int32, device=E.device)
+    ws, n = _workspace(OP_ROUTE, Dims(B, H, Nk, 64, F32), Cq, Ck, E.device)
+    _check("svgear_route_select", lib().svgear_route_select(
+        _ptr(E), _ptr(q_off), Cq, _ptr(k_off), Ck, B, H, Nk, float(density), _ptr(pair_off),
+        _ptr(pair_kc), _ptr(ws), n, _stream()))
+    return pair_off, pair_kc
+
+
+def svgear_route(qbar, q_off, kbar, vbar, k_off, Kp, Vp, density, scale, return_errors=False):
+    kd = _tokens(Kp, "Kp")
+    _tokens(Vp, "Vp")
+    B, H, Cq, d = qbar.shape
+    Ck = kbar.shape[2]
+    dev = Kp.device
+    pair_off = torch.empty((B, H, Cq + 1), dtype=torch.int32, device=dev)
+    pair_kc = torch.empty((B, H, Cq * Ck), dtype=torch.int32, device=dev)
+    E = torch.empty((B, H, Cq, Ck), dtype=torch.float32, device=dev) if return_errors else None
+    ws, n = _workspace(OP_ROUTE, kd, Cq, Ck, dev)
+    _check("svgear_route", lib().svgear_route(
+        _ptr(qbar), _ptr(q_off), Cq, _ptr(kbar), _ptr(vbar), _ptr(k_off), Ck, _ptr(Kp), _ptr(Vp),
+        kd, float(density), float(scale), _ptr(pair_off), _ptr(pair_kc), _ptr(E), _ptr(ws), n,
+        _stream()))
+    return (pair_off, pair_kc, E) if return_errors else (pair_off, pair_kc)
+
+
+def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm, scale, O=None):
+    qd = _tokens(Qp, "Qp")
+    _tokens(Kp, "Kp")
+    _tokens(Vp, "Vp")
+    Cq = q_off.shape[-1] - 1
+    Ck = k_off.shape[-1] - 1
+    Nk = Kp.shape[2]
+    if O is None:
+        O = torch.empty_like(Qp)
+    ws, n = _workspace(OP_ATTEND, qd, Cq, Ck, Qp.device)
+    _check("svgear_attend", lib().svgear_attend(
+        _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Nk, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(pair_off),
+        _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(q_perm), float(scale), _ptr(O), _ptr(ws), n,
+        _stream()))
+    return O
+
+
+def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None):
+    """The whole layer for [B, H, N, d] tensors: cluster Q and K (seeds 2*seed
+    and 2*seed+1), permute V, value centroids, route, attend.  Returns O in the
+    original token order and every intermediate."""
+    d = Q.shape[-1]
+    scale = d ** -0.5 if scale is None else scale
+    cq = svgear_cluster(Q, Cq, iters, warm_q, seed=2 * seed)
+    ck = svgear_cluster(K, Ck, iters, warm_k, seed=2 * seed + 1)
+    Vp = svgear_permute(V, ck.perm)
+    vbar = svgear_centroids(Vp, ck.offsets, Ck)
+    pair_off, pair_kc = svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
+                                     ck.Xp, Vp, density, scale)
+    O = svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, pair_off, pair_kc, ck.centroids,
+                      vbar, cq.perm, scale)
+    return {"O": O, "q": cq, "k": ck, "Vp": Vp, "vbar": vbar, "pair_off": pair_off,
+            "pair_kc": pair_kc}

@@ -1,0 +1,473 @@
+// kmeans.cu -- k-means++ seeding, assignment, segment means and the
+// permutation gather.
+//
+// Method: SVG2 (paper-graph summary, "Sparse VideoGen2 ...", section 3.4,
+// "The clustering operation" and "Fast k-means with centroid cache"):
+// independent k-means over the query and the key tokens of every head,
+// k-means++ seeding for a cold start, centroid = mean of members; the
+// permutation that makes clusters contiguous ("The permutation operation").
+// The SVG-EAR task page (sotabase FrontierCS-2, agent step 1) adds that the
+// k-means returns the sorted order and that a small kernel averages each
+// cluster's values in one pass.
+//
+// B200 design: every pass over a token tensor moves 16-byte chunks with a
+// group of lanes per token row (coalesced 128-bit loads); the assignment is a
+// register-tiled fp32 contraction (tokens x centroids) with the argmin fused
+// into its epilogue, so labels are the only output.
+#include "common.cuh"
+#include "launchers.h"
+
+namespace svgear {
+
+// ---------------------------------------------------------------------------
+// k-means++: per pass j, (1) D^2 <- min(D^2, |x - seed_{j-1}|^2) with a
+// deterministic fp64 scan per block of kKppTokens tokens, (2) one block per
+// head locates the token where the running sum crosses u_j * sum(D^2).
+// ---------------------------------------------------------------------------
+constexpr int kKppThreads = 256;
+
+// Inclusive fp64 prefix of 1024 fp32 values (4 per thread, token order) with
+// a fixed reduction structure, so every call on the same values gives the
+// same bits.  incl_tok receives the prefix at each of the thread's 4 tokens.
+__device__ inline void kpp_block_scan(const float* d2s, double* warp_tot,
+                                      double incl_tok[4]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double s[4], run = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { run += (double)d2s[tid * 4 + i]; s[i] = run; }
+    double x = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    double ex = __shfl_up_sync(0xffffffffu, x, 1);
+    if (lane == 0) ex = 0.0;
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    double wbase = 0.0;
+    for (int w = 0; w < warp; ++w) wbase += warp_tot[w];
+    double base = wbase + ex;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) incl_tok[i] = base + s[i];
+}
+
+template <typename T>
+__global__ void kpp_first_kernel(const T* __restrict__ X, int N, int D, int C,
+                                 uint64_t seed, int32_t* chosen, float* centroids) {
+    const int bh = blockIdx.x;
+    double u = philox_uniform(seed, (uint64_t)bh, 0);
+    long long t = (long long)floor(u * (double)N);
+    if (t >= N) t = N - 1;
+    if (threadIdx.x == 0) chosen[(size_t)bh * C] = (int32_t)t;
+    const T* row = X + ((size_t)bh * N + t) * D;
+    for (int k = threadIdx.x; k < D; k += blockDim.x)
+        centroids[(size_t)bh * C * D + k] = Elem<T>::from(row[k]);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kKppThreads)
+kpp_update_kernel(const T* __restrict__ X, int N, int nblk, const int32_t* chosen,
+                  int C, int j, float* D2, double* blocksum) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int L = D / EPC;                 // lanes per token row
+    constexpr int RP = kKppThreads / L;        // rows per pass
+    __shared__ float cen[D];
+    __shared__ float d2s[kKppTokens];
+    __shared__ double warp_tot[kKppThreads / 32];
+    const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
+    const T* Xh = X + (size_t)bh * N * D;
+    const int st = chosen[(size_t)bh * C + j - 1];
+    for (int k = tid; k < D; k += kKppThreads) cen[k] = Elem<T>::from(Xh[(size_t)st * D + k]);
+    __syncthreads();
+    const int lane = tid % L;
+    for (int r = tid / L; r < kKppTokens; r += RP) {
+        const int t = blk * kKppTokens + r;
+        float part = 0.f;
+        if (t < N) {
+            float x[EPC];
+            Elem<T>::load(Xh + (size_t)t * D + lane * EPC, x);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                float df = x[e] - cen[lane * EPC + e];
+                part = fmaf(df, df, part);
+            }
+        }
+#pragma unroll
+        for (int o = L / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) {
+            float v = 0.f;
+            if (t < N) {
+                v = part;
+                if (j > 1) v = fminf(v, D2[(size_t)bh * N + t]);
+                D2[(size_t)bh * N + t] = v;
+            }
+            d2s[r] = v;
+        }
+    }
+    __syncthreads();
+    double incl[4];
+    kpp_block_scan(d2s, warp_tot, incl);
+    if (tid == kKppThreads - 1) blocksum[(size_t)bh * nblk + blk] = incl[3];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kKppThreads)
+kpp_pick_kernel(const T* __restrict__ X, int N, int D, int nblk, int32_t* chosen, int C,
+                int j, const float* D2, const double* blocksum, uint64_t seed,
+                float* centroids) {
+    __shared__ float d2s[kKppTokens];
+    __shared__ double warp_tot[kKppThreads / 32];
+    __shared__ int s_blk, s_pick;
+    __shared__ double s_base, s_target;
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const double* bs = blocksum + (size_t)bh * nblk;
+    const float* d2 = D2 + (size_t)bh * N;
+    int32_t* ch = chosen + (size_t)bh * C;
+    if (tid == 0) {
+        double total = 0.0;
+        for (int b = 0; b < nblk; ++b) total += bs[b];
+        s_pick = 0x7fffffff;
+        if (total > 0.0) {
+            double target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
+            s_target = target;
+            s_blk = -2;
+            double run = 0.0;
+            for (int b = 0; b < nblk; ++b) {
+                double prev = run;
+                run = prev + bs[b];
+                if (run > target) { s_blk = b; s_base = prev; break; }
+            }
+        } else {
+            s_blk = -3;
+        }
+    }
+    __syncthreads();
+    const int blk = s_blk;
+    if (blk >= 0) {
+        for (int r = tid; r < kKppTokens; r += kKppThreads) {
+            int t = blk * kKppTokens + r;
+            d2s[r] = (t < N) ? d2[t] : 0.f;
+        }
+        __syncthreads();
+        double incl[4];
+        kpp_block_scan(d2s, warp_tot, incl);
+        for (int i = 0; i < 4; ++i) {
+            if (s_base + incl[i] > s_target) {
+                atomicMin(&s_pick, blk * kKppTokens + tid * 4 + i);
+                break;
+            }
+        }
+        __syncthreads();
+    } else if (tid == 0) {
+        int pick = 0;
+        if (blk == -2) {            // rounding left no token above the target
+            for (int t = N - 1; t >= 0; --t)
+                if (d2[t] > 0.f) { pick = t; break; }
+        } else {                    // every D^2 is zero: lowest unchosen token
+            for (int t = 0; t < N; ++t) {
+                bool used = false;
+                for (int q = 0; q < j; ++q) used |= (ch[q] == t);
+                if (!used) { pick = t; break; }
+            }
+        }
+        s_pick = pick;
+    }
+    __syncthreads();
+    const int pick = s_pick < N ? s_pick : N - 1;
+    if (tid == 0) ch[j] = pick;
+    const T* row = X + ((size_t)bh * N + pick) * D;
+    for (int k = tid; k < D; k += kKppThreads)
+        centroids[((size_t)bh * C + j) * D + k] = Elem<T>::from(row[k]);
+}
+
+template <typename T, int D>
+static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed,
+                         float* cent, int32_t* chosen, float* D2, double* blocksum,
+                         cudaStream_t st) {
+    const int BH = dims.B * dims.H, N = dims.N;
+    const int nblk = ceil_div(N, kKppTokens);
+    kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    for (int j = 1; j < C; ++j) {
+        kpp_update_kernel<T, D><<<dim3(nblk, BH), kKppThreads, 0, st>>>(
+            X, N, nblk, chosen, C, j, D2, blocksum);
+        count_launches(1);
+        kpp_pick_kernel<T><<<BH, kKppThreads, 0, st>>>(X, N, D, nblk, chosen, C, j, D2,
+                                                        blocksum, seed, cent);
+        count_launches(1);
+    }
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Assignment: a 128-token x 128-centroid register-tiled fp32 contraction per
+// step (256 threads, 8x8 per thread), distance |c|^2 - 2 x.c, argmin fused.
+// ---------------------------------------------------------------------------
+constexpr int kAsTM = 128, kAsTN = 128, kAsKC = 32, kAsThreads = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kAsThreads, 2)
+assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, int C,
+              int32_t* __restrict__ labels) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    extern __shared__ __align__(16) float smem[];
+    float* Xs = smem;                  // [D][kAsTM]  (transposed tile)
+    float* Cs = Xs + D * kAsTM;        // [kAsKC][kAsTN]
+    float* cn = Cs + kAsKC * kAsTN;    // [kAsTN]
+    const int bh = blockIdx.y, t0 = blockIdx.x * kAsTM, tid = threadIdx.x;
+    const T* Xh = X + (size_t)bh * N * D;
+    const float* Ch = cent + (size_t)bh * C * D;
+
+    for (int q = tid; q < kAsTM * (D / EPC); q += kAsThreads) {
+        const int row = q / (D / EPC), col = (q % (D / EPC)) * EPC;
+        float v[EPC];
+        if (t0 + row < N) Elem<T>::load(Xh + (size_t)(t0 + row) * D + col, v);
+        else
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) v[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) Xs[(col + e) * kAsTM + row] = v[e];
+    }
+
+    const int tx = tid & 15, ty = tid >> 4;
+    float bestd[8];
+    int besti[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { bestd[i] = __int_as_float(0x7f800000); besti[i] = 0; }
+
+    for (int c0 = 0; c0 < C; c0 += kAsTN) {
+        __syncthreads();
+        if (tid < kAsTN) {
+            const int c = c0 + tid;
+            float s = 0.f;
+            if (c < C)
+                for (int k = 0; k < D; ++k) { float v = Ch[(size_t)c * D + k]; s = fmaf(v, v, s); }
+            cn[tid] = s;
+        }
+        float acc[8][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+
+        for (int k0 = 0; k0 < D; k0 += kAsKC) {
+            __syncthreads();
+            for (int q = tid; q < kAsTN * (kAsKC / 4); q += kAsThreads) {
+                const int cc = q / (kAsKC / 4), kk = (q % (kAsKC / 4)) * 4;
+                const int c = c0 + cc;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (c < C) v = __ldg(reinterpret_cast<const float4*>(Ch + (size_t)c * D + k0 + kk));
+                Cs[(kk + 0) * kAsTN + cc] = v.x;
+                Cs[(kk + 1) * kAsTN + cc] = v.y;
+                Cs[(kk + 2) * kAsTN + cc] = v.z;
+                Cs[(kk + 3) * kAsTN + cc] = v.w;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int k = 0; k < kAsKC; ++k) {
+                const float* xr = Xs + (k0 + k) * kAsTM;
+                const float* cr = Cs + k * kAsTN;
+                float4 a0 = *reinterpret_cast<const float4*>(xr + ty * 4);
+                float4 a1 = *reinterpret_cast<const float4*>(xr + 64 + ty * 4);
+                float4 b0 = *reinterpret_cast<const float4*>(cr + tx * 4);
+                float4 b1 = *reinterpret_cast<const float4*>(cr + 64 + tx * 4);
+                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(a[i], b[jj], acc[i][jj]);
+            }
+        }
+        // candidates of this thread come in increasing centroid order
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int cj = (jj < 4) ? tx * 4 + jj : 64 + tx * 4 + (jj - 4);
+            const int c = c0 + cj;
+            if (c < C) {
+                const float cnv = cn[cj];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float dist = fmaf(-2.f, acc[i][jj], cnv);
+                    if (dist < bestd[i]) { bestd[i] = dist; besti[i] = c; }
+                }
+            }
+        }
+    }
+    // lexicographic (distance, index) minimum over the 16 threads of a row group
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float dd = bestd[i];
+        int ix = besti[i];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+            float od = __shfl_xor_sync(0xffffffffu, dd, o);
+            int oi = __shfl_xor_sync(0xffffffffu, ix, o);
+            if (od < dd || (od == dd && oi < ix)) { dd = od; ix = oi; }
+        }
+        if (tx == 0) {
+            const int row = (i < 4) ? ty * 4 + i : 64 + ty * 4 + (i - 4);
+            if (t0 + row < N) labels[(size_t)bh * N + t0 + row] = ix;
+        }
+    }
+}
+
+template <typename T, int D>
+static int assign_impl(const T* X, svgear_dims dims, const float* cent, int C,
+                       int32_t* labels, cudaStream_t st) {
+    const size_t smem = sizeof(float) * (D * kAsTM + kAsKC * kAsTN + kAsTN);
+    // per-device function attribute; cheap enough to set on every call
+    if (cudaFuncSetAttribute(assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return SVGEAR_ERR_CUDA;
+    const int BH = dims.B * dims.H;
+    assign_kernel<T, D><<<dim3(ceil_div(dims.N, kAsTM), BH), kAsThreads, smem, st>>>(
+        X, dims.N, cent, C, labels);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Segment mean: one block per (cluster, head); a group of lanes per row moves
+// 16-byte chunks; fp32 partial sums are combined in a fixed order.
+// ---------------------------------------------------------------------------
+constexpr int kSmThreads = 128;
+
+template <typename T, int D, bool GATHER>
+__global__ void __launch_bounds__(kSmThreads)
+segment_mean_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
+                    const int32_t* __restrict__ offsets, int N, int C, float* out,
+                    bool empty_zero) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int L = D / EPC;
+    constexpr int R = kSmThreads / L;
+    __shared__ float part[R][D];
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int32_t* off = offsets + (size_t)bh * (C + 1);
+    const int a = off[c], b = off[c + 1];
+    float* o = out + ((size_t)bh * C + c) * D;
+    if (b <= a || a < 0 || b > N) {   // empty (or malformed) segment
+        if (empty_zero)
+            for (int k = tid; k < D; k += kSmThreads) o[k] = 0.f;
+        return;
+    }
+    const T* Xh = X + (size_t)bh * N * D;
+    const int lane = tid % L, grp = tid / L;
+    float acc[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    for (int p = a + grp; p < b; p += R) {
+        int row = GATHER ? perm[(size_t)bh * N + p] : p;
+        if ((unsigned)row >= (unsigned)N) continue;
+        float v[EPC];
+        Elem<T>::load(Xh + (size_t)row * D + lane * EPC, v);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] += v[e];
+    }
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) part[grp][lane * EPC + e] = acc[e];
+    __syncthreads();
+    const float n = (float)(b - a);
+    for (int k = tid; k < D; k += kSmThreads) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < R; ++g) s += part[g][k];
+        o[k] = s / n;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Permutation gather: Xp[p] = X[perm[p]], one 16-byte chunk per thread.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void permute_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
+                               int N, T* __restrict__ Xp) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int L = D / EPC;
+    const int bh = blockIdx.y;
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long p = idx / L;
+    const int lane = (int)(idx % L);
+    if (p >= N) return;
+    const int row = perm[(size_t)bh * N + p];
+    if ((unsigned)row >= (unsigned)N) return;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + ((size_t)bh * N + row) * D + lane * EPC));
+    *reinterpret_cast<uint4*>(Xp + ((size_t)bh * N + p) * D + lane * EPC) = v;
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch on (dtype, d).
+// ---------------------------------------------------------------------------
+#define SVGEAR_DISPATCH(dims, FN, ...)                                              \
+    do {                                                                             \
+        if ((dims).dtype == SVGEAR_BF16) {                                           \
+            if ((dims).d == 128) return FN<__nv_bfloat16, 128>(__VA_ARGS__);          \
+            if ((dims).d == 64) return FN<__nv_bfloat16, 64>(__VA_ARGS__);            \
+        } else if ((dims).dtype == SVGEAR_F32) {                                     \
+            if ((dims).d == 128) return FN<float, 128>(__VA_ARGS__);                  \
+            if ((dims).d == 64) return FN<float, 64>(__VA_ARGS__);                    \
+        }                                                                            \
+        return SVGEAR_ERR_UNSUPPORTED;                                               \
+    } while (0)
+
+template <typename T, int D>
+static int kmeanspp_disp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+                         int32_t* chosen, float* D2, double* bs, cudaStream_t st) {
+    return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, cent, chosen, D2, bs, st);
+}
+int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+                    int32_t* chosen, float* D2, double* bs, cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, cent, chosen, D2, bs, st);
+}
+
+template <typename T, int D>
+static int assign_disp(const void* X, svgear_dims dims, const float* cent, int C,
+                       int32_t* labels, cudaStream_t st) {
+    return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, st);
+}
+int launch_assign(const void* X, svgear_dims dims, const float* cent, int C, int32_t* labels,
+                  cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, st);
+}
+
+template <typename T, int D>
+static int segmean_disp(const void* X, const int32_t* perm, const int32_t* offsets, int C,
+                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st) {
+    const int BH = dims.B * dims.H;
+    if (perm)
+        segment_mean_kernel<T, D, true><<<dim3(C, BH), kSmThreads, 0, st>>>(
+            static_cast<const T*>(X), perm, offsets, dims.N, C, out, empty_zero);
+    else
+        segment_mean_kernel<T, D, false><<<dim3(C, BH), kSmThreads, 0, st>>>(
+            static_cast<const T*>(X), nullptr, offsets, dims.N, C, out, empty_zero);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets, int C,
+                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, segmean_disp, X, perm, offsets, C, dims, out, empty_zero, st);
+}
+
+template <typename T, int D>
+static int permute_disp(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
+                        cudaStream_t st) {
+    constexpr int L = D / Elem<T>::kPerChunk;
+    const int BH = dims.B * dims.H;
+    const long long chunks = (long long)dims.N * L;
+    permute_kernel<T, D><<<dim3(ceil_div(chunks, 256), BH), 256, 0, st>>>(
+        static_cast<const T*>(X), perm, dims.N, static_cast<T*>(Xp));
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+int launch_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
+                   cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, permute_disp, X, perm, dims, Xp, st);
+}
+
+}  // namespace svgear

@@ -1,0 +1,53 @@
+// launchers.h -- host-side launch functions of the library's kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "svgear.h"
+
+namespace svgear {
+
+// Tokens per block of the k-means++ D^2 pass and of the label sort.
+constexpr int kKppTokens = 1024;
+constexpr int kSortTokens = 1024;
+
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// kmeans.cu
+int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
+                    float* centroids, int32_t* chosen, float* D2, double* blocksum,
+                    cudaStream_t st);
+int launch_assign(const void* X, svgear_dims dims, const float* centroids, int C,
+                  int32_t* labels, cudaStream_t st);
+// Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
+// empty_zero: an empty segment writes zeros (else leaves the row untouched).
+int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets,
+                        int C, svgear_dims dims, float* out, bool empty_zero,
+                        cudaStream_t st);
+int launch_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
+                   cudaStream_t st);
+
+// sort.cu
+int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm,
+                      int32_t* offsets, int32_t* block_hist, cudaStream_t st);
+
+// route.cu
+int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp,
+                 const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
+                 svgear_dims kdims, float scale, float* E, uint32_t* rowmax,
+                 cudaStream_t st);
+int launch_route_select(const float* E, const int32_t* q_off, int Cq,
+                        const int32_t* k_off, int Ck, int BH, long long budget,
+                        int32_t* lists, int32_t* counts, int32_t* pair_off,
+                        int32_t* pair_kc, cudaStream_t st);
+
+// attend_simt.cu
+int launch_attend_simt(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                       int Nk, const int32_t* q_off, int Cq, const int32_t* k_off,
+                       int Ck, const int32_t* pair_off, const int32_t* pair_kc,
+                       const float* kbar, const float* vbar, const int32_t* q_perm,
+                       float scale, void* O, cudaStream_t st);
+
+}  // namespace svgear

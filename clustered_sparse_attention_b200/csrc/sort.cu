@@ -1,0 +1,118 @@
+// sort.cu -- stable counting sort of cluster labels: the permutation that
+// makes every cluster contiguous and the segment offsets.
+//
+// Method: SVG2 (paper-graph summary, section 3.4, "The permutation operation
+// and its mathematical validity": tokens of cluster 1 first, then cluster 2,
+// ...), and the SVG-EAR task page (agent step 1: the k-means also returns the
+// sorted order).  Ties keep the original token order, so the result is
+// unique and deterministic.
+//
+// Three passes per (batch, head): block histograms (shared-memory integer
+// atomics), a column scan over blocks plus the segment offsets, and a
+// one-warp-per-block scatter that ranks equal labels with __match_any_sync
+// in token order.  Labels outside 0..C-1 are ignored (no write).
+#include "common.cuh"
+#include "launchers.h"
+
+namespace svgear {
+
+__global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int N, int C, int nblk,
+                                 int32_t* __restrict__ hist) {
+    extern __shared__ int32_t h[];
+    const int blk = blockIdx.x, bh = blockIdx.y;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) h[c] = 0;
+    __syncthreads();
+    const int32_t* lab = labels + (size_t)bh * N;
+    for (int r = threadIdx.x; r < kSortTokens; r += blockDim.x) {
+        const int t = blk * kSortTokens + r;
+        if (t < N) {
+            const int c = lab[t];
+            if ((unsigned)c < (unsigned)C) atomicAdd(&h[c], 1);
+        }
+    }
+    __syncthreads();
+    int32_t* out = hist + ((size_t)bh * nblk + blk) * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) out[c] = h[c];
+}
+
+// hist[blk][c] <- global start position of block blk's first token labelled c.
+__global__ void sort_scan_kernel(int N, int C, int nblk, int32_t* __restrict__ hist,
+                                 int32_t* __restrict__ offsets) {
+    extern __shared__ int32_t tot[];   // [C] then [blockDim] partials
+    int32_t* part = tot + C;
+    const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    int32_t* hh = hist + (size_t)bh * nblk * C;
+    for (int c = tid; c < C; c += nt) {
+        int32_t run = 0;
+        for (int b = 0; b < nblk; ++b) {
+            const int32_t v = hh[(size_t)b * C + c];
+            hh[(size_t)b * C + c] = run;
+            run += v;
+        }
+        tot[c] = run;
+    }
+    __syncthreads();
+    // exclusive scan of tot over c: contiguous chunks per thread
+    const int per = (C + nt - 1) / nt;
+    const int c0 = tid * per, c1 = min(C, c0 + per);
+    int32_t s = 0;
+    for (int c = c0; c < c1; ++c) s += tot[c];
+    part[tid] = s;
+    __syncthreads();
+    if (tid == 0) {
+        int32_t run = 0;
+        for (int i = 0; i < nt; ++i) { int32_t v = part[i]; part[i] = run; run += v; }
+    }
+    __syncthreads();
+    int32_t run = part[tid];
+    int32_t* off = offsets + (size_t)bh * (C + 1);
+    for (int c = c0; c < c1; ++c) { const int32_t v = tot[c]; tot[c] = run; off[c] = run; run += v; }
+    if (tid == nt - 1) off[C] = run;   // equals the number of in-range labels
+    __syncthreads();
+    for (int c = tid; c < C; c += nt) {
+        const int32_t base = tot[c];
+        for (int b = 0; b < nblk; ++b) hh[(size_t)b * C + c] += base;
+    }
+}
+
+__global__ void __launch_bounds__(32)
+sort_scatter_kernel(const int32_t* __restrict__ labels, int N, int C, int nblk,
+                    const int32_t* __restrict__ hist, int32_t* __restrict__ perm) {
+    extern __shared__ int32_t cur[];
+    const int blk = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+    const int32_t* hb = hist + ((size_t)bh * nblk + blk) * C;
+    for (int c = lane; c < C; c += 32) cur[c] = hb[c];
+    __syncwarp();
+    const int32_t* lab = labels + (size_t)bh * N;
+    int32_t* pm = perm + (size_t)bh * N;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int step = 0; step < kSortTokens / 32; ++step) {
+        const int t = blk * kSortTokens + step * 32 + lane;
+        int c = (t < N) ? lab[t] : -1;
+        if ((unsigned)c >= (unsigned)C) c = -1;
+        const unsigned same = __match_any_sync(0xffffffffu, c);
+        int pos = 0;
+        if (c >= 0) pos = cur[c] + __popc(same & lt);
+        __syncwarp();
+        if (c >= 0 && (same & lt) == 0) cur[c] += __popc(same);
+        __syncwarp();
+        if (c >= 0) pm[pos] = t;
+    }
+}
+
+int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm,
+                      int32_t* offsets, int32_t* hist, cudaStream_t st) {
+    const int nblk = ceil_div(N, kSortTokens);
+    const size_t sh = sizeof(int32_t) * C;
+    sort_hist_kernel<<<dim3(nblk, BH), 256, sh, st>>>(labels, N, C, nblk, hist);
+    count_launches(1);
+    const int nt = 512;
+    sort_scan_kernel<<<BH, nt, sizeof(int32_t) * (C + nt), st>>>(N, C, nblk, hist, offsets);
+    count_launches(1);
+    sort_scatter_kernel<<<dim3(nblk, BH), 32, sh, st>>>(labels, N, C, nblk, hist, perm);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+}  // namespace svgear

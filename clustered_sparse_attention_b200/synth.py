@@ -154,3 +154,23 @@ def layer_tensor(w: Workload, tensor: str, step: int = 0, heads=None,
     with ThreadPoolExecutor(max(1, threads)) as ex:
         list(ex.map(one, range(len(jobs))))
     return out
+
+
+def layer_tensor_bits(w: Workload, tensor: str, step: int = 0, heads=None,
+                      threads: int = 8, batch_offset: int = 0) -> np.ndarray:
+    """Like layer_tensor, but bfloat16 bit patterns (uint16) for bf16
+    workloads -- half the host memory at the 720p shapes.  Batch index b of
+    the result is drawn as batch b + batch_offset (independent replicas)."""
+    if w.dtype != "bf16":
+        raise ValueError("layer_tensor_bits is for bf16 workloads")
+    heads = list(range(w.H)) if heads is None else list(heads)
+    jobs = [(b + batch_offset, h) for b in range(w.B) for h in heads]
+    out = np.empty((w.B, len(heads), w.N, w.d), dtype=np.uint16)
+
+    def one(i):
+        b, h = jobs[i]
+        out[b - batch_offset, heads.index(h)] = bf16_bits(head_tensor(w, tensor, b, h, step))
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(one, range(len(jobs))))
+    return out

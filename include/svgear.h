@@ -1,0 +1,276 @@
+/*
+ * svgear.h -- C ABI of the B200 clustered sparse attention library
+ * (SVG-EAR's error-aware routing and centroid compensation on top of SVG2's
+ * semantic-aware permutation).
+ *
+ * The layer, for every batch b and head h independently:
+ *   1. k-means over the query tokens and, independently, over the key tokens
+ *      (k-means++ seeding on a cold call, the caller's cached centroids on a
+ *      warm call), returning labels, the permutation that makes every cluster
+ *      contiguous, the segment offsets and the centroids;
+ *   2. the permuted values and one mean value vector per key cluster;
+ *   3. a per-(query cluster, key cluster) compensation-error probe and a
+ *      greedy error-to-cost selection of blocks under a density budget;
+ *   4. one attention pass that computes the selected blocks exactly and adds
+ *      every skipped key cluster as its centroid weighted by its size, inside
+ *      the same online softmax, writing O back in the original token order.
+ *
+ * Sources (page title, section):
+ *   [TASK]   "SVG-EAR" task page (sotabase FrontierCS-2): the three routines
+ *            -- one averages each cluster, one picks which cluster pairs to
+ *            compute, one computes them and estimates the rest; the agent's
+ *            steps 1-3 (k-means returning the sorted order, skipped clusters
+ *            as one key at the centroid with its score raised by log n).
+ *   [BLOG]   "SVG-EAR measured error" (frontier-cs.org blog): worked toy
+ *            example, weight n*e^{s_bar}, the probe error sum, error per pair.
+ *   [REVIEW] "SVG-EAR: Parameter-Free Linear Compensation for Sparse Video
+ *            Generation via Error-aware Routing" (pith.science review): greedy
+ *            error-to-cost routing under a density budget, O(Cq*Nk*d) probe.
+ *   [SVG2]   "Sparse VideoGen2: Accelerate Video Generation with Sparse
+ *            Attention via Semantic-Aware Permutation" (paper-graph summary),
+ *            section 3.4: independent k-means on Q and K, permutation
+ *            validity O = pi_q^T Attn(pi_q Q, pi_k K, pi_k V), k-means++ and
+ *            the centroid cache, the dynamic block-size kernel.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless stated; the caller allocates every
+ *     buffer (outputs and workspace) and keeps ownership.  The library keeps
+ *     no state between calls and never allocates device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and is asynchronous: a return of SVGEAR_OK
+ *     means the arguments were valid and the kernels launched.
+ *   - Tensors are dense row-major with the head dimension d innermost:
+ *     tokens X[B][H][N][d]; per-token ints [B][H][N]; centroids
+ *     float[B][H][C][d]; segment offsets int32[B][H][C+1] holding positions
+ *     0..N within the head.
+ *   - dtype SVGEAR_F32 (float) or SVGEAR_BF16 (bfloat16) for token tensors;
+ *     centroids and errors are always float.  d must be 64 or 128.
+ *   - Errors: a negative svgear_status.  SVGEAR_ERR_INVALID_ARG for a null
+ *     required pointer or sizes out of range, SVGEAR_ERR_UNSUPPORTED for a
+ *     dtype / d / cluster count outside what the kernels implement,
+ *     SVGEAR_ERR_WORKSPACE when ws_bytes is below svgear_workspace_bytes(),
+ *     SVGEAR_ERR_CUDA when a launch fails (the CUDA error stays readable with
+ *     cudaGetLastError).  Nothing is launched when validation fails.
+ */
+#ifndef SVGEAR_H
+#define SVGEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SVGEAR_OK = 0,
+    SVGEAR_ERR_INVALID_ARG = -1,
+    SVGEAR_ERR_UNSUPPORTED = -2,
+    SVGEAR_ERR_CUDA = -3,
+    SVGEAR_ERR_TIMEOUT = -4,
+    SVGEAR_ERR_WORKSPACE = -5
+} svgear_status;
+
+typedef enum { SVGEAR_F32 = 0, SVGEAR_BF16 = 1 } svgear_dtype;
+
+/* Shape of one token tensor X[B][H][N][d]. */
+typedef struct {
+    int32_t B, H, N, d;
+    int32_t dtype; /* svgear_dtype */
+} svgear_dims;
+
+/* Operation selector for svgear_workspace_bytes. */
+typedef enum {
+    SVGEAR_OP_CLUSTER = 0,
+    SVGEAR_OP_KMEANSPP = 1,
+    SVGEAR_OP_LABEL_SORT = 2,
+    SVGEAR_OP_KMEANS_UPDATE = 3,
+    SVGEAR_OP_ROUTE = 4,
+    SVGEAR_OP_ATTEND = 5
+} svgear_op;
+
+/* Largest cluster count any call accepts (shared-memory tables). */
+#define SVGEAR_MAX_CLUSTERS 4096
+
+/* --------------------------------------------------------------------------
+ * svgear_cluster -- k-means over the tokens of every (b, h) and the
+ * semantic-aware permutation ([SVG2] "The clustering operation", "The
+ * permutation operation", "Fast k-means with centroid cache"; [TASK] step 1).
+ *
+ *   X               [B][H][N][d] tokens (dtype).
+ *   C               clusters per head, 1 <= C <= min(N, SVGEAR_MAX_CLUSTERS).
+ *   iters           rounds of (assign, update), >= 1.  The last round's
+ *                   labels are final and its update gives the returned
+ *                   centroids, so every non-empty centroid is exactly the
+ *                   mean of its final members.
+ *   warm_centroids  float[B][H][C][d] starting centroids (the previous
+ *                   step's), or NULL for a cold start with k-means++ seeding
+ *                   driven by Philox4x64-10 draws under `seed` (stream word =
+ *                   b*H + h; see svgear_kmeanspp_init).
+ *   labels          out int32[B][H][N]: argmin_c |x - c|^2, lowest c on ties.
+ *   perm            out int32[B][H][N]: perm[p] = original token index at
+ *                   permuted position p; stable in the original index.
+ *   offsets         out int32[B][H][C+1]: cluster c occupies permuted
+ *                   positions offsets[c] .. offsets[c+1]-1.
+ *   centroids       out float[B][H][C][d]; an empty cluster keeps its
+ *                   previous centroid.  May alias warm_centroids.
+ *   Xp              out [B][H][N][d] (dtype) permuted copy X[perm], or NULL.
+ *   ws, ws_bytes    workspace of svgear_workspace_bytes(SVGEAR_OP_CLUSTER).
+ * ------------------------------------------------------------------------ */
+int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
+                   const float* warm_centroids, uint64_t seed, int32_t* labels,
+                   int32_t* perm, int32_t* offsets, float* centroids, void* Xp,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * Sub-steps of svgear_cluster, exposed for stage-wise use and checking.
+ * ------------------------------------------------------------------------ */
+
+/* k-means++ seeding ([SVG2] "Fast k-means with centroid cache": k-means++
+ * initialisation).  Draw j of head s = b*H + h is u_j = top 53 bits of the
+ * first word of Philox4x64-10(counter = {j, s, 0, 0}, key = {seed, 0}) times
+ * 2^-53.  Seed 0 is token floor(u_0 * N); seed j >= 1 is the smallest token
+ * whose running sum of D^2 (squared distance to the nearest earlier seed,
+ * fp32, summed in fp64) exceeds u_j * sum(D^2); if every D^2 is zero it is the
+ * lowest token not chosen yet.  centroids[c] = X[seed_index[c]] as float.
+ *   seed_index  out int32[B][H][C], or NULL.
+ *   ws          svgear_workspace_bytes(SVGEAR_OP_KMEANSPP). */
+int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t seed,
+                         float* centroids, int32_t* seed_index, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* k-means assignment: labels[t] = argmin_c |x_t - c|^2, lowest c on exact
+ * ties, evaluated in fp32 as |c|^2 - 2 x.c.  Needs no workspace. */
+int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids,
+                         int32_t C, int32_t* labels, void* stream);
+
+/* Stable counting sort of labels ([TASK] step 1: the sorted order).
+ *   labels   int32[B][H][N] in 0..C-1.
+ *   perm     out int32[B][H][N]; offsets out int32[B][H][C+1].
+ *   ws       svgear_workspace_bytes(SVGEAR_OP_LABEL_SORT) (dims.d and
+ *            dims.dtype are ignored). */
+int svgear_label_sort(const int32_t* labels, svgear_dims dims, int32_t C,
+                      int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* k-means update: centroids[c] = mean of the tokens labelled c (fp32 sums in
+ * a fixed order, so the result is deterministic); an empty cluster keeps the
+ * value already in `centroids` (in/out).
+ *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_UPDATE). */
+int svgear_kmeans_update(const void* X, svgear_dims dims, const int32_t* labels,
+                         int32_t C, float* centroids, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_permute -- Xp[p] = X[perm[p]] within every (b, h): the values share
+ * the keys' permutation ([SVG2] "K and V share the same permutation").
+ * ------------------------------------------------------------------------ */
+int svgear_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
+                   void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_centroids -- per-cluster mean of a permuted tensor in one pass
+ * ([TASK] "one averages each cluster"; step 1: a small kernel averages each
+ * cluster's values in one pass).
+ *   Xp        [B][H][N][d] permuted tokens (dtype).
+ *   offsets   int32[B][H][C+1] segments.
+ *   centroids out float[B][H][C][d]; an empty segment gives zeros.
+ * ------------------------------------------------------------------------ */
+int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
+                     svgear_dims dims, float* centroids, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_probe -- compensation-error probe ([BLOG] probe paragraph; [REVIEW]
+ * O(Cq*Nk*d) probe).  With s_it = scale * qbar_i . k_t, sbar_ic = scale *
+ * qbar_i . kbar_c and m_i = max_t s_it over every key of the head:
+ *   E[i][c] = sum_{t in K_c} | e^{sbar_ic - m_i} vbar_c - e^{s_it - m_i} v_t |^2
+ * (fp32).  The shift m_i keeps the exponentials finite and leaves every
+ * ranking within a row unchanged.  E is 0 for an empty key cluster.
+ *   qbar      float[B][H][Cq][d] query centroids (the probes).
+ *   Kp, Vp    [B][H][Nk][d] permuted keys and values (kdims.dtype).
+ *   kbar,vbar float[B][H][Ck][d] key and value centroids.
+ *   k_off     int32[B][H][Ck+1] key segments.
+ *   kdims     shape of Kp (N = Nk).
+ *   E         out float[B][H][Cq][Ck].
+ *   ws        svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck) (holds the
+ *             row maxima).
+ * ------------------------------------------------------------------------ */
+int svgear_probe(const float* qbar, int32_t Cq, const void* Kp, const void* Vp,
+                 const float* kbar, const float* vbar, const int32_t* k_off,
+                 int32_t Ck, svgear_dims kdims, float scale, float* E, void* ws,
+                 size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_route_select -- greedy error-to-cost selection ([REVIEW] greedy
+ * routing under a density budget; [BLOG] error divided by the block's token
+ * pairs, budget spent per query cluster).  For every non-empty query cluster
+ * i: the key r_c = E[i][c] / n_c (one fp32 IEEE division; |Q_i| is constant
+ * within the row) over the non-empty key clusters, ordered by r descending,
+ * ties to the lower c, NaN last; c is taken if the keys taken so far plus n_c
+ * stay within floor(density * Nk), else skipped, and the scan continues.
+ *   pair_off  out int32[B][H][Cq+1]: row i's clusters are
+ *             pair_kc[pair_off[i] .. pair_off[i+1]-1] (relative to the
+ *             head's base B*H-index * Cq*Ck), ascending c.
+ *   pair_kc   out int32[B][H][Cq*Ck].
+ *   density   in (0, 1].
+ *   ws        svgear_workspace_bytes(SVGEAR_OP_ROUTE, ...) suffices.
+ * ------------------------------------------------------------------------ */
+int svgear_route_select(const float* E, const int32_t* q_off, int32_t Cq,
+                        const int32_t* k_off, int32_t Ck, int32_t B, int32_t H,
+                        int32_t Nk, float density, int32_t* pair_off,
+                        int32_t* pair_kc, void* ws, size_t ws_bytes, void* stream);
+
+/* svgear_route -- probe + select in one call ([TASK] "one picks which cluster
+ * pairs to compute").  E_out (float[B][H][Cq][Ck]) may be NULL, in which case
+ * the errors live in the workspace (svgear_workspace_bytes(SVGEAR_OP_ROUTE)). */
+int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq,
+                 const float* kbar, const float* vbar, const int32_t* k_off,
+                 int32_t Ck, const void* Kp, const void* Vp, svgear_dims kdims,
+                 float density, float scale, int32_t* pair_off, int32_t* pair_kc,
+                 float* E_out, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_attend -- exact selected blocks plus centroid compensation in one
+ * online softmax ([TASK] "one computes them and estimates the rest"; [BLOG]
+ * weight n*e^{s_bar} and average value of a skipped cluster; [SVG2]
+ * O = pi_q^T Attn(pi_q Q, pi_k K, pi_k V)).  For permuted query row p of
+ * query cluster i and q = Qp[p]:
+ *   num = sum_{c in S_i} sum_{u in K_c} e^{scale q.k_u} v_u
+ *       + sum_{c not in S_i, n_c > 0} n_c e^{scale q.kbar_c} vbar_c
+ *   den = the same sums with 1 in place of the value vectors
+ *   O[q_perm[p]] = num / den          (O in the original token order).
+ *   Qp        [B][H][Nq][d]; Kp, Vp [B][H][Nk][d] (all qdims.dtype).
+ *   q_off     int32[B][H][Cq+1]; k_off int32[B][H][Ck+1].
+ *   pair_off, pair_kc   from svgear_route / svgear_route_select.
+ *   kbar,vbar float[B][H][Ck][d].
+ *   q_perm    int32[B][H][Nq] (svgear_cluster's perm for the queries).
+ *   O         out [B][H][Nq][d] (qdims.dtype).
+ *   ws        svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck).
+ * bf16 runs on the tcgen05 tensor-core kernel; f32 on an fp32 SIMT kernel.
+ * ------------------------------------------------------------------------ */
+int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                  int32_t Nk, const int32_t* q_off, int32_t Cq, const int32_t* k_off,
+                  int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc,
+                  const float* kbar, const float* vbar, const int32_t* q_perm,
+                  float scale, void* O, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes for `op` at shape `dims` (N = tokens of the clustered
+ * tensor; for SVGEAR_OP_ROUTE and SVGEAR_OP_ATTEND, dims.N = Nq and C2 = Ck),
+ * with C1 = C (or Cq).  Returns 0 for arguments the op would reject. */
+size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t C2);
+
+/* Static description of a status code. */
+const char* svgear_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t svgear_version(void);
+
+/* Number of kernels this library has launched since it was loaded, over all
+ * devices and threads (a host-side counter; no device synchronisation). */
+uint64_t svgear_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVGEAR_H */

@@ -1,0 +1,104 @@
+"""The C-ABI library builds, loads and exports every symbol include/svgear.h
+declares; host-side validation rejects bad arguments before any launch
+(these run without a GPU: no call below reaches the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from clustered_sparse_attention_b200 import build
+    build.build()
+    from clustered_sparse_attention_b200 import _lib
+    return _lib.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "svgear.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svgear_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = _declared()
+    for must in ("svgear_cluster", "svgear_centroids", "svgear_route", "svgear_attend"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    from clustered_sparse_attention_b200 import _lib
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) <= set(_lib.EXPORTED) | set(_declared())
+    assert L.svgear_version() >= 100
+
+
+def test_library_is_built_for_sm100a_only():
+    from clustered_sparse_attention_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH)
+
+
+def _dims(B=1, H=2, N=1000, d=128, dtype=1):
+    from clustered_sparse_attention_b200._lib import Dims
+    return Dims(B, H, N, d, dtype)
+
+
+def test_status_strings(L):
+    assert L.svgear_status_string(0) == b"ok"
+    assert b"workspace" in L.svgear_status_string(-5)
+
+
+def test_workspace_bytes_rejects_bad_sizes(L):
+    from clustered_sparse_attention_b200 import _lib
+    assert L.svgear_workspace_bytes(_lib.OP_CLUSTER, _dims(), 100, 0) > 0
+    assert L.svgear_workspace_bytes(_lib.OP_CLUSTER, _dims(), 1001, 0) == 0      # C > N
+    assert L.svgear_workspace_bytes(_lib.OP_CLUSTER, _dims(d=96), 10, 0) == 0    # d
+    assert L.svgear_workspace_bytes(_lib.OP_CLUSTER, _dims(dtype=7), 10, 0) == 0
+    assert L.svgear_workspace_bytes(_lib.OP_ROUTE, _dims(), 100, 5000) == 0      # > max clusters
+    assert L.svgear_workspace_bytes(99, _dims(), 10, 10) == 0
+
+
+def test_validation_before_launch(L):
+    from clustered_sparse_attention_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+    ws_small = ctypes.c_size_t(16)
+    # null X
+    assert L.svgear_kmeans_assign(None, _dims(), fake, 10, fake, None) == _lib.ERR_INVALID_ARG
+    # unsupported head dimension / dtype
+    assert L.svgear_kmeans_assign(fake, _dims(d=96), fake, 10, fake, None) == _lib.ERR_UNSUPPORTED
+    assert L.svgear_kmeans_assign(fake, _dims(dtype=3), fake, 10, fake, None) == _lib.ERR_UNSUPPORTED
+    # C out of range
+    assert L.svgear_kmeans_assign(fake, _dims(), fake, 0, fake, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_kmeans_assign(fake, _dims(N=5000), fake, 4097, fake, None) == _lib.ERR_UNSUPPORTED
+    # misaligned token pointer
+    assert L.svgear_kmeans_assign(ctypes.c_void_p((1 << 20) + 4), _dims(), fake, 10, fake,
+                                  None) == _lib.ERR_INVALID_ARG
+    # iters < 1
+    assert L.svgear_cluster(fake, _dims(), 10, 0, None, 0, fake, fake, fake, fake, None, fake,
+                            ctypes.c_size_t(1 << 30), None) == _lib.ERR_INVALID_ARG
+    # workspace too small
+    assert L.svgear_cluster(fake, _dims(), 10, 3, None, 0, fake, fake, fake, fake, None, fake,
+                            ws_small, None) == _lib.ERR_WORKSPACE
+    # density outside (0, 1]
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        assert L.svgear_route_select(fake, fake, 10, fake, 20, 1, 2, 1000, bad, fake, fake, fake,
+                                     ctypes.c_size_t(1 << 30), None) == _lib.ERR_INVALID_ARG
+    # Ck > Nk
+    assert L.svgear_route_select(fake, fake, 10, fake, 2000, 1, 2, 1000, 0.5, fake, fake, fake,
+                                 ctypes.c_size_t(1 << 30), None) == _lib.ERR_INVALID_ARG
+    # non-finite scale
+    assert L.svgear_attend(fake, fake, fake, _dims(), 1000, fake, 10, fake, 20, fake, fake, fake,
+                           fake, fake, float("inf"), fake, fake, ctypes.c_size_t(1 << 30),
+                           None) == _lib.ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(L):
+    fake = ctypes.c_void_p(1 << 20)
+    # B = 0: valid, nothing to launch, no CUDA call
+    assert L.svgear_kmeans_assign(fake, _dims(B=0), fake, 10, fake, None) == 0
+    assert L.svgear_centroids(fake, fake, 10, _dims(B=0), fake, None) == 0

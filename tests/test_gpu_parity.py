@@ -1,0 +1,355 @@
+"""CUDA path vs the CPU oracle, stage by stage, through the C ABI.
+
+Labels, permutations, offsets and routed pairs must be bit-exact when the
+oracle is fed the GPU stage's inputs (labels up to documented fp32 near-ties);
+floating-point outputs must lie within bounds derived from the fp32 arithmetic
+(tests/helpers.py); the final O within rel-L2 1e-2 and max-abs 2e-2 for bf16
+and 1e-5 for fp32.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from clustered_sparse_attention_b200 import synth
+from tests.helpers import (U32, check_assign, np64, probe_tolerance, to_torch,
+                           update_tolerance)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _csa():
+    import clustered_sparse_attention_b200 as csa
+    return csa
+
+
+SMALL_BF16 = synth.custom_workload("small_bf16", H=2, frames=2, grid_h=32, grid_w=40, d=128,
+                                   dtype="bf16", Cq=20, Ck=50, iters=5, density=0.3,
+                                   n_centres=32, sigma=0.5, index=50)
+RAGGED_BF16_64 = synth.custom_workload("ragged_bf16_d64", H=3, frames=1, grid_h=25, grid_w=41,
+                                       d=64, dtype="bf16", Cq=7, Ck=33, iters=3, density=0.25,
+                                       n_centres=12, sigma=0.4, index=51)
+TINY = synth.WORKLOADS["tiny"]
+
+
+def _inputs(w, heads=None):
+    t = {n: synth.layer_tensor(w, n, heads=heads) for n in ("q", "k", "v")}
+    return t, {n: to_torch(a, w.dtype) for n, a in t.items()}
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_kmeanspp_stagewise(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    C = w.Ck
+    cent, idx = csa.svgear_kmeanspp_init(dev["k"], C, seed=7)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    cent = cent.cpu().numpy()
+    band = 4 * (w.d + 2) * U32
+    flips = 0
+    for h in range(w.H):
+        X = host["k"][0, h]
+        own, margin = oracle.kmeanspp(X, C, seed=7, stream=h, follow=idx[0, h])
+        assert own[0] == idx[0, h, 0]
+        diff = np.nonzero(own != idx[0, h])[0]
+        for j in diff:
+            assert margin[j] < band, "seed %d of head %d: gpu %d oracle %d margin %.3g" % (
+                j, h, idx[0, h, j], own[j], margin[j])
+        flips += len(diff)
+        assert np.array_equal(cent[0, h], X[idx[0, h]])
+    assert flips <= 2
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_assign_matches_oracle(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    g = np.random.default_rng(1)
+    for C in (w.Cq, w.Ck, 129):
+        C = min(C, w.N)
+        cent = np.stack([host["q"][0, h][g.choice(w.N, C, replace=False)] for h in range(w.H)])[None]
+        cent = cent + 0.01 * g.standard_normal(cent.shape).astype(np.float32)
+        lab = csa.svgear_kmeans_assign(dev["q"], torch.from_numpy(cent).cuda()).cpu().numpy()
+        flips = sum(check_assign(host["q"][0, h], cent[0, h], lab[0, h]) for h in range(w.H))
+        assert flips <= max(2, w.N * w.H // 5000)
+
+
+def test_assign_exact_ties_take_lowest_index():
+    csa = _csa()
+    X = torch.zeros((1, 1, 300, 64), device="cuda")
+    X[0, 0, :, 0] = torch.arange(300, device="cuda").float() % 3
+    cent = torch.zeros((1, 1, 200, 64), device="cuda")
+    cent[0, 0, :, 0] = (torch.arange(200, device="cuda") % 3).float()   # 3 values, many duplicates
+    lab = csa.svgear_kmeans_assign(X, cent).cpu().numpy()[0, 0]
+    assert np.array_equal(lab, np.arange(300) % 3)
+
+
+@pytest.mark.parametrize("N,C", [(5000, 300), (1024, 1), (777, 777), (5000, 4096), (3000, 129)])
+def test_label_sort_bit_exact(N, C):
+    csa = _csa()
+    g = np.random.default_rng(N + C)
+    labels = g.integers(0, C, (2, 3, N)).astype(np.int32)
+    if C > 10:
+        labels[labels % 7 == 3] = 0          # leaves some clusters empty
+    perm, off = csa.svgear_label_sort(torch.from_numpy(labels).cuda(), C)
+    perm, off = perm.cpu().numpy(), off.cpu().numpy()
+    for b in range(2):
+        for h in range(3):
+            p_o, o_o = oracle.stable_sort(labels[b, h], C)
+            assert np.array_equal(perm[b, h], p_o)
+            assert np.array_equal(off[b, h], o_o)
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_update_matches_oracle(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    g = np.random.default_rng(2)
+    C = w.Ck
+    labels = g.integers(0, C - 3, (1, w.H, w.N)).astype(np.int32)   # last clusters empty
+    prev = g.standard_normal((1, w.H, C, w.d)).astype(np.float32)
+    out = csa.svgear_kmeans_update(dev["k"], torch.from_numpy(labels).cuda(),
+                                   torch.from_numpy(prev).cuda()).cpu().numpy()
+    for h in range(w.H):
+        ref = oracle.update(host["k"][0, h], labels[0, h], prev[0, h])
+        tol = update_tolerance(host["k"][0, h], labels[0, h], C)
+        assert np.all(np.abs(out[0, h] - ref) <= tol)
+        assert np.array_equal(out[0, h, C - 3:], prev[0, h, C - 3:])
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16], ids=lambda w: w.name)
+def test_cluster_iteration_chain(w):
+    """cluster(iters=k) returns centroids c^k; cluster(iters=k+1) must hold
+    labels = argmin against c^k, centroids = means of those labels, and the
+    stable sort of those labels; Xp = X[perm]."""
+    csa = _csa()
+    host, dev = _inputs(w)
+    C = w.Ck
+    prev = csa.svgear_cluster(dev["k"], C, 1, seed=11)
+    for k in (1, 2, 3):
+        nxt = csa.svgear_cluster(dev["k"], C, k + 1, seed=11)
+        torch.cuda.synchronize()
+        for h in range(w.H):
+            X = host["k"][0, h]
+            cprev = prev.centroids.cpu().numpy()[0, h]
+            lab = nxt.labels.cpu().numpy()[0, h]
+            check_assign(X, cprev, lab)
+            p_o, o_o = oracle.stable_sort(lab, C)
+            assert np.array_equal(nxt.perm.cpu().numpy()[0, h], p_o)
+            assert np.array_equal(nxt.offsets.cpu().numpy()[0, h], o_o)
+            ref = oracle.update(X, lab, cprev)
+            assert np.all(np.abs(nxt.centroids.cpu().numpy()[0, h] - ref)
+                          <= update_tolerance(X, lab, C))
+            Xp = np64(nxt.Xp)[0, h]
+            assert np.array_equal(Xp, X[p_o].astype(np.float64))
+        prev = nxt
+
+
+def test_warm_start_is_one_round_from_the_cache():
+    csa = _csa()
+    w = SMALL_BF16
+    host, dev = _inputs(w)
+    cold = csa.svgear_cluster(dev["q"], w.Cq, 3, seed=5)
+    warm = csa.svgear_cluster(dev["q"], w.Cq, 1, warm_centroids=cold.centroids.clone())
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        check_assign(host["q"][0, h], cold.centroids.cpu().numpy()[0, h],
+                     warm.labels.cpu().numpy()[0, h])
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_permute_and_value_centroids(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    ck = csa.svgear_cluster(dev["k"], w.Ck, 2, seed=3)
+    Vp = csa.svgear_permute(dev["v"], ck.perm)
+    vbar = csa.svgear_centroids(Vp, ck.offsets, w.Ck)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        perm = ck.perm.cpu().numpy()[0, h]
+        off = ck.offsets.cpu().numpy()[0, h]
+        V = host["v"][0, h]
+        assert np.array_equal(np64(Vp)[0, h], V[perm].astype(np.float64))
+        ref = oracle.segment_mean(V[perm], off)
+        lab = np.repeat(np.arange(w.Ck), np.diff(off))
+        tol = update_tolerance(V[perm], lab, w.Ck)
+        got = vbar.cpu().numpy()[0, h]
+        assert np.all(np.abs(got - ref) <= tol)
+        assert np.all(got[np.diff(off) == 0] == 0)
+
+
+def _clustered(w, dev, seed=3):
+    csa = _csa()
+    cq = csa.svgear_cluster(dev["q"], w.Cq, 2, seed=2 * seed)
+    ck = csa.svgear_cluster(dev["k"], w.Ck, 2, seed=2 * seed + 1)
+    Vp = csa.svgear_permute(dev["v"], ck.perm)
+    vbar = csa.svgear_centroids(Vp, ck.offsets, w.Ck)
+    return cq, ck, Vp, vbar
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_probe_matches_oracle(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    E = csa.svgear_probe(cq.centroids, ck.Xp, Vp, ck.centroids, vbar, ck.offsets, w.scale)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        qbar = cq.centroids.cpu().numpy()[0, h]
+        Kp, Vph = np64(ck.Xp)[0, h], np64(Vp)[0, h]
+        Eo, So = oracle.probe(qbar, Kp, Vph, ck.centroids.cpu().numpy()[0, h],
+                              vbar.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
+                              w.scale, with_scale=True)
+        Eg = E.cpu().numpy()[0, h].astype(np.float64)
+        tol = probe_tolerance(qbar, Kp, Eo, So, w.scale)
+        assert np.all(np.abs(Eg - Eo) <= tol), float(np.max(np.abs(Eg - Eo) / tol))
+        empty = np.diff(ck.offsets.cpu().numpy()[0, h]) == 0
+        assert np.all(Eg[:, empty] == 0)
+
+
+@pytest.mark.parametrize("density", [0.05, 0.25, 0.5, 1.0])
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_route_bit_exact_given_gpu_errors(w, density):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    po, pk, E = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
+                                 Vp, density, w.scale, return_errors=True)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        ref_off, ref_kc = oracle.route(E.cpu().numpy()[0, h], cq.offsets.cpu().numpy()[0, h],
+                                       ck.offsets.cpu().numpy()[0, h], w.N, density)
+        got_off = po.cpu().numpy()[0, h]
+        assert np.array_equal(got_off, ref_off)
+        assert np.array_equal(pk.cpu().numpy()[0, h][:got_off[-1]], ref_kc)
+    # the standalone select on the same errors gives the same pairs
+    po2, pk2 = csa.svgear_route_select(E, cq.offsets, ck.offsets, w.N, density)
+    assert torch.equal(po2, po)
+    n = int(po[0, 0, -1])
+    assert torch.equal(pk2[0, 0, :n], pk[0, 0, :n])
+
+
+def _check_attend(w, dev, density, rows=None):
+    csa = _csa()
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
+                              Vp, density, w.scale)
+    O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
+                          cq.perm, w.scale)
+    torch.cuda.synchronize()
+    Og = np64(O)
+    worst = (0.0, 0.0)
+    for h in range(w.H):
+        args = (np64(cq.Xp)[0, h], np64(ck.Xp)[0, h], np64(Vp)[0, h],
+                cq.offsets.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
+                po.cpu().numpy()[0, h], pk.cpu().numpy()[0, h],
+                ck.centroids.cpu().numpy()[0, h], vbar.cpu().numpy()[0, h],
+                cq.perm.cpu().numpy()[0, h])
+        if rows is None:
+            Oo, _ = oracle.attend(*args, w.scale)
+            Gh = Og[0, h]
+        else:
+            Oo, _ = oracle.attend(*args, w.scale, rows=rows)
+            Gh = Og[0, h][cq.perm.cpu().numpy()[0, h][rows]]
+        worst = (max(worst[0], _rel_l2(Gh, Oo)), max(worst[1], float(np.abs(Gh - Oo).max())))
+    return worst
+
+
+def test_attend_fp32_tiny_within_1e5():
+    host, dev = _inputs(TINY)
+    rel, mx = _check_attend(TINY, dev, TINY.density)
+    assert rel <= 1e-5 and mx <= 1e-5, (rel, mx)
+
+
+@pytest.mark.parametrize("density", [0.1, 0.3, 1.0])
+@pytest.mark.parametrize("w", [SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_attend_bf16_within_tolerance(w, density):
+    host, dev = _inputs(w)
+    rel, mx = _check_attend(w, dev, density)
+    assert rel <= 1e-2 and mx <= 2e-2, (rel, mx)
+
+
+def test_density_one_equals_dense_attention():
+    csa = _csa()
+    w = SMALL_BF16
+    host, dev = _inputs(w)
+    out = csa.layer(dev["q"], dev["k"], dev["v"], w.Cq, w.Ck, 3, 1.0, w.scale, seed=1)
+    torch.cuda.synchronize()
+    O = np64(out["O"])
+    for h in range(w.H):
+        Q, K, V = (host[n][0, h].astype(np.float64) for n in ("q", "k", "v"))
+        S = Q @ K.T * w.scale
+        S -= S.max(1, keepdims=True)
+        P = np.exp(S)
+        ref = (P / P.sum(1, keepdims=True)) @ V
+        assert _rel_l2(O[0, h], ref) <= 1e-2 and np.abs(O[0, h] - ref).max() <= 2e-2
+
+
+def test_singleton_key_clusters_make_compensation_exact():
+    csa = _csa()
+    g = np.random.default_rng(4)
+    N, d = 256, 64
+    Q = g.standard_normal((1, 1, N, d)).astype(np.float32)
+    K = g.standard_normal((1, 1, N, d)).astype(np.float32)
+    V = g.standard_normal((1, 1, N, d)).astype(np.float32)
+    dq, dk, dv = (torch.from_numpy(a).cuda() for a in (Q, K, V))
+    out = csa.layer(dq, dk, dv, 8, N, 2, 0.2, d ** -0.5, seed=2)   # Ck = N: all singletons
+    torch.cuda.synchronize()
+    S = Q[0, 0].astype(np.float64) @ K[0, 0].T.astype(np.float64) * d ** -0.5
+    S -= S.max(1, keepdims=True)
+    P = np.exp(S)
+    ref = (P / P.sum(1, keepdims=True)) @ V[0, 0]
+    got = np64(out["O"])[0, 0]
+    assert _rel_l2(got, ref) <= 1e-5 and np.abs(got - ref).max() <= 1e-5
+
+
+def test_tiny_layer_end_to_end_stagewise():
+    """The tiny fp32 workload through csa.layer, every stage checked."""
+    csa = _csa()
+    w = TINY
+    host, dev = _inputs(w)
+    out = csa.layer(dev["q"], dev["k"], dev["v"], w.Cq, w.Ck, w.iters, w.density, w.scale, seed=0)
+    torch.cuda.synchronize()
+    cq, ck = out["q"], out["k"]
+    for name, cl, X, C in (("q", cq, host["q"][0, 0], w.Cq), ("k", ck, host["k"][0, 0], w.Ck)):
+        lab = cl.labels.cpu().numpy()[0, 0]
+        p_o, o_o = oracle.stable_sort(lab, C)
+        assert np.array_equal(cl.perm.cpu().numpy()[0, 0], p_o)
+        assert np.array_equal(cl.offsets.cpu().numpy()[0, 0], o_o)
+        ref = oracle.segment_mean(X[p_o], o_o, prev=cl.centroids.cpu().numpy()[0, 0])
+        assert np.all(np.abs(cl.centroids.cpu().numpy()[0, 0] - ref)
+                      <= update_tolerance(X, lab, C))
+    pairs = int(out["pair_off"][0, 0, -1])
+    assert pairs > 0
+    Oo, _ = oracle.attend(np64(cq.Xp)[0, 0], np64(ck.Xp)[0, 0], np64(out["Vp"])[0, 0],
+                          cq.offsets.cpu().numpy()[0, 0], ck.offsets.cpu().numpy()[0, 0],
+                          out["pair_off"].cpu().numpy()[0, 0],
+                          out["pair_kc"].cpu().numpy()[0, 0][:pairs],
+                          ck.centroids.cpu().numpy()[0, 0], out["vbar"].cpu().numpy()[0, 0],
+                          cq.perm.cpu().numpy()[0, 0], w.scale)
+    Og = np64(out["O"])[0, 0]
+    assert _rel_l2(Og, Oo) <= 1e-5 and np.abs(Og - Oo).max() <= 1e-5
+
+
+def test_invalid_arguments_are_rejected_before_launch():
+    csa = _csa()
+    from clustered_sparse_attention_b200 import _lib
+    X = torch.zeros((1, 1, 100, 96), device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(_lib.SvgearError) as e:
+        csa.svgear_kmeans_assign(X, torch.zeros((1, 1, 4, 96), device="cuda"))
+    assert e.value.status == _lib.ERR_UNSUPPORTED
+    X = torch.zeros((1, 1, 100, 64), device="cuda")
+    with pytest.raises(_lib.SvgearError) as e:
+        csa.svgear_cluster(X, 101, 1)
+    assert e.value.status == _lib.ERR_INVALID_ARG
+    with pytest.raises(_lib.SvgearError):
+        csa.svgear_cluster(X, 10, 0)
