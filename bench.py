@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    p.add_argument("--heads", type=int, default=None,
+                   help="override the head count (smaller profiling cases)")
     return p.parse_args()
 
 
@@ -289,6 +291,9 @@ def workload_config(w, args):
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name="%s_h%d" % (w.name, args.heads))
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -371,7 +376,7 @@ def main():
     attend_ms = stage_ms["attend"]
     achieved = (f_sel + f_comp) / (attend_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    roofline = {"kernel": "svgear_attend (attend_simt_kernel)", "bound": "tensor",
+    roofline = {"kernel": "attend_sm100_kernel (svgear_attend, bf16)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": "bf16 dense, sustained, %s" % ("of measured" if peaks["source"] == "measured" else "of fallback"),
                 "traffic": None, "flops_per_launch": f_sel + f_comp}

@@ -25,7 +25,7 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_label_sort", "svgear_kmeans_update", "svgear_permute",
             "svgear_centroids", "svgear_probe", "svgear_route_select", "svgear_route",
             "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
-            "svgear_version", "svgear_kernel_launches")
+            "svgear_version", "svgear_kernel_launches", "svgear_attend_status")
 
 
 class Dims(ctypes.Structure):
@@ -69,6 +69,7 @@ def lib():
         "svgear_status_string": [ctypes.c_int],
         "svgear_version": [],
         "svgear_kernel_launches": [],
+        "svgear_attend_status": [P, SZ, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -267,7 +268,10 @@ def svgear_route(qbar, q_off, kbar, vbar, k_off, Kp, Vp, density, scale, return_
     return (pair_off, pair_kc, E) if return_errors else (pair_off, pair_kc)
 
 
-def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm, scale, O=None):
+def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm, scale, O=None,
+                  check_status=False):
+    """O in the original token order.  check_status=True synchronises and
+    raises if any bounded wait inside the kernel gave up."""
     qd = _tokens(Qp, "Qp")
     _tokens(Kp, "Kp")
     _tokens(Vp, "Vp")
@@ -281,6 +285,13 @@ def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_per
         _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Nk, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(pair_off),
         _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(q_perm), float(scale), _ptr(O), _ptr(ws), n,
         _stream()))
+    if check_status:
+        st = (ctypes.c_int32 * 4)()
+        _check("svgear_attend_status", lib().svgear_attend_status(_ptr(ws), n, st, _stream()))
+        if st[0] != OK:
+            raise SvgearError("svgear_attend (device: wait site %d, tile %d, cta %d)"
+                              % (st[1] >> 16, st[1] & 0xFFFF, st[2]), st[0],
+                              lib().svgear_status_string(st[0]).decode())
     return O
 
 

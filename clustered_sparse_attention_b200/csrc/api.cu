@@ -101,6 +101,23 @@ RouteWs carve_route(Carve& cv, size_t BH, int Cq, int Ck) {
     return w;
 }
 
+AttendWs carve_attend(Carve& cv, const svgear_dims& d, int Cq, int Ck) {
+    AttendWs w;
+    const size_t BH = bh_of(d);
+    w.maxT = ceil_div(d.N, 128) + Cq;
+    w.status = cv.take<int>(4);
+    w.kbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
+    w.vbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
+    w.meta = cv.take<int4>(BH * Cq);
+    w.seg_prefix = cv.take<int32_t>(BH * Cq * (size_t)(Ck + 1));
+    w.seg_row = cv.take<int32_t>(BH * Cq * (size_t)Ck);
+    w.comp_idx = cv.take<int32_t>(BH * Cq * (size_t)Ck);
+    w.comp_bias = cv.take<float>(BH * Cq * (size_t)Ck);
+    w.tiles = cv.take<int4>(BH * (size_t)w.maxT);
+    w.ntiles = cv.take<int32_t>(BH);
+    return w;
+}
+
 size_t ws_cluster(const svgear_dims& d, int C) {
     Carve a(nullptr), b(nullptr);
     carve_kpp(a, d, C);
@@ -153,7 +170,7 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             break;
         case SVGEAR_OP_ATTEND:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
-            cv.take<char>(kAlign);
+            carve_attend(cv, dims, C1, C2);
             break;
         default:
             return 0;
@@ -362,8 +379,24 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
         return SVGEAR_ERR_INVALID_ARG;
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(qdims) == 0) return SVGEAR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Carve cv(ws);
+    AttendWs w = carve_attend(cv, qdims, Cq, Ck);
+    if (qdims.dtype == SVGEAR_BF16)
+        return launch_attend_sm100(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc,
+                                   kbar, vbar, q_perm, scale, O, w, st);
+    if (cudaMemsetAsync(w.status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     return launch_attend_simt(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc, kbar,
-                              vbar, q_perm, scale, O, static_cast<cudaStream_t>(stream));
+                              vbar, q_perm, scale, O, st);
+}
+
+int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+    if (!ws || !status || ws_bytes < 4 * sizeof(int)) return SVGEAR_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, ws, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return SVGEAR_ERR_CUDA;
+    return SVGEAR_OK;
 }
 
 }  // extern "C"

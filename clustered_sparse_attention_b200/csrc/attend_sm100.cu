@@ -1,0 +1,550 @@
+// attend_sm100.cu -- bf16 tensor-core attention over the selected cluster
+// blocks plus centroid compensation of every skipped key cluster, in one
+// online softmax, on tcgen05 / TMEM (sm_100a).
+//
+// Method: "SVG-EAR measured error" (frontier-cs.org blog), toy example: a
+// skipped cluster of n keys with centroid score s_bar weighs n e^{s_bar} and
+// carries its mean value; SVG-EAR task page (agent step 3): the skipped
+// cluster is one key at its centroid, its score raised by log n, and every
+// row returns to its place; SVG2 summary, section 3.4: permutation validity
+// and the dynamic block-size kernel, which loads exactly the selected tokens
+// through a per-token address table and computes dense MMAs on them.
+//
+// B200 design (one CTA per 128-row tile of one query cluster):
+//   * the query cluster's selected key clusters form one compacted list of
+//     key rows; 4 producer warps gather 128 rows per tile (K and V) with
+//     16-byte cp.async into 128B-swizzled shared memory -- the per-token
+//     address table of the dynamic block-size kernel, with no padding inside
+//     the list; after the last key tile the skipped clusters' centroids
+//     (bf16) are gathered the same way, 128 per tile;
+//   * one thread issues tcgen05.mma: S = Q K^T (M=128, N=128, K=d) into one
+//     of two TMEM buffers, then O += P V (N=d, V as an MN-major operand)
+//     into a TMEM accumulator;
+//   * 4 softmax warps own one row each (TMEM lane = row): row max, exp2,
+//     the log2(n_c) bias of compensation columns, P to shared memory as bf16;
+//     O is rescaled in TMEM only when the running max grows by more than 2^8;
+//   * the epilogue divides by the row sum and writes O[q_perm[p]].
+// Every wait is bounded (1 s of %globaltimer); on expiry the CTA records
+// SVGEAR_ERR_TIMEOUT in the device status word, drains and returns, and
+// every later wait of the launch gives up at once.
+#include <math.h>
+
+#include "common.cuh"
+#include "launchers.h"
+#include "tc_ptx.cuh"
+
+namespace svgear {
+namespace sm100 {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int BM = 128;            // query rows per CTA
+constexpr int BN = 128;            // keys per tile
+constexpr int STAGES = 2;          // K/V ring
+constexpr int kProducerThreads = 128;
+constexpr int kSoftmaxThreads = 128;
+constexpr int kMmaWarp = 8;
+constexpr int kThreads = kProducerThreads + kSoftmaxThreads + 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s; a tile takes microseconds
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+// Swizzled 16-byte chunk address inside a tile of 128 rows x (regions of
+// 64 bf16): region r covers elements [64r, 64r+64) of every row.
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
+    const int region = chunk >> 3, cc = chunk & 7;
+    return tile + region * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+}
+
+struct Shared {
+    uint64_t q_full;
+    uint64_t kv_full[STAGES];
+    uint64_t kv_empty[STAGES];
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full;
+    uint64_t pv_done;
+    uint64_t o_full;
+    uint32_t tmem_base;
+    int abort_flag;
+    int keep_tmem;
+};
+
+// Bounded wait: gives up when this CTA or any other CTA of the launch has
+// already given up (the device status word is non-zero), or after kTimeoutNs.
+// err[0] is the status word; err[1] records where the first expired wait was
+// (site * 65536 + tile index), err[2] the CTA (blockIdx.y * 65536 + blockIdx.x).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int* err, int where) {
+    const uint32_t b = tc::smem_u32(bar);
+    if (tc::mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = tc::global_timer_ns();
+    volatile int* gerr = err;
+    while (true) {
+        if (tc::mbar_try_wait(b, parity)) return true;
+        if (*abort_flag || *gerr) {
+            *abort_flag = 1;
+            return false;
+        }
+        if (tc::global_timer_ns() - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            if (atomicCAS(err, 0, SVGEAR_ERR_TIMEOUT) == 0) {
+                err[1] = where;
+                err[2] = (int)(blockIdx.y * 65536 + blockIdx.x);
+            }
+            return false;
+        }
+    }
+}
+
+// One lane polls, the whole warp gets the same answer: the softmax and MMA
+// warps stay converged (they run .sync.aligned TMEM instructions and reach
+// the CTA barrier together).
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err, int where) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, err, where) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
+                    const bf16* __restrict__ Vp, int Nq, int Nk, int Cq, int Ck,
+                    const int32_t* __restrict__ q_perm, const bf16* __restrict__ kbar16,
+                    const bf16* __restrict__ vbar16, const int4* __restrict__ tiles,
+                    const int32_t* __restrict__ ntiles, int maxT, const int4* __restrict__ meta,
+                    const int32_t* __restrict__ seg_prefix, const int32_t* __restrict__ seg_row,
+                    const int32_t* __restrict__ comp_idx, const float* __restrict__ comp_bias,
+                    float scale_log2, bf16* __restrict__ O, int* __restrict__ err) {
+    constexpr int REG = D / 64;                 // 64-element regions per row
+    constexpr uint32_t kTileBytes = REG * 16384;
+    constexpr int CPR = D / 8;                  // 16-byte chunks per row
+    const int bh = blockIdx.y;
+    if ((int)blockIdx.x >= ntiles[bh]) return;
+    if (*(volatile int*)err != 0) return;   // an earlier CTA already gave up
+    const int4 tile = tiles[(size_t)bh * maxT + blockIdx.x];
+    const int ci = tile.x, q0 = tile.y, q_end = tile.z;
+    const int4 mt = meta[(size_t)bh * Cq + ci];   // {nseg, L keys, ncomp, 0}
+    const int L = mt.y, ncomp = mt.z;
+    const int T_real = (L + BN - 1) / BN;
+    const int T = T_real + (ncomp + BN - 1) / BN;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ Shared sh;
+    const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t sQ = base;
+    const uint32_t sK0 = sQ + kTileBytes;
+    const uint32_t sV0 = sK0 + STAGES * kTileBytes;
+    const uint32_t sP = sV0 + STAGES * kTileBytes;   // 128 rows x 128 keys
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        tc::mbar_init(tc::smem_u32(&sh.q_full), kProducerThreads);
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(tc::smem_u32(&sh.kv_full[s]), kProducerThreads);
+            tc::mbar_init(tc::smem_u32(&sh.kv_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(tc::smem_u32(&sh.s_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.s_free[s]), kSoftmaxThreads);
+        }
+        tc::mbar_init(tc::smem_u32(&sh.p_full), kSoftmaxThreads);
+        tc::mbar_init(tc::smem_u32(&sh.pv_done), 1);
+        tc::mbar_init(tc::smem_u32(&sh.o_full), 1);
+        sh.abort_flag = 0;
+        sh.keep_tmem = 0;
+        tc::mbar_init_fence();
+    }
+    if (warp == kMmaWarp) {
+        tc::tmem_alloc(tc::smem_u32(&sh.tmem_base), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int* abort_flag = &sh.abort_flag;
+
+    const size_t head = (size_t)bh * Nq * D;
+    const size_t khead = (size_t)bh * Nk * D;
+    const size_t row_meta = ((size_t)bh * Cq + ci) * Ck;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ producer
+        const int r = tid;
+        {
+            const int qrow = q0 + r;
+            const bool ok = qrow < q_end;
+            const bf16* src = Qp + head + (size_t)(ok ? qrow : q0) * D;
+#pragma unroll
+            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(sQ, r, c), src + c * 8, ok ? 16u : 0u);
+            tc::cp_async_commit();
+            tc::cp_async_wait<0>();
+            tc::fence_async_smem();
+            tc::mbar_arrive(tc::smem_u32(&sh.q_full));
+        }
+        const int32_t* pre = seg_prefix + ((size_t)bh * Cq + ci) * (Ck + 1);
+        const int32_t* srow = seg_row + row_meta;
+        const int32_t* cidx = comp_idx + row_meta;
+        const bf16* Kh = Kp + khead;
+        const bf16* Vh = Vp + khead;
+        const bf16* kbh = kbar16 + (size_t)bh * Ck * D;
+        const bf16* vbh = vbar16 + (size_t)bh * Ck * D;
+        int seg = 0;
+        bool ok_run = true;
+        for (int j = 0; j < T; ++j) {
+            const int st = j % STAGES;
+            // publish tile j-1 first: the stage tile j needs is only freed
+            // after the MMA has consumed tile j-1
+            if (j >= 1) {
+                tc::cp_async_wait<0>();
+                tc::fence_async_smem();
+                tc::mbar_arrive(tc::smem_u32(&sh.kv_full[(j - 1) % STAGES]));
+            }
+            if (j >= STAGES &&
+                !wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j)) {
+                ok_run = false;
+                break;
+            }
+            const bf16* sk = Kh;
+            const bf16* sv = Vh;
+            uint32_t bytes = 0;
+            if (j < T_real) {
+                const int p = j * BN + r;
+                if (p < L) {
+                    while (pre[seg + 1] <= p) ++seg;
+                    const int g = srow[seg] + (p - pre[seg]);
+                    sk = Kh + (size_t)g * D;
+                    sv = Vh + (size_t)g * D;
+                    bytes = 16;
+                }
+            } else {
+                const int p = (j - T_real) * BN + r;
+                if (p < ncomp) {
+                    const int c = cidx[p];
+                    sk = kbh + (size_t)c * D;
+                    sv = vbh + (size_t)c * D;
+                    bytes = 16;
+                }
+            }
+            const uint32_t tK = sK0 + st * kTileBytes, tV = sV0 + st * kTileBytes;
+#pragma unroll
+            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tK, r, c), sk + c * 8, bytes);
+#pragma unroll
+            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tV, r, c), sv + c * 8, bytes);
+            tc::cp_async_commit();
+        }
+        tc::cp_async_wait<0>();
+        if (ok_run && T > 0) {
+            tc::fence_async_smem();
+            tc::mbar_arrive(tc::smem_u32(&sh.kv_full[(T - 1) % STAGES]));
+        }
+        __syncwarp();
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax
+        const int r = tid - kProducerThreads;            // row == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const float* cb = comp_bias + row_meta;
+        float m_use = -INFINITY, l = 0.f;
+        bool ok_run = true;
+        for (int j = 0; j < T && ok_run; ++j) {
+            const int sb = j & 1;
+            if (!warp_wait_bar(&sh.s_full[sb], (j >> 1) & 1, abort_flag, err, (2 << 16) + j)) { ok_run = false; break; }
+            tc::fence_after_sync();
+            const bool comp = j >= T_real;
+            const int valid = comp ? min(BN, ncomp - (j - T_real) * BN) : min(BN, L - j * BN);
+            const float* bias = cb + (comp ? (j - T_real) * BN : 0);
+            const uint32_t sS = lane_base + sb * BN;
+            uint32_t v[32];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+                tc::tmem_ld32(sS + c4 * 32, v);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int col = c4 * 32 + e;
+                    float x = __uint_as_float(v[e]) * scale_log2;
+                    if (comp) x += (col < valid) ? bias[col] : 0.f;
+                    if (col < valid) mx = fmaxf(mx, x);
+                }
+            }
+            const float m_new = fmaxf(m_use, mx);
+            if (j >= 1 && !warp_wait_bar(&sh.pv_done, (j - 1) & 1, abort_flag, err, (3 << 16) + j)) { ok_run = false; break; }
+            // Lazy rescale of O: each row decides, but the TMEM loads/stores are
+            // warp-collective, so the warp rescales together when any row must
+            // (rows that need not use alpha = 1).
+            const bool need = j > 0 && m_new > m_use + kRescaleThreshold;
+            if (j == 0) m_use = m_new;
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = need ? tc::ex2(m_use - m_new) : 1.f;
+                const uint32_t sO = lane_base + 2 * BN;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    tc::tmem_ld32(sO + c4 * 32, v);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                    tc::tmem_st32(sO + c4 * 32, v);
+                }
+                tc::tmem_st_wait();
+                if (need) {
+                    l *= alpha;
+                    m_use = m_new;
+                }
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+                tc::tmem_ld32(sS + c4 * 32, v);
+                tc::tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int col = c4 * 32 + e;
+                    float x0 = __uint_as_float(v[e]) * scale_log2;
+                    float x1 = __uint_as_float(v[e + 1]) * scale_log2;
+                    if (comp) {
+                        x0 += (col < valid) ? bias[col] : 0.f;
+                        x1 += (col + 1 < valid) ? bias[col + 1] : 0.f;
+                    }
+                    const float p0 = (col < valid) ? tc::ex2(x0 - m_use) : 0.f;
+                    const float p1 = (col + 1 < valid) ? tc::ex2(x1 - m_use) : 0.f;
+                    sum += p0 + p1;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t dst = swz(sP, r, c4 * 4 + q);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                 "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]),
+                                 "r"(pk[4 * q + 3])
+                                 : "memory");
+                }
+            }
+            l += sum;
+            tc::fence_before_sync();
+            tc::mbar_arrive(tc::smem_u32(&sh.s_free[sb]));
+            tc::fence_async_smem();
+            tc::mbar_arrive(tc::smem_u32(&sh.p_full));
+        }
+        // epilogue: O / l back to the original token order
+        if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
+            tc::fence_after_sync();
+            const int p = q0 + r;
+            const float inv = 1.f / l;
+            const uint32_t sO = lane_base + 2 * BN;
+            const bool write = p < q_end;
+            const int dst = write ? q_perm[(size_t)bh * Nq + p] : 0;
+            bf16* orow = O + head + (size_t)dst * D;
+            uint32_t v[32];
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                tc::tmem_ld32(sO + c4 * 32, v);
+                tc::tmem_ld_wait();
+                if (write && (unsigned)dst < (unsigned)Nq) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[e]) * inv,
+                                                                 __uint_as_float(v[e + 1]) * inv);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    uint4* o4 = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        o4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ MMA issue
+        // The whole warp runs the loop; lane 0 issues the MMAs and commits.
+        constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
+        constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
+        bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
+        for (int j = 0; ok_run && j <= T; ++j) {
+            if (j < T) {
+                const int st = j % STAGES, sb = j & 1;
+                if (!warp_wait_bar(&sh.kv_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
+                    ok_run = false;
+                    break;
+                }
+                if (j >= 2 &&
+                    !warp_wait_bar(&sh.s_free[sb], ((j >> 1) - 1) & 1, abort_flag, err, (7 << 16) + j)) {
+                    ok_run = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t tK = sK0 + st * kTileBytes;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        tc::mma_bf16(tmem + sb * BN, tc::sw128_desc(sQ + off, 16, 1024),
+                                     tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
+                    }
+                    tc::commit(tc::smem_u32(&sh.s_full[sb]));
+                }
+                __syncwarp();
+            }
+            if (j >= 1) {
+                const int jj = j - 1, st = jj % STAGES;
+                if (!warp_wait_bar(&sh.p_full, jj & 1, abort_flag, err, (8 << 16) + jj)) {
+                    ok_run = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t tV = sV0 + st * kTileBytes;
+#pragma unroll
+                    for (int ks = 0; ks < BN / 16; ++ks) {
+                        const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        tc::mma_bf16(tmem + 2 * BN, tc::sw128_desc(sP + offp, 16, 1024),
+                                     tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
+                                     (jj > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    tc::commit(tc::smem_u32(&sh.kv_empty[st]));
+                    tc::commit(tc::smem_u32(&sh.pv_done));
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) tc::commit(tc::smem_u32(&sh.o_full));
+        __syncwarp();
+        // drain: every MMA this CTA issued is complete once o_full flips; if
+        // that wait expires, TMEM is left allocated rather than released under
+        // a running MMA (every later CTA of the launch returns before alloc)
+        if (!warp_wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16)) && lane == 0)
+            sh.keep_tmem = 1;
+        __syncwarp();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == kMmaWarp && !sh.keep_tmem) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Preparation: bf16 centroid tables, per-query-cluster key lists, tile table.
+// ---------------------------------------------------------------------------
+__global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+// One block per (query cluster, head).  Selected clusters in ascending order
+// become segments (prefix positions, first key row); skipped non-empty
+// clusters become the compensation list with bias log2(n_c).
+__global__ void attend_prep_kernel(const int32_t* __restrict__ k_off, int Ck, int Cq, int Nk,
+                                   const int32_t* __restrict__ pair_off,
+                                   const int32_t* __restrict__ pair_kc, int4* __restrict__ meta,
+                                   int32_t* __restrict__ seg_prefix, int32_t* __restrict__ seg_row,
+                                   int32_t* __restrict__ comp_idx, float* __restrict__ comp_bias) {
+    extern __shared__ unsigned char sel[];
+    const int i = blockIdx.x, bh = blockIdx.y;
+    const int32_t* ko = k_off + (size_t)bh * (Ck + 1);
+    const int32_t* po = pair_off + (size_t)bh * (Cq + 1);
+    const int32_t* pk = pair_kc + (size_t)bh * Cq * Ck;
+    for (int c = threadIdx.x; c < Ck; c += blockDim.x) sel[c] = 0;
+    __syncthreads();
+    for (int e = po[i] + threadIdx.x; e < po[i + 1]; e += blockDim.x) {
+        const int c = pk[e];
+        if ((unsigned)c < (unsigned)Ck) sel[c] = 1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const size_t rm = ((size_t)bh * Cq + i) * Ck;
+        int32_t* pre = seg_prefix + ((size_t)bh * Cq + i) * (Ck + 1);
+        int nseg = 0, L = 0, nc = 0;
+        for (int c = 0; c < Ck; ++c) {
+            const int a = ko[c], b = ko[c + 1];
+            if (b <= a || a < 0 || b > Nk) continue;
+            if (sel[c]) {
+                pre[nseg] = L;
+                seg_row[rm + nseg] = a;
+                L += b - a;
+                ++nseg;
+            } else {
+                comp_idx[rm + nc] = c;
+                comp_bias[rm + nc] = log2f((float)(b - a));
+                ++nc;
+            }
+        }
+        pre[nseg] = L;
+        for (int s = nseg + 1; s <= Ck; ++s) pre[s] = L;   // sentinels for the segment walk
+        meta[(size_t)bh * Cq + i] = make_int4(nseg, L, nc, 0);
+    }
+}
+
+// One block per head: every (cluster, 128-row tile) of the query segments.
+__global__ void attend_tiles_kernel(const int32_t* __restrict__ q_off, int Cq, int Nq, int maxT,
+                                    int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+    const int bh = blockIdx.x;
+    if (threadIdx.x != 0) return;
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    int k = 0;
+    for (int i = 0; i < Cq; ++i) {
+        const int a = qo[i], b = qo[i + 1];
+        if (b <= a || a < 0 || b > Nq) continue;
+        for (int r0 = a; r0 < b && k < maxT; r0 += BM) tiles[(size_t)bh * maxT + k++] = make_int4(i, r0, b, 0);
+    }
+    ntiles[bh] = k;
+}
+
+}  // namespace sm100
+
+// Workspace pieces of the tensor-core path (carved by the caller).
+int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd, int Nk,
+                        const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
+                        const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
+                        const float* vbar, const int32_t* q_perm, float scale, void* O,
+                        const AttendWs& w, cudaStream_t st) {
+    using namespace sm100;
+    const int BH = qd.B * qd.H;
+    const int D = qd.d;
+    if (cudaMemsetAsync(w.status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
+    const size_t nc = (size_t)BH * Ck * D;
+    const int cgrid = (int)((nc + 255) / 256 < 4096 ? (nc + 255) / 256 : 4096);
+    to_bf16_kernel<<<cgrid, 256, 0, st>>>(kbar, w.kbar16, nc);
+    count_launches(1);
+    to_bf16_kernel<<<cgrid, 256, 0, st>>>(vbar, w.vbar16, nc);
+    count_launches(1);
+    attend_prep_kernel<<<dim3(Cq, BH), 128, Ck, st>>>(k_off, Ck, Cq, Nk, pair_off, pair_kc, w.meta,
+                                                      w.seg_prefix, w.seg_row, w.comp_idx,
+                                                      w.comp_bias);
+    count_launches(1);
+    attend_tiles_kernel<<<BH, 32, 0, st>>>(q_off, Cq, qd.N, w.maxT, w.tiles, w.ntiles);
+    count_launches(1);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    const size_t smem = (size_t)(1 + 2 * STAGES) * (D / 64) * 16384 + 2 * 16384 + 1024;
+    if (D == 128) {
+        if (cudaFuncSetAttribute(attend_sm100_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        attend_sm100_kernel<128><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
+            static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp),
+            qd.N, Nk, Cq, Ck, q_perm, w.kbar16, w.vbar16, w.tiles, w.ntiles, w.maxT, w.meta,
+            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
+            w.status);
+    } else {
+        if (cudaFuncSetAttribute(attend_sm100_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        attend_sm100_kernel<64><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
+            static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp),
+            qd.N, Nk, Cq, Ck, q_perm, w.kbar16, w.vbar16, w.tiles, w.ntiles, w.maxT, w.meta,
+            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
+            w.status);
+    }
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+}  // namespace svgear

@@ -1,6 +1,7 @@
 // launchers.h -- host-side launch functions of the library's kernels (internal).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -42,6 +43,26 @@ int launch_route_select(const float* E, const int32_t* q_off, int Cq,
                         const int32_t* k_off, int Ck, int BH, long long budget,
                         int32_t* lists, int32_t* counts, int32_t* pair_off,
                         int32_t* pair_kc, cudaStream_t st);
+
+// attend_sm100.cu: workspace of the tensor-core attention
+struct AttendWs {
+    int* status;                 // device status word (0 or SVGEAR_ERR_TIMEOUT)
+    __nv_bfloat16* kbar16;       // [BH][Ck][d] bf16 key centroids
+    __nv_bfloat16* vbar16;       // [BH][Ck][d] bf16 value centroids
+    int4* meta;                  // [BH][Cq] {segments, selected keys, skipped clusters, 0}
+    int32_t* seg_prefix;         // [BH][Cq][Ck+1] list position of each segment
+    int32_t* seg_row;            // [BH][Cq][Ck] first key row of each segment
+    int32_t* comp_idx;           // [BH][Cq][Ck] skipped non-empty clusters
+    float* comp_bias;            // [BH][Cq][Ck] log2(n_c) of those clusters
+    int4* tiles;                 // [BH][maxT] {cluster, first row, end row, 0}
+    int32_t* ntiles;             // [BH]
+    int maxT;
+};
+int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims, int Nk,
+                        const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
+                        const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
+                        const float* vbar, const int32_t* q_perm, float scale, void* O,
+                        const AttendWs& w, cudaStream_t st);
 
 // attend_simt.cu
 int launch_attend_simt(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,

@@ -245,7 +245,9 @@ int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq,
  *   kbar,vbar float[B][H][Ck][d].
  *   q_perm    int32[B][H][Nq] (svgear_cluster's perm for the queries).
  *   O         out [B][H][Nq][d] (qdims.dtype).
- *   ws        svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck).
+ *   ws        svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck); holds
+ *             bf16 centroid copies, the per-query-cluster key lists, the tile
+ *             table and a device status word (svgear_attend_status).
  * bf16 runs on the tcgen05 tensor-core kernel; f32 on an fp32 SIMT kernel.
  * ------------------------------------------------------------------------ */
 int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
@@ -253,6 +255,15 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
                   int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc,
                   const float* kbar, const float* vbar, const int32_t* q_perm,
                   float scale, void* O, void* ws, size_t ws_bytes, void* stream);
+
+/* Device status of the last svgear_attend that used `ws`: copies 4 int32 to
+ * status[0..3] (host memory) and synchronises `stream`.  status[0] is 0 when
+ * every wait in the kernel completed, SVGEAR_ERR_TIMEOUT when a bounded wait
+ * gave up (the kernel drained and returned; O is not valid); status[1] and
+ * status[2] then say which wait (site * 65536 + tile) and which CTA
+ * (blockIdx.y * 65536 + blockIdx.x).  The words sit at the start of the
+ * workspace and every svgear_attend call clears them. */
+int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /* Workspace bytes for `op` at shape `dims` (N = tokens of the clustered
  * tensor; for SVGEAR_OP_ROUTE and SVGEAR_OP_ATTEND, dims.N = Nq and C2 = Ck),

@@ -244,7 +244,7 @@ def _check_attend(w, dev, density, rows=None):
     po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
                               Vp, density, w.scale)
     O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
-                          cq.perm, w.scale)
+                          cq.perm, w.scale, check_status=True)
     torch.cuda.synchronize()
     Og = np64(O)
     worst = (0.0, 0.0)
@@ -353,3 +353,65 @@ def test_invalid_arguments_are_rejected_before_launch():
     assert e.value.status == _lib.ERR_INVALID_ARG
     with pytest.raises(_lib.SvgearError):
         csa.svgear_cluster(X, 10, 0)
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("case", [
+    # (query cluster sizes, key cluster sizes, selected key clusters per query cluster)
+    ([128], [64, 64], [[0, 1]]),                       # one key tile, no compensation
+    ([128], [64, 64], [[1]]),                          # partial key tile + one compensation tile
+    ([200], [100, 150, 7, 300], [[0, 1, 3]]),          # 5 key tiles, ragged query tile
+    ([1, 129, 0, 300], [130, 1, 0, 250, 40], [[2], [0, 1, 3], [], [4]]),
+    ([64, 64], [5] * 300, [list(range(0, 300, 2)), []]),   # 3 compensation tiles
+    ([128], [128, 128, 128], [[0, 1, 2]], "spiky"),    # half the rows rescale O mid-row
+    ([256], [100, 60, 200], [[2], [0]], "spiky"),
+])
+def test_attend_kernel_on_handmade_layouts(D, case):
+    """The attention kernel alone on hand-built segments and pair lists,
+    against the oracle (bf16 inputs, fp32 centroids)."""
+    csa = _csa()
+    qs, ks, sel = case[:3]
+    spiky = len(case) > 3
+    g = np.random.default_rng(len(qs) * 7 + D)
+    Nq, Nk = sum(qs), sum(ks)
+    Cq, Ck = len(qs), len(ks)
+    if spiky:    # route pairs per query cluster: the spiky cases use one list per cluster
+        sel = sel[:Cq]
+    from clustered_sparse_attention_b200.synth import round_to_bf16
+    Q0 = g.standard_normal((Nq, D)).astype(np.float32)
+    K0 = g.standard_normal((Nk, D)).astype(np.float32)
+    if spiky:
+        # rows with an even index see a score jump of ~8.2 (log2 units) in the
+        # keys after the first tile; odd rows do not -> divergent rescales
+        Q0[::2, 0] = 20.0
+        K0[:, 0] = 0.0
+        K0[128:, 0] = 4.0 * (D / 128) ** 0.5
+    Qp = round_to_bf16(Q0)
+    Kp = round_to_bf16(K0)
+    Vp = round_to_bf16(g.standard_normal((Nk, D)).astype(np.float32))
+    q_off = np.concatenate([[0], np.cumsum(qs)]).astype(np.int32)
+    k_off = np.concatenate([[0], np.cumsum(ks)]).astype(np.int32)
+    pair_off = np.concatenate([[0], np.cumsum([len(s) for s in sel])]).astype(np.int32)
+    pair_kc = np.zeros(Cq * Ck, np.int32)
+    flat = [c for s in sel for c in s]
+    pair_kc[:len(flat)] = flat
+    kbar = oracle.segment_mean(Kp, k_off).astype(np.float32)
+    vbar = oracle.segment_mean(Vp, k_off).astype(np.float32)
+    q_perm = g.permutation(Nq).astype(np.int32)
+    scale = D ** -0.5
+
+    def dev(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.to(dt) if dt is not None else t).cuda()
+
+    O = csa.svgear_attend(dev(Qp[None, None], torch.bfloat16), dev(Kp[None, None], torch.bfloat16),
+                          dev(Vp[None, None], torch.bfloat16), dev(q_off[None, None]),
+                          dev(k_off[None, None]), dev(pair_off[None, None]), dev(pair_kc[None, None]),
+                          dev(kbar[None, None]), dev(vbar[None, None]), dev(q_perm[None, None]),
+                          scale, check_status=True)
+    torch.cuda.synchronize()
+    Oo, _ = oracle.attend(Qp, Kp, Vp, q_off, k_off, pair_off, np.array(flat, np.int32), kbar, vbar,
+                          q_perm, scale)
+    Og = np64(O)[0, 0]
+    assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2, (_rel_l2(Og, Oo),
+                                                                        np.abs(Og - Oo).max())
