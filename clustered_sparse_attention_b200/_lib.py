@@ -17,6 +17,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libsvgear.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+ERR_SCRATCH_LIMIT = -6
+NOALLOC_SORT_SCRATCH_INTS = 2 * 1024 * 1024
 F32, BF16 = 0, 1
 OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
 MAX_CLUSTERS = 4096
@@ -25,7 +27,8 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_label_sort", "svgear_kmeans_update", "svgear_permute",
             "svgear_centroids", "svgear_probe", "svgear_route_select", "svgear_route",
             "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
-            "svgear_version", "svgear_kernel_launches", "svgear_attend_status")
+            "svgear_version", "svgear_kernel_launches", "svgear_attend_status",
+            "svgear_label_sort_noalloc")
 
 
 class Dims(ctypes.Structure):
@@ -70,6 +73,7 @@ def lib():
         "svgear_version": [],
         "svgear_kernel_launches": [],
         "svgear_attend_status": [P, SZ, P, P],
+        "svgear_label_sort_noalloc": [P, Dims, I32, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)

@@ -141,6 +141,8 @@ const char* svgear_status_string(int status) {
         case SVGEAR_ERR_CUDA: return "CUDA launch failed";
         case SVGEAR_ERR_TIMEOUT: return "device wait timed out";
         case SVGEAR_ERR_WORKSPACE: return "workspace too small";
+        case SVGEAR_ERR_SCRATCH_LIMIT:
+            return "sizes exceed the fixed scratch of the allocation-free entry point";
         default: return "unknown status";
     }
 }

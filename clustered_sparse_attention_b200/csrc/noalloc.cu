@@ -1,0 +1,62 @@
+// noalloc.cu -- the label sort without a caller-provided workspace.
+//
+// Some callers cannot hand this library any scratch memory: a host framework
+// whose memory planner owns every device byte and forbids side allocations,
+// a real-time loop where cudaMalloc (slow and synchronising) is banned once
+// running, or a plugin interface that passes an operator only its input and
+// output buffers.  svgear_label_sort_noalloc serves them: its scratch (the
+// per-block label histograms of the counting sort) lives in the fixed array
+// below, which every GPU that loads the library keeps until the process
+// exits.  Nothing here calls cudaMalloc, cudaFree or an allocating routine.
+#include <mutex>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace {
+
+// File-scope scratch: block histograms [B*H][ceil(N/1024)][C] of int32.
+static __device__ __align__(256) int32_t g_sort_scratch[SVGEAR_NOALLOC_SORT_SCRATCH_INTS];
+
+// In host code `g_sort_scratch` names a host-side stand-in, not device memory,
+// so the kernels get the device address looked up once per device.
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+int32_t* g_scratch_addr[kMaxDevices] = {};
+
+int scratch_on_current_device(int32_t** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SVGEAR_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SVGEAR_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_sort_scratch) != cudaSuccess || p == nullptr)
+            return SVGEAR_ERR_CUDA;
+        g_scratch_addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = g_scratch_addr[dev];
+    return SVGEAR_OK;
+}
+
+}  // namespace
+
+extern "C" int svgear_label_sort_noalloc(const int32_t* labels, svgear_dims dims, int32_t C,
+                                         int32_t* perm, int32_t* offsets, void* stream) {
+    if (dims.B < 0 || dims.H < 0 || dims.N < 1) return SVGEAR_ERR_INVALID_ARG;
+    const size_t BH = (size_t)dims.B * (size_t)dims.H;
+    if (BH > 65535) return SVGEAR_ERR_UNSUPPORTED;
+    if (C < 1 || C > dims.N) return SVGEAR_ERR_INVALID_ARG;
+    if (C > SVGEAR_MAX_CLUSTERS) return SVGEAR_ERR_UNSUPPORTED;
+    if (!labels || !perm || !offsets) return SVGEAR_ERR_INVALID_ARG;
+    const size_t need = BH * (size_t)svgear::ceil_div(dims.N, svgear::kSortTokens) * (size_t)C;
+    if (need > (size_t)SVGEAR_NOALLOC_SORT_SCRATCH_INTS) return SVGEAR_ERR_SCRATCH_LIMIT;
+    if (BH == 0) return SVGEAR_OK;
+    int32_t* hist = nullptr;
+    const int s = scratch_on_current_device(&hist);
+    if (s != SVGEAR_OK) return s;
+    // The histogram pass overwrites every entry the later passes read, so the
+    // previous call's contents need no clearing.
+    return svgear::launch_label_sort(labels, (int)BH, dims.N, C, perm, offsets, hist,
+                                     static_cast<cudaStream_t>(stream));
+}

@@ -68,7 +68,8 @@ typedef enum {
     SVGEAR_ERR_UNSUPPORTED = -2,
     SVGEAR_ERR_CUDA = -3,
     SVGEAR_ERR_TIMEOUT = -4,
-    SVGEAR_ERR_WORKSPACE = -5
+    SVGEAR_ERR_WORKSPACE = -5,
+    SVGEAR_ERR_SCRATCH_LIMIT = -6
 } svgear_status;
 
 typedef enum { SVGEAR_F32 = 0, SVGEAR_BF16 = 1 } svgear_dtype;
@@ -264,6 +265,33 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
  * (blockIdx.y * 65536 + blockIdx.x).  The words sit at the start of the
  * workspace and every svgear_attend call clears them. */
 int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_label_sort_noalloc -- svgear_label_sort for callers that cannot give
+ * the library any scratch memory: a framework whose memory planner owns all
+ * device memory and forbids side allocations, a real-time loop in which
+ * cudaMalloc (slow and synchronising) is off limits once running, or a plugin
+ * interface that hands an operator only its inputs and outputs.  The paper
+ * has no counterpart; this is an interface convenience.
+ *
+ * Same arguments and results as svgear_label_sort, minus the workspace: the
+ * block histograms live in a fixed device array of
+ * SVGEAR_NOALLOC_SORT_SCRATCH_INTS int32 (8 MiB) that every GPU which loads the
+ * library keeps until the process exits.  B*H*ceil(N/1024)*C must not exceed
+ * that count (the Wan 720p key sort, 40*74*500, fits); larger sizes return
+ * SVGEAR_ERR_SCRATCH_LIMIT without launching.  No call allocates or frees
+ * device memory.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (every entry a call reads is rewritten by that call first), so
+ *     calls that overlap on the GPU -- on different streams, or from several
+ *     threads -- race and corrupt each other's result; serialise them.
+ * ------------------------------------------------------------------------ */
+#define SVGEAR_NOALLOC_SORT_SCRATCH_INTS (2u * 1024u * 1024u)
+int svgear_label_sort_noalloc(const int32_t* labels, svgear_dims dims, int32_t C,
+                              int32_t* perm, int32_t* offsets, void* stream);
 
 /* Workspace bytes for `op` at shape `dims` (N = tokens of the clustered
  * tensor; for SVGEAR_OP_ROUTE and SVGEAR_OP_ATTEND, dims.N = Nq and C2 = Ck),
