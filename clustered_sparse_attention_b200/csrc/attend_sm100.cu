@@ -62,8 +62,8 @@ struct Shared {
     uint64_t kv_empty[STAGES];
     uint64_t s_full[2];
     uint64_t s_free[2];
-    uint64_t p_full;
-    uint64_t pv_done;
+    uint64_t p_full[2];
+    uint64_t pv_done[2];
     uint64_t o_full;
     uint32_t tmem_base;
     int abort_flag;
@@ -121,6 +121,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                     float scale_log2, bf16* __restrict__ O, int* __restrict__ err) {
     constexpr int REG = D / 64;                 // 64-element regions per row
     constexpr uint32_t kTileBytes = REG * 16384;
+    constexpr uint32_t kPBytes = 2 * 16384;     // 128 rows x 128 keys bf16
     constexpr int CPR = D / 8;                  // 16-byte chunks per row
     const int bh = blockIdx.y;
     if ((int)blockIdx.x >= ntiles[bh]) return;
@@ -138,7 +139,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
     const uint32_t sQ = base;
     const uint32_t sK0 = sQ + kTileBytes;
     const uint32_t sV0 = sK0 + STAGES * kTileBytes;
-    const uint32_t sP = sV0 + STAGES * kTileBytes;   // 128 rows x 128 keys
+    const uint32_t sP0 = sV0 + STAGES * kTileBytes;   // two P buffers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -150,9 +151,9 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.s_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.s_free[s]), kSoftmaxThreads);
+            tc::mbar_init(tc::smem_u32(&sh.p_full[s]), kSoftmaxThreads);
+            tc::mbar_init(tc::smem_u32(&sh.pv_done[s]), 1);
         }
-        tc::mbar_init(tc::smem_u32(&sh.p_full), kSoftmaxThreads);
-        tc::mbar_init(tc::smem_u32(&sh.pv_done), 1);
         tc::mbar_init(tc::smem_u32(&sh.o_full), 1);
         sh.abort_flag = 0;
         sh.keep_tmem = 0;
@@ -174,6 +175,9 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
 
     if (warp < 4) {
         // ------------------------------------------------------------ producer
+        // One row per thread.  Copies are published by the cp.async engine
+        // itself (mbarrier arrive on completion), so a producer only ever
+        // waits for a free stage.
         const int r = tid;
         {
             const int qrow = q0 + r;
@@ -181,10 +185,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
             const bf16* src = Qp + head + (size_t)(ok ? qrow : q0) * D;
 #pragma unroll
             for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(sQ, r, c), src + c * 8, ok ? 16u : 0u);
-            tc::cp_async_commit();
-            tc::cp_async_wait<0>();
-            tc::fence_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&sh.q_full));
+            tc::cp_async_arrive_noinc(tc::smem_u32(&sh.q_full));
         }
         const int32_t* pre = seg_prefix + ((size_t)bh * Cq + ci) * (Ck + 1);
         const int32_t* srow = seg_row + row_meta;
@@ -194,21 +195,11 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
         const bf16* kbh = kbar16 + (size_t)bh * Ck * D;
         const bf16* vbh = vbar16 + (size_t)bh * Ck * D;
         int seg = 0;
-        bool ok_run = true;
         for (int j = 0; j < T; ++j) {
             const int st = j % STAGES;
-            // publish tile j-1 first: the stage tile j needs is only freed
-            // after the MMA has consumed tile j-1
-            if (j >= 1) {
-                tc::cp_async_wait<0>();
-                tc::fence_async_smem();
-                tc::mbar_arrive(tc::smem_u32(&sh.kv_full[(j - 1) % STAGES]));
-            }
             if (j >= STAGES &&
-                !wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j)) {
-                ok_run = false;
+                !wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
-            }
             const bf16* sk = Kh;
             const bf16* sv = Vh;
             uint32_t bytes = 0;
@@ -235,13 +226,9 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
             for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tK, r, c), sk + c * 8, bytes);
 #pragma unroll
             for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tV, r, c), sv + c * 8, bytes);
-            tc::cp_async_commit();
+            tc::cp_async_arrive_noinc(tc::smem_u32(&sh.kv_full[st]));
         }
         tc::cp_async_wait<0>();
-        if (ok_run && T > 0) {
-            tc::fence_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&sh.kv_full[(T - 1) % STAGES]));
-        }
         __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
@@ -250,36 +237,51 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
         const float* cb = comp_bias + row_meta;
         float m_use = -INFINITY, l = 0.f;
         bool ok_run = true;
+        uint32_t v[32];
         for (int j = 0; j < T && ok_run; ++j) {
             const int sb = j & 1;
-            if (!warp_wait_bar(&sh.s_full[sb], (j >> 1) & 1, abort_flag, err, (2 << 16) + j)) { ok_run = false; break; }
+            if (!warp_wait_bar(&sh.s_full[sb], (j >> 1) & 1, abort_flag, err, (2 << 16) + j)) {
+                ok_run = false;
+                break;
+            }
             tc::fence_after_sync();
+            const uint32_t sS = lane_base + sb * BN;
             const bool comp = j >= T_real;
             const int valid = comp ? min(BN, ncomp - (j - T_real) * BN) : min(BN, L - j * BN);
             const float* bias = cb + (comp ? (j - T_real) * BN : 0);
-            const uint32_t sS = lane_base + sb * BN;
-            uint32_t v[32];
+            // pass 1: row max of x = s * scale * log2(e) (+ log2 n_c on compensation columns)
             float mx = -INFINITY;
 #pragma unroll
             for (int c4 = 0; c4 < BN / 32; ++c4) {
                 tc::tmem_ld32(sS + c4 * 32, v);
                 tc::tmem_ld_wait();
+                if (comp) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = c4 * 32 + e;
-                    float x = __uint_as_float(v[e]) * scale_log2;
-                    if (comp) x += (col < valid) ? bias[col] : 0.f;
-                    if (col < valid) mx = fmaxf(mx, x);
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = c4 * 32 + e;
+                        if (col < valid) mx = fmaxf(mx, fmaf(__uint_as_float(v[e]), scale_log2, bias[col]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c4 * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
                 }
             }
+            if (!comp) mx *= scale_log2;   // scale > 0: max commutes with scaling
             const float m_new = fmaxf(m_use, mx);
-            if (j >= 1 && !warp_wait_bar(&sh.pv_done, (j - 1) & 1, abort_flag, err, (3 << 16) + j)) { ok_run = false; break; }
+
             // Lazy rescale of O: each row decides, but the TMEM loads/stores are
             // warp-collective, so the warp rescales together when any row must
-            // (rows that need not use alpha = 1).
+            // (rows that need not use alpha = 1).  O must be final up to PV(j-1).
             const bool need = j > 0 && m_new > m_use + kRescaleThreshold;
             if (j == 0) m_use = m_new;
             if (__any_sync(0xffffffffu, need)) {
+                if (!warp_wait_bar(&sh.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, err,
+                                   (3 << 16) + j)) {
+                    ok_run = false;
+                    break;
+                }
+                tc::fence_after_sync();
                 const float alpha = need ? tc::ex2(m_use - m_new) : 1.f;
                 const uint32_t sO = lane_base + 2 * BN;
 #pragma unroll
@@ -296,41 +298,51 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                     m_use = m_new;
                 }
             }
+            // P buffer sb is free once PV(j-2) has completed
+            if (j >= 2 &&
+                !warp_wait_bar(&sh.pv_done[sb], ((j >> 1) - 1) & 1, abort_flag, err, (10 << 16) + j)) {
+                ok_run = false;
+                break;
+            }
+            // pass 2: p = 2^(x - m), row sum, bf16 P into the swizzled buffer
+            const uint32_t sP = sP0 + sb * kPBytes;
+            const float neg_m = -m_use;
             float sum = 0.f;
 #pragma unroll
             for (int c4 = 0; c4 < BN / 32; ++c4) {
                 tc::tmem_ld32(sS + c4 * 32, v);
                 tc::tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int col = c4 * 32 + e;
-                    float x0 = __uint_as_float(v[e]) * scale_log2;
-                    float x1 = __uint_as_float(v[e + 1]) * scale_log2;
-                    if (comp) {
-                        x0 += (col < valid) ? bias[col] : 0.f;
-                        x1 += (col + 1 < valid) ? bias[col + 1] : 0.f;
-                    }
-                    const float p0 = (col < valid) ? tc::ex2(x0 - m_use) : 0.f;
-                    const float p1 = (col + 1 < valid) ? tc::ex2(x1 - m_use) : 0.f;
-                    sum += p0 + p1;
-                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
-                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t dst = swz(sP, r, c4 * 4 + q);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                                 "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]),
-                                 "r"(pk[4 * q + 3])
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const int k0 = q * 8 + e, col = c4 * 32 + k0;
+                        float x0, x1;
+                        if (comp) {
+                            x0 = fmaf(__uint_as_float(v[k0]), scale_log2, bias[col] + neg_m);
+                            x1 = fmaf(__uint_as_float(v[k0 + 1]), scale_log2, bias[col + 1] + neg_m);
+                        } else {
+                            x0 = fmaf(__uint_as_float(v[k0]), scale_log2, neg_m);
+                            x1 = fmaf(__uint_as_float(v[k0 + 1]), scale_log2, neg_m);
+                        }
+                        const float p0 = (col < valid) ? tc::ex2(x0) : 0.f;
+                        const float p1 = (col + 1 < valid) ? tc::ex2(x1) : 0.f;
+                        sum += p0 + p1;
+                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(sP, r, c4 * 4 + q)),
+                                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
                                  : "memory");
                 }
             }
             l += sum;
+            // S(j) consumed and P(j) written
             tc::fence_before_sync();
             tc::mbar_arrive(tc::smem_u32(&sh.s_free[sb]));
             tc::fence_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&sh.p_full));
+            tc::mbar_arrive(tc::smem_u32(&sh.p_full[sb]));
         }
         // epilogue: O / l back to the original token order
         if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
@@ -341,7 +353,6 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
             const bool write = p < q_end;
             const int dst = write ? q_perm[(size_t)bh * Nq + p] : 0;
             bf16* orow = O + head + (size_t)dst * D;
-            uint32_t v[32];
 #pragma unroll
             for (int c4 = 0; c4 < D / 32; ++c4) {
                 tc::tmem_ld32(sO + c4 * 32, v);
@@ -367,6 +378,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
         constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
         constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
         bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
+        if (ok_run) tc::fence_async_smem();
         for (int j = 0; ok_run && j <= T; ++j) {
             if (j < T) {
                 const int st = j % STAGES, sb = j & 1;
@@ -379,6 +391,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                     ok_run = false;
                     break;
                 }
+                tc::fence_async_smem();   // cp.async data -> tensor-core reads
                 tc::fence_after_sync();
                 if (lane == 0) {
                     const uint32_t tK = sK0 + st * kTileBytes;
@@ -393,14 +406,15 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                 __syncwarp();
             }
             if (j >= 1) {
-                const int jj = j - 1, st = jj % STAGES;
-                if (!warp_wait_bar(&sh.p_full, jj & 1, abort_flag, err, (8 << 16) + jj)) {
+                const int jj = j - 1, st = jj % STAGES, pb = jj & 1;
+                if (!warp_wait_bar(&sh.p_full[pb], (jj >> 1) & 1, abort_flag, err, (8 << 16) + jj)) {
                     ok_run = false;
                     break;
                 }
                 tc::fence_after_sync();
                 if (lane == 0) {
                     const uint32_t tV = sV0 + st * kTileBytes;
+                    const uint32_t sP = sP0 + pb * kPBytes;
 #pragma unroll
                     for (int ks = 0; ks < BN / 16; ++ks) {
                         const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -409,7 +423,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                                      (jj > 0 || ks > 0) ? 1u : 0u);
                     }
                     tc::commit(tc::smem_u32(&sh.kv_empty[st]));
-                    tc::commit(tc::smem_u32(&sh.pv_done));
+                    tc::commit(tc::smem_u32(&sh.pv_done[pb]));
                 }
                 __syncwarp();
             }
@@ -522,7 +536,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     attend_tiles_kernel<<<BH, 32, 0, st>>>(q_off, Cq, qd.N, w.maxT, w.tiles, w.ntiles);
     count_launches(1);
     const float scale_log2 = scale * 1.4426950408889634f;
-    const size_t smem = (size_t)(1 + 2 * STAGES) * (D / 64) * 16384 + 2 * 16384 + 1024;
+    const size_t smem = (size_t)(1 + 2 * STAGES) * (D / 64) * 16384 + 2 * 2 * 16384 + 1024;
     if (D == 128) {
         if (cudaFuncSetAttribute(attend_sm100_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
