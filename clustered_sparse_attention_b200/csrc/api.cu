@@ -118,8 +118,22 @@ AttendWs carve_attend(Carve& cv, const svgear_dims& d, int Cq, int Ck) {
     return w;
 }
 
+// svgear_cluster's workspace: per-head fixed-point flags, then the k-means++
+// scratch and the sort histograms (used one after the other, so they overlap).
+struct ClusterFlags {
+    int32_t* done;
+    int32_t* changed;
+};
+ClusterFlags carve_flags(Carve& cv, const svgear_dims& d) {
+    ClusterFlags f;
+    f.done = cv.take<int32_t>(bh_of(d));
+    f.changed = cv.take<int32_t>(bh_of(d));
+    return f;
+}
 size_t ws_cluster(const svgear_dims& d, int C) {
     Carve a(nullptr), b(nullptr);
+    carve_flags(a, d);
+    carve_flags(b, d);
     carve_kpp(a, d, C);
     carve_sort(b, d, C);
     return (a.off > b.off ? a.off : b.off) + kAlign;
@@ -255,6 +269,10 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
     if (bh_of(dims) == 0) return SVGEAR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int BH = (int)bh_of(dims);
+    Carve cf(ws);
+    ClusterFlags fl = carve_flags(cf, dims);
+    const size_t flag_bytes = (size_t)((char*)fl.changed - (char*)fl.done) + sizeof(int32_t) * BH;
+    if (cudaMemsetAsync(fl.done, 0, flag_bytes, st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     if (warm_centroids) {
         if (warm_centroids != centroids &&
             cudaMemcpyAsync(centroids, warm_centroids, sizeof(float) * BH * (size_t)C * dims.d,
@@ -262,16 +280,28 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
             return SVGEAR_ERR_CUDA;
     } else {
         Carve cv(ws);
+        carve_flags(cv, dims);
         KppWs w = carve_kpp(cv, dims, C);
         if ((s = launch_kmeanspp(X, dims, C, seed, centroids, w.chosen, w.D2, w.blocksum, st)))
             return s;
     }
     Carve cv(ws);
+    carve_flags(cv, dims);
     int32_t* hist = carve_sort(cv, dims, C);
+    // Lloyd rounds.  From the second round on, a head whose assignment moved
+    // no label has reached the fixed point (the sort and the deterministic
+    // update would reproduce the current perm, offsets and centroids), so its
+    // remaining kernels return at once; the results are those of all rounds.
     for (int it = 0; it < iters; ++it) {
-        if ((s = launch_assign(X, dims, centroids, C, labels, st))) return s;
-        if ((s = launch_label_sort(labels, BH, dims.N, C, perm, offsets, hist, st))) return s;
-        if ((s = launch_segment_mean(X, perm, offsets, C, dims, centroids, false, st))) return s;
+        const bool track = it > 0;
+        if ((s = launch_assign(X, dims, centroids, C, labels, st, fl.done,
+                               track ? fl.changed : nullptr)))
+            return s;
+        if (track && (s = launch_fixed_point(fl.changed, fl.done, BH, st))) return s;
+        if ((s = launch_label_sort(labels, BH, dims.N, C, perm, offsets, hist, st, fl.done)))
+            return s;
+        if ((s = launch_segment_mean(X, perm, offsets, C, dims, centroids, false, st, fl.done)))
+            return s;
     }
     if (Xp) return launch_permute(X, perm, dims, Xp, st);
     return SVGEAR_OK;

@@ -211,13 +211,15 @@ constexpr int kAsTM = 128, kAsTN = 128, kAsKC = 32, kAsThreads = 256;
 template <typename T, int D>
 __global__ void __launch_bounds__(kAsThreads, 2)
 assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, int C,
-              int32_t* __restrict__ labels) {
+              int32_t* __restrict__ labels, const int32_t* __restrict__ done,
+              int32_t* __restrict__ changed) {
     constexpr int EPC = Elem<T>::kPerChunk;
     extern __shared__ __align__(16) float smem[];
     float* Xs = smem;                  // [D][kAsTM]  (transposed tile)
     float* Cs = Xs + D * kAsTM;        // [kAsKC][kAsTN]
     float* cn = Cs + kAsKC * kAsTN;    // [kAsTN]
     const int bh = blockIdx.y, t0 = blockIdx.x * kAsTM, tid = threadIdx.x;
+    if (done && done[bh]) return;   // this head reached its fixed point
     const T* Xh = X + (size_t)bh * N * D;
     const float* Ch = cent + (size_t)bh * C * D;
 
@@ -310,14 +312,18 @@ assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, in
         }
         if (tx == 0) {
             const int row = (i < 4) ? ty * 4 + i : 64 + ty * 4 + (i - 4);
-            if (t0 + row < N) labels[(size_t)bh * N + t0 + row] = ix;
+            if (t0 + row < N) {
+                int32_t* lp = labels + (size_t)bh * N + t0 + row;
+                if (changed && *lp != ix) changed[bh] = 1;
+                *lp = ix;
+            }
         }
     }
 }
 
 template <typename T, int D>
 static int assign_impl(const T* X, svgear_dims dims, const float* cent, int C,
-                       int32_t* labels, cudaStream_t st) {
+                       int32_t* labels, const int32_t* done, int32_t* changed, cudaStream_t st) {
     const size_t smem = sizeof(float) * (D * kAsTM + kAsKC * kAsTN + kAsTN);
     // per-device function attribute; cheap enough to set on every call
     if (cudaFuncSetAttribute(assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -325,7 +331,7 @@ static int assign_impl(const T* X, svgear_dims dims, const float* cent, int C,
         return SVGEAR_ERR_CUDA;
     const int BH = dims.B * dims.H;
     assign_kernel<T, D><<<dim3(ceil_div(dims.N, kAsTM), BH), kAsThreads, smem, st>>>(
-        X, dims.N, cent, C, labels);
+        X, dims.N, cent, C, labels, done, changed);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
@@ -341,12 +347,13 @@ template <typename T, int D, bool GATHER>
 __global__ void __launch_bounds__(kSmThreads)
 segment_mean_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
                     const int32_t* __restrict__ offsets, int N, int C, float* out,
-                    bool empty_zero) {
+                    bool empty_zero, const int32_t* __restrict__ done) {
     constexpr int EPC = Elem<T>::kPerChunk;
     constexpr int L = D / EPC;
     constexpr int R = kSmThreads / L;
     __shared__ float part[R][D];
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    if (done && done[bh]) return;
     const int32_t* off = offsets + (size_t)bh * (C + 1);
     const int a = off[c], b = off[c + 1];
     float* o = out + ((size_t)bh * C + c) * D;
@@ -426,31 +433,51 @@ int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float
 
 template <typename T, int D>
 static int assign_disp(const void* X, svgear_dims dims, const float* cent, int C,
-                       int32_t* labels, cudaStream_t st) {
-    return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, st);
+                       int32_t* labels, const int32_t* done, int32_t* changed, cudaStream_t st) {
+    return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, done, changed, st);
 }
 int launch_assign(const void* X, svgear_dims dims, const float* cent, int C, int32_t* labels,
-                  cudaStream_t st) {
-    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, st);
+                  cudaStream_t st, const int32_t* done, int32_t* changed) {
+    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, done, changed, st);
+}
+
+// A head whose assignment changed no label has reached the fixed point of
+// Lloyd's iteration: its (deterministic) update would reproduce the current
+// centroids, so every later round is a no-op for it.
+__global__ void kmeans_fixed_point_kernel(int32_t* __restrict__ changed, int32_t* __restrict__ done,
+                                          int BH) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    if (!changed[bh]) done[bh] = 1;
+    changed[bh] = 0;
+}
+
+int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st) {
+    kmeans_fixed_point_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(changed, done, BH);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
 }
 
 template <typename T, int D>
 static int segmean_disp(const void* X, const int32_t* perm, const int32_t* offsets, int C,
-                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st) {
+                        svgear_dims dims, float* out, bool empty_zero, const int32_t* done,
+                        cudaStream_t st) {
     const int BH = dims.B * dims.H;
     if (perm)
         segment_mean_kernel<T, D, true><<<dim3(C, BH), kSmThreads, 0, st>>>(
-            static_cast<const T*>(X), perm, offsets, dims.N, C, out, empty_zero);
+            static_cast<const T*>(X), perm, offsets, dims.N, C, out, empty_zero, done);
     else
         segment_mean_kernel<T, D, false><<<dim3(C, BH), kSmThreads, 0, st>>>(
-            static_cast<const T*>(X), nullptr, offsets, dims.N, C, out, empty_zero);
+            static_cast<const T*>(X), nullptr, offsets, dims.N, C, out, empty_zero, done);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
 }
 int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets, int C,
-                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st) {
-    SVGEAR_DISPATCH(dims, segmean_disp, X, perm, offsets, C, dims, out, empty_zero, st);
+                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st,
+                        const int32_t* done) {
+    SVGEAR_DISPATCH(dims, segmean_disp, X, perm, offsets, C, dims, out, empty_zero, done, st);
 }
 
 template <typename T, int D>

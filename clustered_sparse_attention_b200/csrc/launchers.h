@@ -20,19 +20,23 @@ inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
                     float* centroids, int32_t* chosen, float* D2, double* blocksum,
                     cudaStream_t st);
+// done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
 int launch_assign(const void* X, svgear_dims dims, const float* centroids, int C,
-                  int32_t* labels, cudaStream_t st);
+                  int32_t* labels, cudaStream_t st, const int32_t* done = nullptr,
+                  int32_t* changed = nullptr);
+int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st);
 // Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
 // empty_zero: an empty segment writes zeros (else leaves the row untouched).
 int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets,
                         int C, svgear_dims dims, float* out, bool empty_zero,
-                        cudaStream_t st);
+                        cudaStream_t st, const int32_t* done = nullptr);
 int launch_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
                    cudaStream_t st);
 
 // sort.cu
 int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm,
-                      int32_t* offsets, int32_t* block_hist, cudaStream_t st);
+                      int32_t* offsets, int32_t* block_hist, cudaStream_t st,
+                      const int32_t* done = nullptr);
 
 // route.cu
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp,

@@ -17,9 +17,10 @@
 namespace svgear {
 
 __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int N, int C, int nblk,
-                                 int32_t* __restrict__ hist) {
+                                 int32_t* __restrict__ hist, const int32_t* __restrict__ done) {
     extern __shared__ int32_t h[];
     const int blk = blockIdx.x, bh = blockIdx.y;
+    if (done && done[bh]) return;
     for (int c = threadIdx.x; c < C; c += blockDim.x) h[c] = 0;
     __syncthreads();
     const int32_t* lab = labels + (size_t)bh * N;
@@ -37,10 +38,11 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int N, int 
 
 // hist[blk][c] <- global start position of block blk's first token labelled c.
 __global__ void sort_scan_kernel(int N, int C, int nblk, int32_t* __restrict__ hist,
-                                 int32_t* __restrict__ offsets) {
+                                 int32_t* __restrict__ offsets, const int32_t* __restrict__ done) {
     extern __shared__ int32_t tot[];   // [C] then [blockDim] partials
     int32_t* part = tot + C;
     const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    if (done && done[bh]) return;
     int32_t* hh = hist + (size_t)bh * nblk * C;
     for (int c = tid; c < C; c += nt) {
         int32_t run = 0;
@@ -77,9 +79,11 @@ __global__ void sort_scan_kernel(int N, int C, int nblk, int32_t* __restrict__ h
 
 __global__ void __launch_bounds__(32)
 sort_scatter_kernel(const int32_t* __restrict__ labels, int N, int C, int nblk,
-                    const int32_t* __restrict__ hist, int32_t* __restrict__ perm) {
+                    const int32_t* __restrict__ hist, int32_t* __restrict__ perm,
+                    const int32_t* __restrict__ done) {
     extern __shared__ int32_t cur[];
     const int blk = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+    if (done && done[bh]) return;
     const int32_t* hb = hist + ((size_t)bh * nblk + blk) * C;
     for (int c = lane; c < C; c += 32) cur[c] = hb[c];
     __syncwarp();
@@ -101,15 +105,15 @@ sort_scatter_kernel(const int32_t* __restrict__ labels, int N, int C, int nblk,
 }
 
 int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm,
-                      int32_t* offsets, int32_t* hist, cudaStream_t st) {
+                      int32_t* offsets, int32_t* hist, cudaStream_t st, const int32_t* done) {
     const int nblk = ceil_div(N, kSortTokens);
     const size_t sh = sizeof(int32_t) * C;
-    sort_hist_kernel<<<dim3(nblk, BH), 256, sh, st>>>(labels, N, C, nblk, hist);
+    sort_hist_kernel<<<dim3(nblk, BH), 256, sh, st>>>(labels, N, C, nblk, hist, done);
     count_launches(1);
     const int nt = 512;
-    sort_scan_kernel<<<BH, nt, sizeof(int32_t) * (C + nt), st>>>(N, C, nblk, hist, offsets);
+    sort_scan_kernel<<<BH, nt, sizeof(int32_t) * (C + nt), st>>>(N, C, nblk, hist, offsets, done);
     count_launches(1);
-    sort_scatter_kernel<<<dim3(nblk, BH), 32, sh, st>>>(labels, N, C, nblk, hist, perm);
+    sort_scatter_kernel<<<dim3(nblk, BH), 32, sh, st>>>(labels, N, C, nblk, hist, perm, done);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;

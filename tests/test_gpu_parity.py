@@ -415,3 +415,18 @@ def test_attend_kernel_on_handmade_layouts(D, case):
     Og = np64(O)[0, 0]
     assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2, (_rel_l2(Og, Oo),
                                                                         np.abs(Og - Oo).max())
+
+
+def test_cluster_fixed_point_gives_the_same_result_as_more_rounds():
+    """Once a round moves no label, later rounds are exact no-ops: 60 and 120
+    rounds must agree bit for bit, and one more oracle round moves nothing."""
+    csa = _csa()
+    w = SMALL_BF16
+    host, dev = _inputs(w)
+    a = csa.svgear_cluster(dev["k"], w.Ck, 60, seed=4)
+    b = csa.svgear_cluster(dev["k"], w.Ck, 120, seed=4)
+    torch.cuda.synchronize()
+    for f in ("labels", "perm", "offsets", "centroids", "Xp"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    for h in range(w.H):
+        check_assign(host["k"][0, h], b.centroids.cpu().numpy()[0, h], b.labels.cpu().numpy()[0, h])
