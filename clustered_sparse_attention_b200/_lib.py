@@ -21,6 +21,7 @@ ERR_SCRATCH_LIMIT = -6
 NOALLOC_SORT_SCRATCH_INTS = 2 * 1024 * 1024
 F32, BF16 = 0, 1
 OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
+OP_KMEANS_ASSIGN = 6
 MAX_CLUSTERS = 4096
 
 EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
@@ -59,7 +60,7 @@ def lib():
     sig = {
         "svgear_cluster": [P, Dims, I32, I32, P, U64, P, P, P, P, P, P, SZ, P],
         "svgear_kmeanspp_init": [P, Dims, I32, U64, P, P, P, SZ, P],
-        "svgear_kmeans_assign": [P, Dims, P, I32, P, P],
+        "svgear_kmeans_assign": [P, Dims, P, I32, P, P, SZ, P],
         "svgear_label_sort": [P, Dims, I32, P, P, P, SZ, P],
         "svgear_kmeans_update": [P, Dims, P, I32, P, P, SZ, P],
         "svgear_permute": [P, P, Dims, P, P],
@@ -182,8 +183,9 @@ def svgear_kmeans_assign(X, centroids):
     B, H, N, d = X.shape
     C = centroids.shape[2]
     labels = torch.empty((B, H, N), dtype=torch.int32, device=X.device)
+    ws, n = _workspace(OP_KMEANS_ASSIGN, dims, C, 0, X.device)
     _check("svgear_kmeans_assign", lib().svgear_kmeans_assign(
-        _ptr(X), dims, _ptr(centroids), C, _ptr(labels), _stream()))
+        _ptr(X), dims, _ptr(centroids), C, _ptr(labels), _ptr(ws), n, _stream()))
     return labels
 
 

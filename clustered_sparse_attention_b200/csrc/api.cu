@@ -66,6 +66,9 @@ KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
 int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {
     return cv.take<int32_t>(bh_of(d) * ceil_div(d.N, kSortTokens) * (size_t)C);
 }
+float* carve_assign(Carve& cv, const svgear_dims& d, int C) {
+    return cv.take<float>(assign_scratch_floats((int)bh_of(d), C, d.d));
+}
 struct UpdWs {
     int32_t* perm;
     int32_t* offsets;
@@ -136,6 +139,7 @@ size_t ws_cluster(const svgear_dims& d, int C) {
     carve_flags(b, d);
     carve_kpp(a, d, C);
     carve_sort(b, d, C);
+    carve_assign(b, d, C);
     return (a.off > b.off ? a.off : b.off) + kAlign;
 }
 
@@ -180,6 +184,10 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             if (check_C(C1, dims.N)) return 0;
             carve_update(cv, dims, C1);
             break;
+        case SVGEAR_OP_KMEANS_ASSIGN:
+            if (check_C(C1, dims.N)) return 0;
+            carve_assign(cv, dims, C1);
+            break;
         case SVGEAR_OP_ROUTE:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
             carve_route(cv, bh_of(dims), C1, C2);
@@ -210,14 +218,18 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
 }
 
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids, int32_t C,
-                         int32_t* labels, void* stream) {
+                         int32_t* labels, void* ws, size_t ws_bytes, void* stream) {
     int s = check_dims(dims);
     if (s) return s;
     if ((s = check_C(C, dims.N))) return s;
-    if (!X || !centroids || !labels || !aligned16(X) || !aligned16(centroids))
+    if (!X || !centroids || !labels || !ws || !aligned16(X) || !aligned16(centroids))
         return SVGEAR_ERR_INVALID_ARG;
+    if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN, dims, C, 0))
+        return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
-    return launch_assign(X, dims, centroids, C, labels, static_cast<cudaStream_t>(stream));
+    Carve cv(ws);
+    return launch_assign(X, dims, centroids, C, labels, carve_assign(cv, dims, C),
+                         static_cast<cudaStream_t>(stream));
 }
 
 int svgear_label_sort(const int32_t* labels, svgear_dims dims, int32_t C, int32_t* perm,
@@ -288,13 +300,14 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
     Carve cv(ws);
     carve_flags(cv, dims);
     int32_t* hist = carve_sort(cv, dims, C);
+    float* ascratch = carve_assign(cv, dims, C);
     // Lloyd rounds.  From the second round on, a head whose assignment moved
     // no label has reached the fixed point (the sort and the deterministic
     // update would reproduce the current perm, offsets and centroids), so its
     // remaining kernels return at once; the results are those of all rounds.
     for (int it = 0; it < iters; ++it) {
         const bool track = it > 0;
-        if ((s = launch_assign(X, dims, centroids, C, labels, st, fl.done,
+        if ((s = launch_assign(X, dims, centroids, C, labels, ascratch, st, fl.done,
                                track ? fl.changed : nullptr)))
             return s;
         if (track && (s = launch_fixed_point(fl.changed, fl.done, BH, st))) return s;

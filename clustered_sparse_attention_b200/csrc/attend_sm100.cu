@@ -81,7 +81,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     const uint64_t t0 = tc::global_timer_ns();
     volatile int* gerr = err;
     while (true) {
-        if (tc::mbar_try_wait(b, parity)) return true;
+        // sleep in the instruction (woken by the phase completing), so a
+        // waiting warp takes no issue slots from the working ones
+        if (tc::mbar_try_wait_sleep(b, parity, 20000u)) return true;
         if (*abort_flag || *gerr) {
             *abort_flag = 1;
             return false;
@@ -198,7 +200,7 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
         for (int j = 0; j < T; ++j) {
             const int st = j % STAGES;
             if (j >= STAGES &&
-                !wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
+                !warp_wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
             const bf16* sk = Kh;
             const bf16* sv = Vh;

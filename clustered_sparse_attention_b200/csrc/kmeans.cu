@@ -205,26 +205,76 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed,
 // ---------------------------------------------------------------------------
 // Assignment: a 128-token x 128-centroid register-tiled fp32 contraction per
 // step (256 threads, 8x8 per thread), distance |c|^2 - 2 x.c, argmin fused.
+// The centroids are first re-laid k-major ([d][Cpad], Cpad a multiple of 128,
+// padding norm = +inf), so each 32-deep chunk of a centroid tile is a plain
+// 16-byte cp.async copy into shared memory, double-buffered behind the FMAs.
 // ---------------------------------------------------------------------------
 constexpr int kAsTM = 128, kAsTN = 128, kAsKC = 32, kAsThreads = 256;
 
+__device__ __forceinline__ void cpa16(float* dst_smem, const float* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+
+// cT[bh][k][c] = cent[bh][c][k] (0 for padding), cn[bh][c] = |c|^2 (+inf for padding).
+template <int D>
+__global__ void centroid_kmajor_kernel(const float* __restrict__ cent, int C, int Cpad,
+                                       float* __restrict__ cT, float* __restrict__ cn,
+                                       const int32_t* __restrict__ done) {
+    const int bh = blockIdx.y;
+    if (done && done[bh]) return;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= Cpad) return;
+    const float* src = cent + ((size_t)bh * C + c) * D;
+    float* dst = cT + (size_t)bh * D * Cpad + c;
+    float s = 0.f;
+    if (c < C) {
+        for (int k = 0; k < D; ++k) {
+            const float v = src[k];
+            s = fmaf(v, v, s);
+            dst[(size_t)k * Cpad] = v;
+        }
+        cn[(size_t)bh * Cpad + c] = s;
+    } else {
+        for (int k = 0; k < D; ++k) dst[(size_t)k * Cpad] = 0.f;
+        cn[(size_t)bh * Cpad + c] = __int_as_float(0x7f800000);
+    }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kAsThreads, 2)
-assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, int C,
-              int32_t* __restrict__ labels, const int32_t* __restrict__ done,
-              int32_t* __restrict__ changed) {
+assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cT,
+              const float* __restrict__ cnorm, int C, int Cpad, int32_t* __restrict__ labels,
+              const int32_t* __restrict__ done, int32_t* __restrict__ changed) {
     constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int CPR = D / EPC;               // 16-byte chunks per token row
     extern __shared__ __align__(16) float smem[];
-    float* Xs = smem;                  // [D][kAsTM]  (transposed tile)
-    float* Cs = Xs + D * kAsTM;        // [kAsKC][kAsTN]
-    float* cn = Cs + kAsKC * kAsTN;    // [kAsTN]
+    float* Xs = smem;                          // [D][kAsTM] (transposed tile)
+    float* Cs = Xs + D * kAsTM;                // [2][kAsKC][kAsTN]
     const int bh = blockIdx.y, t0 = blockIdx.x * kAsTM, tid = threadIdx.x;
     if (done && done[bh]) return;   // this head reached its fixed point
     const T* Xh = X + (size_t)bh * N * D;
-    const float* Ch = cent + (size_t)bh * C * D;
+    const float* cTh = cT + (size_t)bh * D * Cpad;
+    const float* cnh = cnorm + (size_t)bh * Cpad;
+    const int nchunks = (Cpad / kAsTN) * (D / kAsKC);
 
-    for (int q = tid; q < kAsTM * (D / EPC); q += kAsThreads) {
-        const int row = q / (D / EPC), col = (q % (D / EPC)) * EPC;
+    // chunk n: centroid tile n / (D/kAsKC), depth slice n % (D/kAsKC)
+    auto load_chunk = [&](int n, int buf) {
+        const int c0 = (n / (D / kAsKC)) * kAsTN, k0 = (n % (D / kAsKC)) * kAsKC;
+        float* dst = Cs + buf * kAsKC * kAsTN;
+#pragma unroll
+        for (int q = tid; q < kAsKC * kAsTN / 4; q += kAsThreads) {
+            const int kk = q / (kAsTN / 4), cc = (q % (kAsTN / 4)) * 4;
+            cpa16(dst + kk * kAsTN + cc, cTh + (size_t)(k0 + kk) * Cpad + c0 + cc);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    load_chunk(0, 0);
+
+    // token tile, transposed; consecutive lanes take consecutive tokens so the
+    // transposed shared-memory stores are conflict-free
+    for (int q = tid; q < kAsTM * CPR; q += kAsThreads) {
+        const int row = q % kAsTM, col = (q / kAsTM) * EPC;
         float v[EPC];
         if (t0 + row < N) Elem<T>::load(Xh + (size_t)(t0 + row) * D + col, v);
         else
@@ -239,65 +289,55 @@ assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, in
     int besti[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) { bestd[i] = __int_as_float(0x7f800000); besti[i] = 0; }
+    float acc[8][8];
 
-    for (int c0 = 0; c0 < C; c0 += kAsTN) {
+    for (int n = 0; n < nchunks; ++n) {
+        const int kslice = n % (D / kAsKC);
+        if (n + 1 < nchunks) {
+            load_chunk(n + 1, (n + 1) & 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();
-        if (tid < kAsTN) {
-            const int c = c0 + tid;
-            float s = 0.f;
-            if (c < C)
-                for (int k = 0; k < D; ++k) { float v = Ch[(size_t)c * D + k]; s = fmaf(v, v, s); }
-            cn[tid] = s;
+        if (kslice == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
         }
-        float acc[8][8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
-
-        for (int k0 = 0; k0 < D; k0 += kAsKC) {
-            __syncthreads();
-            for (int q = tid; q < kAsTN * (kAsKC / 4); q += kAsThreads) {
-                const int cc = q / (kAsKC / 4), kk = (q % (kAsKC / 4)) * 4;
-                const int c = c0 + cc;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (c < C) v = __ldg(reinterpret_cast<const float4*>(Ch + (size_t)c * D + k0 + kk));
-                Cs[(kk + 0) * kAsTN + cc] = v.x;
-                Cs[(kk + 1) * kAsTN + cc] = v.y;
-                Cs[(kk + 2) * kAsTN + cc] = v.z;
-                Cs[(kk + 3) * kAsTN + cc] = v.w;
-            }
-            __syncthreads();
+        const float* cbuf = Cs + (n & 1) * kAsKC * kAsTN;
+        const int k0 = kslice * kAsKC;
 #pragma unroll 4
-            for (int k = 0; k < kAsKC; ++k) {
-                const float* xr = Xs + (k0 + k) * kAsTM;
-                const float* cr = Cs + k * kAsTN;
-                float4 a0 = *reinterpret_cast<const float4*>(xr + ty * 4);
-                float4 a1 = *reinterpret_cast<const float4*>(xr + 64 + ty * 4);
-                float4 b0 = *reinterpret_cast<const float4*>(cr + tx * 4);
-                float4 b1 = *reinterpret_cast<const float4*>(cr + 64 + tx * 4);
-                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        for (int k = 0; k < kAsKC; ++k) {
+            const float* xr = Xs + (k0 + k) * kAsTM;
+            const float* cr = cbuf + k * kAsTN;
+            const float4 a0 = *reinterpret_cast<const float4*>(xr + ty * 4);
+            const float4 a1 = *reinterpret_cast<const float4*>(xr + 64 + ty * 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(cr + tx * 4);
+            const float4 b1 = *reinterpret_cast<const float4*>(cr + 64 + tx * 4);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(a[i], b[jj], acc[i][jj]);
-            }
+                for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(a[i], b[jj], acc[i][jj]);
         }
-        // candidates of this thread come in increasing centroid order
+        if (kslice == D / kAsKC - 1) {
+            // candidates of this thread come in increasing centroid order
+            const int c0 = (n / (D / kAsKC)) * kAsTN;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            const int cj = (jj < 4) ? tx * 4 + jj : 64 + tx * 4 + (jj - 4);
-            const int c = c0 + cj;
-            if (c < C) {
-                const float cnv = cn[cj];
+            for (int jj = 0; jj < 8; ++jj) {
+                const int cj = (jj < 4) ? tx * 4 + jj : 64 + tx * 4 + (jj - 4);
+                const float cnv = __ldg(cnh + c0 + cj);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float dist = fmaf(-2.f, acc[i][jj], cnv);
-                    if (dist < bestd[i]) { bestd[i] = dist; besti[i] = c; }
+                    const float dist = fmaf(-2.f, acc[i][jj], cnv);
+                    if (dist < bestd[i]) { bestd[i] = dist; besti[i] = c0 + cj; }
                 }
             }
         }
+        __syncthreads();   // buffer n&1 is refilled by the next iteration's load
     }
     // lexicographic (distance, index) minimum over the 16 threads of a row group
 #pragma unroll
@@ -306,8 +346,8 @@ assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, in
         int ix = besti[i];
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) {
-            float od = __shfl_xor_sync(0xffffffffu, dd, o);
-            int oi = __shfl_xor_sync(0xffffffffu, ix, o);
+            const float od = __shfl_xor_sync(0xffffffffu, dd, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
             if (od < dd || (od == dd && oi < ix)) { dd = od; ix = oi; }
         }
         if (tx == 0) {
@@ -323,18 +363,28 @@ assign_kernel(const T* __restrict__ X, int N, const float* __restrict__ cent, in
 
 template <typename T, int D>
 static int assign_impl(const T* X, svgear_dims dims, const float* cent, int C,
-                       int32_t* labels, const int32_t* done, int32_t* changed, cudaStream_t st) {
-    const size_t smem = sizeof(float) * (D * kAsTM + kAsKC * kAsTN + kAsTN);
+                       int32_t* labels, const int32_t* done, int32_t* changed, float* cT,
+                       float* cnorm, cudaStream_t st) {
+    const int Cpad = ceil_div(C, kAsTN) * kAsTN;
+    const int BH = dims.B * dims.H;
+    centroid_kmajor_kernel<D><<<dim3(ceil_div(Cpad, 128), BH), 128, 0, st>>>(cent, C, Cpad, cT, cnorm,
+                                                                             done);
+    count_launches(1);
+    const size_t smem = sizeof(float) * (D * kAsTM + 2 * kAsKC * kAsTN);
     // per-device function attribute; cheap enough to set on every call
     if (cudaFuncSetAttribute(assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
-    const int BH = dims.B * dims.H;
     assign_kernel<T, D><<<dim3(ceil_div(dims.N, kAsTM), BH), kAsThreads, smem, st>>>(
-        X, dims.N, cent, C, labels, done, changed);
+        X, dims.N, cT, cnorm, C, Cpad, labels, done, changed);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
+}
+
+size_t assign_scratch_floats(int BH, int C, int D) {
+    const size_t Cpad = (size_t)ceil_div(C, kAsTN) * kAsTN;
+    return (size_t)BH * Cpad * (D + 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -433,12 +483,17 @@ int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float
 
 template <typename T, int D>
 static int assign_disp(const void* X, svgear_dims dims, const float* cent, int C,
-                       int32_t* labels, const int32_t* done, int32_t* changed, cudaStream_t st) {
-    return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, done, changed, st);
+                       int32_t* labels, const int32_t* done, int32_t* changed, float* scratch,
+                       cudaStream_t st) {
+    const size_t Cpad = (size_t)ceil_div(C, kAsTN) * kAsTN;
+    float* cT = scratch;
+    float* cn = scratch + (size_t)dims.B * dims.H * Cpad * D;
+    return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, done, changed, cT,
+                             cn, st);
 }
 int launch_assign(const void* X, svgear_dims dims, const float* cent, int C, int32_t* labels,
-                  cudaStream_t st, const int32_t* done, int32_t* changed) {
-    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, done, changed, st);
+                  float* scratch, cudaStream_t st, const int32_t* done, int32_t* changed) {
+    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, done, changed, scratch, st);
 }
 
 // A head whose assignment changed no label has reached the fixed point of

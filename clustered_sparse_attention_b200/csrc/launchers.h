@@ -21,9 +21,11 @@ int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
                     float* centroids, int32_t* chosen, float* D2, double* blocksum,
                     cudaStream_t st);
 // done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
+// scratch: assign_scratch_floats(B*H, C, d) floats (k-major centroid copy + norms).
 int launch_assign(const void* X, svgear_dims dims, const float* centroids, int C,
-                  int32_t* labels, cudaStream_t st, const int32_t* done = nullptr,
-                  int32_t* changed = nullptr);
+                  int32_t* labels, float* scratch, cudaStream_t st,
+                  const int32_t* done = nullptr, int32_t* changed = nullptr);
+size_t assign_scratch_floats(int BH, int C, int D);
 int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st);
 // Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
 // empty_zero: an empty segment writes zeros (else leaves the row untouched).

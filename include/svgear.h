@@ -87,7 +87,8 @@ typedef enum {
     SVGEAR_OP_LABEL_SORT = 2,
     SVGEAR_OP_KMEANS_UPDATE = 3,
     SVGEAR_OP_ROUTE = 4,
-    SVGEAR_OP_ATTEND = 5
+    SVGEAR_OP_ATTEND = 5,
+    SVGEAR_OP_KMEANS_ASSIGN = 6
 } svgear_op;
 
 /* Largest cluster count any call accepts (shared-memory tables). */
@@ -141,9 +142,12 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
                          size_t ws_bytes, void* stream);
 
 /* k-means assignment: labels[t] = argmin_c |x_t - c|^2, lowest c on exact
- * ties, evaluated in fp32 as |c|^2 - 2 x.c.  Needs no workspace. */
+ * ties, evaluated in fp32 as |c|^2 - 2 x.c.
+ *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN) (a k-major copy of
+ *       the centroids and their norms). */
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids,
-                         int32_t C, int32_t* labels, void* stream);
+                         int32_t C, int32_t* labels, void* ws, size_t ws_bytes,
+                         void* stream);
 
 /* Stable counting sort of labels ([TASK] step 1: the sorted order).
  *   labels   int32[B][H][N] in 0..C-1.

@@ -67,17 +67,22 @@ def test_validation_before_launch(L):
     from clustered_sparse_attention_b200 import _lib
     fake = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
     ws_small = ctypes.c_size_t(16)
+    big = ctypes.c_size_t(1 << 30)
     # null X
-    assert L.svgear_kmeans_assign(None, _dims(), fake, 10, fake, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_kmeans_assign(None, _dims(), fake, 10, fake, fake, big, None) == _lib.ERR_INVALID_ARG
     # unsupported head dimension / dtype
-    assert L.svgear_kmeans_assign(fake, _dims(d=96), fake, 10, fake, None) == _lib.ERR_UNSUPPORTED
-    assert L.svgear_kmeans_assign(fake, _dims(dtype=3), fake, 10, fake, None) == _lib.ERR_UNSUPPORTED
+    assert L.svgear_kmeans_assign(fake, _dims(d=96), fake, 10, fake, fake, big, None) == _lib.ERR_UNSUPPORTED
+    assert L.svgear_kmeans_assign(fake, _dims(dtype=3), fake, 10, fake, fake, big, None) == _lib.ERR_UNSUPPORTED
     # C out of range
-    assert L.svgear_kmeans_assign(fake, _dims(), fake, 0, fake, None) == _lib.ERR_INVALID_ARG
-    assert L.svgear_kmeans_assign(fake, _dims(N=5000), fake, 4097, fake, None) == _lib.ERR_UNSUPPORTED
+    assert L.svgear_kmeans_assign(fake, _dims(), fake, 0, fake, fake, big, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_kmeans_assign(fake, _dims(N=5000), fake, 4097, fake, fake, big,
+                                  None) == _lib.ERR_UNSUPPORTED
     # misaligned token pointer
-    assert L.svgear_kmeans_assign(ctypes.c_void_p((1 << 20) + 4), _dims(), fake, 10, fake,
-                                  None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_kmeans_assign(ctypes.c_void_p((1 << 20) + 4), _dims(), fake, 10, fake, fake,
+                                  big, None) == _lib.ERR_INVALID_ARG
+    # workspace too small
+    assert L.svgear_kmeans_assign(fake, _dims(), fake, 10, fake, fake, ws_small,
+                                  None) == _lib.ERR_WORKSPACE
     # iters < 1
     assert L.svgear_cluster(fake, _dims(), 10, 0, None, 0, fake, fake, fake, fake, None, fake,
                             ctypes.c_size_t(1 << 30), None) == _lib.ERR_INVALID_ARG
@@ -100,5 +105,6 @@ def test_validation_before_launch(L):
 def test_empty_batch_is_a_no_op(L):
     fake = ctypes.c_void_p(1 << 20)
     # B = 0: valid, nothing to launch, no CUDA call
-    assert L.svgear_kmeans_assign(fake, _dims(B=0), fake, 10, fake, None) == 0
+    assert L.svgear_kmeans_assign(fake, _dims(B=0), fake, 10, fake, fake, ctypes.c_size_t(1 << 20),
+                                  None) == 0
     assert L.svgear_centroids(fake, fake, 10, _dims(B=0), fake, None) == 0
