@@ -27,7 +27,11 @@
 // Every wait is bounded (1 s of %globaltimer); on expiry the CTA records
 // SVGEAR_ERR_TIMEOUT in the device status word, drains and returns, and
 // every later wait of the launch gives up at once.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "launchers.h"
@@ -41,13 +45,26 @@ using bf16 = __nv_bfloat16;
 constexpr int BM = 128;            // query rows per CTA
 constexpr int BN = 128;            // keys per tile
 constexpr int STAGES = 2;          // K/V ring
-constexpr int kProducerThreads = 128;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kMmaWarp = 8;
-constexpr int kThreads = kProducerThreads + kSoftmaxThreads + 32;
+constexpr int kSoftmaxThreads = 128;   // warps 0-3: one row each, TMEM lanes 0-127
+constexpr int kProducerWarp0 = 4;      // warps 4-5: K/V gathers, 64 rows each
+constexpr int kProducerWarps = 2;
+constexpr int kMmaWarp = 6;            // issues S = Q K^T (and owns the TMEM allocation)
+// warp 7 issues O += P V
+constexpr int kThreads = 8 * 32;       // 2 warps per SM sub-partition: 255 registers
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s; a tile takes microseconds
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+// Tensor maps of one launch: K and V rows as 2-D boxes of 2^h rows (h = 0..7,
+// for the contiguous runs of a gathered tile), the bf16 centroid tables read a
+// row at a time (tile::gather4), and the query rows as 128-row boxes.
+struct TmaMaps {
+    CUtensorMap k[8];
+    CUtensorMap v[8];
+    CUtensorMap kb;
+    CUtensorMap vb;
+    CUtensorMap q;
+};
 
 // Swizzled 16-byte chunk address inside a tile of 128 rows x (regions of
 // 64 bf16): region r covers elements [64r, 64r+64) of every row.
@@ -58,8 +75,10 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
 
 struct Shared {
     uint64_t q_full;
-    uint64_t kv_full[STAGES];
-    uint64_t kv_empty[STAGES];
+    uint64_t k_full[STAGES];
+    uint64_t k_empty[STAGES];
+    uint64_t v_full[STAGES];
+    uint64_t v_empty[STAGES];
     uint64_t s_full[2];
     uint64_t s_free[2];
     uint64_t p_full[2];
@@ -68,7 +87,19 @@ struct Shared {
     uint32_t tmem_base;
     int abort_flag;
     int keep_tmem;
+    int32_t row[kProducerWarps][BN];        // source row of each gathered row (-1: none)
 };
+
+#ifdef SVGEAR_TRACE
+// Diagnostic build only: per-tile event clocks of one CTA.
+__device__ long long g_trace[8][512];
+#define TRACE(ev, j)                                                                  \
+    do {                                                                              \
+        if (blockIdx.x == 3 && blockIdx.y == 0 && (j) < 512) g_trace[ev][j] = clock64(); \
+    } while (0)
+#else
+#define TRACE(ev, j) do { } while (0)
+#endif
 
 // Bounded wait: gives up when this CTA or any other CTA of the launch has
 // already given up (the device status word is non-zero), or after kTimeoutNs.
@@ -80,10 +111,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     if (tc::mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = tc::global_timer_ns();
     volatile int* gerr = err;
-    while (true) {
-        // sleep in the instruction (woken by the phase completing), so a
-        // waiting warp takes no issue slots from the working ones
-        if (tc::mbar_try_wait_sleep(b, parity, 20000u)) return true;
+    for (uint32_t it = 1;; ++it) {
+        if (tc::mbar_try_wait(b, parity)) return true;
+        if ((it & 63) != 0) continue;   // check the abort flags and the clock now and then
         if (*abort_flag || *gerr) {
             *abort_flag = 1;
             return false;
@@ -113,10 +143,8 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
-                    const bf16* __restrict__ Vp, int Nq, int Nk, int Cq, int Ck,
-                    const int32_t* __restrict__ q_perm, const bf16* __restrict__ kbar16,
-                    const bf16* __restrict__ vbar16, const int4* __restrict__ tiles,
+attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq, int Ck, int BH,
+                    const int32_t* __restrict__ q_perm, const int4* __restrict__ tiles,
                     const int32_t* __restrict__ ntiles, int maxT, const int4* __restrict__ meta,
                     const int32_t* __restrict__ seg_prefix, const int32_t* __restrict__ seg_row,
                     const int32_t* __restrict__ comp_idx, const float* __restrict__ comp_bias,
@@ -145,10 +173,12 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        tc::mbar_init(tc::smem_u32(&sh.q_full), kProducerThreads);
+        tc::mbar_init(tc::smem_u32(&sh.q_full), 1);
         for (int s = 0; s < STAGES; ++s) {
-            tc::mbar_init(tc::smem_u32(&sh.kv_full[s]), kProducerThreads);
-            tc::mbar_init(tc::smem_u32(&sh.kv_empty[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.k_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.k_empty[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.v_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.v_empty[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.s_full[s]), 1);
@@ -172,74 +202,96 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
     volatile int* abort_flag = &sh.abort_flag;
 
     const size_t head = (size_t)bh * Nq * D;
-    const size_t khead = (size_t)bh * Nk * D;
     const size_t row_meta = ((size_t)bh * Cq + ci) * Ck;
 
-    if (warp < 4) {
+    if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
         // ------------------------------------------------------------ producer
-        // One row per thread.  Copies are published by the cp.async engine
-        // itself (mbarrier arrive on completion), so a producer only ever
-        // waits for a free stage.
-        const int r = tid;
-        {
-            const int qrow = q0 + r;
-            const bool ok = qrow < q_end;
-            const bf16* src = Qp + head + (size_t)(ok ? qrow : q0) * D;
+        // Warp 4 fills the K ring (freed by QK), warp 5 the V ring (freed by
+        // PV); lane 0 issues TMA.  A key tile is the next 128 entries of the
+        // query cluster's list of selected keys, which is a concatenation of
+        // contiguous key-cluster segments: every run [g, g+n) of rows that falls
+        // in the tile is copied with 2-D boxes of 2^h rows (the binary digits of
+        // n), landing 128B-swizzled at its place in the tile.  Tile rows past
+        // the list are boxes at an out-of-range row (zeros).  Compensation
+        // tiles gather the skipped clusters' bf16 centroids row by row.
+        const int pw = warp - kProducerWarp0;
+        const bool isK = pw == 0;
+        const CUtensorMap* mrows = isK ? maps.k : maps.v;
+        const CUtensorMap* mcent = isK ? &maps.kb : &maps.vb;
+        uint64_t* ring_full = isK ? sh.k_full : sh.v_full;
+        uint64_t* ring_empty = isK ? sh.k_empty : sh.v_empty;
+        const uint32_t ring0 = isK ? sK0 : sV0;
+        if (isK && lane == 0) {
+            tc::prefetch_tmap(&maps.q);
+            tc::mbar_arrive_expect_tx(tc::smem_u32(&sh.q_full), BM * D * 2);
 #pragma unroll
-            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(sQ, r, c), src + c * 8, ok ? 16u : 0u);
-            tc::cp_async_arrive_noinc(tc::smem_u32(&sh.q_full));
+            for (int h = 0; h < REG; ++h)
+                tc::tma_load_2d(sQ + h * 16384, &maps.q, h * 64, bh * Nq + q0, tc::smem_u32(&sh.q_full));
         }
         const int32_t* pre = seg_prefix + ((size_t)bh * Cq + ci) * (Ck + 1);
         const int32_t* srow = seg_row + row_meta;
         const int32_t* cidx = comp_idx + row_meta;
-        const bf16* Kh = Kp + khead;
-        const bf16* Vh = Vp + khead;
-        const bf16* kbh = kbar16 + (size_t)bh * Ck * D;
-        const bf16* vbh = vbar16 + (size_t)bh * Ck * D;
+        const int krow0 = bh * Nk, kend = BH * Nk;
+        const int crow0 = bh * Ck, cend = BH * Ck;
         int seg = 0;
         for (int j = 0; j < T; ++j) {
             const int st = j % STAGES;
             if (j >= STAGES &&
-                !warp_wait_bar(&sh.kv_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
+                !warp_wait_bar(&ring_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
-            const bf16* sk = Kh;
-            const bf16* sv = Vh;
-            uint32_t bytes = 0;
-            if (j < T_real) {
-                const int p = j * BN + r;
-                if (p < L) {
-                    while (pre[seg + 1] <= p) ++seg;
-                    const int g = srow[seg] + (p - pre[seg]);
-                    sk = Kh + (size_t)g * D;
-                    sv = Vh + (size_t)g * D;
-                    bytes = 16;
+            if (pw == 0 && lane == 0) TRACE(0, j);
+            const uint32_t bar = tc::smem_u32(&ring_full[st]);
+            const uint32_t tX = ring0 + st * kTileBytes;
+            if (j >= T_real) {
+                // compensation tile: lane i gathers tile rows 4i..4i+3
+                int y[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int p = (j - T_real) * BN + 4 * lane + k;
+                    y[k] = (p < ncomp) ? crow0 + cidx[p] : cend;
                 }
-            } else {
-                const int p = (j - T_real) * BN + r;
-                if (p < ncomp) {
-                    const int c = cidx[p];
-                    sk = kbh + (size_t)c * D;
-                    sv = vbh + (size_t)c * D;
-                    bytes = 16;
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar, BN * D * 2);
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < REG; ++h)
+                    tc::tma_gather4(tX + h * 16384 + lane * 512, mcent, h * 64, y[0], y[1], y[2], y[3],
+                                    bar);
+            } else if (lane == 0) {
+                tc::mbar_arrive_expect_tx(bar, BN * D * 2);
+                const int t0 = j * BN, t1 = t0 + BN;
+                int r = 0;   // next tile row to fill
+                while (r < BN) {
+                    const int p = t0 + r;
+                    int g, n;
+                    if (p < L) {
+                        while (pre[seg + 1] <= p) ++seg;
+                        n = min(pre[seg + 1], t1) - p;
+                        g = krow0 + srow[seg] + (p - pre[seg]);
+                    } else {
+                        n = BN - r;
+                        g = kend;   // out of range: zero fill
+                    }
+#pragma unroll 1
+                    for (int hb = 7; hb >= 0; --hb) {
+                        if (!(n >> hb & 1)) continue;
+#pragma unroll
+                        for (int h = 0; h < REG; ++h)
+                            tc::tma_load_2d(tX + h * 16384 + r * 128, &mrows[hb], h * 64, g, bar);
+                        r += 1 << hb;
+                        if (g != kend) g += 1 << hb;
+                    }
                 }
             }
-            const uint32_t tK = sK0 + st * kTileBytes, tV = sV0 + st * kTileBytes;
-#pragma unroll
-            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tK, r, c), sk + c * 8, bytes);
-#pragma unroll
-            for (int c = 0; c < CPR; ++c) tc::cp_async16(swz(tV, r, c), sv + c * 8, bytes);
-            tc::cp_async_arrive_noinc(tc::smem_u32(&sh.kv_full[st]));
+            __syncwarp();
         }
-        tc::cp_async_wait<0>();
-        __syncwarp();
-    } else if (warp < 8) {
+    } else if (warp < 4) {
         // ------------------------------------------------------------ softmax
-        const int r = tid - kProducerThreads;            // row == TMEM lane
+        const int r = tid;                               // row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float* cb = comp_bias + row_meta;
         float m_use = -INFINITY, l = 0.f;
         bool ok_run = true;
-        uint32_t v[32];
+        uint32_t v[BN];
         for (int j = 0; j < T && ok_run; ++j) {
             const int sb = j & 1;
             if (!warp_wait_bar(&sh.s_full[sb], (j >> 1) & 1, abort_flag, err, (2 << 16) + j)) {
@@ -247,29 +299,52 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                 break;
             }
             tc::fence_after_sync();
-            const uint32_t sS = lane_base + sb * BN;
+            if (tid == 0) TRACE(3, j);
+            {
+                const uint32_t sS = lane_base + sb * BN;
+                tc::tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tc::tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tc::tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+                tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+                tc::tmem_ld_wait();
+            }
+            // S(j) is in registers: the MMA may refill this buffer
+            tc::fence_before_sync();
+            tc::mbar_arrive(tc::smem_u32(&sh.s_free[sb]));
+
             const bool comp = j >= T_real;
             const int valid = comp ? min(BN, ncomp - (j - T_real) * BN) : min(BN, L - j * BN);
             const float* bias = cb + (comp ? (j - T_real) * BN : 0);
-            // pass 1: row max of x = s * scale * log2(e) (+ log2 n_c on compensation columns)
-            float mx = -INFINITY;
+            // x = s * scale * log2(e) (+ log2 n_c on compensation columns); masked -> -inf
+            if (comp) {
+                // in 32-column steps (the compiler barrier keeps the bias loads of
+                // one step from being hoisted next to the 128 live scores)
 #pragma unroll
-            for (int c4 = 0; c4 < BN / 32; ++c4) {
-                tc::tmem_ld32(sS + c4 * 32, v);
-                tc::tmem_ld_wait();
-                if (comp) {
+                for (int c4 = 0; c4 < BN / 32; ++c4) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int col = c4 * 32 + e;
-                        if (col < valid) mx = fmaxf(mx, fmaf(__uint_as_float(v[e]), scale_log2, bias[col]));
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (c4 * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+                    for (int e = c4 * 32; e < c4 * 32 + 32; ++e)
+                        v[e] = __float_as_uint((e < valid) ? fmaf(__uint_as_float(v[e]), scale_log2, bias[e])
+                                                           : -INFINITY);
+                    asm volatile("" ::: "memory");
                 }
+            } else if (valid < BN) {
+#pragma unroll
+                for (int e = 0; e < BN; ++e)
+                    v[e] = __float_as_uint((e < valid) ? __uint_as_float(v[e]) * scale_log2 : -INFINITY);
             }
-            if (!comp) mx *= scale_log2;   // scale > 0: max commutes with scaling
+            // full key tiles keep raw scores: the max scales afterwards (scale > 0)
+            // and the exp pass folds the scale into its FFMA
+            const bool raw = !comp && valid == BN;
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < BN; e += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+                mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(v[e + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(v[e + 3]));
+            }
+            float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            if (raw) mx *= scale_log2;
             const float m_new = fmaxf(m_use, mx);
 
             // Lazy rescale of O: each row decides, but the TMEM loads/stores are
@@ -286,13 +361,14 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                 tc::fence_after_sync();
                 const float alpha = need ? tc::ex2(m_use - m_new) : 1.f;
                 const uint32_t sO = lane_base + 2 * BN;
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4) {
-                    tc::tmem_ld32(sO + c4 * 32, v);
+                uint32_t o[16];
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                    tc::tmem_ld16(sO + c * 16, o);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tc::tmem_st32(sO + c4 * 32, v);
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tc::tmem_st16(sO + c * 16, o);
                 }
                 tc::tmem_st_wait();
                 if (need) {
@@ -300,51 +376,37 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                     m_use = m_new;
                 }
             }
+            if (tid == 0) TRACE(4, j);
             // P buffer sb is free once PV(j-2) has completed
             if (j >= 2 &&
                 !warp_wait_bar(&sh.pv_done[sb], ((j >> 1) - 1) & 1, abort_flag, err, (10 << 16) + j)) {
                 ok_run = false;
                 break;
             }
-            // pass 2: p = 2^(x - m), row sum, bf16 P into the swizzled buffer
+            if (tid == 0) TRACE(5, j);
             const uint32_t sP = sP0 + sb * kPBytes;
-            const float neg_m = -m_use;
-            float sum = 0.f;
+            const float xs = raw ? scale_log2 : 1.f, neg_m = -m_use;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int c4 = 0; c4 < BN / 32; ++c4) {
-                tc::tmem_ld32(sS + c4 * 32, v);
-                tc::tmem_ld_wait();
+            for (int q = 0; q < BN / 8; ++q) {
+                uint32_t pk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const int k0 = q * 8 + e, col = c4 * 32 + k0;
-                        float x0, x1;
-                        if (comp) {
-                            x0 = fmaf(__uint_as_float(v[k0]), scale_log2, bias[col] + neg_m);
-                            x1 = fmaf(__uint_as_float(v[k0 + 1]), scale_log2, bias[col + 1] + neg_m);
-                        } else {
-                            x0 = fmaf(__uint_as_float(v[k0]), scale_log2, neg_m);
-                            x1 = fmaf(__uint_as_float(v[k0 + 1]), scale_log2, neg_m);
-                        }
-                        const float p0 = (col < valid) ? tc::ex2(x0) : 0.f;
-                        const float p1 = (col + 1 < valid) ? tc::ex2(x1) : 0.f;
-                        sum += p0 + p1;
-                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(sP, r, c4 * 4 + q)),
-                                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                                 : "memory");
+                for (int e = 0; e < 8; e += 2) {
+                    const float p0 = tc::ex2(fmaf(__uint_as_float(v[q * 8 + e]), xs, neg_m));
+                    const float p1 = tc::ex2(fmaf(__uint_as_float(v[q * 8 + e + 1]), xs, neg_m));
+                    s0 += p0;
+                    s1 += p1;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
                 }
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(sP, r, q)),
+                             "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                             : "memory");
             }
-            l += sum;
-            // S(j) consumed and P(j) written
-            tc::fence_before_sync();
-            tc::mbar_arrive(tc::smem_u32(&sh.s_free[sb]));
+            l += s0 + s1;
             tc::fence_async_smem();
             tc::mbar_arrive(tc::smem_u32(&sh.p_full[sb]));
+            if (tid == 0) TRACE(6, j);
         }
         // epilogue: O / l back to the original token order
         if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
@@ -355,16 +417,17 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
             const bool write = p < q_end;
             const int dst = write ? q_perm[(size_t)bh * Nq + p] : 0;
             bf16* orow = O + head + (size_t)dst * D;
+            uint32_t o[32];
 #pragma unroll
             for (int c4 = 0; c4 < D / 32; ++c4) {
-                tc::tmem_ld32(sO + c4 * 32, v);
+                tc::tmem_ld32(sO + c4 * 32, o);
                 tc::tmem_ld_wait();
                 if (write && (unsigned)dst < (unsigned)Nq) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[e]) * inv,
-                                                                 __uint_as_float(v[e + 1]) * inv);
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[e]) * inv,
+                                                                 __uint_as_float(o[e + 1]) * inv);
                         pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
                     }
                     uint4* o4 = reinterpret_cast<uint4*>(orow + c4 * 32);
@@ -374,67 +437,77 @@ attend_sm100_kernel(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp,
                 }
             }
         }
-    } else {
-        // ------------------------------------------------------------ MMA issue
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ S = Q K^T
         // The whole warp runs the loop; lane 0 issues the MMAs and commits.
         constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
-        constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
         bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
         if (ok_run) tc::fence_async_smem();
-        for (int j = 0; ok_run && j <= T; ++j) {
-            if (j < T) {
-                const int st = j % STAGES, sb = j & 1;
-                if (!warp_wait_bar(&sh.kv_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
-                    ok_run = false;
-                    break;
-                }
-                if (j >= 2 &&
-                    !warp_wait_bar(&sh.s_free[sb], ((j >> 1) - 1) & 1, abort_flag, err, (7 << 16) + j)) {
-                    ok_run = false;
-                    break;
-                }
-                tc::fence_async_smem();   // cp.async data -> tensor-core reads
-                tc::fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t tK = sK0 + st * kTileBytes;
-#pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::mma_bf16(tmem + sb * BN, tc::sw128_desc(sQ + off, 16, 1024),
-                                     tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
-                    }
-                    tc::commit(tc::smem_u32(&sh.s_full[sb]));
-                }
-                __syncwarp();
+        for (int j = 0; ok_run && j < T; ++j) {
+            const int st = j % STAGES, sb = j & 1;
+            if (!warp_wait_bar(&sh.k_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
+                ok_run = false;
+                break;
             }
-            if (j >= 1) {
-                const int jj = j - 1, st = jj % STAGES, pb = jj & 1;
-                if (!warp_wait_bar(&sh.p_full[pb], (jj >> 1) & 1, abort_flag, err, (8 << 16) + jj)) {
-                    ok_run = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t tV = sV0 + st * kTileBytes;
-                    const uint32_t sP = sP0 + pb * kPBytes;
-#pragma unroll
-                    for (int ks = 0; ks < BN / 16; ++ks) {
-                        const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::mma_bf16(tmem + 2 * BN, tc::sw128_desc(sP + offp, 16, 1024),
-                                     tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
-                                     (jj > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    tc::commit(tc::smem_u32(&sh.kv_empty[st]));
-                    tc::commit(tc::smem_u32(&sh.pv_done[pb]));
-                }
-                __syncwarp();
+            if (lane == 0) TRACE(1, j);
+            if (j >= 2 &&
+                !warp_wait_bar(&sh.s_free[sb], ((j >> 1) - 1) & 1, abort_flag, err, (7 << 16) + j)) {
+                ok_run = false;
+                break;
             }
+            tc::fence_async_smem();   // cp.async data -> tensor-core reads
+            tc::fence_after_sync();
+            if (lane == 0) TRACE(2, j);
+            if (lane == 0) {
+                const uint32_t tK = sK0 + st * kTileBytes;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    tc::mma_bf16(tmem + sb * BN, tc::sw128_desc(sQ + off, 16, 1024),
+                                 tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
+                }
+                tc::commit(tc::smem_u32(&sh.k_empty[st]));
+                tc::commit(tc::smem_u32(&sh.s_full[sb]));
+            }
+            __syncwarp();
+        }
+        // S(j) is consumed by the softmax before its P(j) exists, so the PV
+        // warp's last commit covers every MMA of this warp too; nothing to drain.
+    } else {
+        // ------------------------------------------------------------ O += P V
+        constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
+        bool ok_run = true;
+        for (int jj = 0; ok_run && jj < T; ++jj) {
+            const int st = jj % STAGES, pb = jj & 1;
+            if (!warp_wait_bar(&sh.v_full[st], (jj / STAGES) & 1, abort_flag, err, (11 << 16) + jj) ||
+                !warp_wait_bar(&sh.p_full[pb], (jj >> 1) & 1, abort_flag, err, (8 << 16) + jj)) {
+                ok_run = false;
+                break;
+            }
+            tc::fence_async_smem();   // cp.async data -> tensor-core reads
+            tc::fence_after_sync();
+            if (lane == 0) TRACE(7, jj);
+            if (lane == 0) {
+                const uint32_t tV = sV0 + st * kTileBytes;
+                const uint32_t sP = sP0 + pb * kPBytes;
+#pragma unroll
+                for (int ks = 0; ks < BN / 16; ++ks) {
+                    const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    tc::mma_bf16(tmem + 2 * BN, tc::sw128_desc(sP + offp, 16, 1024),
+                                 tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
+                                 (jj > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc::commit(tc::smem_u32(&sh.v_empty[st]));
+                tc::commit(tc::smem_u32(&sh.pv_done[pb]));
+            }
+            __syncwarp();
         }
         if (lane == 0) tc::commit(tc::smem_u32(&sh.o_full));
         __syncwarp();
-        // drain: every MMA this CTA issued is complete once o_full flips; if
-        // that wait expires, TMEM is left allocated rather than released under
-        // a running MMA (every later CTA of the launch returns before alloc)
+        // drain: every MMA of this CTA is complete once o_full flips (the QK
+        // warp's MMAs all precede the last P); if that wait expires, TMEM is
+        // left allocated rather than released under a running MMA (every later
+        // CTA of the launch returns before alloc)
         if (!warp_wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16)) && lane == 0)
             sh.keep_tmem = 1;
         __syncwarp();
@@ -515,7 +588,44 @@ __global__ void attend_tiles_kernel(const int32_t* __restrict__ q_off, int Cq, i
 
 }  // namespace sm100
 
+#ifdef SVGEAR_TRACE
+extern "C" int svgear_debug_trace(long long* host) {
+    return cudaMemcpyFromSymbol(host, sm100::g_trace, sizeof(sm100::g_trace)) == cudaSuccess ? 0 : -3;
+}
+#endif
+
 // Workspace pieces of the tensor-core path (carved by the caller).
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A [rows][D] bf16 matrix seen as 2-D boxes of 64 columns x box_rows rows,
+// 128-byte swizzled on arrival; out-of-range rows read as zeros.
+static bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int D,
+                          uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd, int Nk,
                         const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                         const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
@@ -524,6 +634,16 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     using namespace sm100;
     const int BH = qd.B * qd.H;
     const int D = qd.d;
+    if ((long long)BH * Nk >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;   // int32 TMA rows
+    if ((long long)BH * qd.N >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;
+    TmaMaps maps;
+    bool ok = make_rows_map(&maps.kb, w.kbar16, (uint64_t)BH * Ck, D, 1) &&
+              make_rows_map(&maps.vb, w.vbar16, (uint64_t)BH * Ck, D, 1) &&
+              make_rows_map(&maps.q, Qp, (uint64_t)BH * qd.N, D, BM);
+    for (int h = 0; h < 8 && ok; ++h)
+        ok = make_rows_map(&maps.k[h], Kp, (uint64_t)BH * Nk, D, 1u << h) &&
+             make_rows_map(&maps.v[h], Vp, (uint64_t)BH * Nk, D, 1u << h);
+    if (!ok) return SVGEAR_ERR_CUDA;
     if (cudaMemsetAsync(w.status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     const size_t nc = (size_t)BH * Ck * D;
     const int cgrid = (int)((nc + 255) / 256 < 4096 ? (nc + 255) / 256 : 4096);
@@ -544,8 +664,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
         attend_sm100_kernel<128><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
-            static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp),
-            qd.N, Nk, Cq, Ck, q_perm, w.kbar16, w.vbar16, w.tiles, w.ntiles, w.maxT, w.meta,
+            maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
             w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
             w.status);
     } else {
@@ -553,8 +672,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
         attend_sm100_kernel<64><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
-            static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp),
-            qd.N, Nk, Cq, Ck, q_perm, w.kbar16, w.vbar16, w.tiles, w.ntiles, w.maxT, w.meta,
+            maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
             w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
             w.status);
     }
