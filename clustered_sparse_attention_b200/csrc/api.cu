@@ -55,12 +55,18 @@ struct KppWs {
     float* D2;
     double* blocksum;
     int32_t* chosen;
+    int32_t* counter;
+    int32_t* nearest;
+    float* cc2;
 };
 KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
     KppWs w;
     w.D2 = cv.take<float>(bh_of(d) * d.N);
     w.blocksum = cv.take<double>(bh_of(d) * ceil_div(d.N, kKppTokens));
     w.chosen = cv.take<int32_t>(bh_of(d) * C);
+    w.counter = cv.take<int32_t>(bh_of(d));
+    w.nearest = cv.take<int32_t>(bh_of(d) * d.N);
+    w.cc2 = cv.take<float>(bh_of(d) * C);
     return w;
 }
 int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {
@@ -214,7 +220,8 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
     Carve cv(ws);
     KppWs w = carve_kpp(cv, dims, C);
     return launch_kmeanspp(X, dims, C, seed, centroids, seed_index ? seed_index : w.chosen, w.D2,
-                           w.blocksum, static_cast<cudaStream_t>(stream));
+                           w.nearest, w.cc2, w.blocksum, w.counter,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids, int32_t C,
@@ -294,7 +301,8 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
         Carve cv(ws);
         carve_flags(cv, dims);
         KppWs w = carve_kpp(cv, dims, C);
-        if ((s = launch_kmeanspp(X, dims, C, seed, centroids, w.chosen, w.D2, w.blocksum, st)))
+        if ((s = launch_kmeanspp(X, dims, C, seed, centroids, w.chosen, w.D2, w.nearest, w.cc2,
+                                 w.blocksum, w.counter, st)))
             return s;
     }
     Carve cv(ws);

@@ -65,77 +65,33 @@ __global__ void kpp_first_kernel(const T* __restrict__ X, int N, int D, int C,
         centroids[(size_t)bh * C * D + k] = Elem<T>::from(row[k]);
 }
 
+// Pick of seed j for head bh from the D^2 of this pass (run by the last block
+// of the pass to finish): the block where the running sum of the block sums
+// crosses u_j * sum, then the token inside it, with the same fp64 scan the
+// blocks used, so the two levels agree bit for bit.  Also leaves in cc2 the
+// squared distances from seed j to seeds 0..j-1 for the next pass's pruning.
 template <typename T, int D>
-__global__ void __launch_bounds__(kKppThreads)
-kpp_update_kernel(const T* __restrict__ X, int N, int nblk, const int32_t* chosen,
-                  int C, int j, float* D2, double* blocksum) {
-    constexpr int EPC = Elem<T>::kPerChunk;
-    constexpr int L = D / EPC;                 // lanes per token row
-    constexpr int RP = kKppThreads / L;        // rows per pass
-    __shared__ float cen[D];
-    __shared__ float d2s[kKppTokens];
-    __shared__ double warp_tot[kKppThreads / 32];
-    const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
-    const T* Xh = X + (size_t)bh * N * D;
-    const int st = chosen[(size_t)bh * C + j - 1];
-    for (int k = tid; k < D; k += kKppThreads) cen[k] = Elem<T>::from(Xh[(size_t)st * D + k]);
-    __syncthreads();
-    const int lane = tid % L;
-    for (int r = tid / L; r < kKppTokens; r += RP) {
-        const int t = blk * kKppTokens + r;
-        float part = 0.f;
-        if (t < N) {
-            float x[EPC];
-            Elem<T>::load(Xh + (size_t)t * D + lane * EPC, x);
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-                float df = x[e] - cen[lane * EPC + e];
-                part = fmaf(df, df, part);
-            }
-        }
-#pragma unroll
-        for (int o = L / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (lane == 0) {
-            float v = 0.f;
-            if (t < N) {
-                v = part;
-                if (j > 1) v = fminf(v, D2[(size_t)bh * N + t]);
-                D2[(size_t)bh * N + t] = v;
-            }
-            d2s[r] = v;
-        }
-    }
-    __syncthreads();
-    double incl[4];
-    kpp_block_scan(d2s, warp_tot, incl);
-    if (tid == kKppThreads - 1) blocksum[(size_t)bh * nblk + blk] = incl[3];
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kKppThreads)
-kpp_pick_kernel(const T* __restrict__ X, int N, int D, int nblk, int32_t* chosen, int C,
-                int j, const float* D2, const double* blocksum, uint64_t seed,
-                float* centroids) {
-    __shared__ float d2s[kKppTokens];
-    __shared__ double warp_tot[kKppThreads / 32];
+__device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C, int j,
+                         const float* D2, const double* blocksum, uint64_t seed, float* centroids,
+                         float* cc2, float* d2s, double* warp_tot, float* cnew) {
     __shared__ int s_blk, s_pick;
     __shared__ double s_base, s_target;
-    const int bh = blockIdx.x, tid = threadIdx.x;
+    const int bh = blockIdx.y, tid = threadIdx.x;
     const double* bs = blocksum + (size_t)bh * nblk;
     const float* d2 = D2 + (size_t)bh * N;
     int32_t* ch = chosen + (size_t)bh * C;
     if (tid == 0) {
         double total = 0.0;
-        for (int b = 0; b < nblk; ++b) total += bs[b];
+        for (int b = 0; b < nblk; ++b) total += __ldcg(bs + b);
         s_pick = 0x7fffffff;
         if (total > 0.0) {
-            double target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
+            const double target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
             s_target = target;
             s_blk = -2;
             double run = 0.0;
             for (int b = 0; b < nblk; ++b) {
-                double prev = run;
-                run = prev + bs[b];
+                const double prev = run;
+                run = prev + __ldcg(bs + b);
                 if (run > target) { s_blk = b; s_base = prev; break; }
             }
         } else {
@@ -146,8 +102,8 @@ kpp_pick_kernel(const T* __restrict__ X, int N, int D, int nblk, int32_t* chosen
     const int blk = s_blk;
     if (blk >= 0) {
         for (int r = tid; r < kKppTokens; r += kKppThreads) {
-            int t = blk * kKppTokens + r;
-            d2s[r] = (t < N) ? d2[t] : 0.f;
+            const int t = blk * kKppTokens + r;
+            d2s[r] = (t < N) ? __ldcg(d2 + t) : 0.f;
         }
         __syncthreads();
         double incl[4];
@@ -163,7 +119,7 @@ kpp_pick_kernel(const T* __restrict__ X, int N, int D, int nblk, int32_t* chosen
         int pick = 0;
         if (blk == -2) {            // rounding left no token above the target
             for (int t = N - 1; t >= 0; --t)
-                if (d2[t] > 0.f) { pick = t; break; }
+                if (__ldcg(d2 + t) > 0.f) { pick = t; break; }
         } else {                    // every D^2 is zero: lowest unchosen token
             for (int t = 0; t < N; ++t) {
                 bool used = false;
@@ -177,25 +133,170 @@ kpp_pick_kernel(const T* __restrict__ X, int N, int D, int nblk, int32_t* chosen
     const int pick = s_pick < N ? s_pick : N - 1;
     if (tid == 0) ch[j] = pick;
     const T* row = X + ((size_t)bh * N + pick) * D;
-    for (int k = tid; k < D; k += kKppThreads)
-        centroids[((size_t)bh * C + j) * D + k] = Elem<T>::from(row[k]);
+    for (int k = tid; k < D; k += kKppThreads) {
+        const float v = Elem<T>::from(row[k]);
+        cnew[k] = v;
+        centroids[((size_t)bh * C + j) * D + k] = v;
+    }
+    __syncthreads();
+    // |c_j - c_a|^2 for a < j, one earlier seed per thread (rows of seeds a < j
+    // were written by earlier launches)
+    const float* cen = centroids + (size_t)bh * C * D;
+    for (int a = tid; a < j; a += kKppThreads) {
+        const float4* ra = reinterpret_cast<const float4*>(cen + (size_t)a * D);
+        float acc = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D / 4; ++k) {
+            const float4 v = __ldcg(ra + k);
+            const float d0 = v.x - cnew[4 * k], d1 = v.y - cnew[4 * k + 1];
+            const float d2v = v.z - cnew[4 * k + 2], d3 = v.w - cnew[4 * k + 3];
+            acc = fmaf(d0, d0, acc);
+            acc = fmaf(d1, d1, acc);
+            acc = fmaf(d2v, d2v, acc);
+            acc = fmaf(d3, d3, acc);
+        }
+        cc2[(size_t)bh * C + a] = acc;
+    }
+}
+
+// A token whose nearest seed a lies at squared distance cc2[a] >= kKppPrune *
+// D^2 from the new seed s keeps its D^2: by the triangle inequality
+// |x - c_s| >= |c_s - c_a| - |x - c_a| >= |x - c_a| once |c_s - c_a| >=
+// 2 |x - c_a|.  The factor 4 (1 + 2^-7) leaves a margin far above the fp32
+// rounding of either squared distance (a few units in 2^-24 per term summed),
+// so a pruned token's recomputed fp32 distance would never have been below
+// its D^2 and the pass stays bit-identical to the unpruned one.  A NaN fails
+// the comparison and is recomputed.
+constexpr float kKppPrune = 4.03125f;
+
+// One pass of the seeding: D^2 <- min(D^2, |x - seed_{j-1}|^2) for a block of
+// kKppTokens tokens, the block's fp64 scan total, and -- in the last block of
+// the head to finish -- the pick of seed j.  Tokens are first screened with
+// the triangle bound (8 bytes read per token: D^2 and nearest-seed index);
+// only the survivors' rows are loaded, by groups of lanes, four rows in flight.
+template <typename T, int D>
+__global__ void __launch_bounds__(kKppThreads)
+kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C, int j, float* D2,
+                int32_t* nearest, float* cc2, double* blocksum, int32_t* counter, uint64_t seed,
+                float* centroids) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int L = D / EPC;                 // lanes per token row
+    constexpr int RP = kKppThreads / L;        // rows per sweep of the block
+    constexpr int U = 4;                       // rows in flight per lane group
+    __shared__ float cen[D];
+    __shared__ float d2s[kKppTokens];
+    __shared__ int32_t todo[kKppTokens];
+    __shared__ float ccs[SVGEAR_MAX_CLUSTERS];
+    __shared__ double warp_tot[kKppThreads / 32];
+    __shared__ int s_ntodo, s_last;
+    const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x, wl = tid & 31;
+    const int s = j - 1;                       // the seed this pass adds
+    const T* Xh = X + (size_t)bh * N * D;
+    float* D2h = D2 + (size_t)bh * N;
+    int32_t* nh = nearest + (size_t)bh * N;
+    const int st = chosen[(size_t)bh * C + s];
+    for (int k = tid; k < D; k += kKppThreads) cen[k] = Elem<T>::from(Xh[(size_t)st * D + k]);
+    for (int a = tid; a < s; a += kKppThreads) ccs[a] = cc2[(size_t)bh * C + a];
+    if (tid == 0) s_ntodo = 0;
+    __syncthreads();
+    // screen
+#pragma unroll
+    for (int i = 0; i < kKppTokens / kKppThreads; ++i) {
+        const int r = i * kKppThreads + tid, t = blk * kKppTokens + r;
+        float d = 0.f;
+        bool need = false;
+        if (t < N) {
+            if (s == 0) {
+                need = true;
+            } else {
+                d = D2h[t];
+                const int a = nh[t];
+                need = (unsigned)a >= (unsigned)s || !(ccs[a] >= kKppPrune * d);
+            }
+        }
+        d2s[r] = d;
+        const unsigned m = __ballot_sync(0xffffffffu, need);
+        int base = 0;
+        if (wl == 0 && m) base = atomicAdd(&s_ntodo, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (need) todo[base + __popc(m & ((1u << wl) - 1u))] = r;
+    }
+    __syncthreads();
+    // recompute the survivors
+    const int n = s_ntodo;
+    const int lane = tid % L, grp = tid / L;
+    for (int b0 = 0; b0 < n; b0 += RP * U) {
+        int rr[U];
+        float x[U][EPC];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = b0 + grp + u * RP;
+            rr[u] = i < n ? todo[i] : -1;
+            if (rr[u] >= 0) {
+                Elem<T>::load(Xh + (size_t)(blk * kKppTokens + rr[u]) * D + lane * EPC, x[u]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) x[u][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float part = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                const float df = x[u][e] - cen[lane * EPC + e];
+                part = fmaf(df, df, part);
+            }
+#pragma unroll
+            for (int o = L / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (lane == 0 && rr[u] >= 0) {
+                const int r = rr[u], t = blk * kKppTokens + r;
+                const float old = d2s[r];
+                const float v = s == 0 ? part : fminf(part, old);
+                if (s == 0 || __float_as_int(v) != __float_as_int(old)) {
+                    d2s[r] = v;
+                    D2h[t] = v;
+                    nh[t] = s;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    double incl[4];
+    kpp_block_scan(d2s, warp_tot, incl);
+    if (tid == kKppThreads - 1) blocksum[(size_t)bh * nblk + blk] = incl[3];
+    // the last block of this head to finish picks seed j
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(counter + bh, 1) == nblk - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (j < C)
+        kpp_pick<T, D>(X, N, nblk, chosen, C, j, D2, blocksum, seed, centroids, cc2, d2s, warp_tot,
+                       cen);
+    if (tid == 0) counter[bh] = 0;   // ready for the next pass
+}
+
+__global__ void zero_i32_kernel(int32_t* p, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) p[i] = 0;
 }
 
 template <typename T, int D>
-static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed,
-                         float* cent, int32_t* chosen, float* D2, double* blocksum,
-                         cudaStream_t st) {
+static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+                         int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
+                         double* blocksum, int32_t* counter, cudaStream_t st) {
     const int BH = dims.B * dims.H, N = dims.N;
     const int nblk = ceil_div(N, kKppTokens);
+    zero_i32_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, BH);
+    count_launches(1);
     kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     for (int j = 1; j < C; ++j) {
-        kpp_update_kernel<T, D><<<dim3(nblk, BH), kKppThreads, 0, st>>>(
-            X, N, nblk, chosen, C, j, D2, blocksum);
-        count_launches(1);
-        kpp_pick_kernel<T><<<BH, kKppThreads, 0, st>>>(X, N, D, nblk, chosen, C, j, D2,
-                                                        blocksum, seed, cent);
+        kpp_pass_kernel<T, D><<<dim3(nblk, BH), kKppThreads, 0, st>>>(
+            X, N, nblk, chosen, C, j, D2, nearest, cc2, blocksum, counter, seed, cent);
         count_launches(1);
     }
     SVGEAR_LAUNCH_CHECK();
@@ -417,8 +518,26 @@ segment_mean_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
     float acc[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    for (int p = a + grp; p < b; p += R) {
-        int row = GATHER ? perm[(size_t)bh * N + p] : p;
+    // Four rows in flight per lane group (index loads first, then the rows);
+    // each lane still adds its rows in increasing p, one at a time.
+    constexpr int U = 4;
+    int p = a + grp;
+    for (; p + (U - 1) * R < b; p += U * R) {
+        int row[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) row[u] = GATHER ? perm[(size_t)bh * N + p + u * R] : p + u * R;
+        float v[U][EPC];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if ((unsigned)row[u] < (unsigned)N) Elem<T>::load(Xh + (size_t)row[u] * D + lane * EPC, v[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if ((unsigned)row[u] < (unsigned)N)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] += v[u][e];
+    }
+    for (; p < b; p += R) {
+        const int row = GATHER ? perm[(size_t)bh * N + p] : p;
         if ((unsigned)row >= (unsigned)N) continue;
         float v[EPC];
         Elem<T>::load(Xh + (size_t)row * D + lane * EPC, v);
@@ -473,12 +592,16 @@ __global__ void permute_kernel(const T* __restrict__ X, const int32_t* __restric
 
 template <typename T, int D>
 static int kmeanspp_disp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
-                         int32_t* chosen, float* D2, double* bs, cudaStream_t st) {
-    return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, cent, chosen, D2, bs, st);
+                         int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
+                         int32_t* counter, cudaStream_t st) {
+    return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, cent, chosen, D2, nearest,
+                               cc2, bs, counter, st);
 }
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
-                    int32_t* chosen, float* D2, double* bs, cudaStream_t st) {
-    SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, cent, chosen, D2, bs, st);
+                    int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
+                    int32_t* counter, cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, cent, chosen, D2, nearest, cc2, bs,
+                    counter, st);
 }
 
 template <typename T, int D>

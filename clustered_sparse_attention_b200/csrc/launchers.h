@@ -18,8 +18,8 @@ inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // kmeans.cu
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
-                    float* centroids, int32_t* chosen, float* D2, double* blocksum,
-                    cudaStream_t st);
+                    float* centroids, int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
+                    double* blocksum, int32_t* counter, cudaStream_t st);
 // done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
 // scratch: assign_scratch_floats(B*H, C, d) floats (k-major centroid copy + norms).
 int launch_assign(const void* X, svgear_dims dims, const float* centroids, int C,

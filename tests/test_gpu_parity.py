@@ -33,6 +33,11 @@ RAGGED_BF16_64 = synth.custom_workload("ragged_bf16_d64", H=3, frames=1, grid_h=
                                        d=64, dtype="bf16", Cq=7, Ck=33, iters=3, density=0.25,
                                        n_centres=12, sigma=0.4, index=51)
 TINY = synth.WORKLOADS["tiny"]
+# many seeds over few tokens: most tokens of the late k-means++ passes are
+# screened out by the triangle bound, so the picks exercise the pruned path
+MANY_SEEDS = synth.custom_workload("many_seeds", H=2, frames=2, grid_h=48, grid_w=64, d=128,
+                                   dtype="bf16", Cq=16, Ck=600, iters=2, density=0.3,
+                                   n_centres=48, sigma=0.5, index=52)
 
 
 def _inputs(w, heads=None):
@@ -45,7 +50,8 @@ def _rel_l2(a, b):
 
 
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64, MANY_SEEDS],
+                         ids=lambda w: w.name)
 def test_kmeanspp_stagewise(w):
     csa = _csa()
     host, dev = _inputs(w)
