@@ -29,6 +29,7 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_centroids", "svgear_probe", "svgear_route_select", "svgear_route",
             "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
             "svgear_version", "svgear_kernel_launches", "svgear_attend_status",
+            "svgear_device_status",
             "svgear_label_sort_noalloc")
 
 
@@ -74,6 +75,7 @@ def lib():
         "svgear_version": [],
         "svgear_kernel_launches": [],
         "svgear_attend_status": [P, SZ, P, P],
+        "svgear_device_status": [P, SZ, P, P],
         "svgear_label_sort_noalloc": [P, Dims, I32, P, P, P],
     }
     for name, args in sig.items():
@@ -146,7 +148,21 @@ class Clustering:
     Xp: torch.Tensor | None   # [B, H, N, d] permuted copy
 
 
-def svgear_cluster(X, C, iters, warm_centroids=None, seed=0, permuted=True, out=None):
+def _device_status(fn, ws, n):
+    """Synchronise and raise if a bounded wait inside a tensor-core kernel of
+    the call that used `ws` gave up."""
+    st = (ctypes.c_int32 * 4)()
+    _check("svgear_device_status", lib().svgear_device_status(_ptr(ws), n, st, _stream()))
+    if st[0] != OK:
+        raise SvgearError("%s (device: wait site %d, index %d, cta %d)"
+                          % (fn, st[1] >> 16, st[1] & 0xFFFF, st[2]), st[0],
+                          lib().svgear_status_string(st[0]).decode())
+
+
+def svgear_cluster(X, C, iters, warm_centroids=None, seed=0, permuted=True, out=None,
+                   check_status=False):
+    """check_status=True synchronises and raises if a bounded wait inside the
+    assignment kernel gave up."""
     dims = _tokens(X, "X")
     B, H, N, d = X.shape
     dev = X.device
@@ -163,6 +179,8 @@ def svgear_cluster(X, C, iters, warm_centroids=None, seed=0, permuted=True, out=
     _check("svgear_cluster", lib().svgear_cluster(
         _ptr(X), dims, C, iters, _ptr(warm_centroids), seed, _ptr(out.labels), _ptr(out.perm),
         _ptr(out.offsets), _ptr(out.centroids), _ptr(out.Xp), _ptr(ws), n, _stream()))
+    if check_status:
+        _device_status("svgear_cluster", ws, n)
     return out
 
 
@@ -177,7 +195,7 @@ def svgear_kmeanspp_init(X, C, seed=0):
     return cent, idx
 
 
-def svgear_kmeans_assign(X, centroids):
+def svgear_kmeans_assign(X, centroids, check_status=False):
     dims = _tokens(X, "X")
     _cuda(centroids, "centroids", torch.float32)
     B, H, N, d = X.shape
@@ -186,6 +204,8 @@ def svgear_kmeans_assign(X, centroids):
     ws, n = _workspace(OP_KMEANS_ASSIGN, dims, C, 0, X.device)
     _check("svgear_kmeans_assign", lib().svgear_kmeans_assign(
         _ptr(X), dims, _ptr(centroids), C, _ptr(labels), _ptr(ws), n, _stream()))
+    if check_status:
+        _device_status("svgear_kmeans_assign", ws, n)
     return labels
 
 
@@ -292,12 +312,7 @@ def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_per
         _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(q_perm), float(scale), _ptr(O), _ptr(ws), n,
         _stream()))
     if check_status:
-        st = (ctypes.c_int32 * 4)()
-        _check("svgear_attend_status", lib().svgear_attend_status(_ptr(ws), n, st, _stream()))
-        if st[0] != OK:
-            raise SvgearError("svgear_attend (device: wait site %d, tile %d, cta %d)"
-                              % (st[1] >> 16, st[1] & 0xFFFF, st[2]), st[0],
-                              lib().svgear_status_string(st[0]).decode())
+        _device_status("svgear_attend", ws, n)
     return O
 
 

@@ -72,8 +72,8 @@ KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
 int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {
     return cv.take<int32_t>(bh_of(d) * ceil_div(d.N, kSortTokens) * (size_t)C);
 }
-float* carve_assign(Carve& cv, const svgear_dims& d, int C) {
-    return cv.take<float>(assign_scratch_floats((int)bh_of(d), C, d.d));
+void* carve_assign(Carve& cv, const svgear_dims& d, int C) {
+    return cv.take<char>(assign_scratch_bytes((int)bh_of(d), C, d.d, d.dtype));
 }
 struct UpdWs {
     int32_t* perm;
@@ -127,14 +127,17 @@ AttendWs carve_attend(Carve& cv, const svgear_dims& d, int Cq, int Ck) {
     return w;
 }
 
-// svgear_cluster's workspace: per-head fixed-point flags, then the k-means++
-// scratch and the sort histograms (used one after the other, so they overlap).
+// svgear_cluster's workspace: the device status words, per-head fixed-point
+// flags, then the k-means++ scratch and the sort histograms and assignment
+// scratch (used one after the other, so they overlap).
 struct ClusterFlags {
+    int* status;
     int32_t* done;
     int32_t* changed;
 };
 ClusterFlags carve_flags(Carve& cv, const svgear_dims& d) {
     ClusterFlags f;
+    f.status = cv.take<int>(4);
     f.done = cv.take<int32_t>(bh_of(d));
     f.changed = cv.take<int32_t>(bh_of(d));
     return f;
@@ -192,6 +195,7 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             break;
         case SVGEAR_OP_KMEANS_ASSIGN:
             if (check_C(C1, dims.N)) return 0;
+            cv.take<int>(4);
             carve_assign(cv, dims, C1);
             break;
         case SVGEAR_OP_ROUTE:
@@ -234,9 +238,11 @@ int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN, dims, C, 0))
         return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
-    return launch_assign(X, dims, centroids, C, labels, carve_assign(cv, dims, C),
-                         static_cast<cudaStream_t>(stream));
+    int* status = cv.take<int>(4);
+    if (cudaMemsetAsync(status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
+    return launch_assign(X, dims, centroids, C, labels, carve_assign(cv, dims, C), status, st);
 }
 
 int svgear_label_sort(const int32_t* labels, svgear_dims dims, int32_t C, int32_t* perm,
@@ -290,8 +296,8 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
     const int BH = (int)bh_of(dims);
     Carve cf(ws);
     ClusterFlags fl = carve_flags(cf, dims);
-    const size_t flag_bytes = (size_t)((char*)fl.changed - (char*)fl.done) + sizeof(int32_t) * BH;
-    if (cudaMemsetAsync(fl.done, 0, flag_bytes, st) != cudaSuccess) return SVGEAR_ERR_CUDA;
+    const size_t flag_bytes = (size_t)((char*)fl.changed - (char*)fl.status) + sizeof(int32_t) * BH;
+    if (cudaMemsetAsync(fl.status, 0, flag_bytes, st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     if (warm_centroids) {
         if (warm_centroids != centroids &&
             cudaMemcpyAsync(centroids, warm_centroids, sizeof(float) * BH * (size_t)C * dims.d,
@@ -308,14 +314,14 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
     Carve cv(ws);
     carve_flags(cv, dims);
     int32_t* hist = carve_sort(cv, dims, C);
-    float* ascratch = carve_assign(cv, dims, C);
+    void* ascratch = carve_assign(cv, dims, C);
     // Lloyd rounds.  From the second round on, a head whose assignment moved
     // no label has reached the fixed point (the sort and the deterministic
     // update would reproduce the current perm, offsets and centroids), so its
     // remaining kernels return at once; the results are those of all rounds.
     for (int it = 0; it < iters; ++it) {
         const bool track = it > 0;
-        if ((s = launch_assign(X, dims, centroids, C, labels, ascratch, st, fl.done,
+        if ((s = launch_assign(X, dims, centroids, C, labels, ascratch, fl.status, st, fl.done,
                                track ? fl.changed : nullptr)))
             return s;
         if (track && (s = launch_fixed_point(fl.changed, fl.done, BH, st))) return s;
@@ -443,13 +449,17 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
                               vbar, q_perm, scale, O, st);
 }
 
-int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+int svgear_device_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
     if (!ws || !status || ws_bytes < 4 * sizeof(int)) return SVGEAR_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemcpyAsync(status, ws, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
     return SVGEAR_OK;
+}
+
+int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+    return svgear_device_status(ws, ws_bytes, status, stream);
 }
 
 }  // extern "C"

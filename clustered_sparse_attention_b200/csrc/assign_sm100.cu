@@ -1,0 +1,434 @@
+// assign_sm100.cu -- k-means assignment of bf16 tokens on tcgen05 / TMEM.
+//
+// Method: SVG2 summary ("Sparse VideoGen2 ...", section 3.4, "The clustering
+// operation"): every token joins the centroid nearest in Euclidean distance.
+// argmin_c |x - c|^2 = argmin_c (|c|^2 - 2 x.c), and x.c over all tokens and
+// centroids of a head is a dense contraction, which runs here on the tensor
+// cores; ties keep the lowest centroid index.
+//
+// Precision: x is bf16, exact as an MMA operand.  Each fp32 centroid is split
+// into three bf16 planes, c = h + m + l with h = bf16(c), m = bf16(c - h),
+// l = bf16(c - h - m) (both differences are exact in fp32; what l leaves out
+// is below 2^-26 |c|).  One fp32-accumulated MMA chain of depth 3d sums
+// x.h + x.m + x.l, whose products are exact, so the dot product keeps fp32
+// accuracy; |c|^2 is taken from the fp32 centroid.
+//
+// B200 design: persistent CTAs, one per SM, walk the 128-token tiles of all
+// heads (tiles of heads at their fixed point are skipped).
+//   warp 0     TMA producer: the token tile (2 stages), then a ring of
+//              centroid-plane boxes of Nc rows x 64 dims (128B-swizzled);
+//   warp 1     one lane issues tcgen05.mma (M=128, N=Nc <= 256, K=16) into one
+//              of two TMEM accumulators, each centroid chunk a chain of
+//              3 planes x d/16 steps;
+//   warps 2-5  epilogue, one token per thread (TMEM lane = token row):
+//              dist = |c|^2 - 2 s, running (dist, index) minimum, label out.
+// Every wait is bounded (tc_wait.cuh); on expiry the status word records
+// SVGEAR_ERR_TIMEOUT, copies and MMAs in flight are drained and the CTA
+// returns.
+#include <math.h>
+
+#include "common.cuh"
+#include "launchers.h"
+#include "tc_ptx.cuh"
+#include "tc_wait.cuh"
+#include "tma_host.h"
+
+namespace svgear {
+namespace asg {
+
+using bf16 = __nv_bfloat16;
+using tc::warp_wait_bar;
+
+constexpr int BM = 128;                  // tokens per tile (TMEM lanes)
+constexpr int kPlanes = 3;               // bf16 planes of a centroid
+constexpr int kBStages = 4;              // centroid-plane ring
+constexpr int kThreads = 6 * 32;
+constexpr int kMmaWarp = 1;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;      // two accumulators of up to 256 columns
+constexpr uint32_t kAccCols = 256;
+constexpr uint32_t kBStageBytes = 256 * 128;   // up to 256 rows x 64 bf16
+constexpr uint64_t kDrainNs = 200000000ull;    // 0.2 s to let issued work land
+
+struct Maps {
+    CUtensorMap x;   // tokens [B*H*N][D], boxes of 128 rows x 64
+    CUtensorMap b;   // centroid planes [B*H][3][Cpad][D], boxes of Nc rows x 64
+};
+
+struct Shared {
+    uint64_t a_full[2];
+    uint64_t a_empty[2];
+    uint64_t b_full[kBStages];
+    uint64_t b_empty[kBStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int keep_tmem;
+};
+
+// Wait for a phase without regard to abort flags (used to let copies and MMAs
+// that were issued complete before the CTA exits); false after kDrainNs.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t b = tc::smem_u32(bar);
+    const uint64_t t0 = tc::global_timer_ns();
+    while (!tc::mbar_try_wait(b, parity))
+        if (tc::global_timer_ns() - t0 > kDrainNs) return false;
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc,
+                    const float* __restrict__ cnorm, int32_t* __restrict__ labels,
+                    const int32_t* __restrict__ done, int32_t* __restrict__ changed,
+                    int* __restrict__ err) {
+    constexpr int KH = D / 64;                   // 64-dim halves of a row
+    constexpr uint32_t kABytes = KH * 16384;     // 128 rows x D bf16
+    if (*(volatile int*)err != 0) return;        // an earlier CTA already gave up
+    const int tiles_per_head = (N + BM - 1) / BM;
+    const int total = BH * tiles_per_head;
+    const int nchunk = Cpad / Nc;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ Shared sh;
+    const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t sA0 = base;
+    const uint32_t sB0 = base + 2 * kABytes;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(tc::smem_u32(&sh.a_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.a_empty[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.acc_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.acc_empty[s]), kEpiThreads);
+        }
+        for (int s = 0; s < kBStages; ++s) {
+            tc::mbar_init(tc::smem_u32(&sh.b_full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.b_empty[s]), 1);
+        }
+        tc::mbar_init(tc::smem_u32(&sh.drain), 1);
+        sh.abort_flag = 0;
+        sh.keep_tmem = 0;
+        tc::mbar_init_fence();
+    }
+    if (warp == kMmaWarp) {
+        tc::tmem_alloc(tc::smem_u32(&sh.tmem_base), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int* abort_flag = &sh.abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&maps.x);
+            tc::prefetch_tmap(&maps.b);
+        }
+        int ia = 0, ib = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            const int bh = w / tiles_per_head;
+            if (done && done[bh]) continue;
+            const int t0 = (w - bh * tiles_per_head) * BM;
+            const int sa = ia & 1;
+            if (ia >= 2 &&
+                !warp_wait_bar(&sh.a_empty[sa], ((ia >> 1) - 1) & 1, abort_flag, err, (1 << 16) + ia)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                const uint32_t bar = tc::smem_u32(&sh.a_full[sa]);
+                tc::mbar_arrive_expect_tx(bar, BM * D * 2);
+#pragma unroll
+                for (int kh = 0; kh < KH; ++kh)
+                    tc::tma_load_2d(sA0 + sa * kABytes + kh * 16384, &maps.x, kh * 64, bh * N + t0, bar);
+            }
+            __syncwarp();
+            ++ia;
+            for (int c = 0; ok && c < nchunk; ++c) {
+                for (int p = 0; ok && p < kPlanes; ++p) {
+                    for (int kh = 0; kh < KH; ++kh) {
+                        const int sb = ib % kBStages;
+                        if (ib >= kBStages &&
+                            !warp_wait_bar(&sh.b_empty[sb], ((ib / kBStages) - 1) & 1, abort_flag, err,
+                                           (2 << 16) + (ib & 0xffff))) {
+                            ok = false;
+                            break;
+                        }
+                        if (lane == 0) {
+                            const uint32_t bar = tc::smem_u32(&sh.b_full[sb]);
+                            tc::mbar_arrive_expect_tx(bar, (uint32_t)Nc * 128u);
+                            tc::tma_load_2d(sB0 + sb * kBStageBytes, &maps.b, kh * 64,
+                                            (bh * kPlanes + p) * Cpad + c * Nc, bar);
+                        }
+                        __syncwarp();
+                        ++ib;
+                    }
+                }
+            }
+        }
+        // let the last copy into every stage land before the CTA can exit
+        if (lane == 0) {
+            for (int k = 0; k < 2 && k < ia; ++k) {
+                const int i = ia - 1 - k;
+                drain_wait(&sh.a_full[i & 1], (i >> 1) & 1);
+            }
+            for (int k = 0; k < kBStages && k < ib; ++k) {
+                const int i = ib - 1 - k;
+                drain_wait(&sh.b_full[i % kBStages], (i / kBStages) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issue
+        const uint32_t idesc = tc::idesc_bf16(BM, Nc, false);
+        int ia = 0, ib = 0, ic = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            const int bh = w / tiles_per_head;
+            if (done && done[bh]) continue;
+            const int sa = ia & 1;
+            if (!warp_wait_bar(&sh.a_full[sa], (ia >> 1) & 1, abort_flag, err, (3 << 16) + ia)) {
+                ok = false;
+                break;
+            }
+            for (int c = 0; ok && c < nchunk; ++c) {
+                const int buf = ic & 1;
+                if (ic >= 2 &&
+                    !warp_wait_bar(&sh.acc_empty[buf], ((ic >> 1) - 1) & 1, abort_flag, err,
+                                   (4 << 16) + (ic & 0xffff))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                for (int p = 0; ok && p < kPlanes; ++p) {
+                    for (int kh = 0; kh < KH; ++kh) {
+                        const int sb = ib % kBStages;
+                        if (!warp_wait_bar(&sh.b_full[sb], (ib / kBStages) & 1, abort_flag, err,
+                                           (5 << 16) + (ib & 0xffff))) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                        if (lane == 0) {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                const uint64_t ad = tc::sw128_desc(
+                                    sA0 + sa * kABytes + kh * 16384 + ks * 32, 16, 1024);
+                                const uint64_t bd =
+                                    tc::sw128_desc(sB0 + sb * kBStageBytes + ks * 32, 16, 1024);
+                                tc::mma_bf16(tmem + buf * kAccCols, ad, bd, idesc,
+                                             (p | kh | ks) != 0 ? 1u : 0u);
+                            }
+                            tc::commit(tc::smem_u32(&sh.b_empty[sb]));
+                        }
+                        __syncwarp();
+                        ++ib;
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) tc::commit(tc::smem_u32(&sh.acc_full[buf]));
+                __syncwarp();
+                ++ic;
+            }
+            if (!ok) break;
+            if (lane == 0) tc::commit(tc::smem_u32(&sh.a_empty[sa]));
+            __syncwarp();
+            ++ia;
+        }
+        // every MMA this warp issued has completed once `drain` flips; if it
+        // does not, TMEM stays allocated rather than freed under a running MMA
+        if (lane == 0) {
+            tc::commit(tc::smem_u32(&sh.drain));
+            if (!drain_wait(&sh.drain, 0)) sh.keep_tmem = 1;
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;                  // TMEM lanes this warp may read
+        const int r = quarter * 32 + lane;             // token row in the tile
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        int ic = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            const int bh = w / tiles_per_head;
+            if (done && done[bh]) continue;
+            const int t0 = (w - bh * tiles_per_head) * BM;
+            const float* cn = cnorm + (size_t)bh * Cpad;
+            float best = __int_as_float(0x7f800000);
+            int bi = 0;
+            for (int c = 0; c < nchunk; ++c) {
+                const int buf = ic & 1;
+                if (!warp_wait_bar(&sh.acc_full[buf], (ic >> 1) & 1, abort_flag, err,
+                                   (6 << 16) + (ic & 0xffff))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t tb = lane_base + buf * kAccCols;
+                const int cb = c * Nc;
+                int col = 0;
+                for (; col + 32 <= Nc; col += 32) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(tb + col, v);
+                    float4 n4[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        n4[q] = __ldg(reinterpret_cast<const float4*>(cn + cb + col) + q);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float nn[4] = {n4[q].x, n4[q].y, n4[q].z, n4[q].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
+                            if (dist < best) {
+                                best = dist;
+                                bi = cb + col + 4 * q + e;
+                            }
+                        }
+                    }
+                }
+                if (col < Nc) {   // Nc is a multiple of 16
+                    uint32_t v[16];
+                    tc::tmem_ld16(tb + col, v);
+                    float4 n4[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        n4[q] = __ldg(reinterpret_cast<const float4*>(cn + cb + col) + q);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float nn[4] = {n4[q].x, n4[q].y, n4[q].z, n4[q].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
+                            if (dist < best) {
+                                best = dist;
+                                bi = cb + col + 4 * q + e;
+                            }
+                        }
+                    }
+                }
+                // the accumulator is in registers: the MMA may refill it
+                tc::fence_before_sync();
+                tc::mbar_arrive(tc::smem_u32(&sh.acc_empty[buf]));
+                ++ic;
+            }
+            if (!ok) break;
+            const int t = t0 + r;
+            if (t < N) {
+                int32_t* lp = labels + (size_t)bh * N + t;
+                if (changed && *lp != bi) changed[bh] = 1;
+                *lp = bi;
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == kMmaWarp && !sh.keep_tmem) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// Centroid planes and norms, one warp per centroid: planes[bh][p][c][k] for
+// p = hi, mid, lo; padding rows (c >= C) are zero with norm +inf, so they
+// never win the minimum.
+template <int D>
+__global__ void centroid_planes_kernel(const float* __restrict__ cent, int C, int Cpad,
+                                       bf16* __restrict__ planes, float* __restrict__ cnorm,
+                                       const int32_t* __restrict__ done) {
+    const int bh = blockIdx.y;
+    if (done && done[bh]) return;
+    const int c = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (c >= Cpad) return;
+    float s = 0.f;
+#pragma unroll
+    for (int k = lane; k < D; k += 32) {
+        const float v = c < C ? cent[((size_t)bh * C + c) * D + k] : 0.f;
+        const bf16 h = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(h);
+        const bf16 m = __float2bfloat16_rn(r1);
+        const bf16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+        const size_t row = ((size_t)bh * kPlanes * Cpad + c) * D + k;
+        planes[row] = h;
+        planes[row + (size_t)Cpad * D] = m;
+        planes[row + (size_t)2 * Cpad * D] = l;
+        s = fmaf(v, v, s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) cnorm[(size_t)bh * Cpad + c] = c < C ? s : __int_as_float(0x7f800000);
+}
+
+// Centroid chunking: as few chunks as possible of at most 256 columns, each a
+// multiple of 16 wide.
+inline void chunking(int C, int* nchunk, int* Nc) {
+    *nchunk = (C + 255) / 256;
+    const int per = (C + *nchunk - 1) / *nchunk;
+    *Nc = (per + 15) / 16 * 16;
+}
+
+}  // namespace asg
+
+size_t assign_sm100_scratch_bytes(int BH, int C, int D) {
+    int nchunk, Nc;
+    asg::chunking(C, &nchunk, &Nc);
+    const size_t Cpad = (size_t)nchunk * Nc;
+    return (size_t)BH * Cpad * (asg::kPlanes * D * sizeof(__nv_bfloat16) + sizeof(float));
+}
+
+int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int C,
+                        int32_t* labels, void* scratch, int* err, cudaStream_t st,
+                        const int32_t* done, int32_t* changed) {
+    using namespace asg;
+    const int BH = dims.B * dims.H, N = dims.N, D = dims.d;
+    if ((long long)BH * N >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;   // int32 TMA rows
+    int nchunk, Nc;
+    chunking(C, &nchunk, &Nc);
+    const int Cpad = nchunk * Nc;
+    bf16* planes = static_cast<bf16*>(scratch);
+    float* cn = reinterpret_cast<float*>(planes + (size_t)BH * kPlanes * Cpad * D);
+    Maps maps;
+    if (!make_rows_map(&maps.x, X, (uint64_t)BH * N, D, BM) ||
+        !make_rows_map(&maps.b, planes, (uint64_t)BH * kPlanes * Cpad, D, (uint32_t)Nc))
+        return SVGEAR_ERR_CUDA;
+    static int num_sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SVGEAR_ERR_CUDA;
+    if (num_sms[dev] == 0 &&
+        cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SVGEAR_ERR_CUDA;
+    const int total = BH * ceil_div(N, BM);
+    const int grid = total < num_sms[dev] ? total : num_sms[dev];
+    const size_t smem = (size_t)2 * (D / 64) * 16384 + (size_t)kBStages * kBStageBytes + 1024;
+    if (D == 128) {
+        centroid_planes_kernel<128><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
+                                                                                cn, done);
+        count_launches(1);
+        if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, cn, labels,
+                                                               done, changed, err);
+    } else {
+        centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
+                                                                               cn, done);
+        count_launches(1);
+        if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, cn, labels,
+                                                              done, changed, err);
+    }
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+}  // namespace svgear

@@ -27,15 +27,13 @@
 // Every wait is bounded (1 s of %globaltimer); on expiry the CTA records
 // SVGEAR_ERR_TIMEOUT in the device status word, drains and returns, and
 // every later wait of the launch gives up at once.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <math.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "launchers.h"
 #include "tc_ptx.cuh"
+#include "tc_wait.cuh"
+#include "tma_host.h"
 
 namespace svgear {
 namespace sm100 {
@@ -52,7 +50,6 @@ constexpr int kMmaWarp = 6;            // issues S = Q K^T (and owns the TMEM al
 // warp 7 issues O += P V
 constexpr int kThreads = 8 * 32;       // 2 warps per SM sub-partition: 255 registers
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s; a tile takes microseconds
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 // Tensor maps of one launch: K and V rows as 2-D boxes of 2^h rows (h = 0..7,
@@ -101,45 +98,8 @@ __device__ long long g_trace[8][512];
 #define TRACE(ev, j) do { } while (0)
 #endif
 
-// Bounded wait: gives up when this CTA or any other CTA of the launch has
-// already given up (the device status word is non-zero), or after kTimeoutNs.
-// err[0] is the status word; err[1] records where the first expired wait was
-// (site * 65536 + tile index), err[2] the CTA (blockIdx.y * 65536 + blockIdx.x).
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int* err, int where) {
-    const uint32_t b = tc::smem_u32(bar);
-    if (tc::mbar_try_wait(b, parity)) return true;
-    const uint64_t t0 = tc::global_timer_ns();
-    volatile int* gerr = err;
-    for (uint32_t it = 1;; ++it) {
-        if (tc::mbar_try_wait(b, parity)) return true;
-        if ((it & 63) != 0) continue;   // check the abort flags and the clock now and then
-        if (*abort_flag || *gerr) {
-            *abort_flag = 1;
-            return false;
-        }
-        if (tc::global_timer_ns() - t0 > kTimeoutNs) {
-            *abort_flag = 1;
-            if (atomicCAS(err, 0, SVGEAR_ERR_TIMEOUT) == 0) {
-                err[1] = where;
-                err[2] = (int)(blockIdx.y * 65536 + blockIdx.x);
-            }
-            return false;
-        }
-    }
-}
-
-// One lane polls, the whole warp gets the same answer: the softmax and MMA
-// warps stay converged (they run .sync.aligned TMEM instructions and reach
-// the CTA barrier together).
-__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag, int* err, int where) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, err, where) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok != 0;
-}
+using tc::wait_bar;
+using tc::warp_wait_bar;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -152,7 +112,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     constexpr int REG = D / 64;                 // 64-element regions per row
     constexpr uint32_t kTileBytes = REG * 16384;
     constexpr uint32_t kPBytes = 2 * 16384;     // 128 rows x 128 keys bf16
-    constexpr int CPR = D / 8;                  // 16-byte chunks per row
     const int bh = blockIdx.y;
     if ((int)blockIdx.x >= ntiles[bh]) return;
     if (*(volatile int*)err != 0) return;   // an earlier CTA already gave up
@@ -593,38 +552,6 @@ extern "C" int svgear_debug_trace(long long* host) {
     return cudaMemcpyFromSymbol(host, sm100::g_trace, sizeof(sm100::g_trace)) == cudaSuccess ? 0 : -3;
 }
 #endif
-
-// Workspace pieces of the tensor-core path (carved by the caller).
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against libcuda).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// A [rows][D] bf16 matrix seen as 2-D boxes of 64 columns x box_rows rows,
-// 128-byte swizzled on arrival; out-of-range rows read as zeros.
-static bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int D,
-                          uint32_t box_rows) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd, int Nk,
                         const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,

@@ -483,9 +483,10 @@ static int assign_impl(const T* X, svgear_dims dims, const float* cent, int C,
     return SVGEAR_OK;
 }
 
-size_t assign_scratch_floats(int BH, int C, int D) {
+size_t assign_scratch_bytes(int BH, int C, int D, int dtype) {
+    if (dtype == SVGEAR_BF16) return assign_sm100_scratch_bytes(BH, C, D);
     const size_t Cpad = (size_t)ceil_div(C, kAsTN) * kAsTN;
-    return (size_t)BH * Cpad * (D + 1);
+    return (size_t)BH * Cpad * (D + 1) * sizeof(float);
 }
 
 // ---------------------------------------------------------------------------
@@ -606,17 +607,20 @@ int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float
 
 template <typename T, int D>
 static int assign_disp(const void* X, svgear_dims dims, const float* cent, int C,
-                       int32_t* labels, const int32_t* done, int32_t* changed, float* scratch,
-                       cudaStream_t st) {
+                       int32_t* labels, const int32_t* done, int32_t* changed, void* scratch,
+                       int* err, cudaStream_t st) {
+    if (dims.dtype == SVGEAR_BF16)
+        return launch_assign_sm100(X, dims, cent, C, labels, scratch, err, st, done, changed);
     const size_t Cpad = (size_t)ceil_div(C, kAsTN) * kAsTN;
-    float* cT = scratch;
-    float* cn = scratch + (size_t)dims.B * dims.H * Cpad * D;
+    float* cT = static_cast<float*>(scratch);
+    float* cn = cT + (size_t)dims.B * dims.H * Cpad * D;
     return assign_impl<T, D>(static_cast<const T*>(X), dims, cent, C, labels, done, changed, cT,
                              cn, st);
 }
 int launch_assign(const void* X, svgear_dims dims, const float* cent, int C, int32_t* labels,
-                  float* scratch, cudaStream_t st, const int32_t* done, int32_t* changed) {
-    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, done, changed, scratch, st);
+                  void* scratch, int* err, cudaStream_t st, const int32_t* done,
+                  int32_t* changed) {
+    SVGEAR_DISPATCH(dims, assign_disp, X, dims, cent, C, labels, done, changed, scratch, err, st);
 }
 
 // A head whose assignment changed no label has reached the fixed point of

@@ -21,11 +21,18 @@ int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
                     float* centroids, int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
                     double* blocksum, int32_t* counter, cudaStream_t st);
 // done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
-// scratch: assign_scratch_floats(B*H, C, d) floats (k-major centroid copy + norms).
+// scratch: assign_scratch_bytes(B*H, C, d, dtype) bytes (centroids re-laid
+// for the kernel, and their norms).  bf16 tokens run on the tcgen05 kernel
+// (assign_sm100.cu), whose bounded waits report through err (4 ints; f32
+// tokens run on the SIMT kernel and never touch it).
 int launch_assign(const void* X, svgear_dims dims, const float* centroids, int C,
-                  int32_t* labels, float* scratch, cudaStream_t st,
+                  int32_t* labels, void* scratch, int* err, cudaStream_t st,
                   const int32_t* done = nullptr, int32_t* changed = nullptr);
-size_t assign_scratch_floats(int BH, int C, int D);
+size_t assign_scratch_bytes(int BH, int C, int D, int dtype);
+int launch_assign_sm100(const void* X, svgear_dims dims, const float* centroids, int C,
+                        int32_t* labels, void* scratch, int* err, cudaStream_t st,
+                        const int32_t* done, int32_t* changed);
+size_t assign_sm100_scratch_bytes(int BH, int C, int D);
 int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st);
 // Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
 // empty_zero: an empty segment writes zeros (else leaves the row untouched).

@@ -117,7 +117,9 @@ typedef enum {
  *   centroids       out float[B][H][C][d]; an empty cluster keeps its
  *                   previous centroid.  May alias warm_centroids.
  *   Xp              out [B][H][N][d] (dtype) permuted copy X[perm], or NULL.
- *   ws, ws_bytes    workspace of svgear_workspace_bytes(SVGEAR_OP_CLUSTER).
+ *   ws, ws_bytes    workspace of svgear_workspace_bytes(SVGEAR_OP_CLUSTER); it
+ *                   starts with the device status words of the bf16
+ *                   assignment kernel (svgear_device_status).
  * ------------------------------------------------------------------------ */
 int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
                    const float* warm_centroids, uint64_t seed, int32_t* labels,
@@ -142,9 +144,13 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
                          size_t ws_bytes, void* stream);
 
 /* k-means assignment: labels[t] = argmin_c |x_t - c|^2, lowest c on exact
- * ties, evaluated in fp32 as |c|^2 - 2 x.c.
- *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN) (a k-major copy of
- *       the centroids and their norms). */
+ * ties, evaluated as |c|^2 - 2 x.c with fp32-grade dot products: f32 tokens
+ * by fp32 FMAs; bf16 tokens on the tensor cores, the fp32 centroid split into
+ * three bf16 planes (hi, mid, lo) whose products with the bf16 token are
+ * exact and accumulate in fp32 (what the planes leave out is below 2^-26 |c|).
+ *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN): the device status
+ *       words (svgear_device_status), then the centroids re-laid for the
+ *       kernel and their norms. */
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids,
                          int32_t C, int32_t* labels, void* ws, size_t ws_bytes,
                          void* stream);
@@ -261,13 +267,18 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
                   const float* kbar, const float* vbar, const int32_t* q_perm,
                   float scale, void* O, void* ws, size_t ws_bytes, void* stream);
 
-/* Device status of the last svgear_attend that used `ws`: copies 4 int32 to
- * status[0..3] (host memory) and synchronises `stream`.  status[0] is 0 when
- * every wait in the kernel completed, SVGEAR_ERR_TIMEOUT when a bounded wait
- * gave up (the kernel drained and returned; O is not valid); status[1] and
- * status[2] then say which wait (site * 65536 + tile) and which CTA
- * (blockIdx.y * 65536 + blockIdx.x).  The words sit at the start of the
- * workspace and every svgear_attend call clears them. */
+/* Device status of the last svgear_cluster, svgear_kmeans_assign or
+ * svgear_attend that used `ws`: copies 4 int32 to status[0..3] (host memory)
+ * and synchronises `stream`.  status[0] is 0 when every wait in the
+ * tensor-core kernels completed, SVGEAR_ERR_TIMEOUT when a bounded wait gave
+ * up (the kernel drained what it had issued and returned; its outputs are not
+ * valid); status[1] and status[2] then say which wait (site * 65536 + index)
+ * and which CTA (blockIdx.y * 65536 + blockIdx.x).  The words sit at the start
+ * of the workspace and each of those calls clears them first.  The library's
+ * own extension, with no counterpart in the method. */
+int svgear_device_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* The same as svgear_device_status (kept for svgear_attend callers). */
 int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /* --------------------------------------------------------------------------

@@ -99,6 +99,36 @@ def test_assign_exact_ties_take_lowest_index():
     assert np.array_equal(lab, np.arange(300) % 3)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("C", [16, 100, 256, 257, 500, 1000])
+def test_tensor_core_assign_over_centroid_chunks(d, C):
+    # bf16 tokens take the tcgen05 kernel: one to four centroid chunks of up
+    # to 256 columns, widths rounded to 16, a ragged last token tile
+    csa = _csa()
+    w = synth.custom_workload("assign_tc_d%d" % d, H=2, frames=2, grid_h=30, grid_w=50, d=d,
+                              dtype="bf16", Cq=C, Ck=C, iters=1, density=0.3, n_centres=40,
+                              sigma=0.5, index=53)
+    host, dev = _inputs(w)
+    g = np.random.default_rng(C + d)
+    cent = np.stack([host["k"][0, h][g.choice(w.N, C, replace=False)] for h in range(w.H)])[None]
+    cent = cent + 0.01 * g.standard_normal(cent.shape).astype(np.float32)
+    lab = csa.svgear_kmeans_assign(dev["k"], torch.from_numpy(cent).cuda(),
+                                   check_status=True).cpu().numpy()
+    flips = sum(check_assign(host["k"][0, h], cent[0, h], lab[0, h]) for h in range(w.H))
+    assert flips <= max(2, w.N * w.H // 5000)
+
+
+def test_tensor_core_assign_exact_ties_take_lowest_index():
+    csa = _csa()
+    X = torch.zeros((1, 1, 300, 128), dtype=torch.bfloat16, device="cuda")
+    X[0, 0, :, 0] = (torch.arange(300, device="cuda") % 3).to(torch.bfloat16)
+    cent = torch.zeros((1, 1, 300, 128), device="cuda")
+    cent[0, 0, :, 0] = (torch.arange(300, device="cuda") % 3).float()   # two chunks of duplicates
+    cent[0, 0, :, 5] = 1.0 / 3.0                                        # not on the bf16 grid
+    lab = csa.svgear_kmeans_assign(X, cent, check_status=True).cpu().numpy()[0, 0]
+    assert np.array_equal(lab, np.arange(300) % 3)
+
+
 @pytest.mark.parametrize("N,C", [(5000, 300), (1024, 1), (777, 777), (5000, 4096), (3000, 129)])
 def test_label_sort_bit_exact(N, C):
     csa = _csa()
