@@ -288,6 +288,19 @@ def workload_config(w, args):
             "parallelism": "one independent layer call per GPU (no exchange)"}
 
 
+# DRAM bytes (read + write) of one attend_sm100_kernel launch, from the ncu
+# capture of the 8-head Wan 720p case (profiles/attend_sm100_wan720p_h8.md);
+# traffic grows with the heads of a launch (same per-head routing), so other
+# head counts of that shape scale it.  None for shapes not captured.
+ATTEND_TRAFFIC_H8_WAN720P = 526.024960e6 + 142.095104e6
+
+
+def attend_traffic(w):
+    if w.name.startswith("wan720p") and w.N == 75600 and w.d == 128 and w.Ck == 500:
+        return ATTEND_TRAFFIC_H8_WAN720P * (w.B * w.H) / 8.0
+    return None
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -379,7 +392,7 @@ def main():
     roofline = {"kernel": "attend_sm100_kernel (svgear_attend, bf16)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": "bf16 dense, sustained, %s" % ("of measured" if peaks["source"] == "measured" else "of fallback"),
-                "traffic": None, "flops_per_launch": f_sel + f_comp}
+                "traffic": attend_traffic(w), "flops_per_launch": f_sel + f_comp}
 
     # end to end: pinned host inputs -> device -> layer -> O back to pinned host
     e2e = None
