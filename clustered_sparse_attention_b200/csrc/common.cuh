@@ -22,6 +22,14 @@ template <> struct Elem<float> {
         float4 v = __ldg(reinterpret_cast<const float4*>(p));
         out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
     }
+    // one 16-byte chunk kept packed (fewer live registers), unpacked at use
+    __device__ static inline uint4 load_raw(const float* p) {
+        return __ldg(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ static inline void unpack(const uint4& v, float* out) {
+        out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+        out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+    }
     __device__ static inline float from(float x) { return x; }
     __device__ static inline float to(float x) { return x; }
 };
@@ -29,6 +37,17 @@ template <> struct Elem<__nv_bfloat16> {
     static constexpr int kPerChunk = 8;
     __device__ static inline void load(const __nv_bfloat16* p, float* out) {
         uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            out[2 * i] = __uint_as_float(w[i] << 16);
+            out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+    __device__ static inline uint4 load_raw(const __nv_bfloat16* p) {
+        return __ldg(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ static inline void unpack(const uint4& v, float* out) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

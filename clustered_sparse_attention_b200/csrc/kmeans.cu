@@ -80,9 +80,15 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chos
     const double* bs = blocksum + (size_t)bh * nblk;
     const float* d2 = D2 + (size_t)bh * N;
     int32_t* ch = chosen + (size_t)bh * C;
+    // the block sums, fetched in parallel (the d2s buffer holds 512 doubles);
+    // heads with more blocks than that read the rest from L2 in the loop below
+    double* bsum = reinterpret_cast<double*>(d2s);
+    constexpr int kCached = kKppTokens / 2;
+    for (int b = tid; b < nblk && b < kCached; b += kKppThreads) bsum[b] = __ldcg(bs + b);
+    __syncthreads();
     if (tid == 0) {
         double total = 0.0;
-        for (int b = 0; b < nblk; ++b) total += __ldcg(bs + b);
+        for (int b = 0; b < nblk; ++b) total += b < kCached ? bsum[b] : __ldcg(bs + b);
         s_pick = 0x7fffffff;
         if (total > 0.0) {
             const double target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
@@ -91,7 +97,7 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chos
             double run = 0.0;
             for (int b = 0; b < nblk; ++b) {
                 const double prev = run;
-                run = prev + __ldcg(bs + b);
+                run = prev + (b < kCached ? bsum[b] : __ldcg(bs + b));
                 if (run > target) { s_blk = b; s_base = prev; break; }
             }
         } else {
@@ -175,7 +181,7 @@ constexpr float kKppPrune = 4.03125f;
 // the triangle bound (8 bytes read per token: D^2 and nearest-seed index);
 // only the survivors' rows are loaded, by groups of lanes, four rows in flight.
 template <typename T, int D>
-__global__ void __launch_bounds__(kKppThreads)
+__global__ void __launch_bounds__(kKppThreads, 6)
 kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C, int j, float* D2,
                 int32_t* nearest, float* cc2, double* blocksum, int32_t* counter, uint64_t seed,
                 float* centroids) {
@@ -184,9 +190,9 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
     constexpr int RP = kKppThreads / L;        // rows per sweep of the block
     constexpr int U = 4;                       // rows in flight per lane group
     __shared__ float cen[D];
-    __shared__ float d2s[kKppTokens];
+    __shared__ __align__(16) float d2s[kKppTokens];   // also the pick's fp64 block sums
     __shared__ int32_t todo[kKppTokens];
-    __shared__ float ccs[SVGEAR_MAX_CLUSTERS];
+    extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: s floats)
     __shared__ double warp_tot[kKppThreads / 32];
     __shared__ int s_ntodo, s_last;
     const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x, wl = tid & 31;
@@ -194,14 +200,28 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
     const T* Xh = X + (size_t)bh * N * D;
     float* D2h = D2 + (size_t)bh * N;
     int32_t* nh = nearest + (size_t)bh * N;
-    const int st = chosen[(size_t)bh * C + s];
-    for (int k = tid; k < D; k += kKppThreads) cen[k] = Elem<T>::from(Xh[(size_t)st * D + k]);
+    // issue the per-token state loads first: they do not depend on the seed
+    constexpr int TPT = kKppTokens / kKppThreads;   // tokens per thread
+    float dpre[TPT];
+    int apre[TPT];
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+        const int t = blk * kKppTokens + i * kKppThreads + tid;
+        dpre[i] = 0.f;
+        apre[i] = -1;
+        if (t < N && s > 0) {
+            dpre[i] = D2h[t];
+            apre[i] = nh[t];
+        }
+    }
+    // seed s as fp32 (its row of the centroid table, written by the pick)
+    for (int k = tid; k < D; k += kKppThreads) cen[k] = centroids[((size_t)bh * C + s) * D + k];
     for (int a = tid; a < s; a += kKppThreads) ccs[a] = cc2[(size_t)bh * C + a];
     if (tid == 0) s_ntodo = 0;
     __syncthreads();
     // screen
 #pragma unroll
-    for (int i = 0; i < kKppTokens / kKppThreads; ++i) {
+    for (int i = 0; i < TPT; ++i) {
         const int r = i * kKppThreads + tid, t = blk * kKppTokens + r;
         float d = 0.f;
         bool need = false;
@@ -209,8 +229,8 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
             if (s == 0) {
                 need = true;
             } else {
-                d = D2h[t];
-                const int a = nh[t];
+                d = dpre[i];
+                const int a = apre[i];
                 need = (unsigned)a >= (unsigned)s || !(ccs[a] >= kKppPrune * d);
             }
         }
@@ -227,24 +247,23 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
     const int lane = tid % L, grp = tid / L;
     for (int b0 = 0; b0 < n; b0 += RP * U) {
         int rr[U];
-        float x[U][EPC];
+        uint4 raw[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = b0 + grp + u * RP;
             rr[u] = i < n ? todo[i] : -1;
-            if (rr[u] >= 0) {
-                Elem<T>::load(Xh + (size_t)(blk * kKppTokens + rr[u]) * D + lane * EPC, x[u]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) x[u][e] = 0.f;
-            }
+            raw[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (rr[u] >= 0)
+                raw[u] = Elem<T>::load_raw(Xh + (size_t)(blk * kKppTokens + rr[u]) * D + lane * EPC);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
+            float x[EPC];
+            Elem<T>::unpack(raw[u], x);
             float part = 0.f;
 #pragma unroll
             for (int e = 0; e < EPC; ++e) {
-                const float df = x[u][e] - cen[lane * EPC + e];
+                const float df = x[e] - cen[lane * EPC + e];
                 part = fmaf(df, df, part);
             }
 #pragma unroll
@@ -265,10 +284,13 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
     double incl[4];
     kpp_block_scan(d2s, warp_tot, incl);
     if (tid == kKppThreads - 1) blocksum[(size_t)bh * nblk + blk] = incl[3];
-    // the last block of this head to finish picks seed j
-    __threadfence();
+    // the last block of this head to finish picks seed j (the barrier orders
+    // this block's D^2, label and block-sum stores before thread 0's fence)
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(counter + bh, 1) == nblk - 1);
+    if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(counter + bh, 1) == nblk - 1);
+    }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -295,7 +317,8 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     for (int j = 1; j < C; ++j) {
-        kpp_pass_kernel<T, D><<<dim3(nblk, BH), kKppThreads, 0, st>>>(
+        const size_t ccs_bytes = sizeof(float) * (size_t)(j > 1 ? j - 1 : 1);
+        kpp_pass_kernel<T, D><<<dim3(nblk, BH), kKppThreads, ccs_bytes, st>>>(
             X, N, nblk, chosen, C, j, D2, nearest, cc2, blocksum, counter, seed, cent);
         count_launches(1);
     }

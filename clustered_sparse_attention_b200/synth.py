@@ -73,6 +73,12 @@ WORKLOADS = {
                             100, 500, 40, 0.25, 256, 0.5, True),
     "wan720p_warm": Workload("wan720p_warm", 4, 1, 40, 21, 45, 80, 128, "bf16",
                              100, 500, 1, 0.25, 256, 0.5, True, warm_steps=10),
+    # the SVG-EAR paper's own cluster counts (review page, "What carries the
+    # argument"): 300 or 400 query clusters, 1000 key clusters
+    "wan720p_q300_k1000": Workload("wan720p_q300_k1000", 5, 1, 40, 21, 45, 80, 128, "bf16",
+                                   300, 1000, 40, 0.25, 256, 0.5, True),
+    "wan720p_q400_k1000": Workload("wan720p_q400_k1000", 6, 1, 40, 21, 45, 80, 128, "bf16",
+                                   400, 1000, 40, 0.25, 256, 0.5, True),
 }
 
 

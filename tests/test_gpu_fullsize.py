@@ -1,0 +1,153 @@
+"""The Wan 720p layer at full size (B=1, H=40, N=75600, d=128, Cq=100, Ck=500,
+40 rounds, density 0.25), run through the C ABI exactly as bench.py times it,
+then checked against the oracle on what the oracle can compute one piece at a
+time: sampled heads for the sort, means and routing (whole heads), sampled
+tokens for the assignment, sampled query clusters for the probe and sampled
+rows for the attention output; k-means++ is followed seed by seed on one head.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from clustered_sparse_attention_b200 import synth
+from tests.helpers import U32, check_assign, np64, probe_tolerance, update_tolerance
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+W = synth.WORKLOADS["wan720p"]
+HEADS = (0, 17, 39)          # sampled heads
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+@pytest.fixture(scope="module")
+def run():
+    import clustered_sparse_attention_b200 as csa
+    threads = min(16, os.cpu_count() or 1)
+    bits = {n: synth.layer_tensor_bits(W, n, threads=threads) for n in ("q", "k", "v")}
+    dev = {n: torch.from_numpy(b).view(torch.bfloat16).cuda() for n, b in bits.items()}
+    cq = csa.svgear_cluster(dev["q"], W.Cq, W.iters, seed=0, check_status=True)
+    ck = csa.svgear_cluster(dev["k"], W.Ck, W.iters, seed=1, check_status=True)
+    Vp = csa.svgear_permute(dev["v"], ck.perm)
+    vbar = csa.svgear_centroids(Vp, ck.offsets, W.Ck)
+    po, pk, E = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
+                                 Vp, W.density, W.scale, return_errors=True)
+    O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
+                          cq.perm, W.scale, check_status=True)
+    torch.cuda.synchronize()
+
+    def host(name, h):
+        b = bits[name][0, h].astype(np.uint32) << 16
+        return b.view(np.float32)
+
+    return {"csa": csa, "dev": dev, "host": host, "cq": cq, "ck": ck, "Vp": Vp, "vbar": vbar,
+            "po": po, "pk": pk, "E": E, "O": O}
+
+
+def test_fullsize_kmeanspp_follows_the_oracle_on_one_head(run):
+    csa = run["csa"]
+    h = 17
+    cent, idx = csa.svgear_kmeanspp_init(run["dev"]["k"], W.Ck, seed=1)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()[0, h]
+    X = run["host"]("k", h)
+    own, margin = oracle.kmeanspp(X, W.Ck, seed=1, stream=h, follow=idx)
+    assert own[0] == idx[0]
+    band = 4 * (W.d + 2) * U32
+    diff = np.nonzero(own != idx)[0]
+    for j in diff:
+        assert margin[j] < band, (j, idx[j], own[j], margin[j])
+    assert len(diff) <= 3
+    assert np.array_equal(cent.cpu().numpy()[0, h], X[idx])
+
+
+@pytest.mark.parametrize("name,C", [("q", W.Cq), ("k", W.Ck)])
+def test_fullsize_sort_means_and_permuted_copy(run, name, C):
+    cl = run["cq"] if name == "q" else run["ck"]
+    labels = cl.labels.cpu().numpy()
+    perm = cl.perm.cpu().numpy()
+    offs = cl.offsets.cpu().numpy()
+    cents = cl.centroids.cpu().numpy()
+    g = np.random.default_rng(5)
+    for h in HEADS:
+        X = run["host"](name, h)
+        p_o, o_o = oracle.stable_sort(labels[0, h], C)
+        assert np.array_equal(perm[0, h], p_o)
+        assert np.array_equal(offs[0, h], o_o)
+        ref = oracle.segment_mean(X[p_o], o_o, prev=cents[0, h])
+        assert np.all(np.abs(cents[0, h] - ref) <= update_tolerance(X, labels[0, h], C))
+        pos = g.choice(W.N, 4096, replace=False)
+        Xp = cl.Xp[0, h][torch.from_numpy(pos).cuda()].float().cpu().numpy()
+        assert np.array_equal(Xp, X[perm[0, h][pos]])
+
+
+def test_fullsize_assignment_on_sampled_tokens(run):
+    csa = run["csa"]
+    ck = run["ck"]
+    lab = csa.svgear_kmeans_assign(run["dev"]["k"], ck.centroids, check_status=True).cpu().numpy()
+    cents = ck.centroids.cpu().numpy()
+    g = np.random.default_rng(6)
+    flips = 0
+    for h in HEADS:
+        tok = np.sort(g.choice(W.N, 6000, replace=False))
+        X = run["host"]("k", h)
+        flips += check_assign(X[tok], cents[0, h], lab[0, h][tok])
+    assert flips <= 6
+
+
+def test_fullsize_probe_on_sampled_query_clusters(run):
+    cq, ck = run["cq"], run["ck"]
+    E = run["E"].cpu().numpy()
+    qbar = cq.centroids.cpu().numpy()
+    kbar = ck.centroids.cpu().numpy()
+    vbar = run["vbar"].cpu().numpy()
+    k_off = ck.offsets.cpu().numpy()
+    for h in HEADS[:2]:
+        rows = np.array([0, 37, W.Cq - 1])
+        Kp, Vp = np64(ck.Xp[0, h]), np64(run["Vp"][0, h])
+        Eo, So = oracle.probe(qbar[0, h][rows], Kp, Vp, kbar[0, h], vbar[0, h], k_off[0, h],
+                              W.scale, with_scale=True)
+        tol = probe_tolerance(qbar[0, h][rows], Kp, Eo, So, W.scale)
+        Eg = E[0, h][rows].astype(np.float64)
+        assert np.all(np.abs(Eg - Eo) <= tol), float(np.max(np.abs(Eg - Eo) / tol))
+
+
+def test_fullsize_route_bit_exact_given_gpu_errors(run):
+    cq, ck = run["cq"], run["ck"]
+    E = run["E"].cpu().numpy()
+    po, pk = run["po"].cpu().numpy(), run["pk"].cpu().numpy()
+    for h in HEADS:
+        ref_off, ref_kc = oracle.route(E[0, h], cq.offsets.cpu().numpy()[0, h],
+                                       ck.offsets.cpu().numpy()[0, h], W.N, W.density)
+        assert np.array_equal(po[0, h], ref_off)
+        assert np.array_equal(pk[0, h][:ref_off[-1]], ref_kc)
+
+
+def test_fullsize_attention_on_sampled_rows(run):
+    cq, ck = run["cq"], run["ck"]
+    q_off = cq.offsets.cpu().numpy()
+    g = np.random.default_rng(7)
+    O = run["O"]
+    for h in HEADS[:2]:
+        qo = q_off[0, h]
+        # rows at both ends of a few query clusters (128-row tile boundaries
+        # and the partial last tile) plus random ones
+        rows = set(g.choice(W.N, 32, replace=False).tolist())
+        for i in (0, 1, W.Cq // 2, W.Cq - 1):
+            a, b = int(qo[i]), int(qo[i + 1])
+            rows.update(r for r in (a, a + 127, a + 128, b - 1) if a <= r < b)
+        rows = np.array(sorted(rows))
+        args = (np64(cq.Xp[0, h]), np64(ck.Xp[0, h]), np64(run["Vp"][0, h]), qo,
+                ck.offsets.cpu().numpy()[0, h], run["po"].cpu().numpy()[0, h],
+                run["pk"].cpu().numpy()[0, h], ck.centroids.cpu().numpy()[0, h],
+                run["vbar"].cpu().numpy()[0, h], cq.perm.cpu().numpy()[0, h])
+        Oo, _ = oracle.attend(*args, W.scale, rows=rows)
+        dst = cq.perm.cpu().numpy()[0, h][rows]
+        Og = np64(O[0, h][torch.from_numpy(dst).cuda()])
+        assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2

@@ -33,6 +33,11 @@ RAGGED_BF16_64 = synth.custom_workload("ragged_bf16_d64", H=3, frames=1, grid_h=
                                        d=64, dtype="bf16", Cq=7, Ck=33, iters=3, density=0.25,
                                        n_centres=12, sigma=0.4, index=51)
 TINY = synth.WORKLOADS["tiny"]
+# the SVG-EAR paper's cluster counts (300 query, 1000 key clusters) on a short
+# clip: query clusters of ~16 rows leave most 128-row tiles partial
+EAR_COUNTS = synth.custom_workload("ear_counts", H=2, frames=2, grid_h=40, grid_w=60, d=128,
+                                   dtype="bf16", Cq=300, Ck=1000, iters=3, density=0.25,
+                                   n_centres=64, sigma=0.5, index=54)
 # many seeds over few tokens: most tokens of the late k-means++ passes are
 # screened out by the triangle bound, so the picks exercise the pruned path
 MANY_SEEDS = synth.custom_workload("many_seeds", H=2, frames=2, grid_h=48, grid_w=64, d=128,
@@ -232,7 +237,8 @@ def _clustered(w, dev, seed=3):
     return cq, ck, Vp, vbar
 
 
-@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64, EAR_COUNTS],
+                         ids=lambda w: w.name)
 def test_probe_matches_oracle(w):
     csa = _csa()
     host, dev = _inputs(w)
@@ -253,7 +259,8 @@ def test_probe_matches_oracle(w):
 
 
 @pytest.mark.parametrize("density", [0.05, 0.25, 0.5, 1.0])
-@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64, EAR_COUNTS],
+                         ids=lambda w: w.name)
 def test_route_bit_exact_given_gpu_errors(w, density):
     csa = _csa()
     host, dev = _inputs(w)
@@ -307,7 +314,7 @@ def test_attend_fp32_tiny_within_1e5():
 
 
 @pytest.mark.parametrize("density", [0.1, 0.3, 1.0])
-@pytest.mark.parametrize("w", [SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [SMALL_BF16, RAGGED_BF16_64, EAR_COUNTS], ids=lambda w: w.name)
 def test_attend_bf16_within_tolerance(w, density):
     host, dev = _inputs(w)
     rel, mx = _check_attend(w, dev, density)
