@@ -291,12 +291,14 @@ def workload_config(w, args):
 # DRAM bytes (read + write) of one attend_sm100_kernel launch, from the ncu
 # capture of the 8-head Wan 720p case (profiles/attend_sm100_wan720p_h8.md);
 # traffic grows with the heads of a launch (same per-head routing), so other
-# head counts of that shape scale it.  None for shapes not captured.
-ATTEND_TRAFFIC_H8_WAN720P = 526.024960e6 + 142.095104e6
+# head counts of that shape scale it.  None for shapes not captured, and None
+# while the kernel has changed since the capture.
+ATTEND_TRAFFIC_H8_WAN720P = None
 
 
 def attend_traffic(w):
-    if w.name.startswith("wan720p") and w.N == 75600 and w.d == 128 and w.Ck == 500:
+    if (ATTEND_TRAFFIC_H8_WAN720P is not None and w.name.startswith("wan720p") and w.N == 75600
+            and w.d == 128 and w.Ck == 500):
         return ATTEND_TRAFFIC_H8_WAN720P * (w.B * w.H) / 8.0
     return None
 

@@ -10,23 +10,26 @@
 // and the dynamic block-size kernel, which loads exactly the selected tokens
 // through a per-token address table and computes dense MMAs on them.
 //
-// B200 design (one CTA per 128-row tile of one query cluster):
-//   * the query cluster's selected key clusters form one compacted list of
-//     key rows; 4 producer warps gather 128 rows per tile (K and V) with
-//     16-byte cp.async into 128B-swizzled shared memory -- the per-token
-//     address table of the dynamic block-size kernel, with no padding inside
-//     the list; after the last key tile the skipped clusters' centroids
-//     (bf16) are gathered the same way, 128 per tile;
-//   * one thread issues tcgen05.mma: S = Q K^T (M=128, N=128, K=d) into one
-//     of two TMEM buffers, then O += P V (N=d, V as an MN-major operand)
-//     into a TMEM accumulator;
-//   * 4 softmax warps own one row each (TMEM lane = row): row max, exp2,
-//     the log2(n_c) bias of compensation columns, P to shared memory as bf16;
-//     O is rescaled in TMEM only when the running max grows by more than 2^8;
+// B200 design (one CTA per pair of 128-row tiles of one query cluster, which
+// share every key tile):
+//   * warps 8 and 9 fill the K and V rings by TMA: a key tile is the next 128
+//     entries of the query cluster's compacted list of selected key rows, each
+//     contiguous run copied as 2-D boxes of 2^h rows; after the key tiles the
+//     skipped clusters' bf16 centroids are gathered row by row;
+//   * warp 10 issues every tcgen05.mma in the order PV_0(j-1), QK_0(j),
+//     PV_1(j-1), QK_1(j): S_h = Q_h K^T (M=128, N=128) into TMEM, and
+//     O_h += P_h V with P_h read from TMEM as the A operand;
+//   * warps 0-3 and 4-7 are the softmax of the two halves, one row per thread
+//     (TMEM lane = row): row max, exp2 with the log2(n_c) bias on compensation
+//     columns, bf16 P written over the first 64 columns of its own S in TMEM;
+//     O_h is rescaled in TMEM only when the running max grows by more than
+//     2^8.  While one half's softmax runs, the tensor pipe works on the other
+//     half's PV and QK;
 //   * the epilogue divides by the row sum and writes O[q_perm[p]].
-// Every wait is bounded (1 s of %globaltimer); on expiry the CTA records
-// SVGEAR_ERR_TIMEOUT in the device status word, drains and returns, and
-// every later wait of the launch gives up at once.
+// TMEM: S_0 | S_1 | O_0 | O_1 (128 + 128 + d + d columns).  Every wait is
+// bounded (tc_wait.cuh); on expiry the CTA records SVGEAR_ERR_TIMEOUT in the
+// device status word, drains and returns, and every later wait of the launch
+// gives up at once.
 #include <math.h>
 
 #include "common.cuh"
@@ -39,16 +42,27 @@ namespace svgear {
 namespace sm100 {
 
 using bf16 = __nv_bfloat16;
+using tc::wait_bar;
+using tc::warp_wait_bar;
 
-constexpr int BM = 128;            // query rows per CTA
-constexpr int BN = 128;            // keys per tile
-constexpr int STAGES = 2;          // K/V ring
-constexpr int kSoftmaxThreads = 128;   // warps 0-3: one row each, TMEM lanes 0-127
-constexpr int kProducerWarp0 = 4;      // warps 4-5: K/V gathers, 64 rows each
-constexpr int kProducerWarps = 2;
-constexpr int kMmaWarp = 6;            // issues S = Q K^T (and owns the TMEM allocation)
-// warp 7 issues O += P V
-constexpr int kThreads = 8 * 32;       // 2 warps per SM sub-partition: 255 registers
+constexpr int BM = 128;                // query rows per half
+constexpr int BN = 128;                // keys per tile
+constexpr int STAGES = 2;              // K and V rings
+constexpr int kHalves = 2;             // query halves per CTA
+constexpr int kSoftmaxThreads = 128;   // per half: one row each
+constexpr int kKWarp = 8;              // K ring producer
+constexpr int kVWarp = 9;              // V ring producer
+constexpr int kMmaWarp = 10;           // issues every MMA, owns the TMEM allocation
+constexpr int kThreads = 12 * 32;      // 168 registers per thread at launch
+// Register split: the softmax warpgroups (0-1) grow to kSoftmaxRegs, the
+// producer/MMA warpgroup (2) shrinks to kIssueRegs.  The CTA's pool is
+// kThreads x (registers at launch); the host refuses a build whose launch
+// count is below kMinLaunchRegs, under which the split would not fit.
+constexpr uint32_t kSoftmaxRegs = 232;
+constexpr uint32_t kIssueRegs = 32;
+constexpr int kMinLaunchRegs =
+    (int)((2 * 128 * kSoftmaxRegs + 128 * kIssueRegs + kThreads - 1) / kThreads + 7) / 8 * 8;
+static_assert(kMinLaunchRegs <= 168, "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
@@ -63,33 +77,23 @@ struct TmaMaps {
     CUtensorMap q;
 };
 
-// Swizzled 16-byte chunk address inside a tile of 128 rows x (regions of
-// 64 bf16): region r covers elements [64r, 64r+64) of every row.
-__device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
-    const int region = chunk >> 3, cc = chunk & 7;
-    return tile + region * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-}
-
 struct Shared {
     uint64_t q_full;
     uint64_t k_full[STAGES];
     uint64_t k_empty[STAGES];
     uint64_t v_full[STAGES];
     uint64_t v_empty[STAGES];
-    uint64_t s_full[2];
-    uint64_t s_free[2];
-    uint64_t p_full[2];
-    uint64_t pv_done[2];
+    uint64_t s_full[kHalves];
+    uint64_t p_full[kHalves];
     uint64_t o_full;
     uint32_t tmem_base;
     int abort_flag;
     int keep_tmem;
-    int32_t row[kProducerWarps][BN];        // source row of each gathered row (-1: none)
 };
 
 #ifdef SVGEAR_TRACE
 // Diagnostic build only: per-tile event clocks of one CTA.
-__device__ long long g_trace[8][512];
+__device__ long long g_trace[18][512];
 #define TRACE(ev, j)                                                                  \
     do {                                                                              \
         if (blockIdx.x == 3 && blockIdx.y == 0 && (j) < 512) g_trace[ev][j] = clock64(); \
@@ -97,9 +101,6 @@ __device__ long long g_trace[8][512];
 #else
 #define TRACE(ev, j) do { } while (0)
 #endif
-
-using tc::wait_bar;
-using tc::warp_wait_bar;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -111,12 +112,12 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     float scale_log2, bf16* __restrict__ O, int* __restrict__ err) {
     constexpr int REG = D / 64;                 // 64-element regions per row
     constexpr uint32_t kTileBytes = REG * 16384;
-    constexpr uint32_t kPBytes = 2 * 16384;     // 128 rows x 128 keys bf16
     const int bh = blockIdx.y;
     if ((int)blockIdx.x >= ntiles[bh]) return;
     if (*(volatile int*)err != 0) return;   // an earlier CTA already gave up
     const int4 tile = tiles[(size_t)bh * maxT + blockIdx.x];
     const int ci = tile.x, q0 = tile.y, q_end = tile.z;
+    const int nh = (q0 + BM < q_end) ? 2 : 1;     // query halves with rows
     const int4 mt = meta[(size_t)bh * Cq + ci];   // {nseg, L keys, ncomp, 0}
     const int L = mt.y, ncomp = mt.z;
     const int T_real = (L + BN - 1) / BN;
@@ -125,10 +126,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ Shared sh;
     const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t sQ = base;
-    const uint32_t sK0 = sQ + kTileBytes;
+    const uint32_t sQ0 = base;                          // kHalves query tiles
+    const uint32_t sK0 = sQ0 + kHalves * kTileBytes;
     const uint32_t sV0 = sK0 + STAGES * kTileBytes;
-    const uint32_t sP0 = sV0 + STAGES * kTileBytes;   // two P buffers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -139,11 +139,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             tc::mbar_init(tc::smem_u32(&sh.v_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.v_empty[s]), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(tc::smem_u32(&sh.s_full[s]), 1);
-            tc::mbar_init(tc::smem_u32(&sh.s_free[s]), kSoftmaxThreads);
-            tc::mbar_init(tc::smem_u32(&sh.p_full[s]), kSoftmaxThreads);
-            tc::mbar_init(tc::smem_u32(&sh.pv_done[s]), 1);
+        for (int h = 0; h < kHalves; ++h) {
+            tc::mbar_init(tc::smem_u32(&sh.s_full[h]), 1);
+            tc::mbar_init(tc::smem_u32(&sh.p_full[h]), kSoftmaxThreads);
         }
         tc::mbar_init(tc::smem_u32(&sh.o_full), 1);
         sh.abort_flag = 0;
@@ -163,18 +161,21 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     const size_t head = (size_t)bh * Nq * D;
     const size_t row_meta = ((size_t)bh * Cq + ci) * Ck;
 
-    if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
-        // ------------------------------------------------------------ producer
-        // Warp 4 fills the K ring (freed by QK), warp 5 the V ring (freed by
-        // PV); lane 0 issues TMA.  A key tile is the next 128 entries of the
-        // query cluster's list of selected keys, which is a concatenation of
-        // contiguous key-cluster segments: every run [g, g+n) of rows that falls
-        // in the tile is copied with 2-D boxes of 2^h rows (the binary digits of
-        // n), landing 128B-swizzled at its place in the tile.  Tile rows past
-        // the list are boxes at an out-of-range row (zeros).  Compensation
-        // tiles gather the skipped clusters' bf16 centroids row by row.
-        const int pw = warp - kProducerWarp0;
-        const bool isK = pw == 0;
+    if (warp >= 4 * kHalves) {
+    // ================================================ warpgroup 2: TMA and MMA
+    tc::regs_dec<kIssueRegs>();   // one call site for the whole warpgroup
+    if (warp == kKWarp || warp == kVWarp) {
+        // ------------------------------------------------------------ producers
+        // Warp 8 fills the K ring (freed once both halves' QK are done), warp 9
+        // the V ring (freed once both halves' PV are done); lane 0 issues TMA.
+        // A key tile is the next 128 entries of the query cluster's list of
+        // selected keys, a concatenation of contiguous key-cluster segments:
+        // every run [g, g+n) of rows that falls in the tile is copied with 2-D
+        // boxes of 2^h rows (the binary digits of n), landing 128B-swizzled at
+        // its place in the tile.  Tile rows past the list are boxes at an
+        // out-of-range row (zeros).  Compensation tiles gather the skipped
+        // clusters' bf16 centroids row by row.
+        const bool isK = warp == kKWarp;
         const CUtensorMap* mrows = isK ? maps.k : maps.v;
         const CUtensorMap* mcent = isK ? &maps.kb : &maps.vb;
         uint64_t* ring_full = isK ? sh.k_full : sh.v_full;
@@ -182,10 +183,13 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         const uint32_t ring0 = isK ? sK0 : sV0;
         if (isK && lane == 0) {
             tc::prefetch_tmap(&maps.q);
-            tc::mbar_arrive_expect_tx(tc::smem_u32(&sh.q_full), BM * D * 2);
+            const uint32_t qb = tc::smem_u32(&sh.q_full);
+            tc::mbar_arrive_expect_tx(qb, nh * BM * D * 2);
+            for (int h = 0; h < nh; ++h)
 #pragma unroll
-            for (int h = 0; h < REG; ++h)
-                tc::tma_load_2d(sQ + h * 16384, &maps.q, h * 64, bh * Nq + q0, tc::smem_u32(&sh.q_full));
+                for (int g = 0; g < REG; ++g)
+                    tc::tma_load_2d(sQ0 + h * kTileBytes + g * 16384, &maps.q, g * 64,
+                                    bh * Nq + q0 + h * BM, qb);
         }
         const int32_t* pre = seg_prefix + ((size_t)bh * Cq + ci) * (Ck + 1);
         const int32_t* srow = seg_row + row_meta;
@@ -198,7 +202,8 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             if (j >= STAGES &&
                 !warp_wait_bar(&ring_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
-            if (pw == 0 && lane == 0) TRACE(0, j);
+            if (isK && lane == 0) TRACE(0, j);
+            if (!isK && lane == 0) TRACE(16, j);
             const uint32_t bar = tc::smem_u32(&ring_full[st]);
             const uint32_t tX = ring0 + st * kTileBytes;
             if (j >= T_real) {
@@ -211,9 +216,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 }
                 if (lane == 0) tc::mbar_arrive_expect_tx(bar, BN * D * 2);
                 __syncwarp();
-#pragma unroll
-                for (int h = 0; h < REG; ++h)
-                    tc::tma_gather4(tX + h * 16384 + lane * 512, mcent, h * 64, y[0], y[1], y[2], y[3],
+#pragma unroll 1
+                for (int g = 0; g < REG; ++g)
+                    tc::tma_gather4(tX + g * 16384 + lane * 512, mcent, g * 64, y[0], y[1], y[2], y[3],
                                     bar);
             } else if (lane == 0) {
                 tc::mbar_arrive_expect_tx(bar, BN * D * 2);
@@ -233,9 +238,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
 #pragma unroll 1
                     for (int hb = 7; hb >= 0; --hb) {
                         if (!(n >> hb & 1)) continue;
-#pragma unroll
-                        for (int h = 0; h < REG; ++h)
-                            tc::tma_load_2d(tX + h * 16384 + r * 128, &mrows[hb], h * 64, g, bar);
+#pragma unroll 1
+                        for (int gg = 0; gg < REG; ++gg)
+                            tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, g, bar);
                         r += 1 << hb;
                         if (g != kend) g += 1 << hb;
                     }
@@ -243,33 +248,108 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             }
             __syncwarp();
         }
-    } else if (warp < 4) {
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issue
+        // The whole warp runs the loop (uniform bounded waits); lane 0 issues.
+        // Step j issues, per half h: PV_h(j-1) once P_h(j-1) is in TMEM, then
+        // QK_h(j) into S_h (over P_h(j-1): MMAs of one thread run in order).
+        // While half 0's softmax works on S_0(j), the tensor pipe runs
+        // PV_1(j-1) and QK_1(j), and the other way round; the fixed order keeps
+        // the two softmax warpgroups half a step apart, so they do not contend
+        // for the exp unit at the same time.
+        constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
+        constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
+        bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
+        for (int j = 0; ok_run && j <= T; ++j) {
+            const int st = j % STAGES, pst = (j + STAGES - 1) % STAGES;
+            if (lane == 0) TRACE(1, j);
+            for (int h = 0; h < nh; ++h) {
+                if (j > 0) {
+                    if ((h == 0 && !warp_wait_bar(&sh.v_full[pst], ((j - 1) / STAGES) & 1, abort_flag,
+                                                  err, (11 << 16) + j)) ||
+                        !warp_wait_bar(&sh.p_full[h], (j - 1) & 1, abort_flag, err,
+                                       (8 << 16) + (h << 12) + j)) {
+                        ok_run = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    if (lane == 0) TRACE(h == 0 ? 9 : 13, j);
+                    if (lane == 0) {
+                        const uint32_t tV = sV0 + pst * kTileBytes;
+#pragma unroll 1
+                        for (int ks = 0; ks < BN / 16; ++ks)
+                            tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
+                                            tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
+                                            (j > 1 || ks > 0) ? 1u : 0u);
+                    }
+                    if (lane == 0) TRACE(h == 0 ? 10 : 14, j);
+                    __syncwarp();
+                }
+                if (j < T) {
+                    if (h == 0 &&
+                        !warp_wait_bar(&sh.k_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
+                        ok_run = false;
+                        break;
+                    }
+                    if (lane == 0 && h == 0) TRACE(11, j);
+                    if (lane == 0) {
+                        const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
+#pragma unroll 1
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
+                                         tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
+                        }
+                        tc::commit(tc::smem_u32(&sh.s_full[h]));
+                    }
+                    if (lane == 0) TRACE(h == 0 ? 12 : 15, j);
+                    __syncwarp();
+                }
+            }
+            if (!ok_run) break;
+            if (lane == 0) {
+                if (j < T) tc::commit(tc::smem_u32(&sh.k_empty[st]));
+                if (j > 0) tc::commit(tc::smem_u32(&sh.v_empty[pst]));
+                TRACE(2, j);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) tc::commit(tc::smem_u32(&sh.o_full));
+        __syncwarp();
+        // drain: every MMA of this CTA is complete once o_full flips; if that
+        // wait expires, TMEM is left allocated rather than released under a
+        // running MMA (every later CTA of the launch returns before alloc)
+        if (!warp_wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16)) && lane == 0)
+            sh.keep_tmem = 1;
+        __syncwarp();
+    }
+    } else {
+    // ================================================ warpgroups 0-1: softmax
+    tc::regs_inc<kSoftmaxRegs>();   // one call site for both warpgroups
+    {
         // ------------------------------------------------------------ softmax
-        const int r = tid;                               // row == TMEM lane
+        const int h = warp >> 2;                         // query half
+        const int r = tid & (kSoftmaxThreads - 1);       // row in the half == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t sS = lane_base + h * BN;          // S_h; P_h over its first 64 columns
+        const uint32_t sO = lane_base + kHalves * BN + h * D;
         const float* cb = comp_bias + row_meta;
         float m_use = -INFINITY, l = 0.f;
-        bool ok_run = true;
+        bool ok_run = h < nh;
         uint32_t v[BN];
         for (int j = 0; j < T && ok_run; ++j) {
-            const int sb = j & 1;
-            if (!warp_wait_bar(&sh.s_full[sb], (j >> 1) & 1, abort_flag, err, (2 << 16) + j)) {
+            if (!warp_wait_bar(&sh.s_full[h], j & 1, abort_flag, err, (2 << 16) + j)) {
                 ok_run = false;
                 break;
             }
             tc::fence_after_sync();
             if (tid == 0) TRACE(3, j);
-            {
-                const uint32_t sS = lane_base + sb * BN;
-                tc::tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tc::tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                tc::tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-                tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
-                tc::tmem_ld_wait();
-            }
-            // S(j) is in registers: the MMA may refill this buffer
-            tc::fence_before_sync();
-            tc::mbar_arrive(tc::smem_u32(&sh.s_free[sb]));
+            if (tid == kSoftmaxThreads) TRACE(5, j);
+            tc::tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tc::tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tc::tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+            tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+            tc::tmem_ld_wait();
 
             const bool comp = j >= T_real;
             const int valid = comp ? min(BN, ncomp - (j - T_real) * BN) : min(BN, L - j * BN);
@@ -306,20 +386,41 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             if (raw) mx *= scale_log2;
             const float m_new = fmaxf(m_use, mx);
 
-            // Lazy rescale of O: each row decides, but the TMEM loads/stores are
-            // warp-collective, so the warp rescales together when any row must
-            // (rows that need not use alpha = 1).  O must be final up to PV(j-1).
+            // Lazy rescale of O: a row needs it when its max grew by more than
+            // 2^8; the TMEM loads and stores are warp-collective, so the warp
+            // rescales together when any row must (the others with alpha = 1).
+            // O_h is final up to PV_h(j-1) here: that MMA was issued before
+            // QK_h(j), whose commit completed s_full.
             const bool need = j > 0 && m_new > m_use + kRescaleThreshold;
-            if (j == 0) m_use = m_new;
-            if (__any_sync(0xffffffffu, need)) {
-                if (!warp_wait_bar(&sh.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, err,
-                                   (3 << 16) + j)) {
-                    ok_run = false;
-                    break;
+            const bool any = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (j == 0) {
+                m_use = m_new;
+            } else if (need) {
+                alpha = tc::ex2(m_use - m_new);
+                l *= alpha;
+                m_use = m_new;
+            }
+            if (tid == 0) TRACE(4, j);
+            // P = 2^(x - m) as bf16 pairs over the first 64 columns of S_h
+            const float xs = raw ? scale_log2 : 1.f, neg_m = -m_use;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int q = 0; q < BN / 32; ++q) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = tc::ex2(fmaf(__uint_as_float(v[q * 32 + e]), xs, neg_m));
+                    const float p1 = tc::ex2(fmaf(__uint_as_float(v[q * 32 + e + 1]), xs, neg_m));
+                    s0 += p0;
+                    s1 += p1;
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&hp);
                 }
-                tc::fence_after_sync();
-                const float alpha = need ? tc::ex2(m_use - m_new) : 1.f;
-                const uint32_t sO = lane_base + 2 * BN;
+                tc::tmem_st16(sS + q * 16, pk);
+            }
+            l += s0 + s1;
+            if (any) {
                 uint32_t o[16];
 #pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
@@ -329,50 +430,18 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     tc::tmem_st16(sO + c * 16, o);
                 }
-                tc::tmem_st_wait();
-                if (need) {
-                    l *= alpha;
-                    m_use = m_new;
-                }
             }
-            if (tid == 0) TRACE(4, j);
-            // P buffer sb is free once PV(j-2) has completed
-            if (j >= 2 &&
-                !warp_wait_bar(&sh.pv_done[sb], ((j >> 1) - 1) & 1, abort_flag, err, (10 << 16) + j)) {
-                ok_run = false;
-                break;
-            }
-            if (tid == 0) TRACE(5, j);
-            const uint32_t sP = sP0 + sb * kPBytes;
-            const float xs = raw ? scale_log2 : 1.f, neg_m = -m_use;
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int q = 0; q < BN / 8; ++q) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const float p0 = tc::ex2(fmaf(__uint_as_float(v[q * 8 + e]), xs, neg_m));
-                    const float p1 = tc::ex2(fmaf(__uint_as_float(v[q * 8 + e + 1]), xs, neg_m));
-                    s0 += p0;
-                    s1 += p1;
-                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(sP, r, q)),
-                             "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                             : "memory");
-            }
-            l += s0 + s1;
-            tc::fence_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&sh.p_full[sb]));
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            tc::mbar_arrive(tc::smem_u32(&sh.p_full[h]));
             if (tid == 0) TRACE(6, j);
+            if (tid == kSoftmaxThreads) TRACE(7, j);
         }
         // epilogue: O / l back to the original token order
         if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
             tc::fence_after_sync();
-            const int p = q0 + r;
+            const int p = q0 + h * BM + r;
             const float inv = 1.f / l;
-            const uint32_t sO = lane_base + 2 * BN;
             const bool write = p < q_end;
             const int dst = write ? q_perm[(size_t)bh * Nq + p] : 0;
             bf16* orow = O + head + (size_t)dst * D;
@@ -385,9 +454,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[e]) * inv,
-                                                                 __uint_as_float(o[e + 1]) * inv);
-                        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h);
+                        __nv_bfloat162 hp = __floats2bfloat162_rn(__uint_as_float(o[e]) * inv,
+                                                                  __uint_as_float(o[e + 1]) * inv);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&hp);
                     }
                     uint4* o4 = reinterpret_cast<uint4*>(orow + c4 * 32);
 #pragma unroll
@@ -396,80 +465,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 }
             }
         }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ S = Q K^T
-        // The whole warp runs the loop; lane 0 issues the MMAs and commits.
-        constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
-        bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
-        if (ok_run) tc::fence_async_smem();
-        for (int j = 0; ok_run && j < T; ++j) {
-            const int st = j % STAGES, sb = j & 1;
-            if (!warp_wait_bar(&sh.k_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
-                ok_run = false;
-                break;
-            }
-            if (lane == 0) TRACE(1, j);
-            if (j >= 2 &&
-                !warp_wait_bar(&sh.s_free[sb], ((j >> 1) - 1) & 1, abort_flag, err, (7 << 16) + j)) {
-                ok_run = false;
-                break;
-            }
-            tc::fence_async_smem();   // cp.async data -> tensor-core reads
-            tc::fence_after_sync();
-            if (lane == 0) TRACE(2, j);
-            if (lane == 0) {
-                const uint32_t tK = sK0 + st * kTileBytes;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    tc::mma_bf16(tmem + sb * BN, tc::sw128_desc(sQ + off, 16, 1024),
-                                 tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
-                }
-                tc::commit(tc::smem_u32(&sh.k_empty[st]));
-                tc::commit(tc::smem_u32(&sh.s_full[sb]));
-            }
-            __syncwarp();
-        }
-        // S(j) is consumed by the softmax before its P(j) exists, so the PV
-        // warp's last commit covers every MMA of this warp too; nothing to drain.
-    } else {
-        // ------------------------------------------------------------ O += P V
-        constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
-        bool ok_run = true;
-        for (int jj = 0; ok_run && jj < T; ++jj) {
-            const int st = jj % STAGES, pb = jj & 1;
-            if (!warp_wait_bar(&sh.v_full[st], (jj / STAGES) & 1, abort_flag, err, (11 << 16) + jj) ||
-                !warp_wait_bar(&sh.p_full[pb], (jj >> 1) & 1, abort_flag, err, (8 << 16) + jj)) {
-                ok_run = false;
-                break;
-            }
-            tc::fence_async_smem();   // cp.async data -> tensor-core reads
-            tc::fence_after_sync();
-            if (lane == 0) TRACE(7, jj);
-            if (lane == 0) {
-                const uint32_t tV = sV0 + st * kTileBytes;
-                const uint32_t sP = sP0 + pb * kPBytes;
-#pragma unroll
-                for (int ks = 0; ks < BN / 16; ++ks) {
-                    const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    tc::mma_bf16(tmem + 2 * BN, tc::sw128_desc(sP + offp, 16, 1024),
-                                 tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
-                                 (jj > 0 || ks > 0) ? 1u : 0u);
-                }
-                tc::commit(tc::smem_u32(&sh.v_empty[st]));
-                tc::commit(tc::smem_u32(&sh.pv_done[pb]));
-            }
-            __syncwarp();
-        }
-        if (lane == 0) tc::commit(tc::smem_u32(&sh.o_full));
-        __syncwarp();
-        // drain: every MMA of this CTA is complete once o_full flips (the QK
-        // warp's MMAs all precede the last P); if that wait expires, TMEM is
-        // left allocated rather than released under a running MMA (every later
-        // CTA of the launch returns before alloc)
-        if (!warp_wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16)) && lane == 0)
-            sh.keep_tmem = 1;
-        __syncwarp();
+    }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -530,7 +526,8 @@ __global__ void attend_prep_kernel(const int32_t* __restrict__ k_off, int Ck, in
     }
 }
 
-// One block per head: every (cluster, 128-row tile) of the query segments.
+// One block per head: every (cluster, pair of 128-row tiles) of the query
+// segments; a CTA takes one entry.
 __global__ void attend_tiles_kernel(const int32_t* __restrict__ q_off, int Cq, int Nq, int maxT,
                                     int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
     const int bh = blockIdx.x;
@@ -540,7 +537,8 @@ __global__ void attend_tiles_kernel(const int32_t* __restrict__ q_off, int Cq, i
     for (int i = 0; i < Cq; ++i) {
         const int a = qo[i], b = qo[i + 1];
         if (b <= a || a < 0 || b > Nq) continue;
-        for (int r0 = a; r0 < b && k < maxT; r0 += BM) tiles[(size_t)bh * maxT + k++] = make_int4(i, r0, b, 0);
+        for (int r0 = a; r0 < b && k < maxT; r0 += kHalves * BM)
+            tiles[(size_t)bh * maxT + k++] = make_int4(i, r0, b, 0);
     }
     ntiles[bh] = k;
 }
@@ -584,8 +582,19 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     count_launches(1);
     attend_tiles_kernel<<<BH, 32, 0, st>>>(q_off, Cq, qd.N, w.maxT, w.tiles, w.ntiles);
     count_launches(1);
+    // the register split of the kernel needs its launch allocation
+    static int launch_regs[2] = {0, 0};
+    int& lr = launch_regs[D == 128 ? 1 : 0];
+    if (lr == 0) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, D == 128 ? (const void*)attend_sm100_kernel<128>
+                                                : (const void*)attend_sm100_kernel<64>) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        lr = fa.numRegs;
+    }
+    if (lr < kMinLaunchRegs) return SVGEAR_ERR_UNSUPPORTED;
     const float scale_log2 = scale * 1.4426950408889634f;
-    const size_t smem = (size_t)(1 + 2 * STAGES) * (D / 64) * 16384 + 2 * 2 * 16384 + 1024;
+    const size_t smem = (size_t)(kHalves + 2 * STAGES) * (D / 64) * 16384 + 1024;
     if (D == 128) {
         if (cudaFuncSetAttribute(attend_sm100_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
