@@ -89,10 +89,21 @@ class ClockSampler:
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        # nvidia-smi's first query initialises NVML, which on a fresh machine
+        # takes a while and disturbs the GPU: let it finish before any timing
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 15.0 and self.proc.poll() is None:
+            time.sleep(0.05)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def window(self, t0, t1):
+        """Keep only the samples taken inside [t0, t1] (the timed region)."""
+        inside = [x for x in self.lines if t0 <= x[0] <= t1]
+        if inside:
+            self.lines = inside
 
     def stop(self):
         if self.proc is None:
@@ -106,7 +117,7 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
+        for _, ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -353,25 +364,28 @@ def main():
         mark(5)
         return O, (cq, ck, po, pk)
 
+    # the clock sampler starts (and finishes initialising) before the warm-up
+    clocks = ClockSampler(local if ws > 1 else torch.cuda.current_device())
+    clocks.start()
     for _ in range(max(3, args.warmup)):
         step(Q, K, V)
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local if ws > 1 else torch.cuda.current_device())
-    clocks.start()
-    time.sleep(0.3)
     barrier(ws)
     torch.cuda.synchronize()
     l0 = csa.kernel_launches()
+    t_begin = time.time()
     start.record(stream)
     for s in range(args.steps):
         O, state = step(Q, K, V, evs[s])
     end.record(stream)
     torch.cuda.synchronize()
+    t_end = time.time()
     barrier(ws)
     launches = csa.kernel_launches() - l0
+    clocks.window(t_begin, t_end)
     clk = clocks.stop()
     ms_step = start.elapsed_time(end) / args.steps
     ms_step_max = max_over_ranks(ms_step, ws)

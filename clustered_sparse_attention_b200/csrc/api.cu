@@ -58,6 +58,7 @@ struct KppWs {
     int32_t* counter;
     int32_t* nearest;
     float* cc2;
+    int32_t* gen;
 };
 KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
     KppWs w;
@@ -67,6 +68,7 @@ KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
     w.counter = cv.take<int32_t>(bh_of(d));
     w.nearest = cv.take<int32_t>(bh_of(d) * d.N);
     w.cc2 = cv.take<float>(bh_of(d) * C);
+    w.gen = cv.take<int32_t>(bh_of(d));
     return w;
 }
 int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {
@@ -183,6 +185,7 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             return ws_cluster(dims, C1);
         case SVGEAR_OP_KMEANSPP:
             if (check_C(C1, dims.N)) return 0;
+            cv.take<int>(4);
             carve_kpp(cv, dims, C1);
             break;
         case SVGEAR_OP_LABEL_SORT:
@@ -221,11 +224,13 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
     if (!X || !centroids || !ws || !aligned16(X)) return SVGEAR_ERR_INVALID_ARG;
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_KMEANSPP, dims, C, 0)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
+    int* status = cv.take<int>(4);
+    if (cudaMemsetAsync(status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     KppWs w = carve_kpp(cv, dims, C);
     return launch_kmeanspp(X, dims, C, seed, centroids, seed_index ? seed_index : w.chosen, w.D2,
-                           w.nearest, w.cc2, w.blocksum, w.counter,
-                           static_cast<cudaStream_t>(stream));
+                           w.nearest, w.cc2, w.blocksum, w.counter, w.gen, status, st);
 }
 
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids, int32_t C,
@@ -308,7 +313,7 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
         carve_flags(cv, dims);
         KppWs w = carve_kpp(cv, dims, C);
         if ((s = launch_kmeanspp(X, dims, C, seed, centroids, w.chosen, w.D2, w.nearest, w.cc2,
-                                 w.blocksum, w.counter, st)))
+                                 w.blocksum, w.counter, w.gen, fl.status, st)))
             return s;
     }
     Carve cv(ws);

@@ -15,8 +15,9 @@
 //
 // B200 design: persistent CTAs, one per SM, walk the 128-token tiles of all
 // heads (tiles of heads at their fixed point are skipped).
-//   warp 0     TMA producer: the token tile (2 stages), then a ring of
-//              centroid-plane boxes of Nc rows x 64 dims (128B-swizzled);
+//   warp 0     TMA producer: the token tile (2 to 4 stages, as shared memory
+//              allows), then a ring of centroid-plane boxes of Nc rows x 64
+//              dims (128B-swizzled);
 //   warp 1     one lane issues tcgen05.mma (M=128, N=Nc <= 256, K=16) into one
 //              of two TMEM accumulators, each centroid chunk a chain of
 //              3 planes x d/16 steps;
@@ -47,7 +48,7 @@ constexpr int kMmaWarp = 1;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 512;      // two accumulators of up to 256 columns
 constexpr uint32_t kAccCols = 256;
-constexpr uint32_t kBStageBytes = 256 * 128;   // up to 256 rows x 64 bf16
+constexpr int kMaxAStages = 4;           // token-tile stages: as many as shared memory holds
 constexpr uint64_t kDrainNs = 200000000ull;    // 0.2 s to let issued work land
 
 struct Maps {
@@ -56,8 +57,8 @@ struct Maps {
 };
 
 struct Shared {
-    uint64_t a_full[2];
-    uint64_t a_empty[2];
+    uint64_t a_full[kMaxAStages];
+    uint64_t a_empty[kMaxAStages];
     uint64_t b_full[kBStages];
     uint64_t b_empty[kBStages];
     uint64_t acc_full[2];
@@ -80,7 +81,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc,
+assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc, int nA,
                     const float* __restrict__ cnorm, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
                     int* __restrict__ err) {
@@ -95,13 +96,16 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     __shared__ Shared sh;
     const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t sA0 = base;
-    const uint32_t sB0 = base + 2 * kABytes;
+    const uint32_t sB0 = base + nA * kABytes;
+    const uint32_t kBStageBytes = (uint32_t)Nc * 128u;   // Nc rows x 64 bf16 (multiple of 2 KB)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kMaxAStages; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.a_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.a_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.acc_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.acc_empty[s]), kEpiThreads);
         }
@@ -136,9 +140,9 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             const int bh = w / tiles_per_head;
             if (done && done[bh]) continue;
             const int t0 = (w - bh * tiles_per_head) * BM;
-            const int sa = ia & 1;
-            if (ia >= 2 &&
-                !warp_wait_bar(&sh.a_empty[sa], ((ia >> 1) - 1) & 1, abort_flag, err, (1 << 16) + ia)) {
+            const int sa = ia % nA;
+            if (ia >= nA &&
+                !warp_wait_bar(&sh.a_empty[sa], ((ia / nA) - 1) & 1, abort_flag, err, (1 << 16) + ia)) {
                 ok = false;
                 break;
             }
@@ -175,9 +179,9 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         }
         // let the last copy into every stage land before the CTA can exit
         if (lane == 0) {
-            for (int k = 0; k < 2 && k < ia; ++k) {
+            for (int k = 0; k < nA && k < ia; ++k) {
                 const int i = ia - 1 - k;
-                drain_wait(&sh.a_full[i & 1], (i >> 1) & 1);
+                drain_wait(&sh.a_full[i % nA], (i / nA) & 1);
             }
             for (int k = 0; k < kBStages && k < ib; ++k) {
                 const int i = ib - 1 - k;
@@ -193,8 +197,8 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
             const int bh = w / tiles_per_head;
             if (done && done[bh]) continue;
-            const int sa = ia & 1;
-            if (!warp_wait_bar(&sh.a_full[sa], (ia >> 1) & 1, abort_flag, err, (3 << 16) + ia)) {
+            const int sa = ia % nA;
+            if (!warp_wait_bar(&sh.a_full[sa], (ia / nA) & 1, abort_flag, err, (3 << 16) + ia)) {
                 ok = false;
                 break;
             }
@@ -406,7 +410,14 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         return SVGEAR_ERR_CUDA;
     const int total = BH * ceil_div(N, BM);
     const int grid = total < num_sms[dev] ? total : num_sms[dev];
-    const size_t smem = (size_t)2 * (D / 64) * 16384 + (size_t)kBStages * kBStageBytes + 1024;
+    // the centroid ring takes kBStages boxes of Nc rows; the token-tile stages
+    // take what shared memory has left (2 to kMaxAStages)
+    const size_t a_bytes = (size_t)(D / 64) * 16384, b_bytes = (size_t)kBStages * Nc * 128;
+    const size_t budget = 227 * 1024 - 1024 - sizeof(Shared) - 64;
+    if (budget < b_bytes + 2 * a_bytes) return SVGEAR_ERR_UNSUPPORTED;
+    int nA = (int)((budget - b_bytes) / a_bytes);
+    if (nA > kMaxAStages) nA = kMaxAStages;
+    const size_t smem = (size_t)nA * a_bytes + b_bytes + 1024;
     if (D == 128) {
         centroid_planes_kernel<128><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
                                                                                 cn, done);
@@ -414,7 +425,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, cn, labels,
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, cn, labels,
                                                                done, changed, err);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
@@ -423,7 +434,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, cn, labels,
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, cn, labels,
                                                               done, changed, err);
     }
     count_launches(1);

@@ -71,12 +71,12 @@ __global__ void kpp_first_kernel(const T* __restrict__ X, int N, int D, int C,
 // blocks used, so the two levels agree bit for bit.  Also leaves in cc2 the
 // squared distances from seed j to seeds 0..j-1 for the next pass's pruning.
 template <typename T, int D>
-__device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C, int j,
-                         const float* D2, const double* blocksum, uint64_t seed, float* centroids,
-                         float* cc2, float* d2s, double* warp_tot, float* cnew) {
+__device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32_t* chosen, int C,
+                         int j, const float* D2, const double* blocksum, uint64_t seed,
+                         float* centroids, float* cc2, float* d2s, double* warp_tot, float* cnew) {
     __shared__ int s_blk, s_pick;
     __shared__ double s_base, s_target;
-    const int bh = blockIdx.y, tid = threadIdx.x;
+    const int tid = threadIdx.x;
     const double* bs = blocksum + (size_t)bh * nblk;
     const float* d2 = D2 + (size_t)bh * N;
     int32_t* ch = chosen + (size_t)bh * C;
@@ -129,7 +129,7 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chos
         } else {                    // every D^2 is zero: lowest unchosen token
             for (int t = 0; t < N; ++t) {
                 bool used = false;
-                for (int q = 0; q < j; ++q) used |= (ch[q] == t);
+                for (int q = 0; q < j; ++q) used |= (__ldcg(ch + q) == t);
                 if (!used) { pick = t; break; }
             }
         }
@@ -175,33 +175,33 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int32_t* chos
 // the comparison and is recomputed.
 constexpr float kKppPrune = 4.03125f;
 
-// One pass of the seeding: D^2 <- min(D^2, |x - seed_{j-1}|^2) for a block of
-// kKppTokens tokens, the block's fp64 scan total, and -- in the last block of
-// the head to finish -- the pick of seed j.  Tokens are first screened with
-// the triangle bound (8 bytes read per token: D^2 and nearest-seed index);
-// only the survivors' rows are loaded, by groups of lanes, four rows in flight.
+// Shared memory of one k-means++ CTA.
+template <int D>
+struct KppSmem {
+    float cen[D];                              // the seed this pass adds, fp32
+    __align__(16) float d2s[kKppTokens];       // a block's D^2; also the pick's fp64 block sums
+    int32_t todo[kKppTokens];                  // tokens of the block left by the screen
+    double warp_tot[kKppThreads / 32];
+    int ntodo;
+};
+
+// One 1024-token block of the pass adding seed s: D^2 <- min(D^2, |x - c_s|^2)
+// and the block's fp64 scan total.  Tokens are first screened with the
+// triangle bound (8 bytes read per token: D^2 and nearest-seed index); only
+// the survivors' rows are loaded, by groups of lanes, four rows in flight.
 template <typename T, int D>
-__global__ void __launch_bounds__(kKppThreads, 6)
-kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C, int j, float* D2,
-                int32_t* nearest, float* cc2, double* blocksum, int32_t* counter, uint64_t seed,
-                float* centroids) {
+__device__ void kpp_block_update(const T* __restrict__ X, int N, int nblk, int bh, int blk, int s,
+                                 float* D2, int32_t* nearest, double* blocksum, KppSmem<D>& sm,
+                                 const float* ccs) {
     constexpr int EPC = Elem<T>::kPerChunk;
     constexpr int L = D / EPC;                 // lanes per token row
     constexpr int RP = kKppThreads / L;        // rows per sweep of the block
     constexpr int U = 4;                       // rows in flight per lane group
-    __shared__ float cen[D];
-    __shared__ __align__(16) float d2s[kKppTokens];   // also the pick's fp64 block sums
-    __shared__ int32_t todo[kKppTokens];
-    extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: s floats)
-    __shared__ double warp_tot[kKppThreads / 32];
-    __shared__ int s_ntodo, s_last;
-    const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x, wl = tid & 31;
-    const int s = j - 1;                       // the seed this pass adds
+    constexpr int TPT = kKppTokens / kKppThreads;   // tokens per thread
+    const int tid = threadIdx.x, wl = tid & 31;
     const T* Xh = X + (size_t)bh * N * D;
     float* D2h = D2 + (size_t)bh * N;
     int32_t* nh = nearest + (size_t)bh * N;
-    // issue the per-token state loads first: they do not depend on the seed
-    constexpr int TPT = kKppTokens / kKppThreads;   // tokens per thread
     float dpre[TPT];
     int apre[TPT];
 #pragma unroll
@@ -214,10 +214,7 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
             apre[i] = nh[t];
         }
     }
-    // seed s as fp32 (its row of the centroid table, written by the pick)
-    for (int k = tid; k < D; k += kKppThreads) cen[k] = centroids[((size_t)bh * C + s) * D + k];
-    for (int a = tid; a < s; a += kKppThreads) ccs[a] = cc2[(size_t)bh * C + a];
-    if (tid == 0) s_ntodo = 0;
+    if (tid == 0) sm.ntodo = 0;
     __syncthreads();
     // screen
 #pragma unroll
@@ -234,16 +231,16 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
                 need = (unsigned)a >= (unsigned)s || !(ccs[a] >= kKppPrune * d);
             }
         }
-        d2s[r] = d;
+        sm.d2s[r] = d;
         const unsigned m = __ballot_sync(0xffffffffu, need);
         int base = 0;
-        if (wl == 0 && m) base = atomicAdd(&s_ntodo, __popc(m));
+        if (wl == 0 && m) base = atomicAdd(&sm.ntodo, __popc(m));
         base = __shfl_sync(0xffffffffu, base, 0);
-        if (need) todo[base + __popc(m & ((1u << wl) - 1u))] = r;
+        if (need) sm.todo[base + __popc(m & ((1u << wl) - 1u))] = r;
     }
     __syncthreads();
     // recompute the survivors
-    const int n = s_ntodo;
+    const int n = sm.ntodo;
     const int lane = tid % L, grp = tid / L;
     for (int b0 = 0; b0 < n; b0 += RP * U) {
         int rr[U];
@@ -251,7 +248,7 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = b0 + grp + u * RP;
-            rr[u] = i < n ? todo[i] : -1;
+            rr[u] = i < n ? sm.todo[i] : -1;
             raw[u] = make_uint4(0u, 0u, 0u, 0u);
             if (rr[u] >= 0)
                 raw[u] = Elem<T>::load_raw(Xh + (size_t)(blk * kKppTokens + rr[u]) * D + lane * EPC);
@@ -263,17 +260,17 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
             float part = 0.f;
 #pragma unroll
             for (int e = 0; e < EPC; ++e) {
-                const float df = x[e] - cen[lane * EPC + e];
+                const float df = x[e] - sm.cen[lane * EPC + e];
                 part = fmaf(df, df, part);
             }
 #pragma unroll
             for (int o = L / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             if (lane == 0 && rr[u] >= 0) {
                 const int r = rr[u], t = blk * kKppTokens + r;
-                const float old = d2s[r];
+                const float old = sm.d2s[r];
                 const float v = s == 0 ? part : fminf(part, old);
                 if (s == 0 || __float_as_int(v) != __float_as_int(old)) {
-                    d2s[r] = v;
+                    sm.d2s[r] = v;
                     D2h[t] = v;
                     nh[t] = s;
                 }
@@ -282,47 +279,143 @@ kpp_pass_kernel(const T* __restrict__ X, int N, int nblk, int32_t* chosen, int C
     }
     __syncthreads();
     double incl[4];
-    kpp_block_scan(d2s, warp_tot, incl);
+    kpp_block_scan(sm.d2s, sm.warp_tot, incl);
     if (tid == kKppThreads - 1) blocksum[(size_t)bh * nblk + blk] = incl[3];
-    // the last block of this head to finish picks seed j (the barrier orders
-    // this block's D^2, label and block-sum stores before thread 0's fence)
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        s_last = (atomicAdd(counter + bh, 1) == nblk - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (j < C)
-        kpp_pick<T, D>(X, N, nblk, chosen, C, j, D2, blocksum, seed, centroids, cc2, d2s, warp_tot,
-                       cen);
-    if (tid == 0) counter[bh] = 0;   // ready for the next pass
+    __syncthreads();   // d2s and warp_tot are reused by the next block
 }
 
-__global__ void zero_i32_kernel(int32_t* p, int n) {
+// Persistent seeding: CTA c works for head bh0 + c / cph on its share of the
+// head's 1024-token blocks, for every seed.  Before pass j (which adds seed
+// j-1) it waits until the head's generation word gen[bh] reaches j; after its
+// blocks it arrives on counter[bh]; the last CTA of the head to arrive picks
+// seed j (and the seed-to-seed distances of the next screen), resets the
+// counter and publishes gen[bh] = j + 1.  Heads never wait for each other, so
+// one head's pick overlaps the other heads' passes.  The launch is
+// cooperative (every CTA resident); every wait is bounded and gives up with
+// SVGEAR_ERR_TIMEOUT in err[0] (err[1] = pass, err[2] = CTA).
+constexpr uint64_t kKppWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t tc_global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kKppThreads, 6)
+kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg, int cph, int C,
+                      int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* blocksum,
+                      int32_t* counter, int32_t* gen, uint64_t seed, float* centroids, int* err) {
+    __shared__ KppSmem<D> sm;
+    extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: C floats)
+    __shared__ int s_flag;
+    const int tid = threadIdx.x;
+    const int hl = blockIdx.x / cph, part = blockIdx.x % cph;
+    if (hl >= BHg) return;
+    const int bh = bh0 + hl;
+    const int blk0 = (int)((long long)part * nblk / cph), blk1 = (int)((long long)(part + 1) * nblk / cph);
+    for (int j = 1; j < C; ++j) {
+        const int s = j - 1;
+        // wait for seed s
+        if (tid == 0) {
+            int ok = 1;
+            volatile int* g = gen + bh;
+            if (*g < j) {
+                const uint64_t t0 = tc_global_ns();
+                while (*g < j) {
+                    if (*(volatile int*)err != 0) { ok = 0; break; }
+                    if (tc_global_ns() - t0 > kKppWaitNs) {
+                        if (atomicCAS(err, 0, SVGEAR_ERR_TIMEOUT) == 0) {
+                            err[1] = j;
+                            err[2] = (int)blockIdx.x;
+                        }
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+            }
+            __threadfence();   // acquire: the pick's stores are visible from here on
+            s_flag = ok;
+        }
+        __syncthreads();
+        if (!s_flag) return;
+        for (int k = tid; k < D; k += kKppThreads) sm.cen[k] = __ldcg(centroids + ((size_t)bh * C + s) * D + k);
+        for (int a = tid; a < s; a += kKppThreads) ccs[a] = __ldcg(cc2 + (size_t)bh * C + a);
+        // (the block update's first barrier orders these loads before their use)
+        for (int blk = blk0; blk < blk1; ++blk)
+            kpp_block_update<T, D>(X, N, nblk, bh, blk, s, D2, nearest, blocksum, sm, ccs);
+        // arrive; the barrier inside the block update ordered this CTA's D^2,
+        // label and block-sum stores before thread 0's fence
+        if (tid == 0) {
+            __threadfence();
+            s_flag = (atomicAdd(counter + bh, 1) == cph - 1);
+        }
+        __syncthreads();
+        if (s_flag) {
+            __threadfence();
+            kpp_pick<T, D>(X, N, nblk, bh, chosen, C, j, D2, blocksum, seed, centroids, cc2, sm.d2s,
+                           sm.warp_tot, sm.cen);
+            __syncthreads();
+            if (tid == 0) {
+                counter[bh] = 0;
+                __threadfence();
+                atomicExch(gen + bh, j + 1);   // release seed j
+            }
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void kpp_init_kernel(int32_t* counter, int32_t* gen, int n) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) p[i] = 0;
+    if (i < n) {
+        counter[i] = 0;
+        gen[i] = 1;   // seed 0 comes from kpp_first_kernel, launched before
+    }
 }
 
 template <typename T, int D>
 static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, float* cent,
                          int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
-                         double* blocksum, int32_t* counter, cudaStream_t st) {
+                         double* blocksum, int32_t* counter, int32_t* gen, int* err,
+                         cudaStream_t st) {
     const int BH = dims.B * dims.H, N = dims.N;
     const int nblk = ceil_div(N, kKppTokens);
-    zero_i32_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, BH);
+    kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, gen, BH);
     count_launches(1);
     kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
-    for (int j = 1; j < C; ++j) {
-        const size_t ccs_bytes = sizeof(float) * (size_t)(j > 1 ? j - 1 : 1);
-        kpp_pass_kernel<T, D><<<dim3(nblk, BH), kKppThreads, ccs_bytes, st>>>(
-            X, N, nblk, chosen, C, j, D2, nearest, cc2, blocksum, counter, seed, cent);
+    if (C < 2) return SVGEAR_OK;
+    // cooperative grid: every CTA resident, so CTAs of a head may wait on each other
+    int dev = 0, sms = 0, per_sm = 0;
+    const size_t ccs_bytes = sizeof(float) * (size_t)C;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kpp_persistent_kernel<T, D>,
+                                                      kKppThreads, ccs_bytes) != cudaSuccess ||
+        per_sm < 1)
+        return SVGEAR_ERR_CUDA;
+    const int capacity = per_sm * sms;
+    // heads per launch: all of them when every head gets a CTA, else groups
+    const int BHg_max = BH < capacity ? BH : capacity;
+    for (int bh0 = 0; bh0 < BH; bh0 += BHg_max) {
+        int BHg = BH - bh0 < BHg_max ? BH - bh0 : BHg_max;
+        int cph = capacity / BHg;
+        if (cph > nblk) cph = nblk;
+        if (cph < 1) cph = 1;
+        const int grid = BHg * cph;
+        int n_ = N, nblk_ = nblk, C_ = C;
+        uint64_t seed_ = seed;
+        const T* X_ = X;
+        void* args[] = {&X_, &n_, &nblk_, &bh0, &BHg, &cph, &C_, &chosen, &D2, &nearest, &cc2,
+                        &blocksum, &counter, &gen, &seed_, &cent, &err};
+        if (cudaLaunchCooperativeKernel((const void*)kpp_persistent_kernel<T, D>, dim3(grid),
+                                        dim3(kKppThreads), args, ccs_bytes, st) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
         count_launches(1);
     }
-    SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
 }
 
@@ -516,7 +609,7 @@ size_t assign_scratch_bytes(int BH, int C, int D, int dtype) {
 // Segment mean: one block per (cluster, head); a group of lanes per row moves
 // 16-byte chunks; fp32 partial sums are combined in a fixed order.
 // ---------------------------------------------------------------------------
-constexpr int kSmThreads = 128;
+constexpr int kSmThreads = 256;
 
 template <typename T, int D, bool GATHER>
 __global__ void __launch_bounds__(kSmThreads)
@@ -617,15 +710,15 @@ __global__ void permute_kernel(const T* __restrict__ X, const int32_t* __restric
 template <typename T, int D>
 static int kmeanspp_disp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
                          int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
-                         int32_t* counter, cudaStream_t st) {
+                         int32_t* counter, int32_t* gen, int* err, cudaStream_t st) {
     return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, cent, chosen, D2, nearest,
-                               cc2, bs, counter, st);
+                               cc2, bs, counter, gen, err, st);
 }
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
                     int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
-                    int32_t* counter, cudaStream_t st) {
+                    int32_t* counter, int32_t* gen, int* err, cudaStream_t st) {
     SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, cent, chosen, D2, nearest, cc2, bs,
-                    counter, st);
+                    counter, gen, err, st);
 }
 
 template <typename T, int D>
