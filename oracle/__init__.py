@@ -43,6 +43,8 @@ def lib():
         L.orc_segment_mean.argtypes = [P, i32, P, i32, P, P]
         L.orc_probe.argtypes = [P, i32, P, P, i64, i32, P, P, P, i32, f64, P, P]
         L.orc_route.argtypes = [P, P, i32, P, i32, i64, f32, P, P]
+        L.orc_route_budgets.argtypes = [P, P, i32, P, i32, P, P, P]
+        L.orc_topp_budget.argtypes = [P, i32, P, i32, i32, P, P, f64, f64, P, P]
         L.orc_attend.argtypes = [P, i64, P, P, i32, P, i32, P, i32, P, P, P, P,
                                  P, f64, P, i64, P, P]
         L.orc_num_threads.restype = i32
@@ -144,16 +146,38 @@ def probe(qbar, Kp, Vp, kbar, vbar, k_off, scale: float, with_scale=False):
     return (E, S) if with_scale else E
 
 
-def route(E, q_off, k_off, Nk: int, density: float):
-    """pair_off [Cq+1], pair_kc [nnz] from fp32 errors E [Cq, Ck]."""
+def route(E, q_off, k_off, Nk: int, density: float, budgets=None):
+    """pair_off [Cq+1], pair_kc [nnz] from fp32 errors E [Cq, Ck]; the budget
+    is floor(density * Nk) keys per query cluster, or budgets[i] when given."""
     E = np.ascontiguousarray(E, dtype=np.float32)
     q_off, k_off = _i32(q_off), _i32(k_off)
     Cq, Ck = E.shape
     pair_off = np.zeros(Cq + 1, dtype=np.int32)
     pair_kc = np.zeros(max(1, Cq * Ck), dtype=np.int32)
-    lib().orc_route(_p(E), _p(q_off), Cq, _p(k_off), Ck, int(Nk),
-                    ctypes.c_float(density), _p(pair_off), _p(pair_kc))
+    if budgets is None:
+        lib().orc_route(_p(E), _p(q_off), Cq, _p(k_off), Ck, int(Nk),
+                        ctypes.c_float(density), _p(pair_off), _p(pair_kc))
+    else:
+        b = np.ascontiguousarray(budgets, dtype=np.int64)
+        assert b.shape == (Cq,)
+        lib().orc_route_budgets(_p(E), _p(q_off), Cq, _p(k_off), Ck, _p(b), _p(pair_off),
+                                _p(pair_kc))
     return pair_off, pair_kc[:pair_off[-1]].copy()
+
+
+def topp_budget(qbar, kbar, q_off, k_off, p: float, scale: float):
+    """Per query cluster: keys of the key clusters holding p of the estimated
+    weight P' (budget int64 [Cq]) and the distance of the crossing from p
+    (margin float64 [Cq])."""
+    qbar, kbar = _f64(qbar), _f64(kbar)
+    q_off, k_off = _i32(q_off), _i32(k_off)
+    Cq, d = qbar.shape
+    Ck = kbar.shape[0]
+    budget = np.zeros(Cq, dtype=np.int64)
+    margin = np.zeros(Cq)
+    lib().orc_topp_budget(_p(qbar), Cq, _p(kbar), Ck, d, _p(q_off), _p(k_off), float(p),
+                          float(scale), _p(budget), _p(margin))
+    return budget, margin
 
 
 def attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm,

@@ -305,10 +305,11 @@ static int rank_before(float ra, int ca, float rb, int cb) {
     return ca < cb;
 }
 
-void orc_route(const float *E, const int32_t *q_off, int Cq, const int32_t *k_off,
-               int Ck, int64_t Nk, float density, int32_t *pair_off,
-               int32_t *pair_kc) {
-    int64_t budget = (int64_t)floor((double)density * (double)Nk);
+/* The greedy of orc_route with a budget per query cluster (budgets[i] keys,  */
+/* e.g. from orc_topp_budget); orc_route is the case of one budget for all.  */
+void orc_route_budgets(const float *E, const int32_t *q_off, int Cq,
+                       const int32_t *k_off, int Ck, const int64_t *budgets,
+                       int32_t *pair_off, int32_t *pair_kc) {
     int *order = (int *)malloc(sizeof(int) * (size_t)Ck);
     float *r = (float *)malloc(sizeof(float) * (size_t)Ck);
     unsigned char *take = (unsigned char *)malloc((size_t)Ck);
@@ -333,7 +334,7 @@ void orc_route(const float *E, const int32_t *q_off, int Cq, const int32_t *k_of
             }
             order[b + 1] = c;
         }
-        int64_t used = 0;
+        int64_t used = 0, budget = budgets[i];
         for (int a = 0; a < n; ++a) {
             int c = order[a];
             int64_t nc = k_off[c + 1] - k_off[c];
@@ -346,6 +347,86 @@ void orc_route(const float *E, const int32_t *q_off, int Cq, const int32_t *k_of
     free(order);
     free(r);
     free(take);
+}
+
+void orc_route(const float *E, const int32_t *q_off, int Cq, const int32_t *k_off,
+               int Ck, int64_t Nk, float density, int32_t *pair_off,
+               int32_t *pair_kc) {
+    int64_t budget = (int64_t)floor((double)density * (double)Nk);
+    int64_t *b = (int64_t *)malloc(sizeof(int64_t) * (size_t)(Cq > 0 ? Cq : 1));
+    for (int i = 0; i < Cq; ++i) b[i] = budget;
+    orc_route_budgets(E, q_off, Cq, k_off, Ck, b, pair_off, pair_kc);
+    free(b);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Top-p budget ([SVG2] section 3.4, "From pre-softmax scores to attention   */
+/* probability estimates" and "Top-p selection for dynamic budget           */
+/* allocation"; [BLOG] budget paragraph: per query cluster, the token pairs */
+/* of the blocks that hold p of the estimated weight).  For query cluster i: */
+/*   S_ij  = scale * qbar_i . kbar_j            (centroid score)             */
+/*   P'_ij = n_j e^{S_ij} / sum_l n_l e^{S_il}  (size-weighted, empty l: 0)  */
+/* key clusters in descending P' (ties: lower j first), taken until the     */
+/* running sum of P' reaches p; budget_i = the keys of the taken clusters   */
+/* (|Q_i| times that many token pairs).  An empty query cluster gets 0.     */
+/* margin_i: how far the running sum just before and at the last taken      */
+/* cluster lies from p (the smaller of the two; 1 if nothing was compared), */
+/* so a reimplementation in other rounding can be checked away from ties.   */
+/* Readings: "reaches" = at least p; e^{S - max S} is used (the ratio is    */
+/* unchanged); a NaN score takes no part.                                   */
+/* ------------------------------------------------------------------------ */
+void orc_topp_budget(const double *qbar, int Cq, const double *kbar, int Ck, int d,
+                     const int32_t *q_off, const int32_t *k_off, double p, double scale,
+                     int64_t *budget, double *margin) {
+    double *P = (double *)malloc(sizeof(double) * (size_t)Ck);
+    int *order = (int *)malloc(sizeof(int) * (size_t)Ck);
+    for (int i = 0; i < Cq; ++i) {
+        budget[i] = 0;
+        margin[i] = 1.0;
+        if (q_off[i + 1] == q_off[i]) continue;
+        double smax = -INFINITY;
+        for (int j = 0; j < Ck; ++j) {
+            P[j] = NAN;
+            if (k_off[j + 1] == k_off[j]) continue;
+            P[j] = scale * dot(qbar + (size_t)i * d, kbar + (size_t)j * d, d);
+            if (P[j] > smax) smax = P[j];
+        }
+        double Z = 0.0;
+        int n = 0;
+        for (int j = 0; j < Ck; ++j) {
+            if (isnan(P[j])) continue;
+            P[j] = (double)(k_off[j + 1] - k_off[j]) * exp(P[j] - smax);
+            Z += P[j];
+            order[n++] = j;
+        }
+        if (n == 0) continue;
+        for (int a = 0; a < n; ++a) P[order[a]] /= Z;
+        /* insertion sort: descending P', ties to the lower index */
+        for (int a = 1; a < n; ++a) {
+            int j = order[a], b = a - 1;
+            while (b >= 0 && (P[j] > P[order[b]])) {
+                order[b + 1] = order[b];
+                --b;
+            }
+            order[b + 1] = j;
+        }
+        double cum = 0.0;
+        int64_t keys = 0;
+        for (int a = 0; a < n; ++a) {
+            int j = order[a];
+            double before = cum;
+            cum += P[j];
+            keys += k_off[j + 1] - k_off[j];
+            if (cum >= p) {
+                double m1 = p - before, m2 = cum - p;
+                margin[i] = m1 < m2 ? m1 : m2;
+                break;
+            }
+        }
+        budget[i] = keys;
+    }
+    free(P);
+    free(order);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -468,3 +468,101 @@ def test_layer_at_density_one_equals_dense_attention():
     out = oracle.layer(Q, K, V, Cq=4, Ck=6, iters=3, density=1.0, scale=0.3,
                        seed_q=1, seed_k=2, stream=0)
     assert np.allclose(out["O"], softmax(Q @ K.T * 0.3, axis=-1) @ V, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Top-p budget (SVG2 summary, section 3.4, "Top-p selection for dynamic budget
+# allocation"; SVG-EAR blog, budget paragraph)
+# ---------------------------------------------------------------------------
+def _offsets(sizes):
+    return np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+
+
+def test_topp_identical_centroids_rank_clusters_by_size():
+    # every centroid scores the same, so P'_j = n_j / N: sizes 5, 1, 3, 1 hold
+    # 0.5, 0.1, 0.3, 0.1 of the weight; worked by hand
+    k_off = _offsets([5, 1, 3, 1])
+    q_off = np.array([0, 7], dtype=np.int32)
+    qbar = np.full((1, 8), 0.25)
+    kbar = np.full((4, 8), -0.5)
+    for p, want in ((0.5, 5), (0.55, 8), (0.8, 8), (0.85, 9), (0.95, 10), (1.0, 10), (0.01, 5)):
+        b, _ = oracle.topp_budget(qbar, kbar, q_off, k_off, p, 0.3)
+        assert b[0] == want, (p, b[0], want)
+
+
+def test_topp_dominant_cluster_alone_holds_the_mass():
+    g = np.random.default_rng(40)
+    d = 16
+    kbar = g.standard_normal((6, d)) * 0.1
+    kbar[3] = 4.0 * np.ones(d) / np.sqrt(d)          # the key cluster q points at
+    qbar = (4.0 * np.ones(d) / np.sqrt(d))[None]
+    k_off = _offsets([30, 30, 30, 2, 30, 30])        # small cluster, but e^{16} outweighs size
+    b, _ = oracle.topp_budget(qbar, kbar, np.array([0, 3]), k_off, 0.9, 1.0)
+    assert b[0] == 2
+    # with the score flipped the cluster is the least attended one
+    b, _ = oracle.topp_budget(-qbar, kbar, np.array([0, 3]), k_off, 0.9, 1.0)
+    assert b[0] > 0 and b[0] <= 150 and b[0] != 2
+
+
+def test_topp_p_one_takes_every_nonempty_cluster_and_empties_take_none():
+    g = np.random.default_rng(41)
+    sizes = np.array([4, 0, 7, 3, 0, 9, 1])
+    k_off = _offsets(sizes)
+    q_off = np.array([0, 5, 5, 9], dtype=np.int32)   # query cluster 1 is empty
+    qbar = g.standard_normal((3, 8)) * 0.3
+    kbar = g.standard_normal((7, 8)) * 0.3
+    b, _ = oracle.topp_budget(qbar, kbar, q_off, k_off, 1.0, 0.5)
+    assert list(b) == [sizes.sum(), 0, sizes.sum()]
+
+
+def test_topp_prefix_has_the_fewest_clusters_reaching_p_brute_force():
+    # the descending order makes the taken prefix the smallest number of key
+    # clusters whose weight reaches p: checked over every subset
+    import itertools
+    g = np.random.default_rng(42)
+    for trial in range(30):
+        Ck = 6
+        sizes = g.integers(1, 9, Ck)
+        k_off = _offsets(sizes)
+        qbar = g.standard_normal((1, 5))
+        kbar = g.standard_normal((Ck, 5))
+        p = float(g.uniform(0.2, 0.97))
+        b, margin = oracle.topp_budget(qbar, kbar, np.array([0, 4]), k_off, p, 0.7)
+        w = sizes * np.exp(0.7 * kbar @ qbar[0])
+        w = w / w.sum()
+        kmin = min(len(T) for r in range(1, Ck + 1) for T in itertools.combinations(range(Ck), r)
+                   if w[list(T)].sum() >= p - 1e-12)
+        # the prefix of that length: its sizes must sum to the budget
+        top = np.argsort(-w, kind="stable")[:kmin]
+        if margin[0] > 1e-9:
+            assert b[0] == sizes[top].sum(), (trial, b[0], sizes[top].sum())
+
+
+def test_topp_budget_grows_with_p():
+    g = np.random.default_rng(43)
+    sizes = g.integers(0, 20, 40)
+    k_off = _offsets(sizes)
+    qbar = g.standard_normal((3, 16)) * 0.5
+    kbar = g.standard_normal((40, 16)) * 0.5
+    q_off = np.array([0, 10, 20, 30], dtype=np.int32)
+    prev = np.zeros(3, dtype=np.int64)
+    for p in np.linspace(0.05, 1.0, 20):
+        b, _ = oracle.topp_budget(qbar, kbar, q_off, k_off, p, 0.25)
+        assert np.all(b >= prev)
+        prev = b
+    assert np.all(prev == sizes.sum())
+
+
+def test_route_with_budgets_equals_route_with_the_same_density_per_row():
+    g = np.random.default_rng(44)
+    Cq, Ck, Nk = 5, 12, 100
+    sizes = g.multinomial(Nk, np.ones(Ck) / Ck)
+    k_off = _offsets(sizes)
+    q_off = _offsets([3, 0, 4, 2, 5])
+    E = g.random((Cq, Ck)).astype(np.float32)
+    budgets = np.array([0, 37, 55, 100, 12], dtype=np.int64)
+    off, kc = oracle.route(E, q_off, k_off, Nk, 0.5, budgets=budgets)
+    for i in range(Cq):
+        o1, k1 = oracle.route(E[i:i + 1], q_off[i:i + 2] - q_off[i], k_off, Nk,
+                              (budgets[i] + 0.5) / Nk)
+        assert np.array_equal(kc[off[i]:off[i + 1]], k1)
