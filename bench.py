@@ -43,6 +43,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="wan720p", choices=sorted(synth.WORKLOADS))
     p.add_argument("--density", type=float, default=None)
+    p.add_argument("--topp", type=float, default=None,
+                   help="routing budget per query cluster from the key clusters holding this "
+                        "share of the estimated weight (instead of a fixed density)")
     p.add_argument("--iters", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -164,7 +167,7 @@ def attention_work(q_off, k_off, pair_off, pair_kc, d):
 # ---------------------------------------------------------------------------
 # CPU oracle on a bounded sample, extrapolated to one layer call
 # ---------------------------------------------------------------------------
-def oracle_sample_ms(w, seconds=15.0, density=None, iters=None):
+def oracle_sample_ms(w, seconds=15.0, density=None, iters=None, topp=None):
     """Time the oracle's steps on one head's data with reduced counts, each
     scaled by the ratio of full to sampled work, and return (ms per layer
     call, threads, description).  Setup (inputs, one clustering) is untimed."""
@@ -212,7 +215,13 @@ def oracle_sample_ms(w, seconds=15.0, density=None, iters=None):
     t, Es = timed(lambda: oracle.probe(cent_q[:npr], Kp, Vp, cent_k, vbar, ok, w.scale))
     timings["probe"] = t * w.Cq / npr
     E = np.concatenate([Es, np.tile(Es, (w.Cq // npr + 1, 1))[:w.Cq - npr]], 0)
-    t, (po, pkc) = timed(lambda: oracle.route(E.astype(np.float32), oq, ok, N, density))
+    if topp is None:
+        t, (po, pkc) = timed(lambda: oracle.route(E.astype(np.float32), oq, ok, N, density))
+    else:
+        def topp_route():
+            b, _ = oracle.topp_budget(cent_q, cent_k, oq, ok, topp, w.scale)
+            return oracle.route(E.astype(np.float32), oq, ok, N, 1.0, budgets=b)
+        t, (po, pkc) = timed(topp_route)
     timings["route"] = t
     nr = max(32, int(256 * frac))
     rows = g.choice(N, nr, replace=False)
@@ -270,12 +279,13 @@ def run_reference(args, w):
     oracle.lib()
     secs = min(args.cpu_sample_seconds, 8.0)
     for _ in range(args.warmup):
-        oracle_sample_ms(w, seconds=secs * 0.3, density=args.density, iters=args.iters)
+        oracle_sample_ms(w, seconds=secs * 0.3, density=args.density, iters=args.iters,
+                         topp=args.topp)
     vals = []
     desc = ""
     cores = 1
     for _ in range(args.steps):
-        v, cores, desc, _ = oracle_sample_ms(w, seconds=secs, density=args.density,
+        v, cores, desc, _ = oracle_sample_ms(w, seconds=secs, density=args.density, topp=args.topp,
                                              iters=args.iters)
         vals.append(v)
     value = float(np.mean(vals))
@@ -293,7 +303,10 @@ def run_reference(args, w):
 
 def workload_config(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
-            "iters": args.iters or w.iters, "density": args.density or w.density,
+            "iters": args.iters or w.iters,
+            "budget": ("top-p %g of the estimated weight per query cluster" % args.topp
+                       if args.topp else "density %g (floor(density * N) keys per query cluster)"
+                       % (args.density or w.density)),
             "kmeans_init": "k-means++ (cold)", "inputs": "bf16, seeded Gaussian mixtures",
             "l2": "inputs larger than L2 (3 x %.0f MB)" % (w.B * w.H * w.N * w.d * 2 / 1e6),
             "parallelism": "one independent layer call per GPU (no exchange)"}
@@ -356,8 +369,12 @@ def main():
         Vp = csa.svgear_permute(V, ck.perm)
         vbar = csa.svgear_centroids(Vp, ck.offsets, w.Ck)
         mark(3)
-        po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
-                                  Vp, density, w.scale)
+        if args.topp:
+            po, pk, _ = csa.svgear_route_topp(cq.centroids, cq.offsets, ck.centroids, vbar,
+                                              ck.offsets, ck.Xp, Vp, args.topp, w.scale)
+        else:
+            po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
+                                      ck.Xp, Vp, density, w.scale)
         mark(4)
         O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids,
                               vbar, cq.perm, w.scale)
@@ -441,7 +458,7 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, cores, desc, parts = oracle_sample_ms(w, seconds=args.cpu_sample_seconds,
-                                                 density=density, iters=iters)
+                                                 density=density, iters=iters, topp=args.topp)
         cpu = {"value": v, "unit": "ms", "cores": cores, "kind": "oracle", "sample": desc,
                "stages_ms": parts}
 

@@ -22,6 +22,7 @@ NOALLOC_SORT_SCRATCH_INTS = 2 * 1024 * 1024
 F32, BF16 = 0, 1
 OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
 OP_KMEANS_ASSIGN = 6
+OP_ROUTE_TOPP = 7
 MAX_CLUSTERS = 4096
 
 EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
@@ -29,7 +30,8 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_centroids", "svgear_probe", "svgear_route_select", "svgear_route",
             "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
             "svgear_version", "svgear_kernel_launches", "svgear_attend_status",
-            "svgear_device_status",
+            "svgear_device_status", "svgear_topp_budget", "svgear_route_select_budget",
+            "svgear_route_topp",
             "svgear_label_sort_noalloc")
 
 
@@ -69,6 +71,9 @@ def lib():
         "svgear_probe": [P, I32, P, P, P, P, P, I32, Dims, F, P, P, SZ, P],
         "svgear_route_select": [P, P, I32, P, I32, I32, I32, I32, F, P, P, P, SZ, P],
         "svgear_route": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, SZ, P],
+        "svgear_topp_budget": [P, P, I32, P, P, I32, I32, I32, I32, I32, F, F, P, P],
+        "svgear_route_select_budget": [P, P, I32, P, I32, I32, I32, I32, P, P, P, P, SZ, P],
+        "svgear_route_topp": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, P, SZ, P],
         "svgear_attend": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, P, SZ, P],
         "svgear_workspace_bytes": [I32, Dims, I32, I32],
         "svgear_status_string": [ctypes.c_int],
@@ -277,6 +282,52 @@ def svgear_route_select(E, q_off, k_off, Nk, density):
     return pair_off, pair_kc
 
 
+def svgear_topp_budget(qbar, q_off, kbar, k_off, Nk, p, scale):
+    """Keys per query cluster holding p of the estimated weight: int32 [B, H, Cq]."""
+    _cuda(qbar, "qbar", torch.float32)
+    _cuda(kbar, "kbar", torch.float32)
+    B, H, Cq, d = qbar.shape
+    Ck = kbar.shape[2]
+    budget = torch.empty((B, H, Cq), dtype=torch.int32, device=qbar.device)
+    _check("svgear_topp_budget", lib().svgear_topp_budget(
+        _ptr(qbar), _ptr(q_off), Cq, _ptr(kbar), _ptr(k_off), Ck, B, H, d, int(Nk), float(p),
+        float(scale), _ptr(budget), _stream()))
+    return budget
+
+
+def svgear_route_select_budget(E, q_off, k_off, Nk, budget):
+    _cuda(E, "E", torch.float32)
+    _cuda(budget, "budget", torch.int32)
+    B, H, Cq, Ck = E.shape
+    pair_off = torch.empty((B, H, Cq + 1), dtype=torch.int32, device=E.device)
+    pair_kc = torch.empty((B, H, Cq * Ck), dtype=torch.int32, device=E.device)
+    ws, n = _workspace(OP_ROUTE, Dims(B, H, Nk, 64, F32), Cq, Ck, E.device)
+    _check("svgear_route_select_budget", lib().svgear_route_select_budget(
+        _ptr(E), _ptr(q_off), Cq, _ptr(k_off), Ck, B, H, Nk, _ptr(budget), _ptr(pair_off),
+        _ptr(pair_kc), _ptr(ws), n, _stream()))
+    return pair_off, pair_kc
+
+
+def svgear_route_topp(qbar, q_off, kbar, vbar, k_off, Kp, Vp, p, scale, return_errors=False):
+    """Probe, top-p budget and greedy selection; returns (pair_off, pair_kc,
+    budget[, E])."""
+    kd = _tokens(Kp, "Kp")
+    _tokens(Vp, "Vp")
+    B, H, Cq, d = qbar.shape
+    Ck = kbar.shape[2]
+    dev = Kp.device
+    pair_off = torch.empty((B, H, Cq + 1), dtype=torch.int32, device=dev)
+    pair_kc = torch.empty((B, H, Cq * Ck), dtype=torch.int32, device=dev)
+    budget = torch.empty((B, H, Cq), dtype=torch.int32, device=dev)
+    E = torch.empty((B, H, Cq, Ck), dtype=torch.float32, device=dev) if return_errors else None
+    ws, n = _workspace(OP_ROUTE_TOPP, kd, Cq, Ck, dev)
+    _check("svgear_route_topp", lib().svgear_route_topp(
+        _ptr(qbar), _ptr(q_off), Cq, _ptr(kbar), _ptr(vbar), _ptr(k_off), Ck, _ptr(Kp), _ptr(Vp),
+        kd, float(p), float(scale), _ptr(pair_off), _ptr(pair_kc), _ptr(E), _ptr(budget),
+        _ptr(ws), n, _stream()))
+    return (pair_off, pair_kc, budget, E) if return_errors else (pair_off, pair_kc, budget)
+
+
 def svgear_route(qbar, q_off, kbar, vbar, k_off, Kp, Vp, density, scale, return_errors=False):
     kd = _tokens(Kp, "Kp")
     _tokens(Vp, "Vp")
@@ -316,19 +367,27 @@ def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_per
     return O
 
 
-def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None):
+def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None,
+          topp=None):
     """The whole layer for [B, H, N, d] tensors: cluster Q and K (seeds 2*seed
-    and 2*seed+1), permute V, value centroids, route, attend.  Returns O in the
-    original token order and every intermediate."""
+    and 2*seed+1), permute V, value centroids, route, attend.  The routing
+    budget is floor(density * N) keys per query cluster, or, with topp=p, the
+    keys holding p of the estimated weight (density is then unused).  Returns
+    O in the original token order and every intermediate."""
     d = Q.shape[-1]
     scale = d ** -0.5 if scale is None else scale
     cq = svgear_cluster(Q, Cq, iters, warm_q, seed=2 * seed)
     ck = svgear_cluster(K, Ck, iters, warm_k, seed=2 * seed + 1)
     Vp = svgear_permute(V, ck.perm)
     vbar = svgear_centroids(Vp, ck.offsets, Ck)
-    pair_off, pair_kc = svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
-                                     ck.Xp, Vp, density, scale)
+    budget = None
+    if topp is None:
+        pair_off, pair_kc = svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
+                                         ck.Xp, Vp, density, scale)
+    else:
+        pair_off, pair_kc, budget = svgear_route_topp(cq.centroids, cq.offsets, ck.centroids, vbar,
+                                                      ck.offsets, ck.Xp, Vp, topp, scale)
     O = svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, pair_off, pair_kc, ck.centroids,
                       vbar, cq.perm, scale)
     return {"O": O, "q": cq, "k": ck, "Vp": Vp, "vbar": vbar, "pair_off": pair_off,
-            "pair_kc": pair_kc}
+            "pair_kc": pair_kc, "budget": budget}

@@ -205,6 +205,11 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
             carve_route(cv, bh_of(dims), C1, C2);
             break;
+        case SVGEAR_OP_ROUTE_TOPP:
+            if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
+            carve_route(cv, bh_of(dims), C1, C2);
+            cv.take<int32_t>(bh_of(dims) * C1);
+            break;
         case SVGEAR_OP_ATTEND:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
             carve_attend(cv, dims, C1, C2);
@@ -399,8 +404,8 @@ int svgear_route_select(const float* E, const int32_t* q_off, int32_t Cq, const 
     Carve cv(ws);
     SelWs w = carve_select(cv, BH, Cq, Ck);
     const long long budget = (long long)floor((double)density * (double)Nk);
-    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)BH, budget, w.lists, w.counts,
-                               pair_off, pair_kc, static_cast<cudaStream_t>(stream));
+    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)BH, budget, nullptr, w.lists,
+                               w.counts, pair_off, pair_kc, static_cast<cudaStream_t>(stream));
 }
 
 int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq, const float* kbar,
@@ -423,7 +428,72 @@ int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq, const floa
     if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, st)))
         return s;
     const long long budget = (long long)floor((double)density * (double)kdims.N);
-    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)bh_of(kdims), budget, w.sel.lists,
+    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)bh_of(kdims), budget, nullptr,
+                               w.sel.lists, w.sel.counts, pair_off, pair_kc, st);
+}
+
+int svgear_topp_budget(const float* qbar, const int32_t* q_off, int32_t Cq, const float* kbar,
+                       const int32_t* k_off, int32_t Ck, int32_t B, int32_t H, int32_t d,
+                       int32_t Nk, float p, float scale, int32_t* budget, void* stream) {
+    if (B < 0 || H < 0 || Nk < 1) return SVGEAR_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SVGEAR_ERR_UNSUPPORTED;
+    const size_t BH = (size_t)B * H;
+    if (BH > 65535) return SVGEAR_ERR_UNSUPPORTED;
+    int s = check_route_common(Cq, Ck, Nk, p);
+    if (s) return s;
+    if (!qbar || !q_off || !kbar || !k_off || !budget || !isfinite(scale)) return SVGEAR_ERR_INVALID_ARG;
+    if (BH == 0) return SVGEAR_OK;
+    return launch_topp_budget(qbar, q_off, Cq, kbar, k_off, Ck, (int)BH, d, (double)p,
+                              (double)scale, budget, static_cast<cudaStream_t>(stream));
+}
+
+int svgear_route_select_budget(const float* E, const int32_t* q_off, int32_t Cq,
+                               const int32_t* k_off, int32_t Ck, int32_t B, int32_t H,
+                               int32_t Nk, const int32_t* budget, int32_t* pair_off,
+                               int32_t* pair_kc, void* ws, size_t ws_bytes, void* stream) {
+    if (B < 0 || H < 0 || Nk < 1) return SVGEAR_ERR_INVALID_ARG;
+    const size_t BH = (size_t)B * H;
+    if (BH > 65535) return SVGEAR_ERR_UNSUPPORTED;
+    int s = check_route_common(Cq, Ck, Nk, 1.f);
+    if (s) return s;
+    if (!E || !q_off || !k_off || !budget || !pair_off || !pair_kc || !ws)
+        return SVGEAR_ERR_INVALID_ARG;
+    Carve need(nullptr);
+    carve_select(need, BH, Cq, Ck);
+    if (ws_bytes < need.off + kAlign) return SVGEAR_ERR_WORKSPACE;
+    if (BH == 0) return SVGEAR_OK;
+    Carve cv(ws);
+    SelWs w = carve_select(cv, BH, Cq, Ck);
+    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)BH, 0, budget, w.lists, w.counts,
+                               pair_off, pair_kc, static_cast<cudaStream_t>(stream));
+}
+
+int svgear_route_topp(const float* qbar, const int32_t* q_off, int32_t Cq, const float* kbar,
+                      const float* vbar, const int32_t* k_off, int32_t Ck, const void* Kp,
+                      const void* Vp, svgear_dims kdims, float p, float scale, int32_t* pair_off,
+                      int32_t* pair_kc, float* E_out, int32_t* budget_out, void* ws,
+                      size_t ws_bytes, void* stream) {
+    int s = check_dims(kdims);
+    if (s) return s;
+    if ((s = check_route_common(Cq, Ck, kdims.N, p))) return s;
+    if (!qbar || !q_off || !kbar || !vbar || !k_off || !Kp || !Vp || !pair_off || !pair_kc ||
+        !ws || !aligned16(Kp) || !aligned16(Vp) || !isfinite(scale))
+        return SVGEAR_ERR_INVALID_ARG;
+    if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ROUTE_TOPP, kdims, Cq, Ck))
+        return SVGEAR_ERR_WORKSPACE;
+    if (bh_of(kdims) == 0) return SVGEAR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Carve cv(ws);
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
+    int32_t* bud = cv.take<int32_t>(bh_of(kdims) * Cq);
+    if (budget_out) bud = budget_out;
+    float* E = E_out ? E_out : w.E;
+    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, st)))
+        return s;
+    if ((s = launch_topp_budget(qbar, q_off, Cq, kbar, k_off, Ck, (int)bh_of(kdims), kdims.d,
+                                (double)p, (double)scale, bud, st)))
+        return s;
+    return launch_route_select(E, q_off, Cq, k_off, Ck, (int)bh_of(kdims), 0, bud, w.sel.lists,
                                w.sel.counts, pair_off, pair_kc, st);
 }
 

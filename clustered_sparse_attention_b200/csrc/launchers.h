@@ -54,10 +54,13 @@ int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp,
                  const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
                  svgear_dims kdims, float scale, float* E, uint32_t* rowmax,
                  cudaStream_t st);
-int launch_route_select(const float* E, const int32_t* q_off, int Cq,
-                        const int32_t* k_off, int Ck, int BH, long long budget,
-                        int32_t* lists, int32_t* counts, int32_t* pair_off,
-                        int32_t* pair_kc, cudaStream_t st);
+int launch_route_select(const float* E, const int32_t* q_off, int Cq, const int32_t* k_off,
+                        int Ck, int BH, long long budget, const int32_t* budgets, int32_t* lists,
+                        int32_t* counts, int32_t* pair_off, int32_t* pair_kc, cudaStream_t st);
+// Top-p budget per query cluster (keys), budget int32 [BH][Cq].
+int launch_topp_budget(const float* qbar, const int32_t* q_off, int Cq, const float* kbar,
+                       const int32_t* k_off, int Ck, int BH, int D, double p, double scale,
+                       int32_t* budget, cudaStream_t st);
 
 // attend_sm100.cu: workspace of the tensor-core attention
 struct AttendWs {

@@ -272,8 +272,9 @@ constexpr int kRtThreads = 256;
 
 __global__ void __launch_bounds__(kRtThreads)
 route_select_kernel(const float* __restrict__ E, const int32_t* __restrict__ q_off, int Cq,
-                    const int32_t* __restrict__ k_off, int Ck, long long budget,
-                    int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
+                    const int32_t* __restrict__ k_off, int Ck, long long budget_all,
+                    const int32_t* __restrict__ budgets, int32_t* __restrict__ lists,
+                    int32_t* __restrict__ counts) {
     extern __shared__ __align__(8) unsigned char smraw[];
     const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     int P2 = 1;
@@ -325,6 +326,7 @@ route_select_kernel(const float* __restrict__ E, const int32_t* __restrict__ q_o
         }
     }
     if (tid == 0) {
+        const long long budget = budgets ? (long long)budgets[(size_t)bh * Cq + i] : budget_all;
         long long used = 0;
         for (int x = 0; x < Ck; ++x) {
             const unsigned long long kk = key[x];
@@ -375,8 +377,8 @@ __global__ void route_compact_kernel(const int32_t* __restrict__ lists,
 }
 
 int launch_route_select(const float* E, const int32_t* q_off, int Cq, const int32_t* k_off,
-                        int Ck, int BH, long long budget, int32_t* lists, int32_t* counts,
-                        int32_t* pair_off, int32_t* pair_kc, cudaStream_t st) {
+                        int Ck, int BH, long long budget, const int32_t* budgets, int32_t* lists,
+                        int32_t* counts, int32_t* pair_off, int32_t* pair_kc, cudaStream_t st) {
     int P2 = 1;
     while (P2 < Ck) P2 <<= 1;
     const size_t sm = sizeof(unsigned long long) * P2 + sizeof(int32_t) * Ck + Ck + 16;
@@ -385,10 +387,142 @@ int launch_route_select(const float* E, const int32_t* q_off, int Cq, const int3
                              (int)sm) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
     route_select_kernel<<<dim3(Cq, BH), kRtThreads, sm, st>>>(E, q_off, Cq, k_off, Ck, budget,
-                                                              lists, counts);
+                                                              budgets, lists, counts);
     count_launches(1);
     route_compact_kernel<<<BH, 256, sizeof(int32_t) * (Cq + 1), st>>>(lists, counts, Cq, Ck,
                                                                        pair_off, pair_kc);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+
+// ---------------------------------------------------------------------------
+// Top-p budget (SVG2 summary, section 3.4, "From pre-softmax scores to
+// attention probability estimates" and "Top-p selection for dynamic budget
+// allocation"; SVG-EAR blog, budget paragraph): per query cluster i, the keys
+// of the key clusters that hold p of the size-weighted centroid estimate
+//   P'_ij = n_j e^{S_ij} / sum_l n_l e^{S_il},   S_ij = scale * qbar_i . kbar_j,
+// taken in descending P' (ties: lower j) until the running sum reaches p.
+// One block per (query cluster, head), in fp64 throughout: S (the centroids
+// are fp32), w_j = n_j e^{S_ij - max S}, a bitonic sort of (w, j), and the
+// running sum compared with p * sum(w), both summed in sorted order.  Empty
+// key clusters and NaN scores take no part; an empty query cluster gets 0.
+// ---------------------------------------------------------------------------
+constexpr int kTpThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kTpThreads)
+topp_budget_kernel(const float* __restrict__ qbar, const int32_t* __restrict__ q_off, int Cq,
+                   const float* __restrict__ kbar, const int32_t* __restrict__ k_off, int Ck,
+                   double p, double scale, int32_t* __restrict__ budget) {
+    extern __shared__ __align__(8) unsigned char smraw[];
+    __shared__ double q[D];
+    __shared__ double red[kTpThreads / 32];
+    const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    int P2 = 1;
+    while (P2 < Ck) P2 <<= 1;
+    double* w = reinterpret_cast<double*>(smraw);          // [P2]
+    int32_t* idx = reinterpret_cast<int32_t*>(w + P2);     // [P2]
+    int32_t* nsz = idx + P2;                                // [Ck]
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    if (qo[i + 1] <= qo[i]) {
+        if (tid == 0) budget[(size_t)bh * Cq + i] = 0;
+        return;
+    }
+    const int32_t* ko = k_off + (size_t)bh * (Ck + 1);
+    for (int k = tid; k < D; k += kTpThreads) q[k] = (double)qbar[((size_t)bh * Cq + i) * D + k];
+    __syncthreads();
+    double mx = -INFINITY;
+    for (int c = tid; c < P2; c += kTpThreads) {
+        double sc = NAN;
+        if (c < Ck) {
+            const int n = ko[c + 1] - ko[c];
+            nsz[c] = n;
+            if (n > 0) {
+                const float* kr = kbar + ((size_t)bh * Ck + c) * D;
+                double acc = 0.0;
+                for (int k = 0; k < D; ++k) acc = fma(q[k], (double)kr[k], acc);
+                sc = scale * acc;
+                if (sc > mx) mx = sc;
+            }
+        }
+        w[c] = sc;
+        idx[c] = c;
+    }
+    // block max of the scores
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        double m = red[0];
+        for (int k = 1; k < kTpThreads / 32; ++k) m = fmax(m, red[k]);
+        red[0] = m;
+    }
+    __syncthreads();
+    const double smax = red[0];
+    // weights; excluded entries get -1 and sort last
+    for (int c = tid; c < P2; c += kTpThreads) {
+        const double sc = w[c];
+        w[c] = (c < Ck && sc == sc) ? (double)nsz[c] * exp(sc - smax) : -1.0;
+    }
+    __syncthreads();
+    // bitonic sort: descending w, ties to the lower index
+    for (int k = 2; k <= P2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int x = tid; x < P2; x += kTpThreads) {
+                const int y = x ^ j;
+                if (y > x) {
+                    const double wa = w[x], wb = w[y];
+                    const int ia = idx[x], ib = idx[y];
+                    const bool a_first = wa > wb || (wa == wb && ia < ib);
+                    const bool up = (x & k) == 0;
+                    if (a_first != up) {
+                        w[x] = wb; w[y] = wa;
+                        idx[x] = ib; idx[y] = ia;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (tid == 0) {
+        double total = 0.0;
+        for (int x = 0; x < Ck && w[x] >= 0.0; ++x) total += w[x];
+        const double target = p * total;
+        double cum = 0.0;
+        long long keys = 0;
+        for (int x = 0; x < Ck && w[x] >= 0.0; ++x) {
+            cum += w[x];
+            keys += nsz[idx[x]];
+            if (cum >= target) break;
+        }
+        budget[(size_t)bh * Cq + i] = (int32_t)keys;
+    }
+}
+
+int launch_topp_budget(const float* qbar, const int32_t* q_off, int Cq, const float* kbar,
+                       const int32_t* k_off, int Ck, int BH, int D, double p, double scale,
+                       int32_t* budget, cudaStream_t st) {
+    int P2 = 1;
+    while (P2 < Ck) P2 <<= 1;
+    const size_t sm = (sizeof(double) + sizeof(int32_t)) * P2 + sizeof(int32_t) * Ck + 16;
+    if (D == 128) {
+        if (sm > 48 * 1024 && cudaFuncSetAttribute(topp_budget_kernel<128>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)sm) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        topp_budget_kernel<128><<<dim3(Cq, BH), kTpThreads, sm, st>>>(qbar, q_off, Cq, kbar, k_off,
+                                                                      Ck, p, scale, budget);
+    } else {
+        if (sm > 48 * 1024 && cudaFuncSetAttribute(topp_budget_kernel<64>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)sm) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        topp_budget_kernel<64><<<dim3(Cq, BH), kTpThreads, sm, st>>>(qbar, q_off, Cq, kbar, k_off,
+                                                                     Ck, p, scale, budget);
+    }
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;

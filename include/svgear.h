@@ -88,7 +88,8 @@ typedef enum {
     SVGEAR_OP_KMEANS_UPDATE = 3,
     SVGEAR_OP_ROUTE = 4,
     SVGEAR_OP_ATTEND = 5,
-    SVGEAR_OP_KMEANS_ASSIGN = 6
+    SVGEAR_OP_KMEANS_ASSIGN = 6,
+    SVGEAR_OP_ROUTE_TOPP = 7
 } svgear_op;
 
 /* Largest cluster count any call accepts (shared-memory tables). */
@@ -239,6 +240,50 @@ int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq,
                  int32_t Ck, const void* Kp, const void* Vp, svgear_dims kdims,
                  float density, float scale, int32_t* pair_off, int32_t* pair_kc,
                  float* E_out, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_topp_budget -- the per-query-cluster budget that holds p of the
+ * estimated attention weight ([SVG2] section 3.4, "From pre-softmax scores to
+ * attention probability estimates" and "Top-p selection for dynamic budget
+ * allocation"; [BLOG] budget paragraph: the token pairs of the blocks that
+ * hold 90% of the estimated weight).  For every non-empty query cluster i:
+ *   S_ij  = scale * qbar_i . kbar_j
+ *   P'_ij = n_j e^{S_ij} / sum_l n_l e^{S_il}        (n_j = |K_j|)
+ * the non-empty key clusters in descending P' (ties: lower j), taken until
+ * the running sum of P' reaches p (at least p); budget[i] = the keys of the
+ * taken clusters (|Q_i| * budget[i] token pairs).  fp64 throughout, summed in
+ * the sorted order; NaN scores take no part; an empty query cluster gets 0.
+ *   qbar, kbar  float[B][H][Cq][d], float[B][H][Ck][d] centroids.
+ *   q_off, k_off int32 segments ([B][H][Cq+1], [B][H][Ck+1]); Nk = keys.
+ *   p           in (0, 1].
+ *   budget      out int32[B][H][Cq].
+ * No workspace; asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+int svgear_topp_budget(const float* qbar, const int32_t* q_off, int32_t Cq,
+                       const float* kbar, const int32_t* k_off, int32_t Ck, int32_t B,
+                       int32_t H, int32_t d, int32_t Nk, float p, float scale,
+                       int32_t* budget, void* stream);
+
+/* svgear_route_select with a budget per query cluster: budget int32[B][H][Cq]
+ * keys (e.g. from svgear_topp_budget) in place of floor(density * Nk); the
+ * greedy, ordering and outputs are those of svgear_route_select.  ws as for
+ * svgear_route_select. */
+int svgear_route_select_budget(const float* E, const int32_t* q_off, int32_t Cq,
+                               const int32_t* k_off, int32_t Ck, int32_t B, int32_t H,
+                               int32_t Nk, const int32_t* budget, int32_t* pair_off,
+                               int32_t* pair_kc, void* ws, size_t ws_bytes, void* stream);
+
+/* svgear_route_topp -- probe + top-p budget + select in one call: SVG-EAR
+ * spends the pairs of the blocks that hold p of the estimated weight on the
+ * blocks with the most error per pair ([BLOG] budget paragraph).  E_out and
+ * budget_out (int32[B][H][Cq]) may be NULL (then they live in the workspace,
+ * svgear_workspace_bytes(SVGEAR_OP_ROUTE_TOPP, kdims, Cq, Ck)). */
+int svgear_route_topp(const float* qbar, const int32_t* q_off, int32_t Cq,
+                      const float* kbar, const float* vbar, const int32_t* k_off,
+                      int32_t Ck, const void* Kp, const void* Vp, svgear_dims kdims,
+                      float p, float scale, int32_t* pair_off, int32_t* pair_kc,
+                      float* E_out, int32_t* budget_out, void* ws, size_t ws_bytes,
+                      void* stream);
 
 /* --------------------------------------------------------------------------
  * svgear_attend -- exact selected blocks plus centroid compensation in one

@@ -230,16 +230,21 @@ def cluster(X, C: int, iters: int, seed: int, stream: int, warm=None):
 
 
 def layer(Q, K, V, Cq: int, Ck: int, iters: int, density: float, scale: float,
-          seed_q: int, seed_k: int, stream: int, warm_q=None, warm_k=None):
-    """One head of the layer, every intermediate returned."""
+          seed_q: int, seed_k: int, stream: int, warm_q=None, warm_k=None, topp=None):
+    """One head of the layer, every intermediate returned; with topp=p the
+    routing budget per query cluster is topp_budget's (density unused)."""
     cq = cluster(Q, Cq, iters, seed_q, stream, warm_q)
     ck = cluster(K, Ck, iters, seed_k, stream, warm_k)
     Vp = _f64(V)[ck["perm"]]
     vbar = segment_mean(Vp, ck["offsets"])
     E = probe(cq["centroids"], ck["Xp"], Vp, ck["centroids"], vbar, ck["offsets"], scale)
+    budgets = None
+    if topp is not None:
+        budgets, _ = topp_budget(cq["centroids"], ck["centroids"], cq["offsets"], ck["offsets"],
+                                 topp, scale)
     pair_off, pair_kc = route(E.astype(np.float32), cq["offsets"], ck["offsets"],
-                              K.shape[0], density)
+                              K.shape[0], density if topp is None else 1.0, budgets=budgets)
     O, lse = attend(cq["Xp"], ck["Xp"], Vp, cq["offsets"], ck["offsets"], pair_off,
                     pair_kc, ck["centroids"], vbar, cq["perm"], scale)
     return {"q": cq, "k": ck, "Vp": Vp, "vbar": vbar, "E": E, "pair_off": pair_off,
-            "pair_kc": pair_kc, "O": O, "lse": lse}
+            "pair_kc": pair_kc, "O": O, "lse": lse, "budgets": budgets}

@@ -151,3 +151,23 @@ def test_fullsize_attention_on_sampled_rows(run):
         dst = cq.perm.cpu().numpy()[0, h][rows]
         Og = np64(O[0, h][torch.from_numpy(dst).cuda()])
         assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2
+
+
+def test_fullsize_topp_budget_and_routing(run):
+    csa = run["csa"]
+    cq, ck = run["cq"], run["ck"]
+    budget = csa.svgear_topp_budget(cq.centroids, cq.offsets, ck.centroids, ck.offsets, W.N, 0.9,
+                                    W.scale)
+    po, pk = csa.svgear_route_select_budget(run["E"], cq.offsets, ck.offsets, W.N, budget)
+    b = budget.cpu().numpy()
+    qb, kb = cq.centroids.cpu().numpy(), ck.centroids.cpu().numpy()
+    qo, ko = cq.offsets.cpu().numpy(), ck.offsets.cpu().numpy()
+    E = run["E"].cpu().numpy()
+    for h in HEADS:
+        ref, margin = oracle.topp_budget(qb[0, h], kb[0, h], qo[0, h], ko[0, h], 0.9, W.scale)
+        bad = np.nonzero(ref != b[0, h])[0]
+        assert all(margin[i] < 1e-9 for i in bad) and len(bad) <= 1
+        ref_off, ref_kc = oracle.route(E[0, h], qo[0, h], ko[0, h], W.N, 1.0,
+                                       budgets=b[0, h].astype(np.int64))
+        assert np.array_equal(po.cpu().numpy()[0, h], ref_off)
+        assert np.array_equal(pk.cpu().numpy()[0, h][:ref_off[-1]], ref_kc)

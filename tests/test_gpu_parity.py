@@ -473,3 +473,79 @@ def test_cluster_fixed_point_gives_the_same_result_as_more_rounds():
         assert torch.equal(getattr(a, f), getattr(b, f)), f
     for h in range(w.H):
         check_assign(host["k"][0, h], b.centroids.cpu().numpy()[0, h], b.labels.cpu().numpy()[0, h])
+
+
+# ---------------------------------------------------------------------------
+# Top-p budget (SVG2 summary, section 3.4, top-p selection; SVG-EAR blog,
+# budget paragraph)
+# ---------------------------------------------------------------------------
+def _check_budgets(gpu, qbar, kbar, q_off, k_off, p, scale):
+    """GPU budgets equal the oracle's except where the running weight crosses
+    p within fp64 rounding of it (counted and returned)."""
+    ref, margin = oracle.topp_budget(qbar, kbar, q_off, k_off, p, scale)
+    bad = np.nonzero(ref != gpu)[0]
+    for i in bad:
+        assert margin[i] < 1e-9, (i, int(gpu[i]), int(ref[i]), margin[i])
+    return len(bad)
+
+
+@pytest.mark.parametrize("p", [0.3, 0.9, 1.0])
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64, EAR_COUNTS], ids=lambda w: w.name)
+def test_topp_budget_matches_oracle(w, p):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    budget = csa.svgear_topp_budget(cq.centroids, cq.offsets, ck.centroids, ck.offsets, w.N, p,
+                                    w.scale).cpu().numpy()
+    qb, kb = cq.centroids.cpu().numpy(), ck.centroids.cpu().numpy()
+    qo, ko = cq.offsets.cpu().numpy(), ck.offsets.cpu().numpy()
+    flips = sum(_check_budgets(budget[0, h], qb[0, h], kb[0, h], qo[0, h], ko[0, h], p, w.scale)
+                for h in range(w.H))
+    assert flips <= 1
+    if p == 1.0:
+        nonempty_rows = np.diff(qo, axis=-1) > 0
+        assert np.all(budget[nonempty_rows] == w.N)
+
+
+@pytest.mark.parametrize("w", [SMALL_BF16, EAR_COUNTS], ids=lambda w: w.name)
+def test_route_topp_bit_exact_given_gpu_errors_and_budgets(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    po, pk, budget, E = csa.svgear_route_topp(cq.centroids, cq.offsets, ck.centroids, vbar,
+                                              ck.offsets, ck.Xp, Vp, 0.9, w.scale,
+                                              return_errors=True)
+    torch.cuda.synchronize()
+    b = budget.cpu().numpy()
+    for h in range(w.H):
+        ref_off, ref_kc = oracle.route(E.cpu().numpy()[0, h], cq.offsets.cpu().numpy()[0, h],
+                                       ck.offsets.cpu().numpy()[0, h], w.N, 1.0,
+                                       budgets=b[0, h].astype(np.int64))
+        got = po.cpu().numpy()[0, h]
+        assert np.array_equal(got, ref_off)
+        assert np.array_equal(pk.cpu().numpy()[0, h][:got[-1]], ref_kc)
+        # every taken set fits its budget
+        sizes = np.diff(ck.offsets.cpu().numpy()[0, h])
+        for i in range(w.Cq):
+            assert sizes[ref_kc[ref_off[i]:ref_off[i + 1]]].sum() <= b[0, h, i]
+    # the standalone select with the same budgets gives the same pairs
+    po2, pk2 = csa.svgear_route_select_budget(E, cq.offsets, ck.offsets, w.N, budget)
+    assert torch.equal(po2, po)
+
+
+def test_layer_with_topp_budget_end_to_end():
+    csa = _csa()
+    w = SMALL_BF16
+    host, dev = _inputs(w)
+    out = csa.layer(dev["q"], dev["k"], dev["v"], w.Cq, w.Ck, 3, None, w.scale, seed=2, topp=0.9)
+    torch.cuda.synchronize()
+    cq, ck = out["q"], out["k"]
+    for h in range(w.H):
+        args = (np64(cq.Xp)[0, h], np64(ck.Xp)[0, h], np64(out["Vp"])[0, h],
+                cq.offsets.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
+                out["pair_off"].cpu().numpy()[0, h], out["pair_kc"].cpu().numpy()[0, h],
+                ck.centroids.cpu().numpy()[0, h], out["vbar"].cpu().numpy()[0, h],
+                cq.perm.cpu().numpy()[0, h])
+        Oo, _ = oracle.attend(*args, w.scale)
+        Og = np64(out["O"])[0, h]
+        assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2
