@@ -46,7 +46,8 @@ def lib():
         L.orc_route_budgets.argtypes = [P, P, i32, P, i32, P, P, P]
         L.orc_topp_budget.argtypes = [P, i32, P, i32, i32, P, P, f64, f64, P, P]
         L.orc_attend.argtypes = [P, i64, P, P, i32, P, i32, P, i32, P, P, P, P,
-                                 P, f64, P, i64, P, P]
+                                 P, f64, P, i64, P, P, P, f64]
+        L.orc_segment_var.argtypes = [P, i32, P, i32, P]
         L.orc_num_threads.restype = i32
         _lib = L
     return _lib
@@ -180,11 +181,24 @@ def topp_budget(qbar, kbar, q_off, k_off, p: float, scale: float):
     return budget, margin
 
 
+def segment_var(Xp, offsets):
+    """Per-coordinate population variance of every segment [C, d] (0 if empty)."""
+    Xp = _f64(Xp)
+    offsets = _i32(offsets)
+    C = offsets.shape[0] - 1
+    out = np.zeros((C, Xp.shape[1]))
+    lib().orc_segment_var(_p(Xp), Xp.shape[1], _p(offsets), C, _p(out))
+    return out
+
+
 def attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm,
-           scale: float, rows=None):
+           scale: float, rows=None, kvar=None, lam: float = 0.0):
     """O (original token order) and lse; with ``rows`` (permuted positions),
-    only those rows, in the order given."""
+    only those rows, in the order given.  With ``kvar`` (per-coordinate key
+    variance of every key cluster) a skipped cluster's log-weight gains
+    lam * scale^2 / 2 * sum_k q_k^2 kvar[c][k]."""
     Qp, Kp, Vp, kbar, vbar = map(_f64, (Qp, Kp, Vp, kbar, vbar))
+    kv = None if kvar is None else _f64(kvar)
     q_off, k_off, pair_off, q_perm = map(_i32, (q_off, k_off, pair_off, q_perm))
     pair_kc = _i32(pair_kc if len(pair_kc) else np.zeros(1, np.int32))
     Nq, d = Qp.shape
@@ -200,7 +214,7 @@ def attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm,
         lse = np.zeros(nr)
     lib().orc_attend(_p(Qp), Nq, _p(Kp), _p(Vp), d, _p(q_off), Cq, _p(k_off), Ck,
                      _p(pair_off), _p(pair_kc), _p(kbar), _p(vbar), _p(q_perm),
-                     float(scale), _p(r), nr, _p(O), _p(lse))
+                     float(scale), _p(r), nr, _p(O), _p(lse), _p(kv), float(lam))
     return O, lse
 
 

@@ -242,6 +242,31 @@ void orc_segment_mean(const double *Xp, int d, const int32_t *offsets, int C,
     }
 }
 
+/* Per-coordinate variance of every segment ([BLOG] variance paragraph: one  */
+/* variance per key coordinate, coordinates' co-movement ignored):           */
+/*   out[c][k] = (1/n_c) sum_{t in segment c} (x_tk - mean_ck)^2              */
+/* (population variance, the mean taken first); an empty segment gets 0.    */
+void orc_segment_var(const double *Xp, int d, const int32_t *offsets, int C, double *out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int c = 0; c < C; ++c) {
+        int64_t a = offsets[c], b = offsets[c + 1];
+        for (int k = 0; k < d; ++k) {
+            double v = 0.0;
+            if (b > a) {
+                double mean = 0.0;
+                for (int64_t t = a; t < b; ++t) mean += Xp[(size_t)t * d + k];
+                mean /= (double)(b - a);
+                for (int64_t t = a; t < b; ++t) {
+                    double e = Xp[(size_t)t * d + k] - mean;
+                    v += e * e;
+                }
+                v /= (double)(b - a);
+            }
+            out[(size_t)c * d + k] = v;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Compensation-error probe ([BLOG] probe paragraph; [REVIEW] O(Cq*Nk*d)      */
 /* probe).  The probe of query cluster i is its centroid qbar_i.  For key    */
@@ -444,12 +469,28 @@ void orc_topp_budget(const double *qbar, int Cq, const double *kbar, int Ck, int
 /* rows == NULL: every row, written at O[q_perm[p]] (lse likewise).          */
 /* rows != NULL: only permuted rows rows[r], written at O[r], lse[r].        */
 /* ------------------------------------------------------------------------ */
+/* Variance-corrected compensation ([BLOG] variance paragraph: the average   */
+/* of e^{s_j} over a cluster is about e^{sbar + sigma^2/2}, sigma^2 the      */
+/* variance of the query's scores over the cluster's keys, taken per key     */
+/* coordinate: sigma^2 ~ sum_k q_k^2 Var(k_k) times the square of the score  */
+/* scale (1/d for scale 1/sqrt(d)), at a strength lambda): with kvar != NULL */
+/* a skipped cluster's log-weight gains lambda * scale^2/2 * sum_k q_k^2      */
+/* kvar[c][k]; lambda = 0 or kvar = NULL is plain SVG-EAR.                   */
+/* Reading: the query's own q_p (as in the plain compensation).             */
+static double var_term(const double *q, const double *kv, int d, double coef) {
+    double s = 0.0;
+    for (int k = 0; k < d; ++k) s += q[k] * q[k] * kv[k];
+    return coef * s;
+}
+
 void orc_attend(const double *Qp, int64_t Nq, const double *Kp,
                 const double *Vp, int d, const int32_t *q_off, int Cq,
                 const int32_t *k_off, int Ck, const int32_t *pair_off,
                 const int32_t *pair_kc, const double *kbar, const double *vbar,
                 const int32_t *q_perm, double scale, const int64_t *rows,
-                int64_t n_rows, double *O, double *lse) {
+                int64_t n_rows, double *O, double *lse, const double *kvar,
+                double lambda) {
+    const double coef = lambda * scale * scale / 2.0;
     int64_t count = rows ? n_rows : Nq;
 #pragma omp parallel
     {
@@ -475,6 +516,7 @@ void orc_attend(const double *Qp, int64_t Nq, const double *Kp,
                     }
                 } else {
                     double s = scale * dot(q, kbar + (size_t)c * d, d) + log((double)nc);
+                    if (kvar) s += var_term(q, kvar + (size_t)c * d, d, coef);
                     if (s > m) m = s;
                 }
             }
@@ -491,7 +533,9 @@ void orc_attend(const double *Qp, int64_t Nq, const double *Kp,
                         for (int k = 0; k < d; ++k) num[k] += w * Vp[(size_t)u * d + k];
                     }
                 } else {
-                    double w = (double)nc * exp(scale * dot(q, kbar + (size_t)c * d, d) - m);
+                    double x = scale * dot(q, kbar + (size_t)c * d, d);
+                    if (kvar) x += var_term(q, kvar + (size_t)c * d, d, coef);
+                    double w = (double)nc * exp(x - m);
                     den += w;
                     for (int k = 0; k < d; ++k) num[k] += w * vbar[(size_t)c * d + k];
                 }

@@ -566,3 +566,68 @@ def test_route_with_budgets_equals_route_with_the_same_density_per_row():
         o1, k1 = oracle.route(E[i:i + 1], q_off[i:i + 2] - q_off[i], k_off, Nk,
                               (budgets[i] + 0.5) / Nk)
         assert np.array_equal(kc[off[i]:off[i + 1]], k1)
+
+
+# ---------------------------------------------------------------------------
+# Variance-corrected compensation (SVG-EAR blog, variance paragraph)
+# ---------------------------------------------------------------------------
+def test_segment_variance_closed_forms():
+    Xp = np.array([[0.0, 5.0], [2.0, 5.0],          # segment 0: var 1, 0
+                   [1.0, -3.0], [4.0, 1.0], [7.0, 2.0],  # segment 1
+                   [3.0, 3.0]])                      # segment 2: single row
+    off = np.array([0, 2, 2, 5, 6], dtype=np.int32)  # segment 1 empty
+    v = oracle.segment_var(Xp, off)
+    assert np.allclose(v[0], [1.0, 0.0])
+    assert np.all(v[1] == 0.0)
+    # {1, 4, 7}: mean 4, var (9+0+9)/3 = 6;  {-3, 1, 2}: mean 0, var (9+1+4)/3
+    assert np.allclose(v[2], [6.0, 14.0 / 3.0])
+    assert np.all(v[3] == 0.0)
+
+
+def _weight_of_one_skipped_cluster(keys, q, lam, scale=1.0):
+    """exp(lse) of one query row whose only key cluster is skipped: the
+    cluster's (corrected) estimated weight."""
+    keys = np.asarray(keys, dtype=np.float64)
+    n, d = keys.shape
+    q = np.asarray(q, dtype=np.float64)[None]
+    k_off = np.array([0, n], dtype=np.int32)
+    kbar = keys.mean(0, keepdims=True)
+    kvar = oracle.segment_var(keys, k_off)
+    vbar = np.ones((1, d))
+    _, lse = oracle.attend(q, keys, np.ones((n, d)), np.array([0, 1]), k_off,
+                           np.array([0, 0]), np.zeros(0, np.int32), kbar, vbar,
+                           np.array([0]), scale, kvar=kvar, lam=lam)
+    return float(np.exp(lse[0]))
+
+
+def test_variance_toy_cluster_b_matches_the_printed_estimate():
+    g = json.load(open(os.path.join(GOLDEN, "variance_example.json")))
+    # cluster B of the toy example: scores 0 and 2 for q = 1, d = 1, scale 1
+    w_corr = _weight_of_one_skipped_cluster([[0.0], [2.0]], [1.0], lam=1.0)
+    w_plain = _weight_of_one_skipped_cluster([[0.0], [2.0]], [1.0], lam=0.0)
+    assert abs(w_corr - 2 * math.exp(1.5)) < 1e-12
+    assert abs(w_corr - g["corrected_estimate_B_printed"]) <= g["printed_precision"]
+    assert abs(w_plain - g["uncorrected_estimate_B_printed"]) <= g["printed_precision"]
+    true_b = math.exp(0.0) + math.exp(2.0)
+    assert abs(true_b - g["true_weight_B_printed"]) <= g["printed_precision"]
+    # the corrected estimate lands closer to the truth, from above
+    assert abs(w_corr - true_b) < abs(w_plain - true_b) and w_corr > true_b > w_plain
+
+
+def test_variance_term_vanishes_for_identical_keys_and_scales_with_lambda():
+    g = np.random.default_rng(45)
+    d = 8
+    k = g.standard_normal(d)
+    q = g.standard_normal(d)
+    same = np.tile(k, (5, 1))
+    base = _weight_of_one_skipped_cluster(same, q, lam=0.0, scale=0.4)
+    for lam in (0.5, 1.0, 1.5):
+        assert abs(_weight_of_one_skipped_cluster(same, q, lam, scale=0.4) - base) < 1e-12 * base
+    # spread keys: log-weight grows linearly in lambda by scale^2/2 sum q^2 var
+    keys = g.standard_normal((6, d))
+    var = keys.var(axis=0)
+    w0 = _weight_of_one_skipped_cluster(keys, q, 0.0, scale=0.4)
+    for lam in (0.5, 1.5):
+        w = _weight_of_one_skipped_cluster(keys, q, lam, scale=0.4)
+        want = lam * 0.4 ** 2 / 2 * float((q ** 2 * var).sum())
+        assert abs(math.log(w / w0) - want) < 1e-12
