@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="wan720p", choices=sorted(synth.WORKLOADS))
     p.add_argument("--density", type=float, default=None)
+    p.add_argument("--var-lambda", type=float, default=0.0,
+                   help="strength of the variance-corrected compensation (0: plain)")
     p.add_argument("--topp", type=float, default=None,
                    help="routing budget per query cluster from the key clusters holding this "
                         "share of the estimated weight (instead of a fixed density)")
@@ -304,6 +306,8 @@ def run_reference(args, w):
 def workload_config(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
             "iters": args.iters or w.iters,
+            "compensation": ("variance-corrected, lambda %g" % args.var_lambda if args.var_lambda
+                             else "plain (n e^{score of the centroid})"),
             "budget": ("top-p %g of the estimated weight per query cluster" % args.topp
                        if args.topp else "density %g (floor(density * N) keys per query cluster)"
                        % (args.density or w.density)),
@@ -376,8 +380,9 @@ def main():
             po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
                                       ck.Xp, Vp, density, w.scale)
         mark(4)
+        kvar = csa.svgear_key_variance(ck.Xp, ck.offsets, w.Ck) if args.var_lambda else None
         O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids,
-                              vbar, cq.perm, w.scale)
+                              vbar, cq.perm, w.scale, kvar=kvar, lam=args.var_lambda)
         mark(5)
         return O, (cq, ck, po, pk)
 

@@ -31,7 +31,7 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_attend", "svgear_workspace_bytes", "svgear_status_string",
             "svgear_version", "svgear_kernel_launches", "svgear_attend_status",
             "svgear_device_status", "svgear_topp_budget", "svgear_route_select_budget",
-            "svgear_route_topp",
+            "svgear_route_topp", "svgear_key_variance", "svgear_attend_var",
             "svgear_label_sort_noalloc")
 
 
@@ -74,6 +74,9 @@ def lib():
         "svgear_topp_budget": [P, P, I32, P, P, I32, I32, I32, I32, I32, F, F, P, P],
         "svgear_route_select_budget": [P, P, I32, P, I32, I32, I32, I32, P, P, P, P, SZ, P],
         "svgear_route_topp": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, P, SZ, P],
+        "svgear_key_variance": [P, P, I32, Dims, P, P],
+        "svgear_attend_var": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, F, P, P, SZ,
+                              P],
         "svgear_attend": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, P, SZ, P],
         "svgear_workspace_bytes": [I32, Dims, I32, I32],
         "svgear_status_string": [ctypes.c_int],
@@ -345,10 +348,22 @@ def svgear_route(qbar, q_off, kbar, vbar, k_off, Kp, Vp, density, scale, return_
     return (pair_off, pair_kc, E) if return_errors else (pair_off, pair_kc)
 
 
+def svgear_key_variance(Kp, k_off, Ck):
+    """Per-coordinate variance of every key cluster: float32 [B, H, Ck, d]."""
+    kd = _tokens(Kp, "Kp")
+    B, H, N, d = Kp.shape
+    kvar = torch.empty((B, H, Ck, d), dtype=torch.float32, device=Kp.device)
+    _check("svgear_key_variance", lib().svgear_key_variance(_ptr(Kp), _ptr(k_off), Ck, kd,
+                                                            _ptr(kvar), _stream()))
+    return kvar
+
+
 def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_perm, scale, O=None,
-                  check_status=False):
+                  check_status=False, kvar=None, lam=0.0):
     """O in the original token order.  check_status=True synchronises and
-    raises if any bounded wait inside the kernel gave up."""
+    raises if any bounded wait inside the kernel gave up.  With kvar (key
+    variance per cluster) and lam != 0 the compensation is variance-corrected
+    (svgear_attend_var)."""
     qd = _tokens(Qp, "Qp")
     _tokens(Kp, "Kp")
     _tokens(Vp, "Vp")
@@ -358,22 +373,30 @@ def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_per
     if O is None:
         O = torch.empty_like(Qp)
     ws, n = _workspace(OP_ATTEND, qd, Cq, Ck, Qp.device)
-    _check("svgear_attend", lib().svgear_attend(
-        _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Nk, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(pair_off),
-        _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(q_perm), float(scale), _ptr(O), _ptr(ws), n,
-        _stream()))
+    if kvar is None:
+        _check("svgear_attend", lib().svgear_attend(
+            _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Nk, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(pair_off),
+            _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(q_perm), float(scale), _ptr(O), _ptr(ws),
+            n, _stream()))
+    else:
+        _cuda(kvar, "kvar", torch.float32)
+        _check("svgear_attend_var", lib().svgear_attend_var(
+            _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Nk, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(pair_off),
+            _ptr(pair_kc), _ptr(kbar), _ptr(vbar), _ptr(kvar), float(lam), _ptr(q_perm),
+            float(scale), _ptr(O), _ptr(ws), n, _stream()))
     if check_status:
         _device_status("svgear_attend", ws, n)
     return O
 
 
 def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None,
-          topp=None):
+          topp=None, var_lambda=0.0):
     """The whole layer for [B, H, N, d] tensors: cluster Q and K (seeds 2*seed
     and 2*seed+1), permute V, value centroids, route, attend.  The routing
     budget is floor(density * N) keys per query cluster, or, with topp=p, the
-    keys holding p of the estimated weight (density is then unused).  Returns
-    O in the original token order and every intermediate."""
+    keys holding p of the estimated weight (density is then unused).  With
+    var_lambda != 0 the compensation is variance-corrected.  Returns O in the
+    original token order and every intermediate."""
     d = Q.shape[-1]
     scale = d ** -0.5 if scale is None else scale
     cq = svgear_cluster(Q, Cq, iters, warm_q, seed=2 * seed)
@@ -387,7 +410,8 @@ def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm
     else:
         pair_off, pair_kc, budget = svgear_route_topp(cq.centroids, cq.offsets, ck.centroids, vbar,
                                                       ck.offsets, ck.Xp, Vp, topp, scale)
+    kvar = svgear_key_variance(ck.Xp, ck.offsets, Ck) if var_lambda else None
     O = svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, pair_off, pair_kc, ck.centroids,
-                      vbar, cq.perm, scale)
+                      vbar, cq.perm, scale, kvar=kvar, lam=var_lambda)
     return {"O": O, "q": cq, "k": ck, "Vp": Vp, "vbar": vbar, "pair_off": pair_off,
-            "pair_kc": pair_kc, "budget": budget}
+            "pair_kc": pair_kc, "budget": budget, "kvar": kvar}

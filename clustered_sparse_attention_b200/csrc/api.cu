@@ -119,6 +119,7 @@ AttendWs carve_attend(Carve& cv, const svgear_dims& d, int Cq, int Ck) {
     w.status = cv.take<int>(4);
     w.kbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
     w.vbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
+    w.k2bar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
     w.meta = cv.take<int4>(BH * Cq);
     w.seg_prefix = cv.take<int32_t>(BH * Cq * (size_t)(Ck + 1));
     w.seg_row = cv.take<int32_t>(BH * Cq * (size_t)Ck);
@@ -497,11 +498,12 @@ int svgear_route_topp(const float* qbar, const int32_t* q_off, int32_t Cq, const
                                w.sel.counts, pair_off, pair_kc, st);
 }
 
-int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims, int32_t Nk,
-                  const int32_t* q_off, int32_t Cq, const int32_t* k_off, int32_t Ck,
-                  const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
-                  const float* vbar, const int32_t* q_perm, float scale, void* O, void* ws,
-                  size_t ws_bytes, void* stream) {
+int svgear_attend_var(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                      int32_t Nk, const int32_t* q_off, int32_t Cq, const int32_t* k_off,
+                      int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc,
+                      const float* kbar, const float* vbar, const float* kvar, float lambda,
+                      const int32_t* q_perm, float scale, void* O, void* ws, size_t ws_bytes,
+                      void* stream) {
     int s = check_dims(qdims);
     if (s) return s;
     if (Nk < 1) return SVGEAR_ERR_INVALID_ARG;
@@ -509,19 +511,39 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
     if (Cq > qdims.N) return SVGEAR_ERR_INVALID_ARG;
     if (!Qp || !Kp || !Vp || !q_off || !k_off || !pair_off || !pair_kc || !kbar || !vbar ||
         !q_perm || !O || !ws || !aligned16(Qp) || !aligned16(Kp) || !aligned16(Vp) ||
-        !aligned16(O) || !isfinite(scale))
+        !aligned16(O) || !isfinite(scale) || !isfinite(lambda))
         return SVGEAR_ERR_INVALID_ARG;
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(qdims) == 0) return SVGEAR_OK;
+    if (lambda == 0.f) kvar = nullptr;   // plain SVG-EAR compensation
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
     AttendWs w = carve_attend(cv, qdims, Cq, Ck);
     if (qdims.dtype == SVGEAR_BF16)
         return launch_attend_sm100(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc,
-                                   kbar, vbar, q_perm, scale, O, w, st);
+                                   kbar, vbar, q_perm, scale, O, kvar, lambda, w, st);
     if (cudaMemsetAsync(w.status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     return launch_attend_simt(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc, kbar,
-                              vbar, q_perm, scale, O, st);
+                              vbar, q_perm, scale, O, kvar, lambda * scale * scale * 0.5f, st);
+}
+
+int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims, int32_t Nk,
+                  const int32_t* q_off, int32_t Cq, const int32_t* k_off, int32_t Ck,
+                  const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
+                  const float* vbar, const int32_t* q_perm, float scale, void* O, void* ws,
+                  size_t ws_bytes, void* stream) {
+    return svgear_attend_var(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc, kbar,
+                             vbar, nullptr, 0.f, q_perm, scale, O, ws, ws_bytes, stream);
+}
+
+int svgear_key_variance(const void* Kp, const int32_t* k_off, int32_t Ck, svgear_dims kdims,
+                        float* kvar, void* stream) {
+    int s = check_dims(kdims);
+    if (s) return s;
+    if ((s = check_C(Ck, kdims.N))) return s;
+    if (!Kp || !k_off || !kvar || !aligned16(Kp)) return SVGEAR_ERR_INVALID_ARG;
+    if (bh_of(kdims) == 0) return SVGEAR_OK;
+    return launch_segment_var(Kp, k_off, Ck, kdims, kvar, static_cast<cudaStream_t>(stream));
 }
 
 int svgear_device_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {

@@ -13,7 +13,9 @@
 //
 // One block per 64-row tile of one query cluster.  Keys of each selected
 // cluster are staged 64 at a time; then the skipped, non-empty clusters'
-// centroids are staged 64 at a time with a per-column bias log(n_c).
+// centroids are staged 64 at a time with a per-column bias log(n_c); with a
+// key-variance table the score of a skipped cluster also gains
+// var_coef * sum_k q_k^2 Var_c(k) (SVG-EAR blog, variance paragraph).
 #include <math.h>
 
 #include "common.cuh"
@@ -31,7 +33,8 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
                    const int32_t* __restrict__ k_off, int Ck,
                    const int32_t* __restrict__ pair_off, const int32_t* __restrict__ pair_kc,
                    const float* __restrict__ kbar, const float* __restrict__ vbar,
-                   const int32_t* __restrict__ q_perm, float scale, T* __restrict__ O) {
+                   const int32_t* __restrict__ q_perm, float scale, T* __restrict__ O,
+                   const float* __restrict__ kvar, float var_coef) {
     constexpr int QP = D + 1;
     extern __shared__ __align__(16) float sm[];
     float* Qs = sm;                        // [64][D+1]
@@ -41,6 +44,8 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
     float* bias = Ps + kAtRows * 65;       // [64]
     int32_t* comp = reinterpret_cast<int32_t*>(bias + kAtKeys);   // [Ck]
     unsigned char* sel = reinterpret_cast<unsigned char*>(comp + Ck);  // [Ck]
+    // [64][D+1]: var_coef * key variance of the compensation tile's clusters
+    float* Ws = reinterpret_cast<float*>(sel + ((Ck + 15) & ~15));
     __shared__ int s_i, s_r0, s_r1, s_ncomp;
 
     const int bh = blockIdx.y, tid = threadIdx.x;
@@ -102,7 +107,7 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
     const float* kbh = kbar + (size_t)bh * Ck * D;
     const float* vbh = vbar + (size_t)bh * Ck * D;
 
-    auto process = [&](int nvalid) {
+    auto process = [&](int nvalid, bool with_var) {
         // scores of row `row` against keys sub + 4m
         float s[16];
         float cmax = -INFINITY;
@@ -114,7 +119,15 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
             const float* kr = Ks + j * QP;
 #pragma unroll 8
             for (int k = 0; k < D; ++k) acc = fmaf(qr[k], kr[k], acc);
-            s[mm] = (j < nvalid) ? fmaf(acc, scale, bias[j]) : -INFINITY;
+            if (with_var) {   // + var_coef * sum_k q_k^2 Var_c(k)
+                const float* wr = Ws + j * QP;
+                float vacc = 0.f;
+#pragma unroll 8
+                for (int k = 0; k < D; ++k) vacc = fmaf(qr[k] * qr[k], wr[k], vacc);
+                s[mm] = (j < nvalid) ? fmaf(acc, scale, vacc + bias[j]) : -INFINITY;
+            } else {
+                s[mm] = (j < nvalid) ? fmaf(acc, scale, bias[j]) : -INFINITY;
+            }
             cmax = fmaxf(cmax, s[mm]);
         }
         cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
@@ -162,7 +175,7 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
             }
             if (tid < kAtKeys) bias[tid] = 0.f;
             __syncthreads();
-            process(nv);
+            process(nv, false);
         }
     }
     // compensation: each skipped non-empty cluster as one key at its centroid
@@ -179,6 +192,7 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
             }
             Ks[j * QP + k] = kv;
             Vs[j * D + k] = vv;
+            if (kvar) Ws[j * QP + k] = (j < nv) ? var_coef * kvar[((size_t)bh * Ck + comp[b0 + j]) * D + k] : 0.f;
         }
         if (tid < kAtKeys) {
             float bv = 0.f;
@@ -189,7 +203,7 @@ attend_simt_kernel(const T* __restrict__ Qp, const T* __restrict__ Kp,
             bias[tid] = bv;
         }
         __syncthreads();
-        process(nv);
+        process(nv, kvar != nullptr);
     }
     // epilogue: O[q_perm[p]] = num / den
     const int p = r0 + row;
@@ -209,11 +223,12 @@ static int attend_simt_impl(const void* Qp, const void* Kp, const void* Vp, svge
                             int Nk, const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                             const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
                             const float* vbar, const int32_t* q_perm, float scale, void* O,
-                            cudaStream_t st) {
+                            const float* kvar, float var_coef, cudaStream_t st) {
     constexpr int QP = D + 1;
     const size_t sm = sizeof(float) * (kAtRows * QP + kAtKeys * QP + kAtKeys * D + kAtRows * 65 +
                                        kAtKeys) +
-                      sizeof(int32_t) * Ck + Ck;
+                      sizeof(int32_t) * Ck + ((Ck + 15) & ~15) +
+                      (kvar ? sizeof(float) * kAtKeys * QP : 0);
     if (cudaFuncSetAttribute(attend_simt_kernel<T, D>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
@@ -222,7 +237,7 @@ static int attend_simt_impl(const void* Qp, const void* Kp, const void* Vp, svge
     attend_simt_kernel<T, D><<<dim3(tiles, BH), kAtThreads, sm, st>>>(
         static_cast<const T*>(Qp), static_cast<const T*>(Kp), static_cast<const T*>(Vp), qd.N,
         Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc, kbar, vbar, q_perm, scale,
-        static_cast<T*>(O));
+        static_cast<T*>(O), kvar, var_coef);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
@@ -232,10 +247,10 @@ int launch_attend_simt(const void* Qp, const void* Kp, const void* Vp, svgear_di
                        const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                        const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
                        const float* vbar, const int32_t* q_perm, float scale, void* O,
-                       cudaStream_t st) {
+                       const float* kvar, float var_coef, cudaStream_t st) {
 #define SVGEAR_AT(T, D)                                                                    \
     return attend_simt_impl<T, D>(Qp, Kp, Vp, qd, Nk, q_off, Cq, k_off, Ck, pair_off,       \
-                                  pair_kc, kbar, vbar, q_perm, scale, O, st)
+                                  pair_kc, kbar, vbar, q_perm, scale, O, kvar, var_coef, st)
     if (qd.dtype == SVGEAR_BF16) {
         if (qd.d == 128) SVGEAR_AT(__nv_bfloat16, 128);
         if (qd.d == 64) SVGEAR_AT(__nv_bfloat16, 64);

@@ -74,6 +74,7 @@ struct TmaMaps {
     CUtensorMap v[8];
     CUtensorMap kb;
     CUtensorMap vb;
+    CUtensorMap k2b;   // bf16 lambda*scale/2 * key variance, read a row at a time
     CUtensorMap q;
 };
 
@@ -85,6 +86,7 @@ struct Shared {
     uint64_t v_empty[STAGES];
     uint64_t s_full[kHalves];
     uint64_t p_full[kHalves];
+    uint64_t q2_full[kHalves];   // q^2 of the half in TMEM (variance term, no exact tiles)
     uint64_t o_full;
     uint32_t tmem_base;
     int abort_flag;
@@ -102,6 +104,38 @@ __device__ long long g_trace[18][512];
 #define TRACE(ev, j) do { } while (0)
 #endif
 
+// Swizzled 16-byte chunk address inside a tile of 128 rows x (regions of
+// 64 bf16): region g covers elements [64g, 64g+64) of every row.
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
+    const int region = chunk >> 3, cc = chunk & 7;
+    return tile + region * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+}
+
+// q^2 of this thread's query row (read from the 128B-swizzled Q tile in
+// shared memory) as bf16 pairs -- dimension 2c in the low half of column c --
+// into the D/2 TMEM columns at taddr: the A operand of the variance MMA.
+template <int D>
+__device__ __forceinline__ void write_q2(uint32_t sQh, int r, uint32_t taddr) {
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(swz(sQh, r, half * 8 + c)));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+                __nv_bfloat162 q2 = __floats2bfloat162_rn(lo * lo, hi * hi);
+                pk[4 * c + e] = *reinterpret_cast<uint32_t*>(&q2);
+            }
+        }
+        tc::tmem_st32(taddr + half * 32, pk);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq, int Ck, int BH,
@@ -109,7 +143,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     const int32_t* __restrict__ ntiles, int maxT, const int4* __restrict__ meta,
                     const int32_t* __restrict__ seg_prefix, const int32_t* __restrict__ seg_row,
                     const int32_t* __restrict__ comp_idx, const float* __restrict__ comp_bias,
-                    float scale_log2, bf16* __restrict__ O, int* __restrict__ err) {
+                    float scale_log2, int use_var, bf16* __restrict__ O, int* __restrict__ err) {
     constexpr int REG = D / 64;                 // 64-element regions per row
     constexpr uint32_t kTileBytes = REG * 16384;
     const int bh = blockIdx.y;
@@ -121,7 +155,10 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     const int4 mt = meta[(size_t)bh * Cq + ci];   // {nseg, L keys, ncomp, 0}
     const int L = mt.y, ncomp = mt.z;
     const int T_real = (L + BN - 1) / BN;
-    const int T = T_real + (ncomp + BN - 1) / BN;
+    // compensation tiles take CW skipped clusters: 128, or 64 with the
+    // variance term (the upper 64 columns of S_h then hold q^2 of the half)
+    const int CW = use_var ? BN / 2 : BN;
+    const int T = T_real + (ncomp + CW - 1) / CW;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ Shared sh;
@@ -142,6 +179,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         for (int h = 0; h < kHalves; ++h) {
             tc::mbar_init(tc::smem_u32(&sh.s_full[h]), 1);
             tc::mbar_init(tc::smem_u32(&sh.p_full[h]), kSoftmaxThreads);
+            tc::mbar_init(tc::smem_u32(&sh.q2_full[h]), kSoftmaxThreads);
         }
         tc::mbar_init(tc::smem_u32(&sh.o_full), 1);
         sh.abort_flag = 0;
@@ -207,18 +245,23 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             const uint32_t bar = tc::smem_u32(&ring_full[st]);
             const uint32_t tX = ring0 + st * kTileBytes;
             if (j >= T_real) {
-                // compensation tile: lane i gathers tile rows 4i..4i+3
+                // compensation tile: lane i gathers tile rows 4i..4i+3.  With the
+                // variance term a tile covers 64 clusters: K rows 0-63 are their
+                // centroids and rows 64-127 the same clusters' variance rows; V rows
+                // 64-127 are zeros (read past the table)
+                const int sub = use_var ? (lane & 15) : lane;
+                const CUtensorMap* src = (use_var && isK && lane >= 16) ? &maps.k2b : mcent;
                 int y[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int p = (j - T_real) * BN + 4 * lane + k;
-                    y[k] = (p < ncomp) ? crow0 + cidx[p] : cend;
+                    const int p = (j - T_real) * CW + 4 * sub + k;
+                    y[k] = (p < ncomp && (isK || !use_var || lane < 16)) ? crow0 + cidx[p] : cend;
                 }
                 if (lane == 0) tc::mbar_arrive_expect_tx(bar, BN * D * 2);
                 __syncwarp();
 #pragma unroll 1
                 for (int g = 0; g < REG; ++g)
-                    tc::tma_gather4(tX + g * 16384 + lane * 512, mcent, g * 64, y[0], y[1], y[2], y[3],
+                    tc::tma_gather4(tX + g * 16384 + lane * 512, src, g * 64, y[0], y[1], y[2], y[3],
                                     bar);
             } else if (lane == 0) {
                 tc::mbar_arrive_expect_tx(bar, BN * D * 2);
@@ -258,6 +301,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         // the two softmax warpgroups half a step apart, so they do not contend
         // for the exp unit at the same time.
         constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
+        constexpr uint32_t kIdescQK64 = tc::idesc_bf16(BM, BN / 2, false);
         constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
         bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
         for (int j = 0; ok_run && j <= T; ++j) {
@@ -276,8 +320,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     if (lane == 0) TRACE(h == 0 ? 9 : 13, j);
                     if (lane == 0) {
                         const uint32_t tV = sV0 + pst * kTileBytes;
+                        const int kdepth = (j - 1 >= T_real) ? CW : BN;   // keys of tile j-1
 #pragma unroll 1
-                        for (int ks = 0; ks < BN / 16; ++ks)
+                        for (int ks = 0; ks < kdepth / 16; ++ks)
                             tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
                                             tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
                                             (j > 1 || ks > 0) ? 1u : 0u);
@@ -291,6 +336,16 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         ok_run = false;
                         break;
                     }
+                    const bool var_tile = use_var && j >= T_real;
+                    // q^2 of the half must be in TMEM: written with P(T_real-1), or,
+                    // with no exact tiles, before the first compensation tile
+                    if (var_tile && j == 0) {
+                        if (!warp_wait_bar(&sh.q2_full[h], 0, abort_flag, err, (12 << 16) + h)) {
+                            ok_run = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                    }
                     if (lane == 0 && h == 0) TRACE(11, j);
                     if (lane == 0) {
                         const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
@@ -298,7 +353,18 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                             tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
-                                         tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
+                                         tc::sw128_desc(tK + off, 16, 1024),
+                                         var_tile ? kIdescQK64 : kIdescQK, ks > 0);
+                        }
+                        if (var_tile) {
+                            // S += q^2 . (lambda*scale/2 Var)^T: A = q^2 from TMEM
+                            // (columns 64-127 of S_h), B = tile rows 64-127
+#pragma unroll 1
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks >> 2) * 16384 + 64 * 128 + (ks & 3) * 32;
+                                tc::mma_bf16_ts(tmem + h * BN, tmem + h * BN + BN / 2 + ks * 8,
+                                                tc::sw128_desc(tK + off, 16, 1024), kIdescQK64, 1u);
+                            }
                         }
                         tc::commit(tc::smem_u32(&sh.s_full[h]));
                     }
@@ -336,6 +402,17 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         const float* cb = comp_bias + row_meta;
         float m_use = -INFINITY, l = 0.f;
         bool ok_run = h < nh;
+        const bool need_q2 = use_var && ncomp > 0;
+        if (ok_run && need_q2) {
+            // the Q tile is read from shared memory below: wait for its copy
+            ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (13 << 16) + h);
+            if (ok_run && T_real == 0) {   // no exact tiles: q^2 goes in first
+                write_q2<D>(sQ0 + h * kTileBytes, r, sS + BN / 2);
+                tc::tmem_st_wait();
+                tc::fence_before_sync();
+                tc::mbar_arrive(tc::smem_u32(&sh.q2_full[h]));
+            }
+        }
         uint32_t v[BN];
         for (int j = 0; j < T && ok_run; ++j) {
             if (!warp_wait_bar(&sh.s_full[h], j & 1, abort_flag, err, (2 << 16) + j)) {
@@ -351,9 +428,12 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
             tc::tmem_ld_wait();
 
+            // S_h is in registers: with the variance term, the last exact tile
+            // leaves q^2 in the upper half of S_h for the compensation tiles
+            if (need_q2 && j == T_real - 1) write_q2<D>(sQ0 + h * kTileBytes, r, sS + BN / 2);
             const bool comp = j >= T_real;
-            const int valid = comp ? min(BN, ncomp - (j - T_real) * BN) : min(BN, L - j * BN);
-            const float* bias = cb + (comp ? (j - T_real) * BN : 0);
+            const int valid = comp ? min(CW, ncomp - (j - T_real) * CW) : min(BN, L - j * BN);
+            const float* bias = cb + (comp ? (j - T_real) * CW : 0);
             // x = s * scale * log2(e) (+ log2 n_c on compensation columns); masked -> -inf
             if (comp) {
                 // in 32-column steps (the compiler barrier keeps the bias loads of
@@ -476,10 +556,11 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
 // ---------------------------------------------------------------------------
 // Preparation: bf16 centroid tables, per-query-cluster key lists, tile table.
 // ---------------------------------------------------------------------------
-__global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, size_t n) {
+__global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, size_t n,
+                               float mul) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x)
-        dst[i] = __float2bfloat16_rn(src[i]);
+        dst[i] = __float2bfloat16_rn(src[i] * mul);
 }
 
 // One block per (query cluster, head).  Selected clusters in ascending order
@@ -555,14 +636,16 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
                         const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                         const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
                         const float* vbar, const int32_t* q_perm, float scale, void* O,
-                        const AttendWs& w, cudaStream_t st) {
+                        const float* kvar, float lambda, const AttendWs& w, cudaStream_t st) {
     using namespace sm100;
     const int BH = qd.B * qd.H;
     const int D = qd.d;
     if ((long long)BH * Nk >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;   // int32 TMA rows
     if ((long long)BH * qd.N >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;
     TmaMaps maps;
+    const int use_var = (kvar != nullptr && lambda != 0.f) ? 1 : 0;
     bool ok = make_rows_map(&maps.kb, w.kbar16, (uint64_t)BH * Ck, D, 1) &&
+              make_rows_map(&maps.k2b, w.k2bar16, (uint64_t)BH * Ck, D, 1) &&
               make_rows_map(&maps.vb, w.vbar16, (uint64_t)BH * Ck, D, 1) &&
               make_rows_map(&maps.q, Qp, (uint64_t)BH * qd.N, D, BM);
     for (int h = 0; h < 8 && ok; ++h)
@@ -572,10 +655,16 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     if (cudaMemsetAsync(w.status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     const size_t nc = (size_t)BH * Ck * D;
     const int cgrid = (int)((nc + 255) / 256 < 4096 ? (nc + 255) / 256 : 4096);
-    to_bf16_kernel<<<cgrid, 256, 0, st>>>(kbar, w.kbar16, nc);
+    to_bf16_kernel<<<cgrid, 256, 0, st>>>(kbar, w.kbar16, nc, 1.f);
     count_launches(1);
-    to_bf16_kernel<<<cgrid, 256, 0, st>>>(vbar, w.vbar16, nc);
+    to_bf16_kernel<<<cgrid, 256, 0, st>>>(vbar, w.vbar16, nc, 1.f);
     count_launches(1);
+    if (use_var) {
+        // B operand of the variance MMA: lambda * scale / 2 * Var (the softmax
+        // multiplies the raw scores by scale * log2 e)
+        to_bf16_kernel<<<cgrid, 256, 0, st>>>(kvar, w.k2bar16, nc, lambda * scale * 0.5f);
+        count_launches(1);
+    }
     attend_prep_kernel<<<dim3(Cq, BH), 128, Ck, st>>>(k_off, Ck, Cq, Nk, pair_off, pair_kc, w.meta,
                                                       w.seg_prefix, w.seg_row, w.comp_idx,
                                                       w.comp_bias);
@@ -601,16 +690,16 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
             return SVGEAR_ERR_CUDA;
         attend_sm100_kernel<128><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
             maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
-            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
-            w.status);
+            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, use_var,
+            static_cast<bf16*>(O), w.status);
     } else {
         if (cudaFuncSetAttribute(attend_sm100_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
         attend_sm100_kernel<64><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
             maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
-            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, static_cast<bf16*>(O),
-            w.status);
+            w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, use_var,
+            static_cast<bf16*>(O), w.status);
     }
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();

@@ -674,6 +674,73 @@ segment_mean_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
 }
 
 // ---------------------------------------------------------------------------
+// Per-coordinate variance of every segment (SVG-EAR blog, variance paragraph:
+// one variance per key coordinate): out[c][k] = (1/n) sum_t (x_tk - mean_ck)^2
+// over the contiguous rows of segment c, the mean taken first (two passes,
+// fp32 partial sums combined in a fixed order); an empty segment gets 0.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kSmThreads)
+segment_var_kernel(const T* __restrict__ X, const int32_t* __restrict__ offsets, int N, int C,
+                   float* __restrict__ out) {
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int L = D / EPC;
+    constexpr int R = kSmThreads / L;
+    __shared__ float part[R][D];
+    __shared__ float mean[D];
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int32_t* off = offsets + (size_t)bh * (C + 1);
+    const int a = off[c], b = off[c + 1];
+    float* o = out + ((size_t)bh * C + c) * D;
+    if (b <= a || a < 0 || b > N) {
+        for (int k = tid; k < D; k += kSmThreads) o[k] = 0.f;
+        return;
+    }
+    const T* Xh = X + (size_t)bh * N * D;
+    const int lane = tid % L, grp = tid / L;
+    const float n = (float)(b - a);
+    for (int pass = 0; pass < 2; ++pass) {
+        float acc[EPC];
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+        for (int p = a + grp; p < b; p += R) {
+            float v[EPC];
+            Elem<T>::load(Xh + (size_t)p * D + lane * EPC, v);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                if (pass == 0) {
+                    acc[e] += v[e];
+                } else {
+                    const float dv = v[e] - mean[lane * EPC + e];
+                    acc[e] = fmaf(dv, dv, acc[e]);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) part[grp][lane * EPC + e] = acc[e];
+        __syncthreads();
+        for (int k = tid; k < D; k += kSmThreads) {
+            float s = 0.f;
+#pragma unroll
+            for (int g = 0; g < R; ++g) s += part[g][k];
+            if (pass == 0) mean[k] = s / n;
+            else o[k] = s / n;
+        }
+        __syncthreads();
+    }
+}
+
+template <typename T, int D>
+static int segvar_disp(const void* X, const int32_t* offsets, int C, svgear_dims dims, float* out,
+                       cudaStream_t st) {
+    segment_var_kernel<T, D><<<dim3(C, dims.B * dims.H), kSmThreads, 0, st>>>(
+        static_cast<const T*>(X), offsets, dims.N, C, out);
+    count_launches(1);
+    SVGEAR_LAUNCH_CHECK();
+    return SVGEAR_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Permutation gather: Xp[p] = X[perm[p]], one 16-byte chunk per thread.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
@@ -793,6 +860,11 @@ static int permute_disp(const void* X, const int32_t* perm, svgear_dims dims, vo
 int launch_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
                    cudaStream_t st) {
     SVGEAR_DISPATCH(dims, permute_disp, X, perm, dims, Xp, st);
+}
+
+int launch_segment_var(const void* X, const int32_t* offsets, int C, svgear_dims dims,
+                       float* out, cudaStream_t st) {
+    SVGEAR_DISPATCH(dims, segvar_disp, X, offsets, C, dims, out, st);
 }
 
 }  // namespace svgear

@@ -36,6 +36,9 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* centroids,
                         const int32_t* done, int32_t* changed);
 size_t assign_sm100_scratch_bytes(int BH, int C, int D);
 int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st);
+// Per-coordinate population variance of every contiguous segment of X.
+int launch_segment_var(const void* X, const int32_t* offsets, int C, svgear_dims dims,
+                       float* out, cudaStream_t st);
 // Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
 // empty_zero: an empty segment writes zeros (else leaves the row untouched).
 int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets,
@@ -67,6 +70,7 @@ struct AttendWs {
     int* status;                 // device status word (0 or SVGEAR_ERR_TIMEOUT)
     __nv_bfloat16* kbar16;       // [BH][Ck][d] bf16 key centroids
     __nv_bfloat16* vbar16;       // [BH][Ck][d] bf16 value centroids
+    __nv_bfloat16* k2bar16;      // [BH][Ck][d] bf16 lambda*scale/2 * key variance
     int4* meta;                  // [BH][Cq] {segments, selected keys, skipped clusters, 0}
     int32_t* seg_prefix;         // [BH][Cq][Ck+1] list position of each segment
     int32_t* seg_row;            // [BH][Cq][Ck] first key row of each segment
@@ -80,13 +84,15 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
                         const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                         const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
                         const float* vbar, const int32_t* q_perm, float scale, void* O,
-                        const AttendWs& w, cudaStream_t st);
+                        const float* kvar, float lambda, const AttendWs& w, cudaStream_t st);
 
 // attend_simt.cu
+// kvar (nullable): per-coordinate key variance [B*H][Ck][d]; a skipped
+// cluster's score gains var_coef * sum_k q_k^2 kvar[c][k] (natural-log units).
 int launch_attend_simt(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
                        int Nk, const int32_t* q_off, int Cq, const int32_t* k_off,
                        int Ck, const int32_t* pair_off, const int32_t* pair_kc,
                        const float* kbar, const float* vbar, const int32_t* q_perm,
-                       float scale, void* O, cudaStream_t st);
+                       float scale, void* O, const float* kvar, float var_coef, cudaStream_t st);
 
 }  // namespace svgear

@@ -312,6 +312,41 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
                   const float* kbar, const float* vbar, const int32_t* q_perm,
                   float scale, void* O, void* ws, size_t ws_bytes, void* stream);
 
+/* --------------------------------------------------------------------------
+ * svgear_key_variance -- per-coordinate variance of every key cluster ([BLOG]
+ * variance paragraph: one variance per key coordinate, the coordinates'
+ * co-movement ignored): kvar[c][k] = (1/n_c) sum_{t in K_c} (k_tk - mean_ck)^2
+ * over the contiguous segment c of Kp (population variance, fp32, mean taken
+ * first); an empty cluster gets 0.
+ *   Kp     [B][H][Nk][d] permuted keys (kdims.dtype); k_off int32[B][H][Ck+1].
+ *   kvar   out float[B][H][Ck][d].
+ * No workspace; asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+int svgear_key_variance(const void* Kp, const int32_t* k_off, int32_t Ck, svgear_dims kdims,
+                        float* kvar, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_attend_var -- svgear_attend with variance-corrected compensation
+ * ([BLOG] variance paragraph: the mean of e^{s_j} over a cluster is about
+ * e^{sbar + sigma^2/2}; sigma^2 ~ scale^2 sum_k q_k^2 Var(k_k)).  Every
+ * skipped cluster's log-weight gains
+ *     lambda * scale^2 / 2 * sum_k q_k^2 kvar[c][k]
+ * for each query row q (its own query, as the plain compensation uses);
+ * lambda = 0 (or kvar = NULL) is exactly svgear_attend.
+ *   kvar    float[B][H][Ck][d] (svgear_key_variance), nullable.
+ *   lambda  finite strength of the term (the blog's runs use 0 to 1.5).
+ * Other arguments, layouts, workspace and status word as svgear_attend.  On
+ * the bf16 tensor-core path the term is one more MMA per compensation tile
+ * with bf16 q^2 and bf16 lambda*scale/2*Var operands, and compensation tiles
+ * then take 64 clusters each.
+ * ------------------------------------------------------------------------ */
+int svgear_attend_var(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                      int32_t Nk, const int32_t* q_off, int32_t Cq, const int32_t* k_off,
+                      int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc,
+                      const float* kbar, const float* vbar, const float* kvar, float lambda,
+                      const int32_t* q_perm, float scale, void* O, void* ws, size_t ws_bytes,
+                      void* stream);
+
 /* Device status of the last svgear_cluster, svgear_kmeans_assign or
  * svgear_attend that used `ws`: copies 4 int32 to status[0..3] (host memory)
  * and synchronises `stream`.  status[0] is 0 when every wait in the

@@ -549,3 +549,76 @@ def test_layer_with_topp_budget_end_to_end():
         Oo, _ = oracle.attend(*args, w.scale)
         Og = np64(out["O"])[0, h]
         assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2
+
+
+# ---------------------------------------------------------------------------
+# Variance-corrected compensation (SVG-EAR blog, variance paragraph)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_key_variance_matches_oracle(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    kvar = csa.svgear_key_variance(ck.Xp, ck.offsets, w.Ck).cpu().numpy()
+    for h in range(w.H):
+        Kp = np64(ck.Xp)[0, h]
+        off = ck.offsets.cpu().numpy()[0, h]
+        ref = oracle.segment_var(Kp, off)
+        # fp32 two-pass sums: relative to the segment's second moment
+        m2 = oracle.segment_mean(Kp ** 2, off, prev=np.zeros_like(ref))
+        assert np.all(np.abs(kvar[0, h] - ref) <= 2e-5 * m2 + 1e-7)
+
+
+def _check_attend_var(w, dev, lam, density=None, zero_budget=False):
+    csa = _csa()
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    if zero_budget:   # every cluster compensated: no exact tile at all
+        po, pk = csa.svgear_route_select_budget(
+            torch.zeros((1, w.H, w.Cq, w.Ck), dtype=torch.float32, device="cuda"), cq.offsets,
+            ck.offsets, w.N, torch.zeros((1, w.H, w.Cq), dtype=torch.int32, device="cuda"))
+    else:
+        po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
+                                  Vp, density, w.scale)
+    kvar = csa.svgear_key_variance(ck.Xp, ck.offsets, w.Ck)
+    O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
+                          cq.perm, w.scale, check_status=True, kvar=kvar, lam=lam)
+    O0 = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
+                           cq.perm, w.scale, check_status=True)
+    torch.cuda.synchronize()
+    Og, O0g = np64(O), np64(O0)
+    worst = (0.0, 0.0)
+    for h in range(w.H):
+        Oo, _ = oracle.attend(np64(cq.Xp)[0, h], np64(ck.Xp)[0, h], np64(Vp)[0, h],
+                              cq.offsets.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
+                              po.cpu().numpy()[0, h], pk.cpu().numpy()[0, h],
+                              ck.centroids.cpu().numpy()[0, h], vbar.cpu().numpy()[0, h],
+                              cq.perm.cpu().numpy()[0, h], w.scale,
+                              kvar=kvar.cpu().numpy()[0, h], lam=lam)
+        worst = (max(worst[0], _rel_l2(Og[0, h], Oo)),
+                 max(worst[1], float(np.abs(Og[0, h] - Oo).max())))
+    # the term moves the output well beyond the parity tolerance of the path
+    assert _rel_l2(Og, O0g) > (5e-5 if w.dtype == "f32" else 1e-3)
+    return worst
+
+
+@pytest.mark.parametrize("lam", [0.5, 1.0])
+def test_attend_variance_fp32_tiny_within_1e5(lam):
+    host, dev = _inputs(TINY)
+    rel, mx = _check_attend_var(TINY, dev, lam, density=0.1)
+    assert rel <= 1e-5 and mx <= 1e-5, (rel, mx)
+
+
+@pytest.mark.parametrize("lam", [0.5, 1.5])
+@pytest.mark.parametrize("w", [SMALL_BF16, RAGGED_BF16_64, EAR_COUNTS], ids=lambda w: w.name)
+def test_attend_variance_bf16_within_tolerance(w, lam):
+    host, dev = _inputs(w)
+    rel, mx = _check_attend_var(w, dev, lam, density=0.2)
+    assert rel <= 1e-2 and mx <= 2e-2, (rel, mx)
+
+
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16], ids=lambda w: w.name)
+def test_attend_variance_with_every_cluster_compensated(w):
+    host, dev = _inputs(w)
+    rel, mx = _check_attend_var(w, dev, 1.0, zero_budget=True)
+    tol = (1e-5, 1e-5) if w.dtype == "f32" else (1e-2, 2e-2)
+    assert rel <= tol[0] and mx <= tol[1], (rel, mx)
