@@ -48,6 +48,9 @@ def lib():
         L.orc_attend.argtypes = [P, i64, P, P, i32, P, i32, P, i32, P, P, P, P,
                                  P, f64, P, i64, P, P, P, f64]
         L.orc_segment_var.argtypes = [P, i32, P, i32, P]
+        L.orc_probe_value_free.argtypes = [P, i32, P, i64, i32, P, P, i32, f64, P]
+        L.orc_diagnostics.argtypes = [P, P, P, i64, i32, P, i32, P, i32, P, P, P, P, f64, P,
+                                      i64, P, P, P]
         L.orc_num_threads.restype = i32
         _lib = L
     return _lib
@@ -145,6 +148,35 @@ def probe(qbar, Kp, Vp, kbar, vbar, k_off, scale: float, with_scale=False):
     lib().orc_probe(_p(qbar), Cq, _p(Kp), _p(Vp), Kp.shape[0], d, _p(kbar), _p(vbar),
                     _p(k_off), Ck, float(scale), _p(E), _p(S))
     return (E, S) if with_scale else E
+
+
+def probe_value_free(qbar, Kp, kbar, k_off, scale: float):
+    """Value-free probe error Ehat [Cq, Ck] (the probe without the values)."""
+    qbar, Kp, kbar = map(_f64, (qbar, Kp, kbar))
+    k_off = _i32(k_off)
+    Cq, d = qbar.shape
+    Ck = kbar.shape[0]
+    E = np.zeros((Cq, Ck))
+    lib().orc_probe_value_free(_p(qbar), Cq, _p(Kp), Kp.shape[0], d, _p(kbar), _p(k_off), Ck,
+                               float(scale), _p(E))
+    return E
+
+
+def diagnostics(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, O_sparse, q_perm, scale: float,
+                rows):
+    """Attention recall, |O_sparse - O_dense|^2 and |O_dense|^2 of the query
+    rows ``rows`` (permuted positions); O_sparse in the original order."""
+    Qp, Kp, Vp, O_sparse = map(_f64, (Qp, Kp, Vp, O_sparse))
+    q_off, k_off, pair_off, q_perm = map(_i32, (q_off, k_off, pair_off, q_perm))
+    pair_kc = _i32(pair_kc if len(pair_kc) else np.zeros(1, np.int32))
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+    n = r.shape[0]
+    recall, err2, ref2 = np.zeros(n), np.zeros(n), np.zeros(n)
+    lib().orc_diagnostics(_p(Qp), _p(Kp), _p(Vp), Kp.shape[0], Qp.shape[1], _p(q_off),
+                          q_off.shape[0] - 1, _p(k_off), k_off.shape[0] - 1, _p(pair_off),
+                          _p(pair_kc), _p(O_sparse), _p(q_perm), float(scale), _p(r), n,
+                          _p(recall), _p(err2), _p(ref2))
+    return recall, err2, ref2
 
 
 def route(E, q_off, k_off, Nk: int, density: float, budgets=None):

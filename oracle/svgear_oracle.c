@@ -311,6 +311,91 @@ void orc_probe(const double *qbar, int Cq, const double *Kp, const double *Vp,
     }
 }
 
+/* Value-free probe error ([REVIEW] minor comment 1 names a value-free error  */
+/* beside the value-aware one without printing it).  Reading: the probe error */
+/* of orc_probe with the values left out -- the squared gap between the      */
+/* centroid's and each key's weight:                                         */
+/*   Ehat_ic = sum_{t in K_c} (e^{sbar_ic - m_i} - e^{s_it - m_i})^2           */
+/* (the value-aware error when every value is the same unit vector).         */
+void orc_probe_value_free(const double *qbar, int Cq, const double *Kp, int64_t Nk, int d,
+                          const double *kbar, const int32_t *k_off, int Ck, double scale,
+                          double *E) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < Cq; ++i) {
+        const double *q = qbar + (size_t)i * d;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < Nk; ++t) {
+            double s = scale * dot(q, Kp + (size_t)t * d, d);
+            if (s > m) m = s;
+        }
+        for (int c = 0; c < Ck; ++c) {
+            double a = exp(scale * dot(q, kbar + (size_t)c * d, d) - m);
+            double e = 0.0;
+            for (int64_t t = k_off[c]; t < k_off[c + 1]; ++t) {
+                double b = exp(scale * dot(q, Kp + (size_t)t * d, d) - m);
+                e += (a - b) * (a - b);
+            }
+            E[(size_t)i * Ck + c] = e;
+        }
+    }
+}
+
+/* Recall and output error of the sparse layer against dense attention, on   */
+/* query rows rows[r] (permuted positions) -- the diagnostics of the pages:  */
+/* attention recall, the share of the true softmax mass that the computed    */
+/* blocks hold ([SVG2] section 3.1, oracle policy), and the attention MSE    */
+/* against full attention ([REVIEW] Fig. 6a).  For row p of query cluster i: */
+/*   recall[r] = sum_{u in selected clusters of i} e^{s_pu} / sum_u e^{s_pu}  */
+/*   err2[r]   = | O_sparse[q_perm[p]] - O_dense(p) |^2,  ref2[r] = |O_dense|^2 */
+/* with O_dense(p) = sum_u softmax(s_p)_u v_u over every key (fp64).          */
+void orc_diagnostics(const double *Qp, const double *Kp, const double *Vp, int64_t Nk, int d,
+                     const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
+                     const int32_t *pair_off, const int32_t *pair_kc, const double *O_sparse,
+                     const int32_t *q_perm, double scale, const int64_t *rows, int64_t n_rows,
+                     double *recall, double *err2, double *ref2) {
+#pragma omp parallel
+    {
+        unsigned char *sel = (unsigned char *)malloc((size_t)Ck);
+        double *o = (double *)malloc(sizeof(double) * d);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t p = rows[r];
+            int i = 0;
+            while (!(q_off[i] <= p && p < q_off[i + 1])) ++i;
+            memset(sel, 0, (size_t)Ck);
+            for (int32_t e = pair_off[i]; e < pair_off[i + 1]; ++e) sel[pair_kc[e]] = 1;
+            const double *q = Qp + (size_t)p * d;
+            double m = -INFINITY;
+            for (int64_t u = 0; u < Nk; ++u) {
+                double s = scale * dot(q, Kp + (size_t)u * d, d);
+                if (s > m) m = s;
+            }
+            double Z = 0.0, Zsel = 0.0;
+            for (int k = 0; k < d; ++k) o[k] = 0.0;
+            for (int c = 0; c < Ck; ++c) {
+                for (int64_t u = k_off[c]; u < k_off[c + 1]; ++u) {
+                    double w = exp(scale * dot(q, Kp + (size_t)u * d, d) - m);
+                    Z += w;
+                    if (sel[c]) Zsel += w;
+                    for (int k = 0; k < d; ++k) o[k] += w * Vp[(size_t)u * d + k];
+                }
+            }
+            double e2 = 0.0, r2 = 0.0;
+            const double *os = O_sparse + (size_t)q_perm[p] * d;
+            for (int k = 0; k < d; ++k) {
+                double od = o[k] / Z;
+                e2 += (os[k] - od) * (os[k] - od);
+                r2 += od * od;
+            }
+            recall[r] = Zsel / Z;
+            err2[r] = e2;
+            ref2[r] = r2;
+        }
+        free(sel);
+        free(o);
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Error-to-cost greedy routing ([REVIEW] "greedily selecting highest        */
 /* error-to-cost blocks under a density budget"; [BLOG]: error divided by    */

@@ -631,3 +631,84 @@ def test_variance_term_vanishes_for_identical_keys_and_scales_with_lambda():
         w = _weight_of_one_skipped_cluster(keys, q, lam, scale=0.4)
         want = lam * 0.4 ** 2 / 2 * float((q ** 2 * var).sum())
         assert abs(math.log(w / w0) - want) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Value-free probe error and the recall / MSE diagnostics
+# ---------------------------------------------------------------------------
+def test_value_free_error_is_the_value_aware_error_with_unit_values():
+    g = np.random.default_rng(46)
+    d, N, Cq, Ck = 8, 60, 3, 5
+    Kp = g.standard_normal((N, d))
+    k_off = _offsets([10, 0, 25, 5, 20])
+    kbar = np.stack([Kp[k_off[c]:k_off[c + 1]].mean(0) if k_off[c + 1] > k_off[c]
+                     else np.zeros(d) for c in range(Ck)])
+    qbar = g.standard_normal((Cq, d))
+    u = np.zeros(d)
+    u[3] = 1.0                                          # one unit value vector for all
+    Eaware = oracle.probe(qbar, Kp, np.tile(u, (N, 1)), kbar, np.tile(u, (Ck, 1)), k_off, 0.5)
+    Efree = oracle.probe_value_free(qbar, Kp, kbar, k_off, 0.5)
+    assert np.allclose(Efree, Eaware, rtol=1e-12, atol=1e-300)
+    assert np.all(Efree[:, 1] == 0.0)                   # empty cluster
+
+
+def test_value_free_error_closed_form_and_identical_keys():
+    # cluster B of the toy example: scores 0 and 2 for q = 1, centroid score 1;
+    # the row maximum over the keys is 2
+    E = oracle.probe_value_free(np.array([[1.0]]), np.array([[0.0], [2.0]]), np.array([[1.0]]),
+                                np.array([0, 2], dtype=np.int32), 1.0)
+    want = (math.exp(-1) - math.exp(-2)) ** 2 + (math.exp(-1) - 1.0) ** 2
+    assert abs(E[0, 0] - want) < 1e-15
+    same = np.tile(np.array([0.3, -1.2, 0.5]), (7, 1))
+    E = oracle.probe_value_free(np.array([[0.4, 0.1, -2.0]]), same, same[:1],
+                                np.array([0, 7], dtype=np.int32), 0.8)
+    assert E[0, 0] == 0.0
+
+
+def _toy_setup():
+    # one query (q = 1, d = 1, scale 1); cluster A keys score 1, 1; B keys 0, 2
+    Kp = np.array([[1.0], [1.0], [0.0], [2.0]])
+    Vp = np.array([[0.5], [-1.0], [2.0], [3.0]])
+    k_off = np.array([0, 2, 4], dtype=np.int32)
+    kbar = np.array([[1.0], [1.0]])
+    vbar = np.array([[-0.25], [2.5]])
+    return np.array([[1.0]]), Kp, Vp, np.array([0, 1], dtype=np.int32), k_off, kbar, vbar
+
+
+def test_diagnostics_toy_recall_and_exact_output_when_b_is_computed():
+    gold = json.load(open(os.path.join(GOLDEN, "toy_example.json")))["printed"]
+    Qp, Kp, Vp, q_off, k_off, kbar, vbar = _toy_setup()
+    perm = np.array([0], dtype=np.int32)
+    for sel, recall_want in (([1], (1 + math.e ** 2) / (2 * math.e + 1 + math.e ** 2)),
+                             ([0, 1], 1.0), ([], 0.0)):
+        pair_off = np.array([0, len(sel)], dtype=np.int32)
+        pair_kc = np.array(sel, dtype=np.int32)
+        O, _ = oracle.attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, perm, 1.0)
+        rec, err2, ref2 = oracle.diagnostics(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, O, perm,
+                                             1.0, [0])
+        assert abs(rec[0] - recall_want) < 1e-12
+        if sel:   # B computed: A's keys are identical, so its estimate is exact
+            assert err2[0] < 1e-28 and ref2[0] > 0
+    # the printed weights give the same share for B
+    assert abs(gold["weight_B"] / gold["weight_total"] -
+               (1 + math.e ** 2) / (2 * math.e + 1 + math.e ** 2)) < 0.01
+
+
+def test_diagnostics_full_selection_is_dense_attention():
+    g = np.random.default_rng(47)
+    N, d = 40, 6
+    Qp, Kp, Vp = (g.standard_normal((N, d)) for _ in range(3))
+    q_off, k_off = _offsets([15, 25]), _offsets([12, 8, 20])
+    kbar = np.stack([Kp[k_off[c]:k_off[c + 1]].mean(0) for c in range(3)])
+    vbar = np.stack([Vp[k_off[c]:k_off[c + 1]].mean(0) for c in range(3)])
+    pair_off = np.array([0, 3, 6], dtype=np.int32)
+    pair_kc = np.array([0, 1, 2, 0, 1, 2], dtype=np.int32)
+    perm = g.permutation(N).astype(np.int32)
+    O, _ = oracle.attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, perm, 0.7)
+    rows = np.arange(N)
+    rec, err2, ref2 = oracle.diagnostics(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, O, perm, 0.7,
+                                         rows)
+    assert np.allclose(rec, 1.0) and np.all(err2 < 1e-25)
+    S = Qp @ Kp.T * 0.7
+    ref = softmax(S, axis=1) @ Vp
+    assert np.allclose(ref2, (ref ** 2).sum(1))
