@@ -384,7 +384,7 @@ def main():
         O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids,
                               vbar, cq.perm, w.scale, kvar=kvar, lam=args.var_lambda)
         mark(5)
-        return O, (cq, ck, po, pk)
+        return O, (cq, ck, po, pk, Vp)
 
     # the clock sampler starts (and finishes initialising) before the warm-up
     clocks = ClockSampler(local if ws > 1 else torch.cuda.current_device())
@@ -415,7 +415,7 @@ def main():
                 for i, n in enumerate(ev_names)}
 
     # algorithmic work of the attention pass (from the last step's routing)
-    cq, ck, po, pk = state
+    cq, ck, po, pk, Vp_last = state
     BH = w.B * w.H
     q_off = cq.offsets.view(BH, -1).cpu().numpy()
     k_off = ck.offsets.view(BH, -1).cpu().numpy()
@@ -431,6 +431,19 @@ def main():
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": "bf16 dense, sustained, %s" % ("of measured" if peaks["source"] == "measured" else "of fallback"),
                 "traffic": attend_traffic(w), "flops_per_launch": f_sel + f_comp}
+
+    # quality of the timed configuration (not timed): attention recall and the
+    # output error against dense attention on 64 sampled query rows per head
+    g = np.random.default_rng(1234)
+    R = min(64, w.N)
+    rows = np.stack([np.sort(g.choice(w.N, R, replace=False)) for _ in range(BH)])
+    rec, e2, r2 = csa.svgear_diagnostics(
+        cq.Xp, ck.Xp, Vp_last, cq.offsets, ck.offsets, po, pk, O, cq.perm, w.scale,
+        torch.from_numpy(rows.astype(np.int32)).view(w.B, w.H, R).to(dev))
+    rec, e2, r2 = (t.double().cpu().numpy() for t in (rec, e2, r2))
+    quality = {"rows_per_head": R, "recall_mean": float(rec.mean()),
+               "recall_min": float(rec.min()),
+               "relative_mse": float(e2.sum() / max(r2.sum(), 1e-300))}
 
     # end to end: pinned host inputs -> device -> layer -> O back to pinned host
     e2e = None
@@ -478,6 +491,7 @@ def main():
             "attention_tflops": achieved,
             "stages_ms": stage_ms,
             "roofline": roofline,
+            "quality": quality,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clk,

@@ -32,6 +32,7 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_version", "svgear_kernel_launches", "svgear_attend_status",
             "svgear_device_status", "svgear_topp_budget", "svgear_route_select_budget",
             "svgear_route_topp", "svgear_key_variance", "svgear_attend_var",
+            "svgear_probe_value_free", "svgear_diagnostics",
             "svgear_label_sort_noalloc")
 
 
@@ -75,6 +76,9 @@ def lib():
         "svgear_route_select_budget": [P, P, I32, P, I32, I32, I32, I32, P, P, P, P, SZ, P],
         "svgear_route_topp": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, P, SZ, P],
         "svgear_key_variance": [P, P, I32, Dims, P, P],
+        "svgear_probe_value_free": [P, I32, P, P, P, I32, Dims, F, P, P, SZ, P],
+        "svgear_diagnostics": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, F, P, I32, P, P, P,
+                               P],
         "svgear_attend_var": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, F, P, P, SZ,
                               P],
         "svgear_attend": [P, P, P, Dims, I32, P, I32, P, I32, P, P, P, P, P, F, P, P, SZ, P],
@@ -346,6 +350,37 @@ def svgear_route(qbar, q_off, kbar, vbar, k_off, Kp, Vp, density, scale, return_
         kd, float(density), float(scale), _ptr(pair_off), _ptr(pair_kc), _ptr(E), _ptr(ws), n,
         _stream()))
     return (pair_off, pair_kc, E) if return_errors else (pair_off, pair_kc)
+
+
+def svgear_probe_value_free(qbar, Kp, kbar, k_off, scale):
+    """Value-free probe error Ehat float32 [B, H, Cq, Ck]."""
+    kd = _tokens(Kp, "Kp")
+    B, H, Cq, d = qbar.shape
+    Ck = kbar.shape[2]
+    E = torch.empty((B, H, Cq, Ck), dtype=torch.float32, device=Kp.device)
+    ws, n = _workspace(OP_ROUTE, kd, Cq, Ck, Kp.device)
+    _check("svgear_probe_value_free", lib().svgear_probe_value_free(
+        _ptr(qbar), Cq, _ptr(Kp), _ptr(kbar), _ptr(k_off), Ck, kd, float(scale), _ptr(E),
+        _ptr(ws), n, _stream()))
+    return E
+
+
+def svgear_diagnostics(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, O, q_perm, scale, rows):
+    """Attention recall, |O - O_dense|^2 and |O_dense|^2 on the sampled
+    permuted rows ``rows`` (int32 [B, H, R]); each float32 [B, H, R]."""
+    qd = _tokens(Qp, "Qp")
+    _tokens(Kp, "Kp")
+    _tokens(Vp, "Vp")
+    _cuda(rows, "rows", torch.int32)
+    B, H, R = rows.shape
+    Cq = q_off.shape[-1] - 1
+    Ck = k_off.shape[-1] - 1
+    out = [torch.empty((B, H, R), dtype=torch.float32, device=Qp.device) for _ in range(3)]
+    _check("svgear_diagnostics", lib().svgear_diagnostics(
+        _ptr(Qp), _ptr(Kp), _ptr(Vp), qd, Kp.shape[2], _ptr(q_off), Cq, _ptr(k_off), Ck,
+        _ptr(pair_off), _ptr(pair_kc), _ptr(O), _ptr(q_perm), float(scale), _ptr(rows), R,
+        _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _stream()))
+    return tuple(out)
 
 
 def svgear_key_variance(Kp, k_off, Ck):

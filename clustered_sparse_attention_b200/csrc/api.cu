@@ -536,6 +536,40 @@ int svgear_attend(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd
                              vbar, nullptr, 0.f, q_perm, scale, O, ws, ws_bytes, stream);
 }
 
+int svgear_probe_value_free(const float* qbar, int32_t Cq, const void* Kp, const float* kbar,
+                            const int32_t* k_off, int32_t Ck, svgear_dims kdims, float scale,
+                            float* E, void* ws, size_t ws_bytes, void* stream) {
+    int s = check_dims(kdims);
+    if (s) return s;
+    if ((s = check_route_common(Cq, Ck, kdims.N, 1.f))) return s;
+    if (!qbar || !Kp || !kbar || !k_off || !E || !ws || !aligned16(Kp) || !isfinite(scale))
+        return SVGEAR_ERR_INVALID_ARG;
+    if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
+    if (bh_of(kdims) == 0) return SVGEAR_OK;
+    Carve cv(ws);
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
+    return launch_probe(qbar, Cq, Kp, nullptr, kbar, nullptr, k_off, Ck, kdims, scale, E,
+                        w.rowmax, static_cast<cudaStream_t>(stream), true);
+}
+
+int svgear_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                       int32_t Nk, const int32_t* q_off, int32_t Cq, const int32_t* k_off,
+                       int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc, const void* O,
+                       const int32_t* q_perm, float scale, const int32_t* rows, int32_t R,
+                       float* recall, float* err2, float* ref2, void* stream) {
+    int s = check_dims(qdims);
+    if (s) return s;
+    if (Nk < 1 || R < 0) return SVGEAR_ERR_INVALID_ARG;
+    if ((s = check_route_common(Cq, Ck, Nk, 1.f))) return s;
+    if (!Qp || !Kp || !Vp || !q_off || !k_off || !pair_off || !pair_kc || !O || !q_perm ||
+        !rows || !recall || !err2 || !ref2 || !isfinite(scale))
+        return SVGEAR_ERR_INVALID_ARG;
+    if (bh_of(qdims) == 0 || R == 0) return SVGEAR_OK;
+    return launch_diagnostics(Qp, Kp, Vp, qdims, Nk, q_off, Cq, k_off, Ck, pair_off, pair_kc, O,
+                              q_perm, scale, rows, R, recall, err2, ref2,
+                              static_cast<cudaStream_t>(stream));
+}
+
 int svgear_key_variance(const void* Kp, const int32_t* k_off, int32_t Ck, svgear_dims kdims,
                         float* kvar, void* stream) {
     int s = check_dims(kdims);

@@ -36,6 +36,13 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* centroids,
                         const int32_t* done, int32_t* changed);
 size_t assign_sm100_scratch_bytes(int BH, int C, int D);
 int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st);
+// Recall and output error against dense attention on sampled query rows
+// (diagnostics.cu).
+int launch_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd, int Nk,
+                       const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
+                       const int32_t* pair_off, const int32_t* pair_kc, const void* O,
+                       const int32_t* q_perm, float scale, const int32_t* rows, int R,
+                       float* recall, float* err2, float* ref2, cudaStream_t st);
 // Per-coordinate population variance of every contiguous segment of X.
 int launch_segment_var(const void* X, const int32_t* offsets, int C, svgear_dims dims,
                        float* out, cudaStream_t st);
@@ -56,7 +63,7 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp,
                  const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
                  svgear_dims kdims, float scale, float* E, uint32_t* rowmax,
-                 cudaStream_t st);
+                 cudaStream_t st, bool value_free = false);
 int launch_route_select(const float* E, const int32_t* q_off, int Cq, const int32_t* k_off,
                         int Ck, int BH, long long budget, const int32_t* budgets, int32_t* lists,
                         int32_t* counts, int32_t* pair_off, int32_t* pair_kc, cudaStream_t st);

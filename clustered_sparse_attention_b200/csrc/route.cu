@@ -89,7 +89,8 @@ probe_rowmax_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict_
         atomicMax(rowmax + (size_t)bh * Cq + i0 + lane, float_to_ordered(best));
 }
 
-template <typename T, int D>
+// VF: the value-free error sum_t (a_ic - b_it)^2 (values not read).
+template <typename T, int D, bool VF>
 __global__ void __launch_bounds__(kPrThreads)
 probe_error_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__ Kp,
                    const T* __restrict__ Vp, const float* __restrict__ kbar,
@@ -125,16 +126,18 @@ probe_error_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__
     float dotk = 0.f;
     for (int k = 0; k < D; ++k) dotk = fmaf(Qs[lane * P + k], kb_s[k], dotk);
     const float aic = expf(scale * dotk - m);
-    const float* vb = vbar + ((size_t)bh * Ck + c) * D;
     // every thread needs a_ic of every probe: broadcast through smem
     if (warp == 0) red[lane] = aic;
     __syncthreads();
-    for (int q = tid; q < kPrProbes * D; q += kPrThreads) {
-        const int p = q / D, k = q % D;
-        AV[p * P + k] = red[p] * vb[k];
+    if constexpr (!VF) {   // the value-free error reads no values
+        const float* vb = vbar + ((size_t)bh * Ck + c) * D;
+        for (int q = tid; q < kPrProbes * D; q += kPrThreads) {
+            const int p = q / D, k = q % D;
+            AV[p * P + k] = red[p] * vb[k];
+        }
     }
     const T* Kh = Kp + (size_t)bh * Nk * D;
-    const T* Vh = Vp + (size_t)bh * Nk * D;
+    const T* Vh = VF ? nullptr : Vp + (size_t)bh * Nk * D;
     float err = 0.f;
     for (int tb = a; tb < b; tb += kPrKeys) {
         __syncthreads();
@@ -143,7 +146,12 @@ probe_error_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__
             float kv[EPC], vv[EPC];
             if (tb + r < b) {
                 Elem<T>::load(Kh + (size_t)(tb + r) * D + col, kv);
-                Elem<T>::load(Vh + (size_t)(tb + r) * D + col, vv);
+                if constexpr (!VF) {
+                    Elem<T>::load(Vh + (size_t)(tb + r) * D + col, vv);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) vv[e] = 0.f;
+                }
             } else {
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) { kv[e] = 0.f; vv[e] = 0.f; }
@@ -173,28 +181,34 @@ probe_error_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
             bw[jj] = (tb + warp * 8 + jj < b) ? expf(scale * s[jj] - m) : 0.f;
-        // direct form: sum_k (a vbar_k - b v_k)^2 per key
-        float e8[8];
+        if constexpr (VF) {   // value-free: (a - b)^2 per key
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) e8[jj] = 0.f;
-        const float* avr = AV + lane * P;
+            for (int jj = 0; jj < 8; ++jj)
+                if (tb + warp * 8 + jj < b) err += (aic - bw[jj]) * (aic - bw[jj]);
+        } else {
+            // direct form: sum_k (a vbar_k - b v_k)^2 per key
+            float e8[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) e8[jj] = 0.f;
+            const float* avr = AV + lane * P;
 #pragma unroll 2
-        for (int k = 0; k < D; k += 4) {
-            const float4 av = *reinterpret_cast<const float4*>(avr + k);
+            for (int k = 0; k < D; k += 4) {
+                const float4 av = *reinterpret_cast<const float4*>(avr + k);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const float4 vv = *reinterpret_cast<const float4*>(Vs + (warp * 8 + jj) * P + k);
-                float d0 = fmaf(-bw[jj], vv.x, av.x), d1 = fmaf(-bw[jj], vv.y, av.y);
-                float d2 = fmaf(-bw[jj], vv.z, av.z), d3 = fmaf(-bw[jj], vv.w, av.w);
-                e8[jj] = fmaf(d0, d0, e8[jj]);
-                e8[jj] = fmaf(d1, d1, e8[jj]);
-                e8[jj] = fmaf(d2, d2, e8[jj]);
-                e8[jj] = fmaf(d3, d3, e8[jj]);
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float4 vv = *reinterpret_cast<const float4*>(Vs + (warp * 8 + jj) * P + k);
+                    float d0 = fmaf(-bw[jj], vv.x, av.x), d1 = fmaf(-bw[jj], vv.y, av.y);
+                    float d2 = fmaf(-bw[jj], vv.z, av.z), d3 = fmaf(-bw[jj], vv.w, av.w);
+                    e8[jj] = fmaf(d0, d0, e8[jj]);
+                    e8[jj] = fmaf(d1, d1, e8[jj]);
+                    e8[jj] = fmaf(d2, d2, e8[jj]);
+                    e8[jj] = fmaf(d3, d3, e8[jj]);
+                }
             }
-        }
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-            if (tb + warp * 8 + jj < b) err += e8[jj];
+            for (int jj = 0; jj < 8; ++jj)
+                if (tb + warp * 8 + jj < b) err += e8[jj];
+        }
     }
     __syncthreads();
     red[warp * 32 + lane] = err;
@@ -217,7 +231,7 @@ template <typename T, int D>
 static int probe_impl(const float* qbar, int Cq, const void* Kp, const void* Vp,
                       const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
                       svgear_dims kd, float scale, float* E, uint32_t* rowmax,
-                      cudaStream_t st) {
+                      bool value_free, cudaStream_t st) {
     constexpr int P = ProbeSmem<D>::kPad;
     const int BH = kd.B * kd.H, Nk = kd.N;
     const size_t nrow = (size_t)BH * Cq;
@@ -233,10 +247,11 @@ static int probe_impl(const float* qbar, int Cq, const void* Kp, const void* Vp,
                                                        scale, rowmax);
     count_launches(1);
     const size_t sm2 = sizeof(float) * ((2 * kPrProbes + 2 * kPrKeys) * P + 8 * 32);
-    if (cudaFuncSetAttribute(probe_error_kernel<T, D>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2) != cudaSuccess)
+    auto kern = value_free ? probe_error_kernel<T, D, true> : probe_error_kernel<T, D, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2) !=
+        cudaSuccess)
         return SVGEAR_ERR_CUDA;
-    probe_error_kernel<T, D><<<dim3(Ck, ceil_div(Cq, kPrProbes), BH), kPrThreads, sm2, st>>>(
+    kern<<<dim3(Ck, ceil_div(Cq, kPrProbes), BH), kPrThreads, sm2, st>>>(
         qbar, Cq, static_cast<const T*>(Kp), static_cast<const T*>(Vp), kbar, vbar, k_off, Ck,
         Nk, scale, rowmax, E);
     count_launches(1);
@@ -247,19 +262,20 @@ static int probe_impl(const float* qbar, int Cq, const void* Kp, const void* Vp,
 template <typename T, int D>
 static int probe_disp(const float* qbar, int Cq, const void* Kp, const void* Vp,
                       const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
-                      svgear_dims kd, float scale, float* E, uint32_t* rowmax, cudaStream_t st) {
-    return probe_impl<T, D>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, st);
+                      svgear_dims kd, float scale, float* E, uint32_t* rowmax, bool vf,
+                      cudaStream_t st) {
+    return probe_impl<T, D>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, vf, st);
 }
 
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp, const float* kbar,
                  const float* vbar, const int32_t* k_off, int Ck, svgear_dims kd, float scale,
-                 float* E, uint32_t* rowmax, cudaStream_t st) {
+                 float* E, uint32_t* rowmax, cudaStream_t st, bool value_free) {
     if (kd.dtype == SVGEAR_BF16) {
-        if (kd.d == 128) return probe_disp<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, st);
-        if (kd.d == 64) return probe_disp<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, st);
+        if (kd.d == 128) return probe_disp<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
+        if (kd.d == 64) return probe_disp<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
     } else if (kd.dtype == SVGEAR_F32) {
-        if (kd.d == 128) return probe_disp<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, st);
-        if (kd.d == 64) return probe_disp<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, st);
+        if (kd.d == 128) return probe_disp<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
+        if (kd.d == 64) return probe_disp<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
     }
     return SVGEAR_ERR_UNSUPPORTED;
 }

@@ -347,6 +347,41 @@ int svgear_attend_var(const void* Qp, const void* Kp, const void* Vp, svgear_dim
                       const int32_t* q_perm, float scale, void* O, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* --------------------------------------------------------------------------
+ * svgear_probe_value_free -- the probe error without the values ([REVIEW]
+ * minor comment 1 names a value-free error beside the value-aware one; its
+ * formula is not printed there).  Reading:
+ *   Ehat[i][c] = sum_{t in K_c} ( e^{sbar_ic - m_i} - e^{s_it - m_i} )^2
+ * (the svgear_probe error when every value is the same unit vector; fp32).
+ * Arguments, layouts and workspace as svgear_probe minus the values; the
+ * result feeds svgear_route_select / svgear_route_select_budget like E.
+ * ------------------------------------------------------------------------ */
+int svgear_probe_value_free(const float* qbar, int32_t Cq, const void* Kp, const float* kbar,
+                            const int32_t* k_off, int32_t Ck, svgear_dims kdims, float scale,
+                            float* E, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * svgear_diagnostics -- how close a layer call came to dense attention, on
+ * sampled query rows ([SVG2] section 3.1, attention recall under the oracle
+ * policy; [REVIEW] Fig. 6a, attention MSE against full attention).  For each
+ * sampled row p (a permuted position) of query cluster i:
+ *   recall[r] = sum over the keys of i's selected clusters of e^{s_pu}
+ *               / sum over every key of e^{s_pu}
+ *   err2[r]   = | O[q_perm[p]] - O_dense(p) |^2,  ref2[r] = | O_dense(p) |^2
+ * with O_dense(p) the dense softmax output (fp32, every key).
+ *   Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, q_perm: as for svgear_attend.
+ *   O      [B][H][Nq][d] the layer's output (qdims.dtype), original order.
+ *   rows   int32[B][H][R] permuted row positions; R >= 0.
+ *   recall, err2, ref2  out float[B][H][R] (NaN for a row out of range).
+ * No workspace; asynchronous on `stream`.  A measurement, not part of the
+ * layer: its cost is R * Nk * d multiply-adds per head.
+ * ------------------------------------------------------------------------ */
+int svgear_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,
+                       int32_t Nk, const int32_t* q_off, int32_t Cq, const int32_t* k_off,
+                       int32_t Ck, const int32_t* pair_off, const int32_t* pair_kc, const void* O,
+                       const int32_t* q_perm, float scale, const int32_t* rows, int32_t R,
+                       float* recall, float* err2, float* ref2, void* stream);
+
 /* Device status of the last svgear_cluster, svgear_kmeans_assign or
  * svgear_attend that used `ws`: copies 4 int32 to status[0..3] (host memory)
  * and synchronises `stream`.  status[0] is 0 when every wait in the

@@ -622,3 +622,61 @@ def test_attend_variance_with_every_cluster_compensated(w):
     rel, mx = _check_attend_var(w, dev, 1.0, zero_budget=True)
     tol = (1e-5, 1e-5) if w.dtype == "f32" else (1e-2, 2e-2)
     assert rel <= tol[0] and mx <= tol[1], (rel, mx)
+
+
+# ---------------------------------------------------------------------------
+# Value-free probe error and the recall / MSE diagnostics
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
+def test_value_free_probe_matches_oracle(w):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    E = csa.svgear_probe_value_free(cq.centroids, ck.Xp, ck.centroids, ck.offsets, w.scale)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        qbar = cq.centroids.cpu().numpy()[0, h]
+        Kp = np64(ck.Xp)[0, h]
+        off = ck.offsets.cpu().numpy()[0, h]
+        kb = ck.centroids.cpu().numpy()[0, h]
+        Eo = oracle.probe_value_free(qbar, Kp, kb, off, w.scale)
+        # error scale of the bound: the value-aware probe with unit values
+        u = np.zeros(w.d)
+        u[0] = 1.0
+        _, So = oracle.probe(qbar, Kp, np.tile(u, (w.N, 1)), kb, np.tile(u, (w.Ck, 1)), off,
+                             w.scale, with_scale=True)
+        tol = probe_tolerance(qbar, Kp, Eo, So, w.scale)
+        Eg = E.cpu().numpy()[0, h].astype(np.float64)
+        assert np.all(np.abs(Eg - Eo) <= tol), float(np.max(np.abs(Eg - Eo) / tol))
+
+
+@pytest.mark.parametrize("density", [0.2, 1.0])
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16], ids=lambda w: w.name)
+def test_diagnostics_match_oracle(w, density):
+    csa = _csa()
+    host, dev = _inputs(w)
+    cq, ck, Vp, vbar = _clustered(w, dev)
+    po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets, ck.Xp,
+                              Vp, density, w.scale)
+    O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids, vbar,
+                          cq.perm, w.scale, check_status=True)
+    g = np.random.default_rng(9)
+    R = 48
+    rows = np.stack([np.sort(g.choice(w.N, R, replace=False)) for _ in range(w.H)])[None]
+    rec, e2, r2 = csa.svgear_diagnostics(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, O,
+                                         cq.perm, w.scale,
+                                         torch.from_numpy(rows.astype(np.int32)).cuda())
+    torch.cuda.synchronize()
+    rec, e2, r2 = (t.cpu().numpy().astype(np.float64) for t in (rec, e2, r2))
+    for h in range(w.H):
+        ro, eo, fo = oracle.diagnostics(np64(cq.Xp)[0, h], np64(ck.Xp)[0, h], np64(Vp)[0, h],
+                                        cq.offsets.cpu().numpy()[0, h],
+                                        ck.offsets.cpu().numpy()[0, h], po.cpu().numpy()[0, h],
+                                        pk.cpu().numpy()[0, h], np64(O)[0, h],
+                                        cq.perm.cpu().numpy()[0, h], w.scale, rows[0, h])
+        assert np.all(np.abs(rec[0, h] - ro) <= 1e-5)
+        assert np.all(np.abs(r2[0, h] - fo) <= 1e-5 * fo + 1e-9)
+        # fp32 dense output against fp64: |d err2| <= 2 |O - O_d| |dO_d| + |dO_d|^2
+        assert np.all(np.abs(e2[0, h] - eo) <= 4e-5 * np.sqrt(eo * fo) + 1e-9 * fo + 1e-12)
+        if density == 1.0:
+            assert np.allclose(rec[0, h], 1.0, atol=1e-6)
