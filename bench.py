@@ -242,34 +242,22 @@ def oracle_sample_ms(w, seconds=15.0, density=None, iters=None, topp=None):
 # ---------------------------------------------------------------------------
 def dist_setup(args):
     import torch
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    else:
+
+    from clustered_sparse_attention_b200 import ranks
+    ws, rank, local = ranks.setup("nccl")
+    if ws == 1:
         torch.cuda.set_device(0)
     return ws, rank, local
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from clustered_sparse_attention_b200 import ranks
+    ranks.barrier(ws)
 
 
 def max_over_ranks(x, ws):
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from clustered_sparse_attention_b200 import ranks
+    return ranks.max_over_ranks(x, ws, device="cuda")
 
 
 def run_reference(args, w):
@@ -346,6 +334,7 @@ def main():
     import torch
 
     import clustered_sparse_attention_b200 as csa
+    from clustered_sparse_attention_b200 import ranks as ranks_mod
     ws, rank, local = dist_setup(args)
     iters = args.iters or w.iters
     density = args.density or w.density
@@ -355,8 +344,9 @@ def main():
     def host_tensor(name):
         if w.dtype == "f32":   # the small fp32 workload: every rank draws batch 0
             return torch.from_numpy(synth.layer_tensor(w, name, threads=min(16, os.cpu_count() or 1)))
+        from clustered_sparse_attention_b200 import ranks
         bits = synth.layer_tensor_bits(w, name, threads=min(16, os.cpu_count() or 1),
-                                       batch_offset=rank)
+                                       batch_offset=ranks.batch_offset(rank))
         return torch.from_numpy(bits).view(torch.bfloat16)
 
     host = {n: host_tensor(n).pin_memory() for n in ("q", "k", "v")}
@@ -521,7 +511,8 @@ def main():
         barrier(ws)
         e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, ws)
         nbytes = w.B * w.H * w.N * w.d * 2
-        e2e = {"value": e2e_ms / ws, "unit": "ms", "h2d_bytes_per_step": 3 * nbytes,
+        e2e = {"value": ranks_mod.job_ms_per_call(e2e_ms, ws), "unit": "ms",
+               "h2d_bytes_per_step": 3 * nbytes,
                "d2h_bytes_per_step": nbytes}
 
     cpu = None
@@ -533,7 +524,8 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": ms_step_max / ws, "unit": "ms", "n_gpus": ws,
+            "metric": METRIC, "value": ranks_mod.job_ms_per_call(ms_step_max, ws), "unit": "ms",
+            "n_gpus": ws,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step_max,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic: seeded patch-coherent Gaussian mixtures at the %s shape" % w.name,
@@ -549,9 +541,7 @@ def main():
             "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    ranks_mod.teardown(ws)
 
 
 if __name__ == "__main__":

@@ -42,7 +42,8 @@ using tc::warp_wait_bar;
 
 constexpr int BM = 128;                  // tokens per tile (TMEM lanes)
 constexpr int kPlanes = 3;               // bf16 planes of a centroid
-constexpr int kBStages = 4;              // centroid-plane ring
+constexpr int kMaxBStages = 8;           // centroid-plane ring (barrier arrays)
+constexpr int kBStagesUsed = 4;          // ring depth launched
 constexpr int kThreads = 6 * 32;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiThreads = 128;
@@ -59,8 +60,8 @@ struct Maps {
 struct Shared {
     uint64_t a_full[kMaxAStages];
     uint64_t a_empty[kMaxAStages];
-    uint64_t b_full[kBStages];
-    uint64_t b_empty[kBStages];
+    uint64_t b_full[kMaxBStages];
+    uint64_t b_empty[kMaxBStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -82,6 +83,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc, int nA,
+                    int nB,
                     const float* __restrict__ cnorm, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
                     int* __restrict__ err) {
@@ -109,7 +111,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             tc::mbar_init(tc::smem_u32(&sh.acc_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.acc_empty[s]), kEpiThreads);
         }
-        for (int s = 0; s < kBStages; ++s) {
+        for (int s = 0; s < kMaxBStages; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.b_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.b_empty[s]), 1);
         }
@@ -158,9 +160,9 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             for (int c = 0; ok && c < nchunk; ++c) {
                 for (int p = 0; ok && p < kPlanes; ++p) {
                     for (int kh = 0; kh < KH; ++kh) {
-                        const int sb = ib % kBStages;
-                        if (ib >= kBStages &&
-                            !warp_wait_bar(&sh.b_empty[sb], ((ib / kBStages) - 1) & 1, abort_flag, err,
+                        const int sb = ib % nB;
+                        if (ib >= nB &&
+                            !warp_wait_bar(&sh.b_empty[sb], ((ib / nB) - 1) & 1, abort_flag, err,
                                            (2 << 16) + (ib & 0xffff))) {
                             ok = false;
                             break;
@@ -183,9 +185,9 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 const int i = ia - 1 - k;
                 drain_wait(&sh.a_full[i % nA], (i / nA) & 1);
             }
-            for (int k = 0; k < kBStages && k < ib; ++k) {
+            for (int k = 0; k < nB && k < ib; ++k) {
                 const int i = ib - 1 - k;
-                drain_wait(&sh.b_full[i % kBStages], (i / kBStages) & 1);
+                drain_wait(&sh.b_full[i % nB], (i / nB) & 1);
             }
         }
         __syncwarp();
@@ -213,8 +215,8 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 tc::fence_after_sync();
                 for (int p = 0; ok && p < kPlanes; ++p) {
                     for (int kh = 0; kh < KH; ++kh) {
-                        const int sb = ib % kBStages;
-                        if (!warp_wait_bar(&sh.b_full[sb], (ib / kBStages) & 1, abort_flag, err,
+                        const int sb = ib % nB;
+                        if (!warp_wait_bar(&sh.b_full[sb], (ib / nB) & 1, abort_flag, err,
                                            (5 << 16) + (ib & 0xffff))) {
                             ok = false;
                             break;
@@ -410,11 +412,14 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         return SVGEAR_ERR_CUDA;
     const int total = BH * ceil_div(N, BM);
     const int grid = total < num_sms[dev] ? total : num_sms[dev];
-    // the centroid ring takes kBStages boxes of Nc rows; the token-tile stages
+    // the centroid ring takes kBStagesUsed boxes of Nc rows (a deeper ring,
+    // bought with token-tile stages, measured slower); the token-tile stages
     // take what shared memory has left (2 to kMaxAStages)
-    const size_t a_bytes = (size_t)(D / 64) * 16384, b_bytes = (size_t)kBStages * Nc * 128;
+    const size_t a_bytes = (size_t)(D / 64) * 16384, b_stage = (size_t)Nc * 128;
     const size_t budget = 227 * 1024 - 1024 - sizeof(Shared) - 64;
-    if (budget < b_bytes + 2 * a_bytes) return SVGEAR_ERR_UNSUPPORTED;
+    const int nB = kBStagesUsed;
+    if (budget < 2 * a_bytes + (size_t)nB * b_stage) return SVGEAR_ERR_UNSUPPORTED;
+    const size_t b_bytes = (size_t)nB * b_stage;
     int nA = (int)((budget - b_bytes) / a_bytes);
     if (nA > kMaxAStages) nA = kMaxAStages;
     const size_t smem = (size_t)nA * a_bytes + b_bytes + 1024;
@@ -425,7 +430,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, cn, labels,
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, cn, labels,
                                                                done, changed, err);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
@@ -434,7 +439,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, cn, labels,
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, cn, labels,
                                                               done, changed, err);
     }
     count_launches(1);
