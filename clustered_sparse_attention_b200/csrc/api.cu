@@ -65,7 +65,7 @@ KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
     w.D2 = cv.take<float>(bh_of(d) * d.N);
     w.blocksum = cv.take<double>(bh_of(d) * ceil_div(d.N, kKppTokens));
     w.chosen = cv.take<int32_t>(bh_of(d) * C);
-    w.counter = cv.take<int32_t>(bh_of(d));
+    w.counter = cv.take<int32_t>(2 * bh_of(d));   // arrivals, then block claims
     w.nearest = cv.take<int32_t>(bh_of(d) * d.N);
     w.cc2 = cv.take<float>(bh_of(d) * C);
     w.gen = cv.take<int32_t>(bh_of(d));

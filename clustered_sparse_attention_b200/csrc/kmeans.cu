@@ -74,7 +74,7 @@ template <typename T, int D>
 __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32_t* chosen, int C,
                          int j, const float* D2, const double* blocksum, uint64_t seed,
                          float* centroids, float* cc2, float* d2s, double* warp_tot, float* cnew) {
-    __shared__ int s_blk, s_pick;
+    __shared__ int s_blk, s_pick, s_last;
     __shared__ double s_base, s_target;
     const int tid = threadIdx.x;
     const double* bs = blocksum + (size_t)bh * nblk;
@@ -86,22 +86,53 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32
     constexpr int kCached = kKppTokens / 2;
     for (int b = tid; b < nblk && b < kCached; b += kKppThreads) bsum[b] = __ldcg(bs + b);
     __syncthreads();
-    if (tid == 0) {
-        double total = 0.0;
-        for (int b = 0; b < nblk; ++b) total += b < kCached ? bsum[b] : __ldcg(bs + b);
-        s_pick = 0x7fffffff;
+    if (tid < 32) {
+        // Lane l owns the block sums [l*per, l*per + per).  The running sum at
+        // block b of lane l's chunk is E_l + (the chunk's sequential partial
+        // sum through b), E_l the exclusive shuffle scan of the chunk totals:
+        // a fixed structure, so the pick is the same on every run.
+        const int lane = tid, per = (nblk + 31) / 32;
+        const int b0 = min(lane * per, nblk), b1 = min(b0 + per, nblk);
+        double c = 0.0;
+        for (int b = b0; b < b1; ++b) c += b < kCached ? bsum[b] : __ldcg(bs + b);
+        double x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        double E = __shfl_up_sync(0xffffffffu, x, 1);
+        if (lane == 0) E = 0.0;
+        const double endv = E + c;
+        const double total = __shfl_sync(0xffffffffu, endv, 31);
+        int hit = -3;               // every D^2 is zero
+        double base = 0.0, target = 0.0;
         if (total > 0.0) {
-            const double target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
-            s_target = target;
-            s_blk = -2;
-            double run = 0.0;
-            for (int b = 0; b < nblk; ++b) {
-                const double prev = run;
-                run = prev + (b < kCached ? bsum[b] : __ldcg(bs + b));
-                if (run > target) { s_blk = b; s_base = prev; break; }
+            target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
+            const unsigned m = __ballot_sync(0xffffffffu, b1 > b0 && endv > target);
+            hit = -2;               // rounding left no block above the target
+            if (m) {
+                const int src = __ffs(m) - 1;
+                int h = b1 - 1;     // the chunk's end value is above the target
+                double prev = E, part = 0.0;
+                if (lane == src) {
+                    for (int b = b0; b < b1; ++b) {
+                        part += b < kCached ? bsum[b] : __ldcg(bs + b);
+                        const double run = E + part;
+                        if (run > target) { h = b; break; }
+                        prev = run;
+                    }
+                }
+                hit = __shfl_sync(0xffffffffu, h, src);
+                base = __shfl_sync(0xffffffffu, prev, src);
             }
-        } else {
-            s_blk = -3;
+        }
+        if (lane == 0) {
+            s_pick = 0x7fffffff;
+            s_last = -1;
+            s_blk = hit;
+            s_base = base;
+            s_target = target;
         }
     }
     __syncthreads();
@@ -121,6 +152,15 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32
             }
         }
         __syncthreads();
+        if (s_pick == 0x7fffffff) {
+            // the block-level and token-level sums rounded apart and no token
+            // of the block reaches the target: take its last token with D^2 > 0
+            for (int i = 0; i < 4; ++i)
+                if (d2s[tid * 4 + i] > 0.f) atomicMax(&s_last, blk * kKppTokens + tid * 4 + i);
+            __syncthreads();
+            if (tid == 0 && s_last >= 0) s_pick = s_last;
+            __syncthreads();
+        }
     } else if (tid == 0) {
         int pick = 0;
         if (blk == -2) {            // rounding left no token above the target
@@ -145,21 +185,25 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32
         centroids[((size_t)bh * C + j) * D + k] = v;
     }
     __syncthreads();
-    // |c_j - c_a|^2 for a < j, one earlier seed per thread (rows of seeds a < j
-    // were written by earlier launches)
-    const float* cen = centroids + (size_t)bh * C * D;
+    // |c_j - c_a|^2 for a < j, one earlier seed per thread.  Seeds are rows
+    // of X, so the distances read those rows in X's own type (half the bytes
+    // of the fp32 centroid rows for bf16 inputs); this is the pass's latency
+    // tail, bound by the loads one thread keeps in flight.
+    constexpr int EPC = Elem<T>::kPerChunk;
+    constexpr int NCH = D / EPC;
+    const T* Xh = X + (size_t)bh * N * D;
     for (int a = tid; a < j; a += kKppThreads) {
-        const float4* ra = reinterpret_cast<const float4*>(cen + (size_t)a * D);
+        const T* ra = Xh + (size_t)__ldcg(ch + a) * D;
         float acc = 0.f;
 #pragma unroll 8
-        for (int k = 0; k < D / 4; ++k) {
-            const float4 v = __ldcg(ra + k);
-            const float d0 = v.x - cnew[4 * k], d1 = v.y - cnew[4 * k + 1];
-            const float d2v = v.z - cnew[4 * k + 2], d3 = v.w - cnew[4 * k + 3];
-            acc = fmaf(d0, d0, acc);
-            acc = fmaf(d1, d1, acc);
-            acc = fmaf(d2v, d2v, acc);
-            acc = fmaf(d3, d3, acc);
+        for (int k = 0; k < NCH; ++k) {
+            float v[EPC];
+            Elem<T>::unpack(Elem<T>::load_raw(ra + k * EPC), v);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                const float df = v[e] - cnew[k * EPC + e];
+                acc = fmaf(df, df, acc);
+            }
         }
         cc2[(size_t)bh * C + a] = acc;
     }
@@ -284,12 +328,16 @@ __device__ void kpp_block_update(const T* __restrict__ X, int N, int nblk, int b
     __syncthreads();   // d2s and warp_tot are reused by the next block
 }
 
-// Persistent seeding: CTA c works for head bh0 + c / cph on its share of the
-// head's 1024-token blocks, for every seed.  Before pass j (which adds seed
-// j-1) it waits until the head's generation word gen[bh] reaches j; after its
-// blocks it arrives on counter[bh]; the last CTA of the head to arrive picks
-// seed j (and the seed-to-seed distances of the next screen), resets the
-// counter and publishes gen[bh] = j + 1.  Heads never wait for each other, so
+// Persistent seeding: CTA c works for head bh0 + c / cph, for every seed.
+// Before pass j (which adds seed j-1) it waits until the head's generation
+// word gen[bh] reaches j; it then takes block c % cph and claims further
+// 1024-token blocks from the head's work counter work[bh] until none is left
+// (blocks differ in how many tokens survive the screen, so a fixed share per
+// CTA leaves the head waiting for its slowest CTA); then it arrives on
+// counter[bh].  The last CTA of the head to arrive picks seed j (and the
+// seed-to-seed distances of the next screen), resets both counters and
+// publishes gen[bh] = j + 1.  Every block's arithmetic is the same whichever
+// CTA runs it, so the result does not depend on the claims.  Heads never wait for each other, so
 // one head's pick overlaps the other heads' passes.  The launch is
 // cooperative (every CTA resident); every wait is bounded and gives up with
 // SVGEAR_ERR_TIMEOUT in err[0] (err[1] = pass, err[2] = CTA).
@@ -305,15 +353,15 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kKppThreads, 6)
 kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg, int cph, int C,
                       int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* blocksum,
-                      int32_t* counter, int32_t* gen, uint64_t seed, float* centroids, int* err) {
+                      int32_t* counter, int32_t* work, int32_t* gen, uint64_t seed,
+                      float* centroids, int* err) {
     __shared__ KppSmem<D> sm;
     extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: C floats)
-    __shared__ int s_flag;
+    __shared__ int s_flag, s_next;
     const int tid = threadIdx.x;
     const int hl = blockIdx.x / cph, part = blockIdx.x % cph;
     if (hl >= BHg) return;
     const int bh = bh0 + hl;
-    const int blk0 = (int)((long long)part * nblk / cph), blk1 = (int)((long long)(part + 1) * nblk / cph);
     for (int j = 1; j < C; ++j) {
         const int s = j - 1;
         // wait for seed s
@@ -343,8 +391,16 @@ kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg
         for (int k = tid; k < D; k += kKppThreads) sm.cen[k] = __ldcg(centroids + ((size_t)bh * C + s) * D + k);
         for (int a = tid; a < s; a += kKppThreads) ccs[a] = __ldcg(cc2 + (size_t)bh * C + a);
         // (the block update's first barrier orders these loads before their use)
-        for (int blk = blk0; blk < blk1; ++blk)
+        // block `part` first, then blocks cph, cph + 1, ... as the head's work
+        // counter hands them out (the claim for the next block is issued
+        // before this one is processed, so its latency hides behind it)
+        for (int blk = part; blk < nblk; blk = s_next) {
+            int claim = 0;
+            if (tid == 0) claim = atomicAdd(work + bh, 1);
             kpp_block_update<T, D>(X, N, nblk, bh, blk, s, D2, nearest, blocksum, sm, ccs);
+            if (tid == 0) s_next = cph + claim;
+            __syncthreads();
+        }
         // arrive; the barrier inside the block update ordered this CTA's D^2,
         // label and block-sum stores before thread 0's fence
         if (tid == 0) {
@@ -359,6 +415,7 @@ kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg
             __syncthreads();
             if (tid == 0) {
                 counter[bh] = 0;
+                work[bh] = 0;
                 __threadfence();
                 atomicExch(gen + bh, j + 1);   // release seed j
             }
@@ -367,10 +424,11 @@ kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg
     }
 }
 
-__global__ void kpp_init_kernel(int32_t* counter, int32_t* gen, int n) {
+__global__ void kpp_init_kernel(int32_t* counter, int32_t* work, int32_t* gen, int n) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) {
         counter[i] = 0;
+        work[i] = 0;
         gen[i] = 1;   // seed 0 comes from kpp_first_kernel, launched before
     }
 }
@@ -382,7 +440,8 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
                          cudaStream_t st) {
     const int BH = dims.B * dims.H, N = dims.N;
     const int nblk = ceil_div(N, kKppTokens);
-    kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, gen, BH);
+    int32_t* work = counter + BH;   // the counter array holds 2 BH words
+    kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, work, gen, BH);
     count_launches(1);
     kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
     count_launches(1);
@@ -410,7 +469,7 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
         uint64_t seed_ = seed;
         const T* X_ = X;
         void* args[] = {&X_, &n_, &nblk_, &bh0, &BHg, &cph, &C_, &chosen, &D2, &nearest, &cc2,
-                        &blocksum, &counter, &gen, &seed_, &cent, &err};
+                        &blocksum, &counter, &work, &gen, &seed_, &cent, &err};
         if (cudaLaunchCooperativeKernel((const void*)kpp_persistent_kernel<T, D>, dim3(grid),
                                         dim3(kKppThreads), args, ccs_bytes, st) != cudaSuccess)
             return SVGEAR_ERR_CUDA;

@@ -21,7 +21,8 @@ inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 // (see kpp_persistent_kernel); err: device status words (4 ints).
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
                     float* centroids, int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
-                    double* blocksum, int32_t* counter, int32_t* gen, int* err, cudaStream_t st);
+                    double* blocksum, int32_t* counter /* 2 BH words */, int32_t* gen, int* err,
+                    cudaStream_t st);
 // done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
 // scratch: assign_scratch_bytes(B*H, C, d, dtype) bytes (centroids re-laid
 // for the kernel, and their norms).  bf16 tokens run on the tcgen05 kernel
