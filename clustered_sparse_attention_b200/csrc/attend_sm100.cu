@@ -321,11 +321,17 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     if (lane == 0) {
                         const uint32_t tV = sV0 + pst * kTileBytes;
                         const int kdepth = (j - 1 >= T_real) ? CW : BN;   // keys of tile j-1
+                        if (kdepth == BN) {
+                            tc::mma_bf16_ts_k128(tmem + kHalves * BN + h * D, tmem + h * BN,
+                                                 tc::sw128_desc(tV, 16384, 1024), kIdescPV,
+                                                 j > 1 ? 1u : 0u);
+                        } else {
 #pragma unroll 1
-                        for (int ks = 0; ks < kdepth / 16; ++ks)
-                            tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
-                                            tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
-                                            (j > 1 || ks > 0) ? 1u : 0u);
+                            for (int ks = 0; ks < kdepth / 16; ++ks)
+                                tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
+                                                tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
+                                                (j > 1 || ks > 0) ? 1u : 0u);
+                        }
                     }
                     if (lane == 0) TRACE(h == 0 ? 10 : 14, j);
                     __syncwarp();
@@ -349,12 +355,17 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     if (lane == 0 && h == 0) TRACE(11, j);
                     if (lane == 0) {
                         const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
+                        if (D == 128 && !var_tile) {
+                            tc::mma_bf16_k128(tmem + h * BN, tc::sw128_desc(tQ, 16, 1024),
+                                              tc::sw128_desc(tK, 16, 1024), kIdescQK, 0u);
+                        } else {
 #pragma unroll 1
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
-                                         tc::sw128_desc(tK + off, 16, 1024),
-                                         var_tile ? kIdescQK64 : kIdescQK, ks > 0);
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                                tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
+                                             tc::sw128_desc(tK + off, 16, 1024),
+                                             var_tile ? kIdescQK64 : kIdescQK, ks > 0);
+                            }
                         }
                         if (var_tile) {
                             // S += q^2 . (lambda*scale/2 Var)^T: A = q^2 from TMEM
