@@ -95,7 +95,7 @@ struct Shared {
 
 #ifdef SVGEAR_TRACE
 // Diagnostic build only: per-tile event clocks of one CTA.
-__device__ long long g_trace[18][512];
+__device__ long long g_trace[32][512];
 #define TRACE(ev, j)                                                                  \
     do {                                                                              \
         if (blockIdx.x == 3 && blockIdx.y == 0 && (j) < 512) g_trace[ev][j] = clock64(); \
@@ -289,6 +289,8 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     }
                 }
             }
+            if (isK && lane == 0) TRACE(27, j);
+            if (!isK && lane == 0) TRACE(28, j);
             __syncwarp();
         }
     } else if (warp == kMmaWarp) {
@@ -433,38 +435,66 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             tc::fence_after_sync();
             if (tid == 0) TRACE(3, j);
             if (tid == kSoftmaxThreads) TRACE(5, j);
+            const bool comp = j >= T_real;
+            const int valid = comp ? min(CW, ncomp - (j - T_real) * CW) : min(BN, L - j * BN);
+            const float* bias = cb + (comp ? (j - T_real) * CW : 0);
+            // full key tiles keep raw scores: the max scales afterwards (scale > 0)
+            // and the exp pass folds the scale into its FFMA
+            const bool raw = !comp && valid == BN;
+            if (!raw) {
+                // Compensation and partial tiles: x = s * scale * log2(e) (+ log2 n_c
+                // on compensation columns), -inf past the valid columns, rewritten
+                // in TMEM 32 columns at a time before the row is loaded, so this
+                // rare path's registers stay out of the main one.  Chunks wholly
+                // past the valid columns are left as they are (with the variance
+                // term the upper half of S_h holds q^2) and masked after the load.
+#pragma unroll 1
+                for (int c4 = 0; c4 * 32 < valid; ++c4) {
+                    uint32_t t[32];
+                    tc::tmem_ld32(sS + c4 * 32, t);
+                    tc::tmem_ld_wait();
+                    if (comp) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int col = c4 * 32 + e;
+                            t[e] = __float_as_uint(col < valid ? fmaf(__uint_as_float(t[e]), scale_log2, bias[col])
+                                                               : -INFINITY);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int col = c4 * 32 + e;
+                            t[e] = __float_as_uint(col < valid ? __uint_as_float(t[e]) * scale_log2 : -INFINITY);
+                        }
+                    }
+                    tc::tmem_st32(sS + c4 * 32, t);
+                }
+                tc::tmem_st_wait();
+            }
             tc::tmem_ld32(sS + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tc::tmem_ld32(sS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
             tc::tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
             tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
             tc::tmem_ld_wait();
+#ifdef SVGEAR_TRACE
+            {   // stamp once the loaded registers are usable (the add waits on them)
+                const float t = __uint_as_float(v[0]) + __uint_as_float(v[63]) + __uint_as_float(v[127]);
+                if (tid == 0) g_trace[22][j & 511] = __float_as_int(t) == 0x7fffffff;
+            }
+#endif
+            if (tid == 0) TRACE(19, j);
+            if (tid == kSoftmaxThreads) TRACE(24, j);
 
             // S_h is in registers: with the variance term, the last exact tile
             // leaves q^2 in the upper half of S_h for the compensation tiles
             if (need_q2 && j == T_real - 1) write_q2<D>(sQ0 + h * kTileBytes, r, sS + BN / 2);
-            const bool comp = j >= T_real;
-            const int valid = comp ? min(CW, ncomp - (j - T_real) * CW) : min(BN, L - j * BN);
-            const float* bias = cb + (comp ? (j - T_real) * CW : 0);
-            // x = s * scale * log2(e) (+ log2 n_c on compensation columns); masked -> -inf
-            if (comp) {
-                // in 32-column steps (the compiler barrier keeps the bias loads of
-                // one step from being hoisted next to the 128 live scores)
+            if (!raw) {
 #pragma unroll
-                for (int c4 = 0; c4 < BN / 32; ++c4) {
+                for (int c4 = 0; c4 < BN / 32; ++c4)
+                    if (c4 * 32 >= valid)
 #pragma unroll
-                    for (int e = c4 * 32; e < c4 * 32 + 32; ++e)
-                        v[e] = __float_as_uint((e < valid) ? fmaf(__uint_as_float(v[e]), scale_log2, bias[e])
-                                                           : -INFINITY);
-                    asm volatile("" ::: "memory");
-                }
-            } else if (valid < BN) {
-#pragma unroll
-                for (int e = 0; e < BN; ++e)
-                    v[e] = __float_as_uint((e < valid) ? __uint_as_float(v[e]) * scale_log2 : -INFINITY);
+                        for (int e = 0; e < 32; ++e) v[c4 * 32 + e] = __float_as_uint(-INFINITY);
             }
-            // full key tiles keep raw scores: the max scales afterwards (scale > 0)
-            // and the exp pass folds the scale into its FFMA
-            const bool raw = !comp && valid == BN;
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
             for (int e = 0; e < BN; e += 4) {
@@ -474,6 +504,11 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 mx3 = fmaxf(mx3, __uint_as_float(v[e + 3]));
             }
             float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+#ifdef SVGEAR_TRACE
+            if (tid == 0) g_trace[23][j & 511] = __float_as_int(mx) == 0x7fffffff;
+#endif
+            if (tid == 0) TRACE(17, j);
+            if (tid == kSoftmaxThreads) TRACE(25, j);
             if (raw) mx *= scale_log2;
             const float m_new = fmaxf(m_use, mx);
 
@@ -511,6 +546,8 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 tc::tmem_st16(sS + q * 16, pk);
             }
             l += s0 + s1;
+            if (tid == 0) TRACE(20, j);
+            if (tid == kSoftmaxThreads) TRACE(26, j);
             if (any) {
                 uint32_t o[16];
 #pragma unroll 1
@@ -523,9 +560,11 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 }
             }
             tc::tmem_st_wait();
+            if (tid == 0) TRACE(21, j);
             tc::fence_before_sync();
             tc::mbar_arrive(tc::smem_u32(&sh.p_full[h]));
             if (tid == 0) TRACE(6, j);
+            if (tid == 96) TRACE(18, j);
             if (tid == kSoftmaxThreads) TRACE(7, j);
         }
         // epilogue: O / l back to the original token order
