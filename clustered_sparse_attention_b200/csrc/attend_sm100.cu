@@ -59,7 +59,7 @@ constexpr int kThreads = 12 * 32;      // 168 registers per thread at launch
 // kThreads x (registers at launch); the host refuses a build whose launch
 // count is below kMinLaunchRegs, under which the split would not fit.
 constexpr uint32_t kSoftmaxRegs = 232;
-constexpr uint32_t kIssueRegs = 32;
+constexpr uint32_t kIssueRegs = 40;
 constexpr int kMinLaunchRegs =
     (int)((2 * 128 * kSoftmaxRegs + 128 * kIssueRegs + kThreads - 1) / kThreads + 7) / 8 * 8;
 static_assert(kMinLaunchRegs <= 168, "register split exceeds the launch allocation");
@@ -153,7 +153,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     const int ci = tile.x, q0 = tile.y, q_end = tile.z;
     const int nh = (q0 + BM < q_end) ? 2 : 1;     // query halves with rows
     const int4 mt = meta[(size_t)bh * Cq + ci];   // {nseg, L keys, ncomp, 0}
-    const int L = mt.y, ncomp = mt.z;
+    const int nseg = mt.x, L = mt.y, ncomp = mt.z;
     const int T_real = (L + BN - 1) / BN;
     // compensation tiles take CW skipped clusters: 128, or 64 with the
     // variance term (the upper 64 columns of S_h then hold q^2 of the half)
@@ -263,29 +263,55 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 for (int g = 0; g < REG; ++g)
                     tc::tma_gather4(tX + g * 16384 + lane * 512, src, g * 64, y[0], y[1], y[2], y[3],
                                     bar);
-            } else if (lane == 0) {
-                tc::mbar_arrive_expect_tx(bar, BN * D * 2);
-                const int t0 = j * BN, t1 = t0 + BN;
-                int r = 0;   // next tile row to fill
-                while (r < BN) {
-                    const int p = t0 + r;
-                    int g, n;
-                    if (p < L) {
-                        while (pre[seg + 1] <= p) ++seg;
-                        n = min(pre[seg + 1], t1) - p;
-                        g = krow0 + srow[seg] + (p - pre[seg]);
-                    } else {
-                        n = BN - r;
-                        g = kend;   // out of range: zero fill
+            } else {
+                // Lane i copies the run of segment seg + i that falls in the tile
+                // (a window of 32 segments: the bounds and first rows come in with
+                // two coalesced loads; a tile that spans more segments takes
+                // further windows), and lane 0 zero-fills the rows past the list.
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar, BN * D * 2);
+                __syncwarp();
+                const int t0 = j * BN, t1 = t0 + BN, tend = min(t1, L);
+                int s0 = seg;
+                unsigned done_mask;
+                for (;;) {
+                    const int s = s0 + lane;
+                    int a = L, b = L;
+                    if (s < nseg) {
+                        a = __ldg(pre + s);
+                        b = __ldg(pre + s + 1);
                     }
+                    const int lo = max(a, t0), hi = min(b, tend);
+                    if (lo < hi) {
+                        int g = krow0 + __ldg(srow + s) + (lo - a), r = lo - t0;
+                        const int n = hi - lo;
+#pragma unroll 1
+                        for (int hb = 7; hb >= 0; --hb) {
+                            if (!(n >> hb & 1)) continue;
+#pragma unroll 1
+                            for (int gg = 0; gg < REG; ++gg)
+                                tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, g, bar);
+                            r += 1 << hb;
+                            g += 1 << hb;
+                        }
+                    }
+                    // segments of the window that end by t1: the next tile starts
+                    // in the first one that does not
+                    done_mask = __ballot_sync(0xffffffffu, s < nseg && b <= t1);
+                    const int last_end = __shfl_sync(0xffffffffu, b, 31);
+                    if (last_end >= tend || s0 + 32 >= nseg) break;
+                    s0 += 32;
+                }
+                seg = s0 + __popc(done_mask);
+                if (lane == 0 && tend < t1) {   // rows past the list: zeros
+                    int r = tend - t0;
+                    const int n = t1 - tend;
 #pragma unroll 1
                     for (int hb = 7; hb >= 0; --hb) {
                         if (!(n >> hb & 1)) continue;
 #pragma unroll 1
                         for (int gg = 0; gg < REG; ++gg)
-                            tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, g, bar);
+                            tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, kend, bar);
                         r += 1 << hb;
-                        if (g != kend) g += 1 << hb;
                     }
                 }
             }
