@@ -47,7 +47,8 @@ using tc::warp_wait_bar;
 
 constexpr int BM = 128;                // query rows per half
 constexpr int BN = 128;                // keys per tile
-constexpr int STAGES = 2;              // K and V rings
+constexpr int KSTAGES = 2;             // K ring (a third stage measured no faster)
+constexpr int VSTAGES = 2;             // V ring
 constexpr int kHalves = 2;             // query halves per CTA
 constexpr int kSoftmaxThreads = 128;   // per half: one row each
 constexpr int kKWarp = 8;              // K ring producer
@@ -80,10 +81,10 @@ struct TmaMaps {
 
 struct Shared {
     uint64_t q_full;
-    uint64_t k_full[STAGES];
-    uint64_t k_empty[STAGES];
-    uint64_t v_full[STAGES];
-    uint64_t v_empty[STAGES];
+    uint64_t k_full[KSTAGES];
+    uint64_t k_empty[KSTAGES];
+    uint64_t v_full[VSTAGES];
+    uint64_t v_empty[VSTAGES];
     uint64_t s_full[kHalves];
     uint64_t p_full[kHalves];
     uint64_t q2_full[kHalves];   // q^2 of the half in TMEM (variance term, no exact tiles)
@@ -165,14 +166,16 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t sQ0 = base;                          // kHalves query tiles
     const uint32_t sK0 = sQ0 + kHalves * kTileBytes;
-    const uint32_t sV0 = sK0 + STAGES * kTileBytes;
+    const uint32_t sV0 = sK0 + KSTAGES * kTileBytes;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         tc::mbar_init(tc::smem_u32(&sh.q_full), 1);
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < KSTAGES; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.k_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.k_empty[s]), 1);
+        }
+        for (int s = 0; s < VSTAGES; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.v_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.v_empty[s]), 1);
         }
@@ -236,9 +239,10 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         const int crow0 = bh * Ck, cend = BH * Ck;
         int seg = 0;
         for (int j = 0; j < T; ++j) {
-            const int st = j % STAGES;
-            if (j >= STAGES &&
-                !warp_wait_bar(&ring_empty[st], ((j / STAGES) - 1) & 1, abort_flag, err, (1 << 16) + j))
+            const int NS = isK ? KSTAGES : VSTAGES;
+            const int st = j % NS;
+            if (j >= NS &&
+                !warp_wait_bar(&ring_empty[st], ((j / NS) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
             if (isK && lane == 0) TRACE(0, j);
             if (!isK && lane == 0) TRACE(16, j);
@@ -268,9 +272,25 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 // (a window of 32 segments: the bounds and first rows come in with
                 // two coalesced loads; a tile that spans more segments takes
                 // further windows), and lane 0 zero-fills the rows past the list.
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar, BN * D * 2);
-                __syncwarp();
+                // A run of n rows is covered by at most two boxes of 2^k rows,
+                // k = floor(log2 n): one at its start and one ending at its end;
+                // where they overlap both write the same bytes.  Each lane adds
+                // its boxes' bytes to the barrier's expected count before issuing
+                // them, and lane 0 arrives once every lane has done so.
                 const int t0 = j * BN, t1 = t0 + BN, tend = min(t1, L);
+                auto issue_run = [&](int r, int g, int n) {   // tile rows [r, r+n) <- rows [g, g+n)
+                    const int k = 31 - __clz(n), h2 = 1 << k;
+                    tc::mbar_expect_tx(bar, (n == h2 ? 1u : 2u) * (uint32_t)h2 * (uint32_t)(D * 2));
+#pragma unroll 1
+                    for (int gg = 0; gg < REG; ++gg)
+                        tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[k], gg * 64, g, bar);
+                    if (n != h2) {
+                        const int r2 = r + n - h2, g2 = (g == kend) ? kend : g + n - h2;
+#pragma unroll 1
+                        for (int gg = 0; gg < REG; ++gg)
+                            tc::tma_load_2d(tX + gg * 16384 + r2 * 128, &mrows[k], gg * 64, g2, bar);
+                    }
+                };
                 int s0 = seg;
                 unsigned done_mask;
                 for (;;) {
@@ -281,19 +301,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         b = __ldg(pre + s + 1);
                     }
                     const int lo = max(a, t0), hi = min(b, tend);
-                    if (lo < hi) {
-                        int g = krow0 + __ldg(srow + s) + (lo - a), r = lo - t0;
-                        const int n = hi - lo;
-#pragma unroll 1
-                        for (int hb = 7; hb >= 0; --hb) {
-                            if (!(n >> hb & 1)) continue;
-#pragma unroll 1
-                            for (int gg = 0; gg < REG; ++gg)
-                                tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, g, bar);
-                            r += 1 << hb;
-                            g += 1 << hb;
-                        }
-                    }
+                    if (lo < hi) issue_run(lo - t0, krow0 + __ldg(srow + s) + (lo - a), hi - lo);
                     // segments of the window that end by t1: the next tile starts
                     // in the first one that does not
                     done_mask = __ballot_sync(0xffffffffu, s < nseg && b <= t1);
@@ -302,18 +310,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     s0 += 32;
                 }
                 seg = s0 + __popc(done_mask);
-                if (lane == 0 && tend < t1) {   // rows past the list: zeros
-                    int r = tend - t0;
-                    const int n = t1 - tend;
-#pragma unroll 1
-                    for (int hb = 7; hb >= 0; --hb) {
-                        if (!(n >> hb & 1)) continue;
-#pragma unroll 1
-                        for (int gg = 0; gg < REG; ++gg)
-                            tc::tma_load_2d(tX + gg * 16384 + r * 128, &mrows[hb], gg * 64, kend, bar);
-                        r += 1 << hb;
-                    }
-                }
+                if (lane == 0 && tend < t1) issue_run(tend - t0, kend, t1 - tend);   // zeros
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar);
             }
             if (isK && lane == 0) TRACE(27, j);
             if (!isK && lane == 0) TRACE(28, j);
@@ -333,11 +332,11 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
         bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
         for (int j = 0; ok_run && j <= T; ++j) {
-            const int st = j % STAGES, pst = (j + STAGES - 1) % STAGES;
+            const int st = j % KSTAGES, pst = (j + VSTAGES - 1) % VSTAGES;
             if (lane == 0) TRACE(1, j);
             for (int h = 0; h < nh; ++h) {
                 if (j > 0) {
-                    if ((h == 0 && !warp_wait_bar(&sh.v_full[pst], ((j - 1) / STAGES) & 1, abort_flag,
+                    if ((h == 0 && !warp_wait_bar(&sh.v_full[pst], ((j - 1) / VSTAGES) & 1, abort_flag,
                                                   err, (11 << 16) + j)) ||
                         !warp_wait_bar(&sh.p_full[h], (j - 1) & 1, abort_flag, err,
                                        (8 << 16) + (h << 12) + j)) {
@@ -366,7 +365,7 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 }
                 if (j < T) {
                     if (h == 0 &&
-                        !warp_wait_bar(&sh.k_full[st], (j / STAGES) & 1, abort_flag, err, (6 << 16) + j)) {
+                        !warp_wait_bar(&sh.k_full[st], (j / KSTAGES) & 1, abort_flag, err, (6 << 16) + j)) {
                         ok_run = false;
                         break;
                     }
@@ -759,7 +758,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     }
     if (lr < kMinLaunchRegs) return SVGEAR_ERR_UNSUPPORTED;
     const float scale_log2 = scale * 1.4426950408889634f;
-    const size_t smem = (size_t)(kHalves + 2 * STAGES) * (D / 64) * 16384 + 1024;
+    const size_t smem = (size_t)(kHalves + KSTAGES + VSTAGES) * (D / 64) * 16384 + 1024;
     if (D == 128) {
         if (cudaFuncSetAttribute(attend_sm100_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
