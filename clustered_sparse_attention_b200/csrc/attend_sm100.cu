@@ -320,7 +320,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
-        // The whole warp runs the loop (uniform bounded waits); lane 0 issues.
+        // Lane 0 runs the loop alone (MMA, commit and fence are single-thread
+        // operations; the warp meets again after the drain), so nothing in the
+        // loop makes it wait for the tensor core to take its queued MMAs.
         // Step j issues, per half h: PV_h(j-1) once P_h(j-1) is in TMEM, then
         // QK_h(j) into S_h (over P_h(j-1): MMAs of one thread run in order).
         // While half 0's softmax works on S_0(j), the tensor pipe runs
@@ -330,42 +332,37 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         constexpr uint32_t kIdescQK = tc::idesc_bf16(BM, BN, false);
         constexpr uint32_t kIdescQK64 = tc::idesc_bf16(BM, BN / 2, false);
         constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
-        bool ok_run = warp_wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
+        if (lane == 0) {
+        bool ok_run = wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
         for (int j = 0; ok_run && j <= T; ++j) {
             const int st = j % KSTAGES, pst = (j + VSTAGES - 1) % VSTAGES;
-            if (lane == 0) TRACE(1, j);
+            TRACE(1, j);
             for (int h = 0; h < nh; ++h) {
                 if (j > 0) {
-                    if ((h == 0 && !warp_wait_bar(&sh.v_full[pst], ((j - 1) / VSTAGES) & 1, abort_flag,
-                                                  err, (11 << 16) + j)) ||
-                        !warp_wait_bar(&sh.p_full[h], (j - 1) & 1, abort_flag, err,
-                                       (8 << 16) + (h << 12) + j)) {
+                    if ((h == 0 && !wait_bar(&sh.v_full[pst], ((j - 1) / VSTAGES) & 1, abort_flag, err,
+                                             (11 << 16) + j)) ||
+                        !wait_bar(&sh.p_full[h], (j - 1) & 1, abort_flag, err, (8 << 16) + (h << 12) + j)) {
                         ok_run = false;
                         break;
                     }
                     tc::fence_after_sync();
-                    if (lane == 0) TRACE(h == 0 ? 9 : 13, j);
-                    if (lane == 0) {
-                        const uint32_t tV = sV0 + pst * kTileBytes;
-                        const int kdepth = (j - 1 >= T_real) ? CW : BN;   // keys of tile j-1
-                        if (kdepth == BN) {
-                            tc::mma_bf16_ts_k128(tmem + kHalves * BN + h * D, tmem + h * BN,
-                                                 tc::sw128_desc(tV, 16384, 1024), kIdescPV,
-                                                 j > 1 ? 1u : 0u);
-                        } else {
+                    TRACE(h == 0 ? 9 : 13, j);
+                    const uint32_t tV = sV0 + pst * kTileBytes;
+                    const int kdepth = (j - 1 >= T_real) ? CW : BN;   // keys of tile j-1
+                    if (kdepth == BN) {
+                        tc::mma_bf16_ts_k128(tmem + kHalves * BN + h * D, tmem + h * BN,
+                                             tc::sw128_desc(tV, 16384, 1024), kIdescPV, j > 1 ? 1u : 0u);
+                    } else {
 #pragma unroll 1
-                            for (int ks = 0; ks < kdepth / 16; ++ks)
-                                tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
-                                                tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
-                                                (j > 1 || ks > 0) ? 1u : 0u);
-                        }
+                        for (int ks = 0; ks < kdepth / 16; ++ks)
+                            tc::mma_bf16_ts(tmem + kHalves * BN + h * D, tmem + h * BN + ks * 8,
+                                            tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
+                                            (j > 1 || ks > 0) ? 1u : 0u);
                     }
-                    if (lane == 0) TRACE(h == 0 ? 10 : 14, j);
-                    __syncwarp();
+                    TRACE(h == 0 ? 10 : 14, j);
                 }
                 if (j < T) {
-                    if (h == 0 &&
-                        !warp_wait_bar(&sh.k_full[st], (j / KSTAGES) & 1, abort_flag, err, (6 << 16) + j)) {
+                    if (h == 0 && !wait_bar(&sh.k_full[st], (j / KSTAGES) & 1, abort_flag, err, (6 << 16) + j)) {
                         ok_run = false;
                         break;
                     }
@@ -373,58 +370,51 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     // q^2 of the half must be in TMEM: written with P(T_real-1), or,
                     // with no exact tiles, before the first compensation tile
                     if (var_tile && j == 0) {
-                        if (!warp_wait_bar(&sh.q2_full[h], 0, abort_flag, err, (12 << 16) + h)) {
+                        if (!wait_bar(&sh.q2_full[h], 0, abort_flag, err, (12 << 16) + h)) {
                             ok_run = false;
                             break;
                         }
                         tc::fence_after_sync();
                     }
-                    if (lane == 0 && h == 0) TRACE(11, j);
-                    if (lane == 0) {
-                        const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
-                        if (D == 128 && !var_tile) {
-                            tc::mma_bf16_k128(tmem + h * BN, tc::sw128_desc(tQ, 16, 1024),
-                                              tc::sw128_desc(tK, 16, 1024), kIdescQK, 0u);
-                        } else {
+                    if (h == 0) TRACE(11, j);
+                    const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
+                    if (D == 128 && !var_tile) {
+                        tc::mma_bf16_k128(tmem + h * BN, tc::sw128_desc(tQ, 16, 1024),
+                                          tc::sw128_desc(tK, 16, 1024), kIdescQK, 0u);
+                    } else {
 #pragma unroll 1
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                                tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
-                                             tc::sw128_desc(tK + off, 16, 1024),
-                                             var_tile ? kIdescQK64 : kIdescQK, ks > 0);
-                            }
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            tc::mma_bf16(tmem + h * BN, tc::sw128_desc(tQ + off, 16, 1024),
+                                         tc::sw128_desc(tK + off, 16, 1024),
+                                         var_tile ? kIdescQK64 : kIdescQK, ks > 0);
                         }
-                        if (var_tile) {
-                            // S += q^2 . (lambda*scale/2 Var)^T: A = q^2 from TMEM
-                            // (columns 64-127 of S_h), B = tile rows 64-127
-#pragma unroll 1
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t off = (ks >> 2) * 16384 + 64 * 128 + (ks & 3) * 32;
-                                tc::mma_bf16_ts(tmem + h * BN, tmem + h * BN + BN / 2 + ks * 8,
-                                                tc::sw128_desc(tK + off, 16, 1024), kIdescQK64, 1u);
-                            }
-                        }
-                        tc::commit(tc::smem_u32(&sh.s_full[h]));
                     }
-                    if (lane == 0) TRACE(h == 0 ? 12 : 15, j);
-                    __syncwarp();
+                    if (var_tile) {
+                        // S += q^2 . (lambda*scale/2 Var)^T: A = q^2 from TMEM
+                        // (columns 64-127 of S_h), B = tile rows 64-127
+#pragma unroll 1
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + 64 * 128 + (ks & 3) * 32;
+                            tc::mma_bf16_ts(tmem + h * BN, tmem + h * BN + BN / 2 + ks * 8,
+                                            tc::sw128_desc(tK + off, 16, 1024), kIdescQK64, 1u);
+                        }
+                    }
+                    tc::commit(tc::smem_u32(&sh.s_full[h]));
+                    TRACE(h == 0 ? 12 : 15, j);
                 }
             }
             if (!ok_run) break;
-            if (lane == 0) {
-                if (j < T) tc::commit(tc::smem_u32(&sh.k_empty[st]));
-                if (j > 0) tc::commit(tc::smem_u32(&sh.v_empty[pst]));
-                TRACE(2, j);
-            }
-            __syncwarp();
+            if (j < T) tc::commit(tc::smem_u32(&sh.k_empty[st]));
+            if (j > 0) tc::commit(tc::smem_u32(&sh.v_empty[pst]));
+            TRACE(2, j);
         }
-        if (lane == 0) tc::commit(tc::smem_u32(&sh.o_full));
-        __syncwarp();
+        tc::commit(tc::smem_u32(&sh.o_full));
         // drain: every MMA of this CTA is complete once o_full flips; if that
         // wait expires, TMEM is left allocated rather than released under a
         // running MMA (every later CTA of the launch returns before alloc)
-        if (!warp_wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16)) && lane == 0)
-            sh.keep_tmem = 1;
+        if (!wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16))) sh.keep_tmem = 1;
+        }
         __syncwarp();
     }
     } else {
