@@ -105,6 +105,27 @@ __device__ long long g_trace[32][512];
 #define TRACE(ev, j) do { } while (0)
 #endif
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+// (o0, o1) = (x0, x1) * m + a on packed fp32 pairs
+__device__ __forceinline__ void fma2(uint32_t x0, uint32_t x1, uint64_t m, uint64_t a, uint32_t& o0,
+                                     uint32_t& o1) {
+    asm("{\n\t.reg .b64 x, r;\n\tmov.b64 x, {%2, %3};\n\t"
+        "fma.rn.f32x2 r, x, %4, %5;\n\tmov.b64 {%0, %1}, r;\n\t}"
+        : "=r"(o0), "=r"(o1) : "r"(x0), "r"(x1), "l"(m), "l"(a));
+}
+// s += (p0, p1) on a packed fp32 pair
+__device__ __forceinline__ void add2(uint64_t& s, float p0, float p1) {
+    asm("{\n\t.reg .b64 x;\n\tmov.b64 x, {%1, %2};\n\tadd.rn.f32x2 %0, %0, x;\n\t}"
+        : "+l"(s) : "f"(p0), "f"(p1));
+}
+
 // Swizzled 16-byte chunk address inside a tile of 128 rows x (regions of
 // 64 bf16): region g covers elements [64g, 64g+64) of every row.
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
@@ -512,11 +533,11 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             }
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < BN; e += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(v[e]));
-                mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(v[e + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(v[e + 3]));
+            for (int e = 0; e < BN; e += 8) {   // three-input max: half the instructions
+                mx0 = fmax3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
             }
             float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
 #ifdef SVGEAR_TRACE
@@ -545,22 +566,26 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             if (tid == 0) TRACE(4, j);
             // P = 2^(x - m) as bf16 pairs over the first 64 columns of S_h
             const float xs = raw ? scale_log2 : 1.f, neg_m = -m_use;
-            float s0 = 0.f, s1 = 0.f;
+            // (even, odd) columns in packed fp32 pairs: one FFMA2 and one FADD2
+            // per two scores, elementwise round-to-nearest like the scalar forms
+            uint64_t s01 = 0ull;
+            const uint64_t xs2 = pack2(xs, xs), nm2 = pack2(neg_m, neg_m);
 #pragma unroll
             for (int q = 0; q < BN / 32; ++q) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float p0 = tc::ex2(fmaf(__uint_as_float(v[q * 32 + e]), xs, neg_m));
-                    const float p1 = tc::ex2(fmaf(__uint_as_float(v[q * 32 + e + 1]), xs, neg_m));
-                    s0 += p0;
-                    s1 += p1;
+                    uint32_t a0, a1;
+                    fma2(v[q * 32 + e], v[q * 32 + e + 1], xs2, nm2, a0, a1);
+                    const float p0 = tc::ex2(__uint_as_float(a0));
+                    const float p1 = tc::ex2(__uint_as_float(a1));
+                    add2(s01, p0, p1);
                     __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
                     pk[e >> 1] = *reinterpret_cast<uint32_t*>(&hp);
                 }
                 tc::tmem_st16(sS + q * 16, pk);
             }
-            l += s0 + s1;
+            l += __uint_as_float((uint32_t)s01) + __uint_as_float((uint32_t)(s01 >> 32));
             if (tid == 0) TRACE(20, j);
             if (tid == kSoftmaxThreads) TRACE(26, j);
             if (any) {
