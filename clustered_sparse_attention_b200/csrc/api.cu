@@ -102,12 +102,14 @@ SelWs carve_select(Carve& cv, size_t BH, int Cq, int Ck) {
 struct RouteWs {
     float* E;
     uint32_t* rowmax;
+    float* qT;   // probes transposed in blocks of 128: [BH][ceil(Cq/128)][d][128]
     SelWs sel;
 };
-RouteWs carve_route(Carve& cv, size_t BH, int Cq, int Ck) {
+RouteWs carve_route(Carve& cv, size_t BH, int Cq, int Ck, int d) {
     RouteWs w;
     w.E = cv.take<float>(BH * Cq * (size_t)Ck);
     w.rowmax = cv.take<uint32_t>(BH * Cq);
+    w.qT = cv.take<float>(BH * (size_t)ceil_div(Cq, 128) * 128 * (size_t)d);
     w.sel = carve_select(cv, BH, Cq, Ck);
     return w;
 }
@@ -204,11 +206,11 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             break;
         case SVGEAR_OP_ROUTE:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
-            carve_route(cv, bh_of(dims), C1, C2);
+            carve_route(cv, bh_of(dims), C1, C2, dims.d);
             break;
         case SVGEAR_OP_ROUTE_TOPP:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
-            carve_route(cv, bh_of(dims), C1, C2);
+            carve_route(cv, bh_of(dims), C1, C2, dims.d);
             cv.take<int32_t>(bh_of(dims) * C1);
             break;
         case SVGEAR_OP_ATTEND:
@@ -383,8 +385,8 @@ int svgear_probe(const float* qbar, int32_t Cq, const void* Kp, const void* Vp, 
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     Carve cv(ws);
-    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
-    return launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax,
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
+    return launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -424,9 +426,9 @@ int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq, const floa
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
-    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
     float* E = E_out ? E_out : w.E;
-    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, st)))
+    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT, st)))
         return s;
     const long long budget = (long long)floor((double)density * (double)kdims.N);
     return launch_route_select(E, q_off, Cq, k_off, Ck, (int)bh_of(kdims), budget, nullptr,
@@ -485,11 +487,11 @@ int svgear_route_topp(const float* qbar, const int32_t* q_off, int32_t Cq, const
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
-    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
     int32_t* bud = cv.take<int32_t>(bh_of(kdims) * Cq);
     if (budget_out) bud = budget_out;
     float* E = E_out ? E_out : w.E;
-    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, st)))
+    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT, st)))
         return s;
     if ((s = launch_topp_budget(qbar, q_off, Cq, kbar, k_off, Ck, (int)bh_of(kdims), kdims.d,
                                 (double)p, (double)scale, bud, st)))
@@ -547,9 +549,9 @@ int svgear_probe_value_free(const float* qbar, int32_t Cq, const void* Kp, const
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     Carve cv(ws);
-    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck);
+    RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
     return launch_probe(qbar, Cq, Kp, nullptr, kbar, nullptr, k_off, Ck, kdims, scale, E,
-                        w.rowmax, static_cast<cudaStream_t>(stream), true);
+                        w.rowmax, w.qT, static_cast<cudaStream_t>(stream), true);
 }
 
 int svgear_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,

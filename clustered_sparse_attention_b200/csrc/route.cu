@@ -12,9 +12,10 @@
 // Kernels (fp32 throughout):
 //   probe_rowmax  m_i = max_t scale*qbar_i.k_t, by an order-independent
 //                 atomicMax on order-preserving integer keys (deterministic);
-//   probe_error   one block per (key cluster, 32 probes, head): every probe
-//                 against every key of the cluster, direct form of the error
-//                 (no expansion, so small errors are not lost to cancellation);
+//   probe_error   one block per (key cluster, 128 probes, head): every probe
+//                 against every key of the cluster, the error expanded around
+//                 the key's residual from its cluster's value mean (see the
+//                 register-tiled section below), summed in a fixed order;
 //   route_select  one block per (query cluster, head): r_c = E/n_c, a bitonic
 //                 sort on (r desc, c asc), the greedy take-if-fits scan, and
 //                 an ascending list of the taken clusters;
@@ -24,201 +25,243 @@
 
 namespace svgear {
 
-constexpr int kPrProbes = 32;    // probes per block (one per lane)
-constexpr int kPrKeys = 64;      // keys staged per step
-constexpr int kPrThreads = 256;  // 8 warps, 8 keys each per step
+// ---------------------------------------------------------------------------
+// Probe, register-tiled: a block of up to 128 probes against a tile of 64
+// keys, each thread 8 probes x 8 keys (probes 4pi..4pi+3 and 64+4pi..,
+// keys 4ki..4ki+3 and 32+4ki.., so both shared-memory reads are free of
+// bank conflicts).  Scores accumulate over k in order, like the plain form.
+// The error of key t (cluster c, residual w_t = v_t - vbar_c) is evaluated
+// as (a-b)^2 |vbar_c|^2 - 2 (a-b) b vbar_c.w_t + b^2 |w_t|^2 -- the same
+// quantity as |a vbar_c - b v_t|^2 -- so a (probe, key) pair costs its score
+// and a handful of scalar operations; vbar_c.w_t and |w_t|^2 come once per
+// key from the cluster's value rows.
+// ---------------------------------------------------------------------------
+constexpr int kPbP = 128;        // probes per block
+constexpr int kPbK = 64;         // keys per tile
+constexpr int kPbThreads = 128;
 
-template <int D> struct ProbeSmem {
-    static constexpr int kPad = D + 4;   // float4-aligned rows, conflict-free
-};
-
-template <typename T, int D>
-__global__ void __launch_bounds__(kPrThreads)
-probe_rowmax_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__ Kp,
-                    int Nk, float scale, uint32_t* __restrict__ rowmax) {
-    constexpr int P = ProbeSmem<D>::kPad;
-    constexpr int EPC = Elem<T>::kPerChunk;
-    extern __shared__ __align__(16) float sm[];
-    float* Qs = sm;                 // [32][P]
-    float* Ks = Qs + kPrProbes * P; // [kPrKeys][P]
-    const int bh = blockIdx.z, i0 = blockIdx.y * kPrProbes, tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const int keys_per_block = kPrKeys * 4;
-    const int t_begin = blockIdx.x * keys_per_block;
-    for (int q = tid; q < kPrProbes * D; q += kPrThreads) {
-        const int p = q / D, k = q % D;
-        Qs[p * P + k] = (i0 + p < Cq) ? qbar[((size_t)bh * Cq + i0 + p) * D + k] : 0.f;
+// qT[bh][blk][k][p] = qbar[bh][blk * 128 + p][k] (0 past Cq)
+template <int D>
+__global__ void probe_qT_kernel(const float* __restrict__ qbar, int Cq, int nPB,
+                                float* __restrict__ qT) {
+    const int blk = blockIdx.x, bh = blockIdx.y;
+    float* out = qT + ((size_t)bh * nPB + blk) * D * kPbP;
+    for (int e = threadIdx.x; e < D * kPbP; e += blockDim.x) {
+        const int k = e / kPbP, p = e % kPbP, i = blk * kPbP + p;
+        out[e] = i < Cq ? qbar[((size_t)bh * Cq + i) * D + k] : 0.f;
     }
-    const T* Kh = Kp + (size_t)bh * Nk * D;
-    float best = __int_as_float(0xff800000);
-    for (int kb = 0; kb < 4; ++kb) {
-        const int tb = t_begin + kb * kPrKeys;
-        __syncthreads();
-        for (int q = tid; q < kPrKeys * (D / EPC); q += kPrThreads) {
-            const int r = q / (D / EPC), col = (q % (D / EPC)) * EPC;
-            float v[EPC];
-            if (tb + r < Nk) Elem<T>::load(Kh + (size_t)(tb + r) * D + col, v);
-            else
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) v[e] = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) Ks[r * P + col + e] = v[e];
-        }
-        __syncthreads();
-        float acc[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.f;
-        const float* qr = Qs + lane * P;
-#pragma unroll 2
-        for (int k = 0; k < D; k += 4) {
-            const float4 qv = *reinterpret_cast<const float4*>(qr + k);
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const float4 kv = *reinterpret_cast<const float4*>(Ks + (warp * 8 + jj) * P + k);
-                acc[jj] = fmaf(qv.x, kv.x, acc[jj]);
-                acc[jj] = fmaf(qv.y, kv.y, acc[jj]);
-                acc[jj] = fmaf(qv.z, kv.z, acc[jj]);
-                acc[jj] = fmaf(qv.w, kv.w, acc[jj]);
-            }
-        }
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-            if (tb + warp * 8 + jj < Nk) best = fmaxf(best, scale * acc[jj]);
-    }
-    if (i0 + lane < Cq)
-        atomicMax(rowmax + (size_t)bh * Cq + i0 + lane, float_to_ordered(best));
 }
 
-// VF: the value-free error sum_t (a_ic - b_it)^2 (values not read).
-template <typename T, int D, bool VF>
-__global__ void __launch_bounds__(kPrThreads)
-probe_error_kernel(const float* __restrict__ qbar, int Cq, const T* __restrict__ Kp,
-                   const T* __restrict__ Vp, const float* __restrict__ kbar,
-                   const float* __restrict__ vbar, const int32_t* __restrict__ k_off,
-                   int Ck, int Nk, float scale, const uint32_t* __restrict__ rowmax,
-                   float* __restrict__ E) {
-    constexpr int P = ProbeSmem<D>::kPad;
+template <int D>
+__device__ __forceinline__ void pb_load_q(const float* __restrict__ qT, float* Qs) {
+    const float4* src = reinterpret_cast<const float4*>(qT);
+    float4* dst = reinterpret_cast<float4*>(Qs);
+    for (int e = threadIdx.x; e < D * kPbP / 4; e += kPbThreads) dst[e] = __ldg(src + e);
+}
+
+// Ks[k][t] = key t0 + t, dimension k (0 past t_end)
+template <typename T, int D>
+__device__ __forceinline__ void pb_load_k(const T* __restrict__ Kh, int t0, int t_end, float* Ks) {
     constexpr int EPC = Elem<T>::kPerChunk;
-    extern __shared__ __align__(16) float sm[];
-    float* Qs = sm;                    // [32][P] probes
-    float* AV = Qs + kPrProbes * P;    // [32][P] a_ic * vbar_c
-    float* Ks = AV + kPrProbes * P;    // [kPrKeys][P]
-    float* Vs = Ks + kPrKeys * P;      // [kPrKeys][P]
-    float* red = Vs + kPrKeys * P;     // [8][32]
-    __shared__ float kb_s[D];
-    const int c = blockIdx.x, i0 = blockIdx.y * kPrProbes, bh = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NCH = D / EPC;
+    for (int idx = threadIdx.x; idx < kPbK * NCH; idx += kPbThreads) {
+        const int t = idx % kPbK, ch = idx / kPbK;
+        float x[EPC];
+        if (t0 + t < t_end) {
+            Elem<T>::unpack(Elem<T>::load_raw(Kh + (size_t)(t0 + t) * D + ch * EPC), x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) x[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) Ks[(ch * EPC + e) * kPbK + t] = x[e];
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int pi, int ki,
+                                          float (&acc)[8][8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+    for (int k = 0; k < D; ++k) {
+        const float4 qa = *reinterpret_cast<const float4*>(Qs + k * kPbP + pi * 4);
+        const float4 qb = *reinterpret_cast<const float4*>(Qs + k * kPbP + 64 + pi * 4);
+        const float4 ka = *reinterpret_cast<const float4*>(Ks + k * kPbK + ki * 4);
+        const float4 kb = *reinterpret_cast<const float4*>(Ks + k * kPbK + 32 + ki * 4);
+        const float q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(q[i], kk[j], acc[i][j]);
+    }
+}
+__device__ __forceinline__ int pb_probe(int pi, int i) { return pi * 4 + (i & 3) + (i >> 2) * 64; }
+__device__ __forceinline__ int pb_key(int ki, int j) { return ki * 4 + (j & 3) + (j >> 2) * 32; }
+
+// m_i = max over keys [t_begin, t_end) of scale * qbar_i . k_t, merged into
+// rowmax by an order-independent atomicMax on order-preserving integers.
+template <typename T, int D>
+__global__ void __launch_bounds__(kPbThreads, 2)
+probe_rowmax_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __restrict__ Kp,
+                       int Nk, float scale, int keys_per_cta, uint32_t* __restrict__ rowmax) {
+    extern __shared__ __align__(16) float pbs[];
+    float* Qs = pbs;                 // [D][128]
+    float* Ks = Qs + D * kPbP;       // [D][64]
+    float* red = Ks + D * kPbK;      // [4][128]
+    const int part = blockIdx.x, blk = blockIdx.y, bh = blockIdx.z, tid = threadIdx.x;
+    const int pi = tid & 15, ki = tid >> 4, lane = tid & 31, warp = tid >> 5;
+    const int t_begin = part * keys_per_cta, t_end = min(Nk, t_begin + keys_per_cta);
+    pb_load_q<D>(qT + ((size_t)bh * nPB + blk) * D * kPbP, Qs);
+    const T* Kh = Kp + (size_t)bh * Nk * D;
+    float mx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+    for (int t0 = t_begin; t0 < t_end; t0 += kPbK) {
+        __syncthreads();
+        pb_load_k<T, D>(Kh, t0, t_end, Ks);
+        __syncthreads();
+        float acc[8][8];
+        pb_scores<D>(Qs, Ks, pi, ki, acc);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (t0 + pb_key(ki, j) < t_end)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], scale * acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 16));
+    __syncthreads();
+    if (lane < 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp * kPbP + pb_probe(pi, i)] = mx[i];
+    __syncthreads();
+    const int p = blk * kPbP + tid;
+    if (p < Cq) {
+        const float m = fmaxf(fmaxf(red[tid], red[kPbP + tid]), fmaxf(red[2 * kPbP + tid], red[3 * kPbP + tid]));
+        atomicMax(rowmax + (size_t)bh * Cq + p, float_to_ordered(m));
+    }
+}
+
+// E[bh][i][c] for the block's probes, one CTA per (key cluster c, probe
+// block, head).  VF: the value-free error sum_t (a - b)^2.
+template <typename T, int D, bool VF>
+__global__ void __launch_bounds__(kPbThreads, 2)
+probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __restrict__ Kp,
+                      const T* __restrict__ Vp, const float* __restrict__ kbar,
+                      const float* __restrict__ vbar, const int32_t* __restrict__ k_off, int Ck,
+                      int Nk, float scale, const uint32_t* __restrict__ rowmax,
+                      float* __restrict__ E) {
+    extern __shared__ __align__(16) float pbs[];
+    float* Qs = pbs;                 // [D][128]
+    float* Ks = Qs + D * kPbP;       // [D][64]
+    float* red = Ks + D * kPbK;      // [4][128]
+    float* kb = red + 4 * kPbP;      // [D] kbar_c
+    float* vb = kb + D;              // [D] vbar_c
+    float* al = vb + D;              // [64] vbar_c . w_t
+    float* be = al + kPbK;           // [64] |w_t|^2
+    const int c = blockIdx.x, blk = blockIdx.y, bh = blockIdx.z, tid = threadIdx.x;
+    const int pi = tid & 15, ki = tid >> 4, lane = tid & 31, warp = tid >> 5;
     const int32_t* off = k_off + (size_t)bh * (Ck + 1);
-    const int a = off[c], b = off[c + 1];
-    const int ip = i0 + lane;
-    if (b <= a || a < 0 || b > Nk) {   // empty (or malformed) key cluster: no error
-        if (warp == 0 && ip < Cq) E[((size_t)bh * Cq + ip) * Ck + c] = 0.f;
+    const int a0 = off[c], a1 = off[c + 1];
+    if (a1 <= a0 || a0 < 0 || a1 > Nk) {   // empty (or malformed) key cluster: no error
+        const int p = blk * kPbP + tid;
+        if (p < Cq) E[((size_t)bh * Cq + p) * Ck + c] = 0.f;
         return;
     }
-    for (int q = tid; q < kPrProbes * D; q += kPrThreads) {
-        const int p = q / D, k = q % D;
-        Qs[p * P + k] = (i0 + p < Cq) ? qbar[((size_t)bh * Cq + i0 + p) * D + k] : 0.f;
+    pb_load_q<D>(qT + ((size_t)bh * nPB + blk) * D * kPbP, Qs);
+    for (int k = tid; k < D; k += kPbThreads) {
+        kb[k] = kbar[((size_t)bh * Ck + c) * D + k];
+        if (!VF) vb[k] = vbar[((size_t)bh * Ck + c) * D + k];
     }
-    for (int k = tid; k < D; k += kPrThreads) kb_s[k] = kbar[((size_t)bh * Ck + c) * D + k];
     __syncthreads();
-    // a_ic = exp(scale * qbar_i . kbar_c - m_i), one lane per probe
-    const float m = (ip < Cq) ? ordered_to_float(rowmax[(size_t)bh * Cq + ip]) : 0.f;
-    float dotk = 0.f;
-    for (int k = 0; k < D; ++k) dotk = fmaf(Qs[lane * P + k], kb_s[k], dotk);
-    const float aic = expf(scale * dotk - m);
-    // every thread needs a_ic of every probe: broadcast through smem
-    if (warp == 0) red[lane] = aic;
-    __syncthreads();
-    if constexpr (!VF) {   // the value-free error reads no values
-        const float* vb = vbar + ((size_t)bh * Ck + c) * D;
-        for (int q = tid; q < kPrProbes * D; q += kPrThreads) {
-            const int p = q / D, k = q % D;
-            AV[p * P + k] = red[p] * vb[k];
-        }
+    // a_i = exp(scale * qbar_i . kbar_c - m_i) for this thread's probes
+    float ai[8], mi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int p = blk * kPbP + pb_probe(pi, i);
+        mi[i] = p < Cq ? ordered_to_float(rowmax[(size_t)bh * Cq + p]) : 0.f;
+        float dotk = 0.f;
+        for (int k = 0; k < D; ++k) dotk = fmaf(Qs[k * kPbP + pb_probe(pi, i)], kb[k], dotk);
+        ai[i] = expf(scale * dotk - mi[i]);
     }
+    float gamma = 0.f;
+    if (!VF)
+        for (int k = 0; k < D; ++k) gamma = fmaf(vb[k], vb[k], gamma);
     const T* Kh = Kp + (size_t)bh * Nk * D;
     const T* Vh = VF ? nullptr : Vp + (size_t)bh * Nk * D;
-    float err = 0.f;
-    for (int tb = a; tb < b; tb += kPrKeys) {
+    float err[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) err[i] = 0.f;
+    for (int t0 = a0; t0 < a1; t0 += kPbK) {
         __syncthreads();
-        for (int q = tid; q < kPrKeys * (D / EPC); q += kPrThreads) {
-            const int r = q / (D / EPC), col = (q % (D / EPC)) * EPC;
-            float kv[EPC], vv[EPC];
-            if (tb + r < b) {
-                Elem<T>::load(Kh + (size_t)(tb + r) * D + col, kv);
-                if constexpr (!VF) {
-                    Elem<T>::load(Vh + (size_t)(tb + r) * D + col, vv);
+        pb_load_k<T, D>(Kh, t0, a1, Ks);
+        if constexpr (!VF) {
+            // per key: alpha = vbar_c . w, beta = |w|^2, two threads per key
+            constexpr int EPC = Elem<T>::kPerChunk;
+            const int t = tid >> 1, half = tid & 1;
+            float sa = 0.f, sb = 0.f;
+            if (t0 + t < a1) {
+                const T* vr = Vh + (size_t)(t0 + t) * D + half * (D / 2);
+#pragma unroll 4
+                for (int ch = 0; ch < D / 2 / EPC; ++ch) {
+                    float x[EPC];
+                    Elem<T>::unpack(Elem<T>::load_raw(vr + ch * EPC), x);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) {
+                        const int k = half * (D / 2) + ch * EPC + e;
+                        const float w = x[e] - vb[k];
+                        sa = fmaf(vb[k], w, sa);
+                        sb = fmaf(w, w, sb);
+                    }
+                }
+            }
+            sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+            sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+            if (half == 0) {
+                al[t] = sa;
+                be[t] = sb;
+            }
+        }
+        __syncthreads();
+        float acc[8][8];
+        pb_scores<D>(Qs, Ks, pi, ki, acc);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int tj = pb_key(ki, j);
+            if (t0 + tj >= a1) continue;
+            float alj = 0.f, bej = 0.f;
+            if (!VF) {
+                alj = al[tj];
+                bej = be[tj];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float b = expf(scale * acc[i][j] - mi[i]);
+                const float dab = ai[i] - b;
+                if (VF) {
+                    err[i] = fmaf(dab, dab, err[i]);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) vv[e] = 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) { kv[e] = 0.f; vv[e] = 0.f; }
-            }
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) { Ks[r * P + col + e] = kv[e]; Vs[r * P + col + e] = vv[e]; }
-        }
-        __syncthreads();
-        // scores of this lane's probe against the warp's 8 keys
-        float s[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) s[jj] = 0.f;
-        const float* qr = Qs + lane * P;
-#pragma unroll 2
-        for (int k = 0; k < D; k += 4) {
-            const float4 qv = *reinterpret_cast<const float4*>(qr + k);
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const float4 kv = *reinterpret_cast<const float4*>(Ks + (warp * 8 + jj) * P + k);
-                s[jj] = fmaf(qv.x, kv.x, s[jj]);
-                s[jj] = fmaf(qv.y, kv.y, s[jj]);
-                s[jj] = fmaf(qv.z, kv.z, s[jj]);
-                s[jj] = fmaf(qv.w, kv.w, s[jj]);
-            }
-        }
-        float bw[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-            bw[jj] = (tb + warp * 8 + jj < b) ? expf(scale * s[jj] - m) : 0.f;
-        if constexpr (VF) {   // value-free: (a - b)^2 per key
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                if (tb + warp * 8 + jj < b) err += (aic - bw[jj]) * (aic - bw[jj]);
-        } else {
-            // direct form: sum_k (a vbar_k - b v_k)^2 per key
-            float e8[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) e8[jj] = 0.f;
-            const float* avr = AV + lane * P;
-#pragma unroll 2
-            for (int k = 0; k < D; k += 4) {
-                const float4 av = *reinterpret_cast<const float4*>(avr + k);
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const float4 vv = *reinterpret_cast<const float4*>(Vs + (warp * 8 + jj) * P + k);
-                    float d0 = fmaf(-bw[jj], vv.x, av.x), d1 = fmaf(-bw[jj], vv.y, av.y);
-                    float d2 = fmaf(-bw[jj], vv.z, av.z), d3 = fmaf(-bw[jj], vv.w, av.w);
-                    e8[jj] = fmaf(d0, d0, e8[jj]);
-                    e8[jj] = fmaf(d1, d1, e8[jj]);
-                    e8[jj] = fmaf(d2, d2, e8[jj]);
-                    e8[jj] = fmaf(d3, d3, e8[jj]);
+                    const float e = fmaf(b * b, bej, fmaf(dab * dab, gamma, -2.f * dab * b * alj));
+                    err[i] += e;
                 }
             }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                if (tb + warp * 8 + jj < b) err += e8[jj];
         }
     }
-    __syncthreads();
-    red[warp * 32 + lane] = err;
-    __syncthreads();
-    if (warp == 0 && ip < Cq) {
-        float tot = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) tot += red[w * 32 + lane];
-        E[((size_t)bh * Cq + ip) * Ck + c] = tot;
-    }
+    for (int i = 0; i < 8; ++i) err[i] += __shfl_xor_sync(0xffffffffu, err[i], 16);
+    __syncthreads();
+    if (lane < 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp * kPbP + pb_probe(pi, i)] = err[i];
+    __syncthreads();
+    const int p = blk * kPbP + tid;
+    if (p < Cq)
+        E[((size_t)bh * Cq + p) * Ck + c] =
+            ((red[tid] + red[kPbP + tid]) + red[2 * kPbP + tid]) + red[3 * kPbP + tid];
 }
 
 __global__ void fill_u32_kernel(uint32_t* p, size_t n, uint32_t v) {
@@ -230,52 +273,59 @@ __global__ void fill_u32_kernel(uint32_t* p, size_t n, uint32_t v) {
 template <typename T, int D>
 static int probe_impl(const float* qbar, int Cq, const void* Kp, const void* Vp,
                       const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
-                      svgear_dims kd, float scale, float* E, uint32_t* rowmax,
+                      svgear_dims kd, float scale, float* E, uint32_t* rowmax, float* qT,
                       bool value_free, cudaStream_t st) {
-    constexpr int P = ProbeSmem<D>::kPad;
     const int BH = kd.B * kd.H, Nk = kd.N;
+    const int nPB = ceil_div(Cq, kPbP);
     const size_t nrow = (size_t)BH * Cq;
+    probe_qT_kernel<D><<<dim3(nPB, BH), 256, 0, st>>>(qbar, Cq, nPB, qT);
+    count_launches(1);
     fill_u32_kernel<<<ceil_div((long long)nrow, 256) < 1024 ? ceil_div((long long)nrow, 256) : 1024,
                       256, 0, st>>>(rowmax, nrow, 0x007FFFFFu);  // ordered(-inf)
-    const size_t sm1 = sizeof(float) * (kPrProbes + kPrKeys) * P;
     count_launches(1);
-    if (cudaFuncSetAttribute(probe_rowmax_kernel<T, D>,
+    // row maxima: about four CTAs per SM over all (part, probe block, head)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SVGEAR_ERR_CUDA;
+    const long long want = 4LL * sms;
+    int parts = (int)((want + (long long)nPB * BH - 1) / ((long long)nPB * BH));
+    const int max_parts = ceil_div(Nk, kPbK);
+    if (parts > max_parts) parts = max_parts;
+    if (parts < 1) parts = 1;
+    const int keys_per_cta = ceil_div(ceil_div(Nk, parts), kPbK) * kPbK;
+    parts = ceil_div(Nk, keys_per_cta);
+    const size_t sm1 = sizeof(float) * ((size_t)D * (kPbP + kPbK) + 4 * kPbP);
+    if (cudaFuncSetAttribute(probe_rowmax_v2_kernel<T, D>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
-    probe_rowmax_kernel<T, D><<<dim3(ceil_div(Nk, kPrKeys * 4), ceil_div(Cq, kPrProbes), BH),
-                                kPrThreads, sm1, st>>>(qbar, Cq, static_cast<const T*>(Kp), Nk,
-                                                       scale, rowmax);
-    count_launches(1);
-    const size_t sm2 = sizeof(float) * ((2 * kPrProbes + 2 * kPrKeys) * P + 8 * 32);
-    auto kern = value_free ? probe_error_kernel<T, D, true> : probe_error_kernel<T, D, false>;
+    if (Nk > 0) {
+        probe_rowmax_v2_kernel<T, D><<<dim3(parts, nPB, BH), kPbThreads, sm1, st>>>(
+            qT, Cq, nPB, static_cast<const T*>(Kp), Nk, scale, keys_per_cta, rowmax);
+        count_launches(1);
+    }
+    const size_t sm2 = sm1 + sizeof(float) * (2 * D + 2 * kPbK);
+    auto kern = value_free ? probe_error_v2_kernel<T, D, true> : probe_error_v2_kernel<T, D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2) !=
         cudaSuccess)
         return SVGEAR_ERR_CUDA;
-    kern<<<dim3(Ck, ceil_div(Cq, kPrProbes), BH), kPrThreads, sm2, st>>>(
-        qbar, Cq, static_cast<const T*>(Kp), static_cast<const T*>(Vp), kbar, vbar, k_off, Ck,
+    kern<<<dim3(Ck, nPB, BH), kPbThreads, sm2, st>>>(
+        qT, Cq, nPB, static_cast<const T*>(Kp), static_cast<const T*>(Vp), kbar, vbar, k_off, Ck,
         Nk, scale, rowmax, E);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
 }
 
-template <typename T, int D>
-static int probe_disp(const float* qbar, int Cq, const void* Kp, const void* Vp,
-                      const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
-                      svgear_dims kd, float scale, float* E, uint32_t* rowmax, bool vf,
-                      cudaStream_t st) {
-    return probe_impl<T, D>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, vf, st);
-}
-
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp, const float* kbar,
                  const float* vbar, const int32_t* k_off, int Ck, svgear_dims kd, float scale,
-                 float* E, uint32_t* rowmax, cudaStream_t st, bool value_free) {
+                 float* E, uint32_t* rowmax, float* qT, cudaStream_t st, bool value_free) {
     if (kd.dtype == SVGEAR_BF16) {
-        if (kd.d == 128) return probe_disp<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
-        if (kd.d == 64) return probe_disp<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
+        if (kd.d == 128) return probe_impl<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
+        if (kd.d == 64) return probe_impl<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
     } else if (kd.dtype == SVGEAR_F32) {
-        if (kd.d == 128) return probe_disp<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
-        if (kd.d == 64) return probe_disp<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, value_free, st);
+        if (kd.d == 128) return probe_impl<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
+        if (kd.d == 64) return probe_impl<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
     }
     return SVGEAR_ERR_UNSUPPORTED;
 }

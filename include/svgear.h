@@ -197,7 +197,10 @@ int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
  * qbar_i . kbar_c and m_i = max_t s_it over every key of the head:
  *   E[i][c] = sum_{t in K_c} | e^{sbar_ic - m_i} vbar_c - e^{s_it - m_i} v_t |^2
  * (fp32).  The shift m_i keeps the exponentials finite and leaves every
- * ranking within a row unchanged.  E is 0 for an empty key cluster.
+ * ranking within a row unchanged.  E is 0 for an empty key cluster.  Each
+ * term is evaluated expanded around the key's residual w_t = v_t - vbar_c,
+ * (a-b)^2 |vbar_c|^2 - 2 (a-b) b vbar_c.w_t + b^2 |w_t|^2 with a = e^{sbar-m},
+ * b = e^{s-m} (the same quantity), summed in a fixed order.
  *   qbar      float[B][H][Cq][d] query centroids (the probes).
  *   Kp, Vp    [B][H][Nk][d] permuted keys and values (kdims.dtype).
  *   kbar,vbar float[B][H][Ck][d] key and value centroids.
@@ -205,7 +208,7 @@ int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
  *   kdims     shape of Kp (N = Nk).
  *   E         out float[B][H][Cq][Ck].
  *   ws        svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck) (holds the
- *             row maxima).
+ *             row maxima and the probes transposed in blocks of 128).
  * ------------------------------------------------------------------------ */
 int svgear_probe(const float* qbar, int32_t Cq, const void* Kp, const void* Vp,
                  const float* kbar, const float* vbar, const int32_t* k_off,

@@ -41,7 +41,7 @@ def lib():
         L.orc_update.argtypes = [P, i64, i32, P, i32, P, P]
         L.orc_stable_sort.argtypes = [P, i64, i32, P, P]
         L.orc_segment_mean.argtypes = [P, i32, P, i32, P, P]
-        L.orc_probe.argtypes = [P, i32, P, P, i64, i32, P, P, P, i32, f64, P, P]
+        L.orc_probe.argtypes = [P, i32, P, P, i64, i32, P, P, P, i32, f64, P, P, P]
         L.orc_route.argtypes = [P, P, i32, P, i32, i64, f32, P, P]
         L.orc_route_budgets.argtypes = [P, P, i32, P, i32, P, P, P]
         L.orc_topp_budget.argtypes = [P, i32, P, i32, i32, P, P, f64, f64, P, P]
@@ -138,15 +138,21 @@ def segment_mean(Xp, offsets, prev=None):
     return out
 
 
-def probe(qbar, Kp, Vp, kbar, vbar, k_off, scale: float, with_scale=False):
+def probe(qbar, Kp, Vp, kbar, vbar, k_off, scale: float, with_scale=False, with_parts=False):
+    """Probe errors E [Cq, Ck]; with_scale adds the error scale S, with_parts
+    also P (the bound on the terms of the error expanded around v_t - vbar_c);
+    S and P serve tolerance bounds only."""
     qbar, Kp, Vp, kbar, vbar = map(_f64, (qbar, Kp, Vp, kbar, vbar))
     k_off = _i32(k_off)
     Cq, d = qbar.shape
     Ck = kbar.shape[0]
     E = np.zeros((Cq, Ck))
-    S = np.zeros((Cq, Ck)) if with_scale else None
+    S = np.zeros((Cq, Ck)) if (with_scale or with_parts) else None
+    P = np.zeros((Cq, Ck)) if with_parts else None
     lib().orc_probe(_p(qbar), Cq, _p(Kp), _p(Vp), Kp.shape[0], d, _p(kbar), _p(vbar),
-                    _p(k_off), Ck, float(scale), _p(E), _p(S))
+                    _p(k_off), Ck, float(scale), _p(E), _p(S), _p(P))
+    if with_parts:
+        return E, S, P
     return (E, S) if with_scale else E
 
 

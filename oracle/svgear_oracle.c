@@ -275,13 +275,15 @@ void orc_segment_var(const double *Xp, int d, const int32_t *offsets, int C, dou
 /* with s_it = scale*qbar_i.k_t, sbar_ic = scale*qbar_i.kbar_c.              */
 /* Reading: m_i = max over all keys t of s_it, a per-row shift that keeps    */
 /* the exponentials finite and does not change any ranking within the row.   */
-/* S_ic = sum_t (e^{sbar-m}|vbar_c| + e^{s_it-m}|v_t|)^2 is an error scale   */
-/* the tests use to bound fp32 rounding; it is not part of the method.       */
+/* S_ic = sum_t (e^{sbar-m}|vbar_c| + e^{s_it-m}|v_t|)^2 and                  */
+/* P_ic = sum_t (|a - b| |vbar_c| + b |v_t - vbar_c|)^2 (a, b the two weights)  */
+/* are error scales the tests use to bound fp32 rounding (P bounds the terms  */
+/* of the error expanded around v_t - vbar_c); neither is part of the method. */
 /* ------------------------------------------------------------------------ */
 void orc_probe(const double *qbar, int Cq, const double *Kp, const double *Vp,
                int64_t Nk, int d, const double *kbar, const double *vbar,
                const int32_t *k_off, int Ck, double scale, double *E,
-               double *S) {
+               double *S, double *P) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < Cq; ++i) {
         const double *q = qbar + (size_t)i * d;
@@ -295,7 +297,7 @@ void orc_probe(const double *qbar, int Cq, const double *Kp, const double *Vp,
             const double *kb = kbar + (size_t)c * d, *vb = vbar + (size_t)c * d;
             double a = exp(scale * dot(q, kb, d) - m);
             double nvb = sqrt(dot(vb, vb, d));
-            double e = 0.0, sc = 0.0;
+            double e = 0.0, sc = 0.0, pc = 0.0;
             for (int64_t t = k_off[c]; t < k_off[c + 1]; ++t) {
                 const double *v = Vp + (size_t)t * d;
                 double b = exp(scale * dot(q, Kp + (size_t)t * d, d) - m);
@@ -303,9 +305,16 @@ void orc_probe(const double *qbar, int Cq, const double *Kp, const double *Vp,
                 e += dot(diff, diff, d);
                 double w = a * nvb + b * sqrt(dot(v, v, d));
                 sc += w * w;
+                if (P) {
+                    double r2 = 0.0;
+                    for (int k = 0; k < d; ++k) r2 += (v[k] - vb[k]) * (v[k] - vb[k]);
+                    double u = fabs(a - b) * nvb + b * sqrt(r2);
+                    pc += u * u;
+                }
             }
             E[(size_t)i * Ck + c] = e;
             if (S) S[(size_t)i * Ck + c] = sc;
+            if (P) P[(size_t)i * Ck + c] = pc;
         }
         free(diff);
     }

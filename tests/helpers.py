@@ -59,13 +59,18 @@ def update_tolerance(X, labels, C):
     return (n[:, None] / 8 + 40) * U32 * mean_abs * 2 + 1e-30
 
 
-def probe_tolerance(qbar, Kp, E, S, scale):
-    """|dE| <= 2.5 k sqrt(E S) + k^2 S + 1e-5 E, with k the relative error of
+def probe_tolerance(qbar, Kp, E, S, scale, P=None):
+    """|dE| <= 2.5 k sqrt(E S) + k^2 S + 1e-5 P, with k the relative error of
     the fp32 weights e^{s-m}: twice the dot-product bound d u scale |q||k|_max
-    plus the exp rounding."""
+    plus the exp rounding.  The last term bounds the fp32 evaluation and
+    summation of the per-key terms: the kernel evaluates each term expanded
+    around v_t - vbar_c, whose parts can differ in sign, so the bound is on
+    the sum of their magnitudes P (>= E); with all terms non-negative (the
+    value-free error) P = E."""
     qbar = np.asarray(qbar, np.float64)
     kmax = float(np.sqrt((np.asarray(Kp, np.float64) ** 2).sum(1).max()))
     d = qbar.shape[1]
     kappa = 2 * d * U32 * scale * np.sqrt((qbar ** 2).sum(1)) * kmax + 4e-7
     kappa = kappa[:, None]
-    return 2.5 * kappa * np.sqrt(E * S) + kappa ** 2 * S + 1e-5 * E + 1e-37
+    P = E if P is None else P
+    return 2.5 * kappa * np.sqrt(E * S) + kappa ** 2 * S + 1e-5 * P + 1e-37

@@ -111,9 +111,9 @@ def test_fullsize_probe_on_sampled_query_clusters(run):
     for h in HEADS[:2]:
         rows = np.array([0, 37, W.Cq - 1])
         Kp, Vp = np64(ck.Xp[0, h]), np64(run["Vp"][0, h])
-        Eo, So = oracle.probe(qbar[0, h][rows], Kp, Vp, kbar[0, h], vbar[0, h], k_off[0, h],
-                              W.scale, with_scale=True)
-        tol = probe_tolerance(qbar[0, h][rows], Kp, Eo, So, W.scale)
+        Eo, So, Po = oracle.probe(qbar[0, h][rows], Kp, Vp, kbar[0, h], vbar[0, h], k_off[0, h],
+                                  W.scale, with_parts=True)
+        tol = probe_tolerance(qbar[0, h][rows], Kp, Eo, So, W.scale, P=Po)
         Eg = E[0, h][rows].astype(np.float64)
         assert np.all(np.abs(Eg - Eo) <= tol), float(np.max(np.abs(Eg - Eo) / tol))
 

@@ -248,11 +248,11 @@ def test_probe_matches_oracle(w):
     for h in range(w.H):
         qbar = cq.centroids.cpu().numpy()[0, h]
         Kp, Vph = np64(ck.Xp)[0, h], np64(Vp)[0, h]
-        Eo, So = oracle.probe(qbar, Kp, Vph, ck.centroids.cpu().numpy()[0, h],
-                              vbar.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
-                              w.scale, with_scale=True)
+        Eo, So, Po = oracle.probe(qbar, Kp, Vph, ck.centroids.cpu().numpy()[0, h],
+                                  vbar.cpu().numpy()[0, h], ck.offsets.cpu().numpy()[0, h],
+                                  w.scale, with_parts=True)
         Eg = E.cpu().numpy()[0, h].astype(np.float64)
-        tol = probe_tolerance(qbar, Kp, Eo, So, w.scale)
+        tol = probe_tolerance(qbar, Kp, Eo, So, w.scale, P=Po)
         assert np.all(np.abs(Eg - Eo) <= tol), float(np.max(np.abs(Eg - Eo) / tol))
         empty = np.diff(ck.offsets.cpu().numpy()[0, h]) == 0
         assert np.all(Eg[:, empty] == 0)

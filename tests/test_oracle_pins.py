@@ -712,3 +712,37 @@ def test_diagnostics_full_selection_is_dense_attention():
     S = Qp @ Kp.T * 0.7
     ref = softmax(S, axis=1) @ Vp
     assert np.allclose(ref2, (ref ** 2).sum(1))
+
+def test_probe_error_equals_its_expansion_and_parts_bound_the_terms():
+    """E_ic = sum_t |a vbar - b v_t|^2 equals, term by term, the expansion
+    (a-b)^2|vbar|^2 - 2(a-b) b vbar.w_t + b^2|w_t|^2 with w_t = v_t - vbar
+    (brute force on a tiny case), and P_ic bounds the terms' absolute values."""
+    rng = np.random.default_rng(11)
+    d, Nk, Cq, Ck = 8, 40, 3, 4
+    q = rng.normal(size=(Cq, d))
+    K = rng.normal(size=(Nk, d))
+    V = rng.normal(size=(Nk, d)) + 2.0
+    off = np.array([0, 7, 7, 22, 40], np.int32)
+    kb = np.stack([K[off[c]:off[c + 1]].mean(0) if off[c + 1] > off[c] else np.zeros(d)
+                   for c in range(Ck)])
+    vb = np.stack([V[off[c]:off[c + 1]].mean(0) if off[c + 1] > off[c] else np.zeros(d)
+                   for c in range(Ck)])
+    scale = 0.3
+    E, S, P = oracle.probe(q, K, V, kb, vb, off, scale, with_parts=True)
+    for i in range(Cq):
+        m = max(scale * float(q[i] @ K[t]) for t in range(Nk))
+        for c in range(Ck):
+            a = np.exp(scale * float(q[i] @ kb[c]) - m)
+            terms, absum = 0.0, 0.0
+            for t in range(off[c], off[c + 1]):
+                b = np.exp(scale * float(q[i] @ K[t]) - m)
+                w = V[t] - vb[c]
+                t1 = (a - b) ** 2 * float(vb[c] @ vb[c])
+                t2 = -2.0 * (a - b) * b * float(vb[c] @ w)
+                t3 = b * b * float(w @ w)
+                terms += t1 + t2 + t3
+                absum += abs(t1) + abs(t2) + abs(t3)
+            assert abs(E[i, c] - terms) <= 1e-12 * max(1.0, abs(terms))
+            assert P[i, c] >= absum * (1 - 1e-12) and P[i, c] >= E[i, c] * (1 - 1e-12)
+            if off[c + 1] == off[c]:
+                assert E[i, c] == 0.0 and P[i, c] == 0.0
