@@ -83,7 +83,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc, int nA,
-                    int nB,
+                    int nB, int resident,
                     const float* __restrict__ cnorm, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
                     int* __restrict__ err) {
@@ -137,6 +137,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             tc::prefetch_tmap(&maps.b);
         }
         int ia = 0, ib = 0;
+        int loaded_bh = -1, hc = 0;   // resident mode: head in the slots, head changes
         bool ok = true;
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
             const int bh = w / tiles_per_head;
@@ -157,6 +158,32 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             }
             __syncwarp();
             ++ia;
+            if (resident) {
+                // the head's planes stay in slots 0..nB-1 (b_full[0] / b_empty[0]
+                // serve as "planes full" / "planes free"); copied at a head change
+                // once the MMAs of the previous head have completed
+                if (bh != loaded_bh) {
+                    if (hc > 0 &&
+                        !warp_wait_bar(&sh.b_empty[0], (hc - 1) & 1, abort_flag, err, (2 << 16) + hc)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        const uint32_t bar = tc::smem_u32(&sh.b_full[0]);
+                        tc::mbar_arrive_expect_tx(bar, (uint32_t)(nB * Nc * 128));
+                        for (int c = 0; c < nchunk; ++c)
+                            for (int p = 0; p < kPlanes; ++p)
+#pragma unroll
+                                for (int kh = 0; kh < KH; ++kh)
+                                    tc::tma_load_2d(sB0 + ((c * kPlanes + p) * KH + kh) * kBStageBytes,
+                                                    &maps.b, kh * 64, (bh * kPlanes + p) * Cpad + c * Nc, bar);
+                    }
+                    __syncwarp();
+                    loaded_bh = bh;
+                    ++hc;
+                }
+                continue;
+            }
             for (int c = 0; ok && c < nchunk; ++c) {
                 for (int p = 0; ok && p < kPlanes; ++p) {
                     for (int kh = 0; kh < KH; ++kh) {
@@ -185,74 +212,101 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 const int i = ia - 1 - k;
                 drain_wait(&sh.a_full[i % nA], (i / nA) & 1);
             }
-            for (int k = 0; k < nB && k < ib; ++k) {
-                const int i = ib - 1 - k;
-                drain_wait(&sh.b_full[i % nB], (i / nB) & 1);
+            if (resident) {
+                if (hc > 0) drain_wait(&sh.b_full[0], (hc - 1) & 1);
+            } else {
+                for (int k = 0; k < nB && k < ib; ++k) {
+                    const int i = ib - 1 - k;
+                    drain_wait(&sh.b_full[i % nB], (i / nB) & 1);
+                }
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
+        // Lane 0 runs the loop alone (MMA, commit and fence are single-thread
+        // operations; the warp meets again after the drain), so no warp
+        // barrier makes it wait for the tensor core to take its queued MMAs.
         const uint32_t idesc = tc::idesc_bf16(BM, Nc, false);
+        if (lane == 0) {
         int ia = 0, ib = 0, ic = 0;
+        int cur_bh = -1, hc = 0;   // resident mode: head whose planes are in use, head changes
         bool ok = true;
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
             const int bh = w / tiles_per_head;
             if (done && done[bh]) continue;
             const int sa = ia % nA;
-            if (!warp_wait_bar(&sh.a_full[sa], (ia / nA) & 1, abort_flag, err, (3 << 16) + ia)) {
+            if (!tc::wait_bar(&sh.a_full[sa], (ia / nA) & 1, abort_flag, err, (3 << 16) + ia)) {
                 ok = false;
                 break;
             }
             for (int c = 0; ok && c < nchunk; ++c) {
                 const int buf = ic & 1;
                 if (ic >= 2 &&
-                    !warp_wait_bar(&sh.acc_empty[buf], ((ic >> 1) - 1) & 1, abort_flag, err,
-                                   (4 << 16) + (ic & 0xffff))) {
+                    !tc::wait_bar(&sh.acc_empty[buf], ((ic >> 1) - 1) & 1, abort_flag, err,
+                                  (4 << 16) + (ic & 0xffff))) {
                     ok = false;
                     break;
                 }
                 tc::fence_after_sync();
-                for (int p = 0; ok && p < kPlanes; ++p) {
-                    for (int kh = 0; kh < KH; ++kh) {
-                        const int sb = ib % nB;
-                        if (!warp_wait_bar(&sh.b_full[sb], (ib / nB) & 1, abort_flag, err,
-                                           (5 << 16) + (ib & 0xffff))) {
+                if (resident) {
+                    if (bh != cur_bh) {
+                        // planes of the previous head are free once its MMAs complete;
+                        // then wait for this head's planes
+                        if (hc > 0) tc::commit(tc::smem_u32(&sh.b_empty[0]));
+                        if (!tc::wait_bar(&sh.b_full[0], hc & 1, abort_flag, err, (5 << 16) + hc)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after_sync();
-                        if (lane == 0) {
+                        cur_bh = bh;
+                        ++hc;
+                    }
+                    for (int p = 0; p < kPlanes; ++p)
+                        for (int kh = 0; kh < KH; ++kh) {
+                            const int sb = (c * kPlanes + p) * KH + kh;
+                            const uint64_t ad0 = tc::sw128_desc(sA0 + sa * kABytes + kh * 16384, 16, 1024);
+                            const uint64_t bd0 = tc::sw128_desc(sB0 + sb * kBStageBytes, 16, 1024);
 #pragma unroll
-                            for (int ks = 0; ks < 4; ++ks) {
-                                const uint64_t ad = tc::sw128_desc(
-                                    sA0 + sa * kABytes + kh * 16384 + ks * 32, 16, 1024);
-                                const uint64_t bd =
-                                    tc::sw128_desc(sB0 + sb * kBStageBytes + ks * 32, 16, 1024);
-                                tc::mma_bf16(tmem + buf * kAccCols, ad, bd, idesc,
+                            for (int ks = 0; ks < 4; ++ks)
+                                tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
                                              (p | kh | ks) != 0 ? 1u : 0u);
-                            }
-                            tc::commit(tc::smem_u32(&sh.b_empty[sb]));
                         }
-                        __syncwarp();
+                    tc::commit(tc::smem_u32(&sh.acc_full[buf]));
+                    ++ic;
+                    continue;
+                }
+                for (int p = 0; ok && p < kPlanes; ++p) {
+                    for (int kh = 0; kh < KH; ++kh) {
+                        const int sb = ib % nB;
+                        if (!tc::wait_bar(&sh.b_full[sb], (ib / nB) & 1, abort_flag, err,
+                                          (5 << 16) + (ib & 0xffff))) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                        const uint64_t ad0 = tc::sw128_desc(sA0 + sa * kABytes + kh * 16384, 16, 1024);
+                        const uint64_t bd0 = tc::sw128_desc(sB0 + sb * kBStageBytes, 16, 1024);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)   // +32 bytes per K=16 step
+                            tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
+                                         (p | kh | ks) != 0 ? 1u : 0u);
+                        tc::commit(tc::smem_u32(&sh.b_empty[sb]));
                         ++ib;
                     }
                 }
                 if (!ok) break;
-                if (lane == 0) tc::commit(tc::smem_u32(&sh.acc_full[buf]));
-                __syncwarp();
+                tc::commit(tc::smem_u32(&sh.acc_full[buf]));
                 ++ic;
             }
             if (!ok) break;
-            if (lane == 0) tc::commit(tc::smem_u32(&sh.a_empty[sa]));
-            __syncwarp();
+            tc::commit(tc::smem_u32(&sh.a_empty[sa]));
             ++ia;
         }
         // every MMA this warp issued has completed once `drain` flips; if it
         // does not, TMEM stays allocated rather than freed under a running MMA
-        if (lane == 0) {
-            tc::commit(tc::smem_u32(&sh.drain));
-            if (!drain_wait(&sh.drain, 0)) sh.keep_tmem = 1;
+        tc::commit(tc::smem_u32(&sh.drain));
+        if (!drain_wait(&sh.drain, 0)) sh.keep_tmem = 1;
         }
         __syncwarp();
     } else {
@@ -267,8 +321,36 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             if (done && done[bh]) continue;
             const int t0 = (w - bh * tiles_per_head) * BM;
             const float* cn = cnorm + (size_t)bh * Cpad;
-            float best = __int_as_float(0x7f800000);
-            int bi = 0;
+            const int t = t0 + r;
+            int32_t* lp = labels + (size_t)bh * N + t;
+            // the previous label, loaded now and compared once the tile is done
+            const int old = (changed && t < N) ? *lp : -1;
+            // four interleaved running minima (columns e mod 4), merged with ties
+            // to the lower index: the first minimum of the sequential scan
+            float best[4];
+            int bi[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                best[e] = __int_as_float(0x7f800000);
+                bi[e] = 0;
+            }
+            auto scan = [&](const uint32_t* v, int nq, int base, const float* cnc) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (q < nq) {
+                        const float4 n4 = __ldg(reinterpret_cast<const float4*>(cnc) + q);
+                        const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
+                            if (dist < best[e]) {
+                                best[e] = dist;
+                                bi[e] = base + 4 * q + e;
+                            }
+                        }
+                    }
+                }
+            };
             for (int c = 0; c < nchunk; ++c) {
                 const int buf = ic & 1;
                 if (!warp_wait_bar(&sh.acc_full[buf], (ic >> 1) & 1, abort_flag, err,
@@ -279,48 +361,25 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 tc::fence_after_sync();
                 const uint32_t tb = lane_base + buf * kAccCols;
                 const int cb = c * Nc;
-                int col = 0;
-                for (; col + 32 <= Nc; col += 32) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tb + col, v);
-                    float4 n4[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        n4[q] = __ldg(reinterpret_cast<const float4*>(cn + cb + col) + q);
+                const int nfull = Nc / 32;   // 32-column steps; Nc is a multiple of 16
+                uint32_t va[32], vb[32];
+                // double-buffered: the next step's load is in flight while one is scanned
+                if (nfull > 0) tc::tmem_ld32(tb, va);
+                for (int k = 0; k < nfull; k += 2) {
                     tc::tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float nn[4] = {n4[q].x, n4[q].y, n4[q].z, n4[q].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
-                            if (dist < best) {
-                                best = dist;
-                                bi = cb + col + 4 * q + e;
-                            }
-                        }
+                    if (k + 1 < nfull) tc::tmem_ld32(tb + (k + 1) * 32, vb);
+                    scan(va, 8, cb + k * 32, cn + cb + k * 32);
+                    if (k + 1 < nfull) {
+                        tc::tmem_ld_wait();
+                        if (k + 2 < nfull) tc::tmem_ld32(tb + (k + 2) * 32, va);
+                        scan(vb, 8, cb + (k + 1) * 32, cn + cb + (k + 1) * 32);
                     }
                 }
-                if (col < Nc) {   // Nc is a multiple of 16
-                    uint32_t v[16];
-                    tc::tmem_ld16(tb + col, v);
-                    float4 n4[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        n4[q] = __ldg(reinterpret_cast<const float4*>(cn + cb + col) + q);
+                if (Nc & 16) {
+                    uint32_t v16[16];
+                    tc::tmem_ld16(tb + nfull * 32, v16);
                     tc::tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float nn[4] = {n4[q].x, n4[q].y, n4[q].z, n4[q].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
-                            if (dist < best) {
-                                best = dist;
-                                bi = cb + col + 4 * q + e;
-                            }
-                        }
-                    }
+                    scan(v16, 4, cb + nfull * 32, cn + cb + nfull * 32);
                 }
                 // the accumulator is in registers: the MMA may refill it
                 tc::fence_before_sync();
@@ -328,11 +387,17 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 ++ic;
             }
             if (!ok) break;
-            const int t = t0 + r;
+            float bb = best[0];
+            int bx = bi[0];
+#pragma unroll
+            for (int e = 1; e < 4; ++e)
+                if (best[e] < bb || (best[e] == bb && bi[e] < bx)) {
+                    bb = best[e];
+                    bx = bi[e];
+                }
             if (t < N) {
-                int32_t* lp = labels + (size_t)bh * N + t;
-                if (changed && *lp != bi) changed[bh] = 1;
-                *lp = bi;
+                if (changed && old != bx) changed[bh] = 1;
+                *lp = bx;
             }
         }
     }
@@ -414,10 +479,16 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
     const int grid = total < num_sms[dev] ? total : num_sms[dev];
     // the centroid ring takes kBStagesUsed boxes of Nc rows (a deeper ring,
     // bought with token-tile stages, measured slower); the token-tile stages
-    // take what shared memory has left (2 to kMaxAStages)
+    // take what shared memory has left (2 to kMaxAStages).  When every box of
+    // a head's planes fits in the ring (one slot per box, at most kMaxBStages)
+    // the planes stay resident: a slot is copied again only when the CTA moves
+    // to another head.
     const size_t a_bytes = (size_t)(D / 64) * 16384, b_stage = (size_t)Nc * 128;
     const size_t budget = 227 * 1024 - 1024 - sizeof(Shared) - 64;
-    const int nB = kBStagesUsed;
+    const int boxes = nchunk * kPlanes * (D / 64);
+    const int resident = (boxes <= kMaxBStages &&
+                          budget >= 2 * a_bytes + (size_t)boxes * b_stage) ? 1 : 0;
+    const int nB = resident ? boxes : kBStagesUsed;
     if (budget < 2 * a_bytes + (size_t)nB * b_stage) return SVGEAR_ERR_UNSUPPORTED;
     const size_t b_bytes = (size_t)nB * b_stage;
     int nA = (int)((budget - b_bytes) / a_bytes);
@@ -430,7 +501,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, cn, labels,
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, cn, labels,
                                                                done, changed, err);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
@@ -439,7 +510,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, cn, labels,
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, cn, labels,
                                                               done, changed, err);
     }
     count_launches(1);
