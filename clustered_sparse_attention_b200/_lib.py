@@ -425,17 +425,27 @@ def svgear_attend(Qp, Kp, Vp, q_off, k_off, pair_off, pair_kc, kbar, vbar, q_per
 
 
 def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None,
-          topp=None, var_lambda=0.0):
+          topp=None, var_lambda=0.0, ready=None):
     """The whole layer for [B, H, N, d] tensors: cluster Q and K (seeds 2*seed
     and 2*seed+1), permute V, value centroids, route, attend.  The routing
     budget is floor(density * N) keys per query cluster, or, with topp=p, the
     keys holding p of the estimated weight (density is then unused).  With
-    var_lambda != 0 the compensation is variance-corrected.  Returns O in the
-    original token order and every intermediate."""
+    var_lambda != 0 the compensation is variance-corrected.  ready may map
+    "q", "k", "v" to CUDA events the current stream waits for before the
+    tensor's first use (inputs still arriving on another stream).  Returns O
+    in the original token order and every intermediate."""
     d = Q.shape[-1]
     scale = d ** -0.5 if scale is None else scale
+
+    def wait(name):
+        if ready is not None and ready.get(name) is not None:
+            torch.cuda.current_stream().wait_event(ready[name])
+
+    wait("q")
     cq = svgear_cluster(Q, Cq, iters, warm_q, seed=2 * seed)
+    wait("k")
     ck = svgear_cluster(K, Ck, iters, warm_k, seed=2 * seed + 1)
+    wait("v")
     Vp = svgear_permute(V, ck.perm)
     vbar = svgear_centroids(Vp, ck.offsets, Ck)
     budget = None
@@ -450,3 +460,42 @@ def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm
                       vbar, cq.perm, scale, kvar=kvar, lam=var_lambda)
     return {"O": O, "q": cq, "k": ck, "Vp": Vp, "vbar": vbar, "pair_off": pair_off,
             "pair_kc": pair_kc, "budget": budget, "kvar": kvar}
+
+
+_copy_streams = {}
+
+
+def layer_host(Qh, Kh, Vh, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None,
+               warm_k=None, topp=None, var_lambda=0.0, out=None):
+    """The layer for host tensors (pinned for the copies to overlap): Q, K and
+    V go to the device on a side stream, and each stage of the layer waits
+    only for the input it reads, so clustering Q runs while K and V are still
+    on their way.  O comes back into out (a pinned host tensor like Qh, made if
+    None), ordered after the layer on the current stream.  Returns the layer's
+    dict with "O_host" added; the host tensor is complete once the current
+    stream has passed this call."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cs = torch.cuda.current_stream(dev)
+    xs = _copy_streams.get(dev.index)
+    if xs is None:
+        xs = _copy_streams[dev.index] = torch.cuda.Stream(dev)
+    ready = {}
+    with torch.cuda.stream(xs):
+        # the device copies belong to the copy stream; record_stream keeps them
+        # from reuse until the layer's stream is done with them
+        Qd, Kd, Vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (Qh, Kh, Vh))
+        for name, d, h in (("q", Qd, Qh), ("k", Kd, Kh), ("v", Vd, Vh)):
+            d.copy_(h, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(xs)
+            ready[name] = ev
+    for d in (Qd, Kd, Vd):
+        d.record_stream(cs)
+    res = layer(Qd, Kd, Vd, Cq, Ck, iters, density, scale=scale, seed=seed, warm_q=warm_q,
+                warm_k=warm_k, topp=topp, var_lambda=var_lambda, ready=ready)
+    if out is None:
+        out = torch.empty(res["O"].shape, dtype=res["O"].dtype, pin_memory=True)
+    out.copy_(res["O"], non_blocking=True)
+    res["O_host"] = out
+    return res
+

@@ -551,6 +551,24 @@ def test_layer_with_topp_budget_end_to_end():
         assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2
 
 
+@pytest.mark.parametrize("w", [TINY, SMALL_BF16], ids=lambda w: w.name)
+def test_layer_from_host_buffers_equals_the_device_layer(w):
+    """layer_host (inputs copied on a side stream while the first stages run)
+    returns exactly the device layer's O, and the same every time."""
+    csa = _csa()
+    host, dev = _inputs(w)
+    ref = csa.layer(dev["q"], dev["k"], dev["v"], w.Cq, w.Ck, w.iters, w.density, w.scale,
+                    seed=1)["O"].cpu()
+    hp = {n: t.cpu().pin_memory() for n, t in dev.items()}
+    out = torch.empty(ref.shape, dtype=ref.dtype).pin_memory()
+    for _ in range(3):
+        res = csa.layer_host(hp["q"], hp["k"], hp["v"], w.Cq, w.Ck, w.iters, w.density,
+                             w.scale, seed=1, out=out)
+        torch.cuda.synchronize()
+        assert res["O_host"] is out
+        assert torch.equal(out, ref)
+
+
 # ---------------------------------------------------------------------------
 # Variance-corrected compensation (SVG-EAR blog, variance paragraph)
 # ---------------------------------------------------------------------------
