@@ -312,7 +312,7 @@ def workload_config(w, args):
 # traffic grows with the heads of a launch (same per-head routing), so other
 # head counts of that shape scale it.  None for shapes not captured, and None
 # while the kernel has changed since the capture.
-ATTEND_TRAFFIC_H8_WAN720P = 621.823744e6 + 144.791296e6
+ATTEND_TRAFFIC_H8_WAN720P = 561.704960e6 + 139.453696e6
 
 
 def attend_traffic(w):
