@@ -65,10 +65,10 @@ KppWs carve_kpp(Carve& cv, const svgear_dims& d, int C) {
     w.D2 = cv.take<float>(bh_of(d) * d.N);
     w.blocksum = cv.take<double>(bh_of(d) * ceil_div(d.N, kKppTokens));
     w.chosen = cv.take<int32_t>(bh_of(d) * C);
-    w.counter = cv.take<int32_t>(2 * bh_of(d));   // arrivals, then block claims
+    w.counter = cv.take<int32_t>(2 * bh_of(d));   // per-head 64-bit claim words
     w.nearest = cv.take<int32_t>(bh_of(d) * d.N);
     w.cc2 = cv.take<float>(bh_of(d) * C);
-    w.gen = cv.take<int32_t>(bh_of(d));
+    w.gen = cv.take<int32_t>(bh_of(d) + 1);   // per-head arrivals, then the finished-head count
     return w;
 }
 int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {

@@ -328,19 +328,19 @@ __device__ void kpp_block_update(const T* __restrict__ X, int N, int nblk, int b
     __syncthreads();   // d2s and warp_tot are reused by the next block
 }
 
-// Persistent seeding: CTA c works for head bh0 + c / cph, for every seed.
-// Before pass j (which adds seed j-1) it waits until the head's generation
-// word gen[bh] reaches j; it then takes block c % cph and claims further
-// 1024-token blocks from the head's work counter work[bh] until none is left
-// (blocks differ in how many tokens survive the screen, so a fixed share per
-// CTA leaves the head waiting for its slowest CTA); then it arrives on
-// counter[bh].  The last CTA of the head to arrive picks seed j (and the
-// seed-to-seed distances of the next screen), resets both counters and
-// publishes gen[bh] = j + 1.  Every block's arithmetic is the same whichever
-// CTA runs it, so the result does not depend on the claims.  Heads never wait for each other, so
-// one head's pick overlaps the other heads' passes.  The launch is
-// cooperative (every CTA resident); every wait is bounded and gives up with
-// SVGEAR_ERR_TIMEOUT in err[0] (err[1] = pass, err[2] = CTA).
+// Persistent seeding over a shared pool of work: every CTA serves every head.
+// Head h's state is claim[h] (pass index p in the high 32 bits, blocks claimed
+// in that pass in the low 32) and arrive[h] (blocks of pass p finished).  A
+// CTA claims a 1024-token block of pass p (which adds seed p-1) from its own
+// head c % BH first and from the other heads when that one has none left,
+// processes it and arrives; the CTA that finishes the last block of the pass
+// picks seed p (and the seed-to-seed distances of the next screen), resets
+// arrive[h] and publishes pass p+1 by swapping claim[h] to (p+1) << 32.  No
+// CTA waits for a particular head or CTA: while one head's pick runs, its
+// CTAs work on the other heads' passes.  Every block's arithmetic is the same
+// whichever CTA runs it, so the result does not depend on the schedule.  A
+// CTA that finds no block anywhere for kKppWaitNs gives up with
+// SVGEAR_ERR_TIMEOUT (err[1] = pass of its own head, err[2] = CTA).
 constexpr uint64_t kKppWaitNs = 2000000000ull;
 
 __device__ __forceinline__ uint64_t tc_global_ns() {
@@ -351,86 +351,127 @@ __device__ __forceinline__ uint64_t tc_global_ns() {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kKppThreads, 6)
-kpp_persistent_kernel(const T* __restrict__ X, int N, int nblk, int bh0, int BHg, int cph, int C,
-                      int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* blocksum,
-                      int32_t* counter, int32_t* work, int32_t* gen, uint64_t seed,
-                      float* centroids, int* err) {
+kpp_pool_kernel(const T* __restrict__ X, int N, int nblk, int BH, int C, int32_t* chosen,
+                float* D2, int32_t* nearest, float* cc2, double* blocksum,
+                unsigned long long* claim, int32_t* arrive, int32_t* heads_done, uint64_t seed,
+                float* centroids, int* err) {
     __shared__ KppSmem<D> sm;
     extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: C floats)
-    __shared__ int s_flag, s_next;
+    __shared__ int s_bh, s_pass, s_blk, s_last;
     const int tid = threadIdx.x;
-    const int hl = blockIdx.x / cph, part = blockIdx.x % cph;
-    if (hl >= BHg) return;
-    const int bh = bh0 + hl;
-    for (int j = 1; j < C; ++j) {
-        const int s = j - 1;
-        // wait for seed s
-        if (tid == 0) {
-            int ok = 1;
-            volatile int* g = gen + bh;
-            if (*g < j) {
-                const uint64_t t0 = tc_global_ns();
-                while (*g < j) {
-                    if (*(volatile int*)err != 0) { ok = 0; break; }
-                    if (tc_global_ns() - t0 > kKppWaitNs) {
-                        if (atomicCAS(err, 0, SVGEAR_ERR_TIMEOUT) == 0) {
-                            err[1] = j;
-                            err[2] = (int)blockIdx.x;
-                        }
-                        ok = 0;
-                        break;
-                    }
-                    __nanosleep(64);
+    const int home = blockIdx.x % BH;
+    int cur_bh = -1, cur_pass = -1;            // seed row and screen distances in shared memory
+    for (;;) {
+        if (tid < 32) {
+            // warp 0 looks for a block: lane l reads head home + l (+ 32 k), a
+            // ballot picks the nearest head with unclaimed blocks, its lane claims
+            const int lane = tid;
+            int fbh = -1, fpass = 0, fblk = 0;
+            const uint64_t t0 = tc_global_ns();
+            for (;;) {
+                int stop = 0;
+                if (lane == 0) {
+                    if (*(volatile int*)err != 0) stop = -2;
+                    else if (*(volatile int*)heads_done >= BH) stop = -3;
                 }
+                stop = __shfl_sync(0xffffffffu, stop, 0);
+                if (stop) { fbh = stop; break; }
+                for (int k0 = 0; k0 < BH && fbh < 0; k0 += 32) {
+                    const int k = k0 + lane;
+                    int h = home + k;
+                    if (h >= BH) h -= BH;
+                    bool open = false;
+                    if (k < BH) {
+                        const unsigned long long w = *(volatile unsigned long long*)(claim + h);
+                        open = (int)(w >> 32) < C && (uint32_t)w < (uint32_t)nblk;
+                    }
+                    unsigned m = __ballot_sync(0xffffffffu, open);
+                    while (m && fbh < 0) {
+                        const int src = __ffs(m) - 1;
+                        m &= m - 1;
+                        int got_bh = -1, got_pass = 0, got_blk = 0;
+                        if (lane == src) {
+                            const unsigned long long got = atomicAdd(claim + h, 1ull);
+                            if ((int)(got >> 32) < C && (uint32_t)got < (uint32_t)nblk) {
+                                got_bh = h;
+                                got_pass = (int)(got >> 32);
+                                got_blk = (int)(uint32_t)got;
+                            }
+                        }
+                        got_bh = __shfl_sync(0xffffffffu, got_bh, src);
+                        if (got_bh >= 0) {
+                            fbh = got_bh;
+                            fpass = __shfl_sync(0xffffffffu, got_pass, src);
+                            fblk = __shfl_sync(0xffffffffu, got_blk, src);
+                        }
+                    }
+                }
+                if (fbh >= 0) break;
+                // lane 0 alone reads the clock, so the warp leaves together
+                const int expired = __shfl_sync(0xffffffffu,
+                                                lane == 0 && tc_global_ns() - t0 > kKppWaitNs, 0);
+                if (expired) {
+                    if (lane == 0 && atomicCAS(err, 0, SVGEAR_ERR_TIMEOUT) == 0) {
+                        err[1] = (int)(*(volatile unsigned long long*)(claim + home) >> 32);
+                        err[2] = (int)blockIdx.x;
+                    }
+                    fbh = -2;
+                    break;
+                }
+                __nanosleep(128);
             }
-            __threadfence();   // acquire: the pick's stores are visible from here on
-            s_flag = ok;
+            __threadfence();   // acquire: the pick that published this pass is visible
+            if (lane == 0) {
+                s_bh = fbh;
+                s_pass = fpass;
+                s_blk = fblk;
+            }
         }
         __syncthreads();
-        if (!s_flag) return;
-        for (int k = tid; k < D; k += kKppThreads) sm.cen[k] = __ldcg(centroids + ((size_t)bh * C + s) * D + k);
-        for (int a = tid; a < s; a += kKppThreads) ccs[a] = __ldcg(cc2 + (size_t)bh * C + a);
-        // (the block update's first barrier orders these loads before their use)
-        // block `part` first, then blocks cph, cph + 1, ... as the head's work
-        // counter hands them out (the claim for the next block is issued
-        // before this one is processed, so its latency hides behind it)
-        for (int blk = part; blk < nblk; blk = s_next) {
-            int claim = 0;
-            if (tid == 0) claim = atomicAdd(work + bh, 1);
-            kpp_block_update<T, D>(X, N, nblk, bh, blk, s, D2, nearest, blocksum, sm, ccs);
-            if (tid == 0) s_next = cph + claim;
-            __syncthreads();
+        const int bh = s_bh, pass = s_pass, blk = s_blk;
+        if (bh < 0) return;
+        const int s = pass - 1;
+        if (bh != cur_bh || pass != cur_pass) {
+            for (int k = tid; k < D; k += kKppThreads)
+                sm.cen[k] = __ldcg(centroids + ((size_t)bh * C + s) * D + k);
+            for (int a = tid; a < s; a += kKppThreads) ccs[a] = __ldcg(cc2 + (size_t)bh * C + a);
+            cur_bh = bh;
+            cur_pass = pass;
+            // (the block update's first barrier orders these loads before their use)
         }
-        // arrive; the barrier inside the block update ordered this CTA's D^2,
-        // label and block-sum stores before thread 0's fence
+        kpp_block_update<T, D>(X, N, nblk, bh, blk, s, D2, nearest, blocksum, sm, ccs);
+        // arrive; the block update's last barrier ordered its D^2, label and
+        // block-sum stores before thread 0's fence
         if (tid == 0) {
             __threadfence();
-            s_flag = (atomicAdd(counter + bh, 1) == cph - 1);
+            s_last = (atomicAdd(arrive + bh, 1) == nblk - 1);
         }
         __syncthreads();
-        if (s_flag) {
+        if (s_last) {
             __threadfence();
-            kpp_pick<T, D>(X, N, nblk, bh, chosen, C, j, D2, blocksum, seed, centroids, cc2, sm.d2s,
-                           sm.warp_tot, sm.cen);
+            kpp_pick<T, D>(X, N, nblk, bh, chosen, C, pass, D2, blocksum, seed, centroids, cc2,
+                           sm.d2s, sm.warp_tot, sm.cen);
             __syncthreads();
             if (tid == 0) {
-                counter[bh] = 0;
-                work[bh] = 0;
+                arrive[bh] = 0;
                 __threadfence();
-                atomicExch(gen + bh, j + 1);   // release seed j
+                atomicExch(claim + bh, (unsigned long long)(pass + 1) << 32);   // release pass + 1
+                if (pass + 1 >= C) atomicAdd(heads_done, 1);
             }
+            cur_bh = -1;   // shared memory now holds the new seed, not the next screen's distances
         }
         __syncthreads();
     }
 }
 
-__global__ void kpp_init_kernel(int32_t* counter, int32_t* work, int32_t* gen, int n) {
+__global__ void kpp_init_kernel(unsigned long long* claim, int32_t* arrive, int32_t* heads_done,
+                                int n) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) {
-        counter[i] = 0;
-        work[i] = 0;
-        gen[i] = 1;   // seed 0 comes from kpp_first_kernel, launched before
+        claim[i] = 1ull << 32;   // pass 1: seed 0 comes from kpp_first_kernel, launched before
+        arrive[i] = 0;
     }
+    if (i == 0) *heads_done = 0;
 }
 
 template <typename T, int D>
@@ -440,41 +481,38 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
                          cudaStream_t st) {
     const int BH = dims.B * dims.H, N = dims.N;
     const int nblk = ceil_div(N, kKppTokens);
-    int32_t* work = counter + BH;   // the counter array holds 2 BH words
-    kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(counter, work, gen, BH);
+    // the counter array (2 BH words) holds the heads' claim words, gen (BH + 1
+    // words) the arrival counts and the finished-head count
+    unsigned long long* claim = reinterpret_cast<unsigned long long*>(counter);
+    int32_t* arrive = gen;
+    int32_t* heads_done = gen + BH;
+    kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(claim, arrive, heads_done, BH);
     count_launches(1);
     kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     if (C < 2) return SVGEAR_OK;
-    // cooperative grid: every CTA resident, so CTAs of a head may wait on each other
+    // every CTA resident (cooperative launch), as many as fit, at most one per
+    // block of a pass over all heads
     int dev = 0, sms = 0, per_sm = 0;
     const size_t ccs_bytes = sizeof(float) * (size_t)C;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kpp_persistent_kernel<T, D>,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kpp_pool_kernel<T, D>,
                                                       kKppThreads, ccs_bytes) != cudaSuccess ||
         per_sm < 1)
         return SVGEAR_ERR_CUDA;
-    const int capacity = per_sm * sms;
-    // heads per launch: all of them when every head gets a CTA, else groups
-    const int BHg_max = BH < capacity ? BH : capacity;
-    for (int bh0 = 0; bh0 < BH; bh0 += BHg_max) {
-        int BHg = BH - bh0 < BHg_max ? BH - bh0 : BHg_max;
-        int cph = capacity / BHg;
-        if (cph > nblk) cph = nblk;
-        if (cph < 1) cph = 1;
-        const int grid = BHg * cph;
-        int n_ = N, nblk_ = nblk, C_ = C;
-        uint64_t seed_ = seed;
-        const T* X_ = X;
-        void* args[] = {&X_, &n_, &nblk_, &bh0, &BHg, &cph, &C_, &chosen, &D2, &nearest, &cc2,
-                        &blocksum, &counter, &work, &gen, &seed_, &cent, &err};
-        if (cudaLaunchCooperativeKernel((const void*)kpp_persistent_kernel<T, D>, dim3(grid),
-                                        dim3(kKppThreads), args, ccs_bytes, st) != cudaSuccess)
-            return SVGEAR_ERR_CUDA;
-        count_launches(1);
-    }
+    long long grid = (long long)per_sm * sms;
+    if (grid > (long long)BH * nblk) grid = (long long)BH * nblk;
+    int n_ = N, nblk_ = nblk, BH_ = BH, C_ = C;
+    uint64_t seed_ = seed;
+    const T* X_ = X;
+    void* args[] = {&X_, &n_, &nblk_, &BH_, &C_, &chosen, &D2, &nearest, &cc2, &blocksum,
+                    &claim, &arrive, &heads_done, &seed_, &cent, &err};
+    if (cudaLaunchCooperativeKernel((const void*)kpp_pool_kernel<T, D>, dim3((unsigned)grid),
+                                    dim3(kKppThreads), args, ccs_bytes, st) != cudaSuccess)
+        return SVGEAR_ERR_CUDA;
+    count_launches(1);
     return SVGEAR_OK;
 }
 

@@ -17,11 +17,12 @@ constexpr int kSortTokens = 1024;
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // kmeans.cu
-// k-means++ seeding: one cooperative persistent launch per group of heads
-// (see kpp_persistent_kernel); err: device status words (4 ints).
+// k-means++ seeding: one cooperative persistent launch over a shared pool of
+// work (see kpp_pool_kernel); err: device status words (4 ints).
 int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
                     float* centroids, int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
-                    double* blocksum, int32_t* counter /* 2 BH words */, int32_t* gen, int* err,
+                    double* blocksum, int32_t* counter /* 2 BH words */,
+                    int32_t* gen /* BH + 1 words */, int* err,
                     cudaStream_t st);
 // done[bh] != 0 skips head bh; changed[bh] is set to 1 when a label moves.
 // scratch: assign_scratch_bytes(B*H, C, d, dtype) bytes (centroids re-laid
