@@ -80,6 +80,40 @@ def test_kmeanspp_stagewise(w):
     assert flips <= 2
 
 
+# more heads than resident CTAs, one 1024-token block each: most heads have no
+# CTA of their own and are served by CTAs homed on other heads
+MANY_HEADS = synth.custom_workload("many_heads", H=1200, frames=1, grid_h=16, grid_w=40, d=64,
+                                   dtype="bf16", Cq=4, Ck=12, iters=2, density=0.5,
+                                   n_centres=8, sigma=0.5, index=55)
+
+
+def test_kmeanspp_with_more_heads_than_ctas():
+    csa = _csa()
+    w = MANY_HEADS
+    heads = list(range(0, w.H, 97)) + [w.H - 1]
+    host, dev = _inputs(w)
+    C = w.Ck
+    cent, idx = csa.svgear_kmeanspp_init(dev["k"], C, seed=3)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    cent = cent.cpu().numpy()
+    band = 4 * (w.d + 2) * U32
+    flips = 0
+    for h in heads:
+        X = host["k"][0, h]
+        own, margin = oracle.kmeanspp(X, C, seed=3, stream=h, follow=idx[0, h])
+        assert own[0] == idx[0, h, 0]
+        diff = np.nonzero(own != idx[0, h])[0]
+        for j in diff:
+            assert margin[j] < band
+        flips += len(diff)
+        assert np.array_equal(cent[0, h], X[idx[0, h]])
+    assert flips <= 2
+    # every head: distinct seeds, all of them tokens of the head
+    assert np.all((idx >= 0) & (idx < w.N))
+    assert all(len(set(idx[0, h].tolist())) == C for h in range(w.H))
+
+
 @pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
 def test_assign_matches_oracle(w):
     csa = _csa()
