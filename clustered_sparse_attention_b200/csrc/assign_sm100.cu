@@ -7,20 +7,27 @@
 // cores; ties keep the lowest centroid index.
 //
 // Precision: x is bf16, exact as an MMA operand.  Each fp32 centroid is split
-// into three bf16 planes, c = h + m + l with h = bf16(c), m = bf16(c - h),
-// l = bf16(c - h - m) (both differences are exact in fp32; what l leaves out
-// is below 2^-26 |c|).  One fp32-accumulated MMA chain of depth 3d sums
-// x.h + x.m + x.l, whose products are exact, so the dot product keeps fp32
-// accuracy; |c|^2 is taken from the fp32 centroid.
+// into two bf16 planes, c ~ h + m with h = bf16(c), m = bf16(c - h) (the
+// difference is exact in fp32); what m leaves out is at most 2^-18 |c_k| per
+// element, so |x.(c - h - m)| <= 2^-18 sum_k |x_k c_k|: half the worst-case
+// rounding error of an fp32 dot product of length 128 (d u sum_k |x_k c_k|).
+// One fp32-accumulated MMA chain of depth 2d sums x.h + x.m, whose products
+// are exact, so the distances keep fp32 accuracy in that worst-case sense;
+// |c|^2 is taken from the fp32 centroid.  (A third plane, bf16(c - h - m),
+// would make the split exact for a third more MMAs and plane traffic.)
 //
 // B200 design: persistent CTAs, one per SM, walk the 128-token tiles of all
-// heads (tiles of heads at their fixed point are skipped).
+// heads (tiles of heads at their fixed point are skipped).  Centroid planes
+// stay in shared memory: all of a head's when they fit (each tile then runs
+// every chunk), else one chunk's at a time, run against a group of up to
+// kGroupTiles token tiles of the head before the next chunk's planes replace
+// them (each token's running minimum is carried from chunk to chunk).
 //   warp 0     TMA producer: the token tile (2 to 4 stages, as shared memory
-//              allows), then a ring of centroid-plane boxes of Nc rows x 64
-//              dims (128B-swizzled);
+//              allows) and, when the plane set changes, its boxes of Nc rows
+//              x 64 dims (128B-swizzled);
 //   warp 1     one lane issues tcgen05.mma (M=128, N=Nc <= 256, K=16) into one
 //              of two TMEM accumulators, each centroid chunk a chain of
-//              3 planes x d/16 steps;
+//              2 planes x d/16 steps;
 //   warps 2-5  epilogue, one token per thread (TMEM lane = token row):
 //              dist = |c|^2 - 2 s, running (dist, index) minimum, label out.
 // Every wait is bounded (tc_wait.cuh); on expiry the status word records
@@ -41,9 +48,9 @@ using bf16 = __nv_bfloat16;
 using tc::warp_wait_bar;
 
 constexpr int BM = 128;                  // tokens per tile (TMEM lanes)
-constexpr int kPlanes = 3;               // bf16 planes of a centroid
-constexpr int kMaxBStages = 8;           // centroid-plane ring (barrier arrays)
-constexpr int kBStagesUsed = 4;          // ring depth launched
+constexpr int kPlanes = 2;               // bf16 planes of a centroid
+constexpr int kGroupTiles = 16;          // token tiles per unit when one chunk's planes are resident
+constexpr int kMaxGroup = 16;            // carried minima per epilogue thread
 constexpr int kThreads = 6 * 32;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiThreads = 128;
@@ -54,14 +61,14 @@ constexpr uint64_t kDrainNs = 200000000ull;    // 0.2 s to let issued work land
 
 struct Maps {
     CUtensorMap x;   // tokens [B*H*N][D], boxes of 128 rows x 64
-    CUtensorMap b;   // centroid planes [B*H][3][Cpad][D], boxes of Nc rows x 64
+    CUtensorMap b;   // centroid planes [B*H][2][Cpad][D], boxes of Nc rows x 64
 };
 
 struct Shared {
     uint64_t a_full[kMaxAStages];
     uint64_t a_empty[kMaxAStages];
-    uint64_t b_full[kMaxBStages];
-    uint64_t b_empty[kMaxBStages];
+    uint64_t b_full;    // the current plane set is in its slots
+    uint64_t b_empty;   // the MMAs of the previous plane set have completed
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -83,7 +90,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc, int nA,
-                    int nB, int resident,
+                    int nB, int resident, int G,
                     const float* __restrict__ cnorm, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
                     int* __restrict__ err) {
@@ -91,8 +98,18 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     constexpr uint32_t kABytes = KH * 16384;     // 128 rows x D bf16
     if (*(volatile int*)err != 0) return;        // an earlier CTA already gave up
     const int tiles_per_head = (N + BM - 1) / BM;
-    const int total = BH * tiles_per_head;
     const int nchunk = Cpad / Nc;
+    // Work units and plane sets.  Resident: a unit is one token tile, every
+    // chunk's planes form one set per head, and each tile runs all chunks.
+    // Grouped: a unit is up to G tiles of one head, a set is one chunk's
+    // planes, and the unit's tiles run chunk by chunk (one phase per chunk),
+    // carrying each token's running minimum from phase to phase.
+    if (resident || G < 1) G = 1;
+    if (G > kMaxGroup) G = kMaxGroup;
+    const int units_per_head = (tiles_per_head + G - 1) / G;
+    const int total = BH * units_per_head;
+    const int phases = resident ? 1 : nchunk;
+    const int chunks_per_step = resident ? nchunk : 1;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ Shared sh;
@@ -111,10 +128,8 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             tc::mbar_init(tc::smem_u32(&sh.acc_full[s]), 1);
             tc::mbar_init(tc::smem_u32(&sh.acc_empty[s]), kEpiThreads);
         }
-        for (int s = 0; s < kMaxBStages; ++s) {
-            tc::mbar_init(tc::smem_u32(&sh.b_full[s]), 1);
-            tc::mbar_init(tc::smem_u32(&sh.b_empty[s]), 1);
-        }
+        tc::mbar_init(tc::smem_u32(&sh.b_full), 1);
+        tc::mbar_init(tc::smem_u32(&sh.b_empty), 1);
         tc::mbar_init(tc::smem_u32(&sh.drain), 1);
         sh.abort_flag = 0;
         sh.keep_tmem = 0;
@@ -136,72 +151,57 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             tc::prefetch_tmap(&maps.x);
             tc::prefetch_tmap(&maps.b);
         }
-        int ia = 0, ib = 0;
-        int loaded_bh = -1, hc = 0;   // resident mode: head in the slots, head changes
+        int ia = 0;
+        int loaded = -1, hc = 0;   // plane set in the slots, plane-set changes
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-            const int bh = w / tiles_per_head;
+        for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+            const int bh = u / units_per_head;
             if (done && done[bh]) continue;
-            const int t0 = (w - bh * tiles_per_head) * BM;
-            const int sa = ia % nA;
-            if (ia >= nA &&
-                !warp_wait_bar(&sh.a_empty[sa], ((ia / nA) - 1) & 1, abort_flag, err, (1 << 16) + ia)) {
-                ok = false;
-                break;
-            }
-            if (lane == 0) {
-                const uint32_t bar = tc::smem_u32(&sh.a_full[sa]);
-                tc::mbar_arrive_expect_tx(bar, BM * D * 2);
-#pragma unroll
-                for (int kh = 0; kh < KH; ++kh)
-                    tc::tma_load_2d(sA0 + sa * kABytes + kh * 16384, &maps.x, kh * 64, bh * N + t0, bar);
-            }
-            __syncwarp();
-            ++ia;
-            if (resident) {
-                // the head's planes stay in slots 0..nB-1 (b_full[0] / b_empty[0]
-                // serve as "planes full" / "planes free"); copied at a head change
-                // once the MMAs of the previous head have completed
-                if (bh != loaded_bh) {
-                    if (hc > 0 &&
-                        !warp_wait_bar(&sh.b_empty[0], (hc - 1) & 1, abort_flag, err, (2 << 16) + hc)) {
+            const int tlo = (u - bh * units_per_head) * G;
+            const int thi = min(tlo + G, tiles_per_head);
+            for (int ph = 0; ok && ph < phases; ++ph) {
+                const int set = resident ? bh : bh * nchunk + ph;
+                for (int ti = tlo; ti < thi; ++ti) {
+                    const int sa = ia % nA;
+                    if (ia >= nA &&
+                        !warp_wait_bar(&sh.a_empty[sa], ((ia / nA) - 1) & 1, abort_flag, err, (1 << 16) + ia)) {
                         ok = false;
                         break;
                     }
                     if (lane == 0) {
-                        const uint32_t bar = tc::smem_u32(&sh.b_full[0]);
-                        tc::mbar_arrive_expect_tx(bar, (uint32_t)(nB * Nc * 128));
-                        for (int c = 0; c < nchunk; ++c)
-                            for (int p = 0; p < kPlanes; ++p)
+                        const uint32_t bar = tc::smem_u32(&sh.a_full[sa]);
+                        tc::mbar_arrive_expect_tx(bar, BM * D * 2);
 #pragma unroll
-                                for (int kh = 0; kh < KH; ++kh)
-                                    tc::tma_load_2d(sB0 + ((c * kPlanes + p) * KH + kh) * kBStageBytes,
-                                                    &maps.b, kh * 64, (bh * kPlanes + p) * Cpad + c * Nc, bar);
+                        for (int kh = 0; kh < KH; ++kh)
+                            tc::tma_load_2d(sA0 + sa * kABytes + kh * 16384, &maps.x, kh * 64, bh * N + ti * BM,
+                                            bar);
                     }
                     __syncwarp();
-                    loaded_bh = bh;
-                    ++hc;
-                }
-                continue;
-            }
-            for (int c = 0; ok && c < nchunk; ++c) {
-                for (int p = 0; ok && p < kPlanes; ++p) {
-                    for (int kh = 0; kh < KH; ++kh) {
-                        const int sb = ib % nB;
-                        if (ib >= nB &&
-                            !warp_wait_bar(&sh.b_empty[sb], ((ib / nB) - 1) & 1, abort_flag, err,
-                                           (2 << 16) + (ib & 0xffff))) {
+                    ++ia;
+                    // the set's planes go into slots 0..nB-1 once the MMAs of the
+                    // previous set have completed (after this tile's copy was issued,
+                    // which the MMA warp needs before it releases the previous set)
+                    if (set != loaded) {
+                        if (hc > 0 &&
+                            !warp_wait_bar(&sh.b_empty, (hc - 1) & 1, abort_flag, err, (2 << 16) + hc)) {
                             ok = false;
                             break;
                         }
                         if (lane == 0) {
-                            const uint32_t bar = tc::smem_u32(&sh.b_full[sb]);
-                            tc::mbar_arrive_expect_tx(bar, (uint32_t)Nc * 128u);
-                            tc::tma_load_2d(sB0 + sb * kBStageBytes, &maps.b, kh * 64,
-                                            (bh * kPlanes + p) * Cpad + c * Nc, bar);
+                            const uint32_t bar = tc::smem_u32(&sh.b_full);
+                            tc::mbar_arrive_expect_tx(bar, (uint32_t)(nB * Nc * 128));
+                            const int c0 = resident ? 0 : ph;
+                            for (int c = 0; c < chunks_per_step; ++c)
+                                for (int p = 0; p < kPlanes; ++p)
+#pragma unroll
+                                    for (int kh = 0; kh < KH; ++kh)
+                                        tc::tma_load_2d(sB0 + ((c * kPlanes + p) * KH + kh) * kBStageBytes,
+                                                        &maps.b, kh * 64,
+                                                        (bh * kPlanes + p) * Cpad + (c0 + c) * Nc, bar);
                         }
                         __syncwarp();
-                        ++ib;
+                        loaded = set;
+                        ++hc;
                     }
                 }
             }
@@ -212,14 +212,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                 const int i = ia - 1 - k;
                 drain_wait(&sh.a_full[i % nA], (i / nA) & 1);
             }
-            if (resident) {
-                if (hc > 0) drain_wait(&sh.b_full[0], (hc - 1) & 1);
-            } else {
-                for (int k = 0; k < nB && k < ib; ++k) {
-                    const int i = ib - 1 - k;
-                    drain_wait(&sh.b_full[i % nB], (i / nB) & 1);
-                }
-            }
+            if (hc > 0) drain_wait(&sh.b_full, (hc - 1) & 1);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -229,79 +222,61 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         // barrier makes it wait for the tensor core to take its queued MMAs.
         const uint32_t idesc = tc::idesc_bf16(BM, Nc, false);
         if (lane == 0) {
-        int ia = 0, ib = 0, ic = 0;
-        int cur_bh = -1, hc = 0;   // resident mode: head whose planes are in use, head changes
+        int ia = 0, ic = 0;
+        int cur = -1, hc = 0;   // plane set in use, plane-set changes
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-            const int bh = w / tiles_per_head;
+        for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+            const int bh = u / units_per_head;
             if (done && done[bh]) continue;
-            const int sa = ia % nA;
-            if (!tc::wait_bar(&sh.a_full[sa], (ia / nA) & 1, abort_flag, err, (3 << 16) + ia)) {
-                ok = false;
-                break;
-            }
-            for (int c = 0; ok && c < nchunk; ++c) {
-                const int buf = ic & 1;
-                if (ic >= 2 &&
-                    !tc::wait_bar(&sh.acc_empty[buf], ((ic >> 1) - 1) & 1, abort_flag, err,
-                                  (4 << 16) + (ic & 0xffff))) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                if (resident) {
-                    if (bh != cur_bh) {
-                        // planes of the previous head are free once its MMAs complete;
-                        // then wait for this head's planes
-                        if (hc > 0) tc::commit(tc::smem_u32(&sh.b_empty[0]));
-                        if (!tc::wait_bar(&sh.b_full[0], hc & 1, abort_flag, err, (5 << 16) + hc)) {
+            const int tlo = (u - bh * units_per_head) * G;
+            const int thi = min(tlo + G, tiles_per_head);
+            for (int ph = 0; ok && ph < phases; ++ph) {
+                const int set = resident ? bh : bh * nchunk + ph;
+                for (int ti = tlo; ok && ti < thi; ++ti) {
+                    const int sa = ia % nA;
+                    if (!tc::wait_bar(&sh.a_full[sa], (ia / nA) & 1, abort_flag, err, (3 << 16) + ia)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int c = 0; c < chunks_per_step; ++c) {
+                        const int buf = ic & 1;
+                        if (ic >= 2 &&
+                            !tc::wait_bar(&sh.acc_empty[buf], ((ic >> 1) - 1) & 1, abort_flag, err,
+                                          (4 << 16) + (ic & 0xffff))) {
                             ok = false;
                             break;
                         }
                         tc::fence_after_sync();
-                        cur_bh = bh;
-                        ++hc;
-                    }
-                    for (int p = 0; p < kPlanes; ++p)
-                        for (int kh = 0; kh < KH; ++kh) {
-                            const int sb = (c * kPlanes + p) * KH + kh;
-                            const uint64_t ad0 = tc::sw128_desc(sA0 + sa * kABytes + kh * 16384, 16, 1024);
-                            const uint64_t bd0 = tc::sw128_desc(sB0 + sb * kBStageBytes, 16, 1024);
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
-                                             (p | kh | ks) != 0 ? 1u : 0u);
+                        if (set != cur) {
+                            // the previous set's slots are free once its MMAs
+                            // complete; then wait for this set's planes
+                            if (hc > 0) tc::commit(tc::smem_u32(&sh.b_empty));
+                            if (!tc::wait_bar(&sh.b_full, hc & 1, abort_flag, err, (5 << 16) + hc)) {
+                                ok = false;
+                                break;
+                            }
+                            tc::fence_after_sync();
+                            cur = set;
+                            ++hc;
                         }
-                    tc::commit(tc::smem_u32(&sh.acc_full[buf]));
-                    ++ic;
-                    continue;
-                }
-                for (int p = 0; ok && p < kPlanes; ++p) {
-                    for (int kh = 0; kh < KH; ++kh) {
-                        const int sb = ib % nB;
-                        if (!tc::wait_bar(&sh.b_full[sb], (ib / nB) & 1, abort_flag, err,
-                                          (5 << 16) + (ib & 0xffff))) {
-                            ok = false;
-                            break;
-                        }
-                        tc::fence_after_sync();
-                        const uint64_t ad0 = tc::sw128_desc(sA0 + sa * kABytes + kh * 16384, 16, 1024);
-                        const uint64_t bd0 = tc::sw128_desc(sB0 + sb * kBStageBytes, 16, 1024);
+                        for (int p = 0; p < kPlanes; ++p)
+                            for (int kh = 0; kh < KH; ++kh) {
+                                const int sb = (c * kPlanes + p) * KH + kh;
+                                const uint64_t ad0 = tc::sw128_desc(sA0 + sa * kABytes + kh * 16384, 16, 1024);
+                                const uint64_t bd0 = tc::sw128_desc(sB0 + sb * kBStageBytes, 16, 1024);
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)   // +32 bytes per K=16 step
-                            tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
-                                         (p | kh | ks) != 0 ? 1u : 0u);
-                        tc::commit(tc::smem_u32(&sh.b_empty[sb]));
-                        ++ib;
+                                for (int ks = 0; ks < 4; ++ks)   // +32 bytes per K=16 step
+                                    tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
+                                                 (p | kh | ks) != 0 ? 1u : 0u);
+                            }
+                        tc::commit(tc::smem_u32(&sh.acc_full[buf]));
+                        ++ic;
                     }
+                    if (!ok) break;
+                    tc::commit(tc::smem_u32(&sh.a_empty[sa]));
+                    ++ia;
                 }
-                if (!ok) break;
-                tc::commit(tc::smem_u32(&sh.acc_full[buf]));
-                ++ic;
             }
-            if (!ok) break;
-            tc::commit(tc::smem_u32(&sh.a_empty[sa]));
-            ++ia;
         }
         // every MMA this warp issued has completed once `drain` flips; if it
         // does not, TMEM stays allocated rather than freed under a running MMA
@@ -314,90 +289,111 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         const int quarter = warp & 3;                  // TMEM lanes this warp may read
         const int r = quarter * 32 + lane;             // token row in the tile
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        // running minimum of this thread's token in each tile of a unit,
+        // carried from one phase to the next (grouped units)
+        float carry_d[kMaxGroup];
+        int carry_i[kMaxGroup];
         int ic = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-            const int bh = w / tiles_per_head;
+        for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+            const int bh = u / units_per_head;
             if (done && done[bh]) continue;
-            const int t0 = (w - bh * tiles_per_head) * BM;
+            const int tlo = (u - bh * units_per_head) * G;
+            const int thi = min(tlo + G, tiles_per_head);
             const float* cn = cnorm + (size_t)bh * Cpad;
-            const int t = t0 + r;
-            int32_t* lp = labels + (size_t)bh * N + t;
-            // the previous label, loaded now and compared once the tile is done
-            const int old = (changed && t < N) ? *lp : -1;
-            // four interleaved running minima (columns e mod 4), merged with ties
-            // to the lower index: the first minimum of the sequential scan
-            float best[4];
-            int bi[4];
+            for (int ph = 0; ok && ph < phases; ++ph) {
+                const bool last = ph == phases - 1;
+                for (int ti = tlo; ok && ti < thi; ++ti) {
+                    const int t = ti * BM + r;
+                    int32_t* lp = labels + (size_t)bh * N + t;
+                    // the previous label, loaded now and compared once the tile is done
+                    const int old = (last && changed && t < N) ? *lp : -1;
+                    // four interleaved running minima (columns e mod 4), merged with
+                    // ties to the lower index: the first minimum of the sequential scan
+                    float best[4];
+                    int bi[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                best[e] = __int_as_float(0x7f800000);
-                bi[e] = 0;
-            }
-            auto scan = [&](const uint32_t* v, int nq, int base, const float* cnc) {
+                    for (int e = 0; e < 4; ++e) {
+                        best[e] = __int_as_float(0x7f800000);
+                        bi[e] = 0;
+                    }
+                    auto scan = [&](const uint32_t* v, int nq, int base, const float* cnc) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    if (q < nq) {
-                        const float4 n4 = __ldg(reinterpret_cast<const float4*>(cnc) + q);
-                        const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+                        for (int q = 0; q < 8; ++q) {
+                            if (q < nq) {
+                                const float4 n4 = __ldg(reinterpret_cast<const float4*>(cnc) + q);
+                                const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
-                            if (dist < best[e]) {
-                                best[e] = dist;
-                                bi[e] = base + 4 * q + e;
+                                for (int e = 0; e < 4; ++e) {
+                                    const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
+                                    if (dist < best[e]) {
+                                        best[e] = dist;
+                                        bi[e] = base + 4 * q + e;
+                                    }
+                                }
                             }
                         }
+                    };
+                    for (int c = 0; c < chunks_per_step; ++c) {
+                        const int buf = ic & 1;
+                        if (!warp_wait_bar(&sh.acc_full[buf], (ic >> 1) & 1, abort_flag, err,
+                                           (6 << 16) + (ic & 0xffff))) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                        const uint32_t tb = lane_base + buf * kAccCols;
+                        const int cb = (resident ? c : ph) * Nc;
+                        const int nfull = Nc / 32;   // 32-column steps; Nc is a multiple of 16
+                        uint32_t va[32], vb[32];
+                        // double-buffered: the next step's load is in flight while one is scanned
+                        if (nfull > 0) tc::tmem_ld32(tb, va);
+                        for (int k = 0; k < nfull; k += 2) {
+                            tc::tmem_ld_wait();
+                            if (k + 1 < nfull) tc::tmem_ld32(tb + (k + 1) * 32, vb);
+                            scan(va, 8, cb + k * 32, cn + cb + k * 32);
+                            if (k + 1 < nfull) {
+                                tc::tmem_ld_wait();
+                                if (k + 2 < nfull) tc::tmem_ld32(tb + (k + 2) * 32, va);
+                                scan(vb, 8, cb + (k + 1) * 32, cn + cb + (k + 1) * 32);
+                            }
+                        }
+                        if (Nc & 16) {
+                            uint32_t v16[16];
+                            tc::tmem_ld16(tb + nfull * 32, v16);
+                            tc::tmem_ld_wait();
+                            scan(v16, 4, cb + nfull * 32, cn + cb + nfull * 32);
+                        }
+                        // the accumulator is in registers: the MMA may refill it
+                        tc::fence_before_sync();
+                        tc::mbar_arrive(tc::smem_u32(&sh.acc_empty[buf]));
+                        ++ic;
                     }
-                }
-            };
-            for (int c = 0; c < nchunk; ++c) {
-                const int buf = ic & 1;
-                if (!warp_wait_bar(&sh.acc_full[buf], (ic >> 1) & 1, abort_flag, err,
-                                   (6 << 16) + (ic & 0xffff))) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const uint32_t tb = lane_base + buf * kAccCols;
-                const int cb = c * Nc;
-                const int nfull = Nc / 32;   // 32-column steps; Nc is a multiple of 16
-                uint32_t va[32], vb[32];
-                // double-buffered: the next step's load is in flight while one is scanned
-                if (nfull > 0) tc::tmem_ld32(tb, va);
-                for (int k = 0; k < nfull; k += 2) {
-                    tc::tmem_ld_wait();
-                    if (k + 1 < nfull) tc::tmem_ld32(tb + (k + 1) * 32, vb);
-                    scan(va, 8, cb + k * 32, cn + cb + k * 32);
-                    if (k + 1 < nfull) {
-                        tc::tmem_ld_wait();
-                        if (k + 2 < nfull) tc::tmem_ld32(tb + (k + 2) * 32, va);
-                        scan(vb, 8, cb + (k + 1) * 32, cn + cb + (k + 1) * 32);
-                    }
-                }
-                if (Nc & 16) {
-                    uint32_t v16[16];
-                    tc::tmem_ld16(tb + nfull * 32, v16);
-                    tc::tmem_ld_wait();
-                    scan(v16, 4, cb + nfull * 32, cn + cb + nfull * 32);
-                }
-                // the accumulator is in registers: the MMA may refill it
-                tc::fence_before_sync();
-                tc::mbar_arrive(tc::smem_u32(&sh.acc_empty[buf]));
-                ++ic;
-            }
-            if (!ok) break;
-            float bb = best[0];
-            int bx = bi[0];
+                    if (!ok) break;
+                    float bb = best[0];
+                    int bx = bi[0];
 #pragma unroll
-            for (int e = 1; e < 4; ++e)
-                if (best[e] < bb || (best[e] == bb && bi[e] < bx)) {
-                    bb = best[e];
-                    bx = bi[e];
+                    for (int e = 1; e < 4; ++e)
+                        if (best[e] < bb || (best[e] == bb && bi[e] < bx)) {
+                            bb = best[e];
+                            bx = bi[e];
+                        }
+                    if (ph > 0) {
+                        // earlier phases hold lower indices: they keep ties
+                        const int g = ti - tlo;
+                        if (!(bb < carry_d[g])) {
+                            bb = carry_d[g];
+                            bx = carry_i[g];
+                        }
+                    }
+                    if (!last) {
+                        carry_d[ti - tlo] = bb;
+                        carry_i[ti - tlo] = bx;
+                    } else if (t < N) {
+                        if (changed && old != bx) changed[bh] = 1;
+                        *lp = bx;
+                    }
                 }
-            if (t < N) {
-                if (changed && old != bx) changed[bh] = 1;
-                *lp = bx;
             }
         }
     }
@@ -408,7 +404,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
 }
 
 // Centroid planes and norms, one warp per centroid: planes[bh][p][c][k] for
-// p = hi, mid, lo; padding rows (c >= C) are zero with norm +inf, so they
+// p = hi, lo; padding rows (c >= C) are zero with norm +inf, so they
 // never win the minimum.
 template <int D>
 __global__ void centroid_planes_kernel(const float* __restrict__ cent, int C, int Cpad,
@@ -425,11 +421,9 @@ __global__ void centroid_planes_kernel(const float* __restrict__ cent, int C, in
         const bf16 h = __float2bfloat16_rn(v);
         const float r1 = v - __bfloat162float(h);
         const bf16 m = __float2bfloat16_rn(r1);
-        const bf16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
         const size_t row = ((size_t)bh * kPlanes * Cpad + c) * D + k;
         planes[row] = h;
         planes[row + (size_t)Cpad * D] = m;
-        planes[row + (size_t)2 * Cpad * D] = l;
         s = fmaf(v, v, s);
     }
 #pragma unroll
@@ -475,21 +469,20 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
     if (num_sms[dev] == 0 &&
         cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
-    const int total = BH * ceil_div(N, BM);
-    const int grid = total < num_sms[dev] ? total : num_sms[dev];
-    // the centroid ring takes kBStagesUsed boxes of Nc rows (a deeper ring,
-    // bought with token-tile stages, measured slower); the token-tile stages
-    // take what shared memory has left (2 to kMaxAStages).  When every box of
-    // a head's planes fits in the ring (one slot per box, at most kMaxBStages)
-    // the planes stay resident: a slot is copied again only when the CTA moves
-    // to another head.
+    const int tiles = BH * ceil_div(N, BM);
+    // Shared memory: the plane slots, then as many token-tile stages as fit
+    // (2 to kMaxAStages).  All of a head's planes stay resident when they fit
+    // beside two token stages; otherwise one chunk's planes are resident per
+    // phase of a group of kGroupTiles tiles.
     const size_t a_bytes = (size_t)(D / 64) * 16384, b_stage = (size_t)Nc * 128;
     const size_t budget = 227 * 1024 - 1024 - sizeof(Shared) - 64;
-    const int boxes = nchunk * kPlanes * (D / 64);
-    const int resident = (boxes <= kMaxBStages &&
-                          budget >= 2 * a_bytes + (size_t)boxes * b_stage) ? 1 : 0;
-    const int nB = resident ? boxes : kBStagesUsed;
+    const int boxes_head = nchunk * kPlanes * (D / 64);
+    const int resident = budget >= 2 * a_bytes + (size_t)boxes_head * b_stage ? 1 : 0;
+    const int nB = resident ? boxes_head : kPlanes * (D / 64);
     if (budget < 2 * a_bytes + (size_t)nB * b_stage) return SVGEAR_ERR_UNSUPPORTED;
+    const int G = resident ? 1 : (kGroupTiles < kMaxGroup ? kGroupTiles : kMaxGroup);
+    const int units = resident ? tiles : BH * ceil_div(ceil_div(N, BM), G);
+    const int grid = units < num_sms[dev] ? units : num_sms[dev];
     const size_t b_bytes = (size_t)nB * b_stage;
     int nA = (int)((budget - b_bytes) / a_bytes);
     if (nA > kMaxAStages) nA = kMaxAStages;
@@ -501,7 +494,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, cn, labels,
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
                                                                done, changed, err);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
@@ -510,7 +503,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, cn, labels,
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
                                                               done, changed, err);
     }
     count_launches(1);
