@@ -28,8 +28,11 @@
 //   warp 1     one lane issues tcgen05.mma (M=128, N=Nc <= 256, K=16) into one
 //              of two TMEM accumulators, each centroid chunk a chain of
 //              2 planes x d/16 steps;
-//   warps 2-5  epilogue, one token per thread (TMEM lane = token row):
-//              dist = |c|^2 - 2 s, running (dist, index) minimum, label out.
+//   warps 2-9  epilogue, two warps per TMEM lane quarter (TMEM lane = token
+//              row), each scanning half of every chunk's columns:
+//              dist = |c|^2 - 2 s, running (dist, index) minimum; the upper
+//              half hands its minimum to the lower through shared memory,
+//              which merges (ties to the lower index) and writes the label.
 // Every wait is bounded (tc_wait.cuh); on expiry the status word records
 // SVGEAR_ERR_TIMEOUT, copies and MMAs in flight are drained and the CTA
 // returns.
@@ -51,9 +54,9 @@ constexpr int BM = 128;                  // tokens per tile (TMEM lanes)
 constexpr int kPlanes = 2;               // bf16 planes of a centroid
 constexpr int kGroupTiles = 16;          // token tiles per unit when one chunk's planes are resident
 constexpr int kMaxGroup = 16;            // carried minima per epilogue thread
-constexpr int kThreads = 6 * 32;
+constexpr int kThreads = 10 * 32;
 constexpr int kMmaWarp = 1;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiThreads = 256;
 constexpr uint32_t kTmemCols = 512;      // two accumulators of up to 256 columns
 constexpr uint32_t kAccCols = 256;
 constexpr int kMaxAStages = 4;           // token-tile stages: as many as shared memory holds
@@ -72,6 +75,10 @@ struct Shared {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t pair_full[4][2];    // per lane quarter and slot: the upper half's minimum is stored
+    uint64_t pair_empty[4][2];   // the lower half has read it
+    float pair_d[2][BM];         // the upper half's running minimum, double-buffered by tile
+    uint16_t pair_i[2][BM];      // and its centroid index (C <= SVGEAR_MAX_CLUSTERS)
     uint32_t tmem_base;
     int abort_flag;
     int keep_tmem;
@@ -131,6 +138,11 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         tc::mbar_init(tc::smem_u32(&sh.b_full), 1);
         tc::mbar_init(tc::smem_u32(&sh.b_empty), 1);
         tc::mbar_init(tc::smem_u32(&sh.drain), 1);
+        for (int q = 0; q < 4; ++q)
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(tc::smem_u32(&sh.pair_full[q][s]), 32);
+                tc::mbar_init(tc::smem_u32(&sh.pair_empty[q][s]), 32);
+            }
         sh.abort_flag = 0;
         sh.keep_tmem = 0;
         tc::mbar_init_fence();
@@ -287,8 +299,16 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                  // TMEM lanes this warp may read
+        const int upper = (warp - 2) >> 2;             // 0: warps 2-5, 1: warps 6-9
         const int r = quarter * 32 + lane;             // token row in the tile
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        // a chunk's columns in steps of 32 (and a last step of 16 when Nc is
+        // an odd multiple of 16): the lower half takes the first ceil(n/2)
+        const int nfull = Nc / 32;
+        const int nsteps = nfull + ((Nc & 16) ? 1 : 0);
+        const int s_lo = upper ? (nsteps + 1) / 2 : 0;
+        const int s_hi = upper ? nsteps : (nsteps + 1) / 2;
+        int it = 0;   // tiles handed over, for the slot and its phase
         // running minimum of this thread's token in each tile of a unit,
         // carried from one phase to the next (grouped units)
         float carry_d[kMaxGroup];
@@ -307,7 +327,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                     const int t = ti * BM + r;
                     int32_t* lp = labels + (size_t)bh * N + t;
                     // the previous label, loaded now and compared once the tile is done
-                    const int old = (last && changed && t < N) ? *lp : -1;
+                    const int old = (last && changed && !upper && t < N) ? *lp : -1;
                     // four interleaved running minima (columns e mod 4), merged with
                     // ties to the lower index: the first minimum of the sequential scan
                     float best[4];
@@ -344,21 +364,21 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                         tc::fence_after_sync();
                         const uint32_t tb = lane_base + buf * kAccCols;
                         const int cb = (resident ? c : ph) * Nc;
-                        const int nfull = Nc / 32;   // 32-column steps; Nc is a multiple of 16
+                        const int hi_full = s_hi < nfull ? s_hi : nfull;   // full steps of this half
                         uint32_t va[32], vb[32];
                         // double-buffered: the next step's load is in flight while one is scanned
-                        if (nfull > 0) tc::tmem_ld32(tb, va);
-                        for (int k = 0; k < nfull; k += 2) {
+                        if (s_lo < hi_full) tc::tmem_ld32(tb + s_lo * 32, va);
+                        for (int k = s_lo; k < hi_full; k += 2) {
                             tc::tmem_ld_wait();
-                            if (k + 1 < nfull) tc::tmem_ld32(tb + (k + 1) * 32, vb);
+                            if (k + 1 < hi_full) tc::tmem_ld32(tb + (k + 1) * 32, vb);
                             scan(va, 8, cb + k * 32, cn + cb + k * 32);
-                            if (k + 1 < nfull) {
+                            if (k + 1 < hi_full) {
                                 tc::tmem_ld_wait();
-                                if (k + 2 < nfull) tc::tmem_ld32(tb + (k + 2) * 32, va);
+                                if (k + 2 < hi_full) tc::tmem_ld32(tb + (k + 2) * 32, va);
                                 scan(vb, 8, cb + (k + 1) * 32, cn + cb + (k + 1) * 32);
                             }
                         }
-                        if (Nc & 16) {
+                        if ((Nc & 16) && s_hi == nsteps && s_lo <= nfull) {   // the 16-column step
                             uint32_t v16[16];
                             tc::tmem_ld16(tb + nfull * 32, v16);
                             tc::tmem_ld_wait();
@@ -378,6 +398,35 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                             bb = best[e];
                             bx = bi[e];
                         }
+                    // the upper half hands its minimum to the lower half of the same rows
+                    const int slot = it & 1;
+                    const uint32_t use = (uint32_t)(it >> 1);
+                    ++it;
+                    if (upper) {
+                        if (use > 0 && !warp_wait_bar(&sh.pair_empty[quarter][slot], (use - 1) & 1, abort_flag,
+                                                      err, (7 << 16) + (it & 0xffff))) {
+                            ok = false;
+                            break;
+                        }
+                        sh.pair_d[slot][r] = bb;
+                        sh.pair_i[slot][r] = (uint16_t)bx;
+                        tc::mbar_arrive(tc::smem_u32(&sh.pair_full[quarter][slot]));
+                        continue;
+                    }
+                    if (!warp_wait_bar(&sh.pair_full[quarter][slot], use & 1, abort_flag, err,
+                                       (8 << 16) + (it & 0xffff))) {
+                        ok = false;
+                        break;
+                    }
+                    {
+                        const float ud = sh.pair_d[slot][r];
+                        const int ux = sh.pair_i[slot][r];
+                        tc::mbar_arrive(tc::smem_u32(&sh.pair_empty[quarter][slot]));
+                        if (ud < bb || (ud == bb && ux < bx)) {
+                            bb = ud;
+                            bx = ux;
+                        }
+                    }
                     if (ph > 0) {
                         // earlier phases hold lower indices: they keep ties
                         const int g = ti - tlo;
@@ -475,7 +524,9 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
     // beside two token stages; otherwise one chunk's planes are resident per
     // phase of a group of kGroupTiles tiles.
     const size_t a_bytes = (size_t)(D / 64) * 16384, b_stage = (size_t)Nc * 128;
-    const size_t budget = 227 * 1024 - 1024 - sizeof(Shared) - 64;
+    // the static Shared block is placed before the 1024-aligned dynamic block
+    const size_t static_bytes = (sizeof(Shared) + 1023) / 1024 * 1024;
+    const size_t budget = 227 * 1024 - static_bytes - 1024;
     const int boxes_head = nchunk * kPlanes * (D / 64);
     const int resident = budget >= 2 * a_bytes + (size_t)boxes_head * b_stage ? 1 : 0;
     const int nB = resident ? boxes_head : kPlanes * (D / 64);
