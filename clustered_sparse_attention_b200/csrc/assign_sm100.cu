@@ -8,13 +8,14 @@
 //
 // Precision: x is bf16, exact as an MMA operand.  Each fp32 centroid is split
 // into two bf16 planes, c ~ h + m with h = bf16(c), m = bf16(c - h) (the
-// difference is exact in fp32); what m leaves out is at most 2^-18 |c_k| per
-// element, so |x.(c - h - m)| <= 2^-18 sum_k |x_k c_k|: half the worst-case
-// rounding error of an fp32 dot product of length 128 (d u sum_k |x_k c_k|).
-// One fp32-accumulated MMA chain of depth 2d sums x.h + x.m, whose products
-// are exact, so the distances keep fp32 accuracy in that worst-case sense;
-// |c|^2 is taken from the fp32 centroid.  (A third plane, bf16(c - h - m),
-// would make the split exact for a third more MMAs and plane traffic.)
+// difference is exact in fp32).  The residual c - h lies below half a bf16
+// ulp of c, so rounding it loses at most 2^-17 |c_k| per element, and the
+// split changes x.c by at most 2^-17 sum_k |x_k c_k|: the worst-case rounding
+// of an fp32 dot product of length 128.  One fp32-accumulated MMA chain of
+// depth 2d sums x.h + x.m, whose products are exact; for d = 128 split and
+// accumulation together bound the error by the same 1.5 * 2^-16 sum_k
+// |x_k c_k| as an exact three-plane split accumulated over depth 3d, for a
+// third fewer MMAs and plane bytes.  |c|^2 is taken from the fp32 centroid.
 //
 // B200 design: persistent CTAs, one per SM, walk the 128-token tiles of all
 // heads (tiles of heads at their fixed point are skipped).  Centroid planes

@@ -148,8 +148,8 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
  * ties, evaluated as |c|^2 - 2 x.c with fp32-grade dot products: f32 tokens
  * by fp32 FMAs; bf16 tokens on the tensor cores, the fp32 centroid split into
  * two bf16 planes (hi, lo) whose products with the bf16 token are exact and
- * accumulate in fp32 (what the planes leave out is at most 2^-18 |c_k| per
- * element: half the worst-case rounding of an fp32 dot product of length 128).
+ * accumulate in fp32 (what the planes leave out is at most 2^-17 |c_k| per
+ * element: the worst-case rounding of an fp32 dot product of length 128).
  *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN): the device status
  *       words (svgear_device_status), then the centroids re-laid for the
  *       kernel and their norms. */
