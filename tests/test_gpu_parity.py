@@ -80,7 +80,7 @@ def test_kmeanspp_stagewise(w):
     assert flips <= 2
 
 
-# more heads than resident CTAs, one 1024-token block each: most heads have no
+# more heads than resident CTAs, 640 tokens (one partial block) each: many heads have no
 # CTA of their own and are served by CTAs homed on other heads
 MANY_HEADS = synth.custom_workload("many_heads", H=1200, frames=1, grid_h=16, grid_w=40, d=64,
                                    dtype="bf16", Cq=4, Ck=12, iters=2, density=0.5,
