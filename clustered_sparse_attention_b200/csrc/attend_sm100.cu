@@ -94,17 +94,6 @@ struct Shared {
     int keep_tmem;
 };
 
-#ifdef SVGEAR_TRACE
-// Diagnostic build only: per-tile event clocks of one CTA.
-__device__ long long g_trace[32][512];
-#define TRACE(ev, j)                                                                  \
-    do {                                                                              \
-        if (blockIdx.x == 3 && blockIdx.y == 0 && (j) < 512) g_trace[ev][j] = clock64(); \
-    } while (0)
-#else
-#define TRACE(ev, j) do { } while (0)
-#endif
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -165,12 +154,14 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                     const int32_t* __restrict__ ntiles, int maxT, const int4* __restrict__ meta,
                     const int32_t* __restrict__ seg_prefix, const int32_t* __restrict__ seg_row,
                     const int32_t* __restrict__ comp_idx, const float* __restrict__ comp_bias,
-                    float scale_log2, int use_var, bf16* __restrict__ O, int* __restrict__ err) {
+                    float scale_log2, int use_var, bf16* __restrict__ O, int* __restrict__ err,
+                    int* __restrict__ lost) {
     constexpr int REG = D / 64;                 // 64-element regions per row
     constexpr uint32_t kTileBytes = REG * 16384;
     const int bh = blockIdx.y;
     if ((int)blockIdx.x >= ntiles[bh]) return;
-    if (*(volatile int*)err != 0) return;   // an earlier CTA already gave up
+    // an earlier CTA already gave up, or the device's TMEM was lost before
+    if (tc::refuse_start(lost, err)) return;
     const int4 tile = tiles[(size_t)bh * maxT + blockIdx.x];
     const int ci = tile.x, q0 = tile.y, q_end = tile.z;
     const int nh = (q0 + BM < q_end) ? 2 : 1;     // query halves with rows
@@ -265,8 +256,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             if (j >= NS &&
                 !warp_wait_bar(&ring_empty[st], ((j / NS) - 1) & 1, abort_flag, err, (1 << 16) + j))
                 break;
-            if (isK && lane == 0) TRACE(0, j);
-            if (!isK && lane == 0) TRACE(16, j);
             const uint32_t bar = tc::smem_u32(&ring_full[st]);
             const uint32_t tX = ring0 + st * kTileBytes;
             if (j >= T_real) {
@@ -335,8 +324,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar);
             }
-            if (isK && lane == 0) TRACE(27, j);
-            if (!isK && lane == 0) TRACE(28, j);
             __syncwarp();
         }
     } else if (warp == kMmaWarp) {
@@ -357,7 +344,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         bool ok_run = wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
         for (int j = 0; ok_run && j <= T; ++j) {
             const int st = j % KSTAGES, pst = (j + VSTAGES - 1) % VSTAGES;
-            TRACE(1, j);
             for (int h = 0; h < nh; ++h) {
                 if (j > 0) {
                     if ((h == 0 && !wait_bar(&sh.v_full[pst], ((j - 1) / VSTAGES) & 1, abort_flag, err,
@@ -367,7 +353,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         break;
                     }
                     tc::fence_after_sync();
-                    TRACE(h == 0 ? 9 : 13, j);
                     const uint32_t tV = sV0 + pst * kTileBytes;
                     const int kdepth = (j - 1 >= T_real) ? CW : BN;   // keys of tile j-1
                     if (kdepth == BN) {
@@ -380,7 +365,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                                             tc::sw128_desc(tV + ks * 2048, 16384, 1024), kIdescPV,
                                             (j > 1 || ks > 0) ? 1u : 0u);
                     }
-                    TRACE(h == 0 ? 10 : 14, j);
                 }
                 if (j < T) {
                     if (h == 0 && !wait_bar(&sh.k_full[st], (j / KSTAGES) & 1, abort_flag, err, (6 << 16) + j)) {
@@ -397,7 +381,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         }
                         tc::fence_after_sync();
                     }
-                    if (h == 0) TRACE(11, j);
                     const uint32_t tQ = sQ0 + h * kTileBytes, tK = sK0 + st * kTileBytes;
                     if (D == 128 && !var_tile) {
                         tc::mma_bf16_k128(tmem + h * BN, tc::sw128_desc(tQ, 16, 1024),
@@ -422,19 +405,21 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                         }
                     }
                     tc::commit(tc::smem_u32(&sh.s_full[h]));
-                    TRACE(h == 0 ? 12 : 15, j);
                 }
             }
             if (!ok_run) break;
             if (j < T) tc::commit(tc::smem_u32(&sh.k_empty[st]));
             if (j > 0) tc::commit(tc::smem_u32(&sh.v_empty[pst]));
-            TRACE(2, j);
         }
         tc::commit(tc::smem_u32(&sh.o_full));
         // drain: every MMA of this CTA is complete once o_full flips; if that
         // wait expires, TMEM is left allocated rather than released under a
-        // running MMA (every later CTA of the launch returns before alloc)
-        if (!wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16))) sh.keep_tmem = 1;
+        // running MMA, and the device's lost word makes every later CTA and
+        // launch return before it allocates
+        if (!wait_bar(&sh.o_full, 0, abort_flag, err, (9 << 16))) {
+            sh.keep_tmem = 1;
+            tc::mark_tmem_lost(lost);
+        }
         }
         __syncwarp();
     }
@@ -469,8 +454,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 break;
             }
             tc::fence_after_sync();
-            if (tid == 0) TRACE(3, j);
-            if (tid == kSoftmaxThreads) TRACE(5, j);
             const bool comp = j >= T_real;
             const int valid = comp ? min(CW, ncomp - (j - T_real) * CW) : min(BN, L - j * BN);
             const float* bias = cb + (comp ? (j - T_real) * CW : 0);
@@ -512,14 +495,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             tc::tmem_ld32(sS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
             tc::tmem_ld32(sS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
             tc::tmem_ld_wait();
-#ifdef SVGEAR_TRACE
-            {   // stamp once the loaded registers are usable (the add waits on them)
-                const float t = __uint_as_float(v[0]) + __uint_as_float(v[63]) + __uint_as_float(v[127]);
-                if (tid == 0) g_trace[22][j & 511] = __float_as_int(t) == 0x7fffffff;
-            }
-#endif
-            if (tid == 0) TRACE(19, j);
-            if (tid == kSoftmaxThreads) TRACE(24, j);
 
             // S_h is in registers: with the variance term, the last exact tile
             // leaves q^2 in the upper half of S_h for the compensation tiles
@@ -540,11 +515,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 mx3 = fmax3(mx3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
             }
             float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-#ifdef SVGEAR_TRACE
-            if (tid == 0) g_trace[23][j & 511] = __float_as_int(mx) == 0x7fffffff;
-#endif
-            if (tid == 0) TRACE(17, j);
-            if (tid == kSoftmaxThreads) TRACE(25, j);
             if (raw) mx *= scale_log2;
             const float m_new = fmaxf(m_use, mx);
 
@@ -563,7 +533,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 l *= alpha;
                 m_use = m_new;
             }
-            if (tid == 0) TRACE(4, j);
             // P = 2^(x - m) as bf16 pairs over the first 64 columns of S_h
             const float xs = raw ? scale_log2 : 1.f, neg_m = -m_use;
             // (even, odd) columns in packed fp32 pairs: one FFMA2 and one FADD2
@@ -586,8 +555,6 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 tc::tmem_st16(sS + q * 16, pk);
             }
             l += __uint_as_float((uint32_t)s01) + __uint_as_float((uint32_t)(s01 >> 32));
-            if (tid == 0) TRACE(20, j);
-            if (tid == kSoftmaxThreads) TRACE(26, j);
             if (any) {
                 uint32_t o[16];
 #pragma unroll 1
@@ -600,12 +567,8 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
                 }
             }
             tc::tmem_st_wait();
-            if (tid == 0) TRACE(21, j);
             tc::fence_before_sync();
             tc::mbar_arrive(tc::smem_u32(&sh.p_full[h]));
-            if (tid == 0) TRACE(6, j);
-            if (tid == 96) TRACE(18, j);
-            if (tid == kSoftmaxThreads) TRACE(7, j);
         }
         // epilogue: O / l back to the original token order
         if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
@@ -716,12 +679,6 @@ __global__ void attend_tiles_kernel(const int32_t* __restrict__ q_off, int Cq, i
 
 }  // namespace sm100
 
-#ifdef SVGEAR_TRACE
-extern "C" int svgear_debug_trace(long long* host) {
-    return cudaMemcpyFromSymbol(host, sm100::g_trace, sizeof(sm100::g_trace)) == cudaSuccess ? 0 : -3;
-}
-#endif
-
 int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_dims qd, int Nk,
                         const int32_t* q_off, int Cq, const int32_t* k_off, int Ck,
                         const int32_t* pair_off, const int32_t* pair_kc, const float* kbar,
@@ -730,6 +687,9 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
     using namespace sm100;
     const int BH = qd.B * qd.H;
     const int D = qd.d;
+    if (tmem_lost_latched()) return SVGEAR_ERR_TMEM_LOST;
+    int* lost = nullptr;
+    if (int s = tmem_lost_word(&lost)) return s;
     if ((long long)BH * Nk >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;   // int32 TMA rows
     if ((long long)BH * qd.N >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;
     TmaMaps maps;
@@ -781,7 +741,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
         attend_sm100_kernel<128><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
             maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
             w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, use_var,
-            static_cast<bf16*>(O), w.status);
+            static_cast<bf16*>(O), w.status, lost);
     } else {
         if (cudaFuncSetAttribute(attend_sm100_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -789,7 +749,7 @@ int launch_attend_sm100(const void* Qp, const void* Kp, const void* Vp, svgear_d
         attend_sm100_kernel<64><<<dim3(w.maxT, BH), kThreads, smem, st>>>(
             maps, qd.N, Nk, Cq, Ck, BH, q_perm, w.tiles, w.ntiles, w.maxT, w.meta,
             w.seg_prefix, w.seg_row, w.comp_idx, w.comp_bias, scale_log2, use_var,
-            static_cast<bf16*>(O), w.status);
+            static_cast<bf16*>(O), w.status, lost);
     }
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
