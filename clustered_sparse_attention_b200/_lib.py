@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libsvgear.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
 ERR_SCRATCH_LIMIT = -6
+ERR_TMEM_LOST = -7
 NOALLOC_SORT_SCRATCH_INTS = 2 * 1024 * 1024
 F32, BF16 = 0, 1
 OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
@@ -33,7 +34,7 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_device_status", "svgear_topp_budget", "svgear_route_select_budget",
             "svgear_route_topp", "svgear_key_variance", "svgear_attend_var",
             "svgear_probe_value_free", "svgear_diagnostics",
-            "svgear_label_sort_noalloc")
+            "svgear_label_sort_noalloc", "svgear_selftest_wait")
 
 
 class Dims(ctypes.Structure):
@@ -89,6 +90,7 @@ def lib():
         "svgear_attend_status": [P, SZ, P, P],
         "svgear_device_status": [P, SZ, P, P],
         "svgear_label_sort_noalloc": [P, Dims, I32, P, P, P],
+        "svgear_selftest_wait": [P, SZ, I32, I32, I32, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -160,15 +162,34 @@ class Clustering:
     Xp: torch.Tensor | None   # [B, H, N, d] permuted copy
 
 
-def _device_status(fn, ws, n):
-    """Synchronise and raise if a bounded wait inside a tensor-core kernel of
-    the call that used `ws` gave up."""
+def device_status(ws, n=None):
+    """The four device status words of the call that used workspace `ws`
+    (synchronises the current stream): [status, wait site * 65536 + index,
+    CTA, 1 if the device's tensor memory is lost else 0]."""
+    n = ws.numel() * ws.element_size() if n is None else n
     st = (ctypes.c_int32 * 4)()
     _check("svgear_device_status", lib().svgear_device_status(_ptr(ws), n, st, _stream()))
+    return [int(x) for x in st]
+
+
+def _device_status(fn, ws, n):
+    """Synchronise and raise if a bounded wait inside a tensor-core kernel of
+    the call that used `ws` gave up, or the kernel refused to start because
+    the device's tensor memory was lost earlier."""
+    st = device_status(ws, n)
     if st[0] != OK:
-        raise SvgearError("%s (device: wait site %d, index %d, cta %d)"
-                          % (fn, st[1] >> 16, st[1] & 0xFFFF, st[2]), st[0],
+        raise SvgearError("%s (device: wait site %d, index %d, cta %d, tensor memory lost %d)"
+                          % (fn, st[1] >> 16, st[1] & 0xFFFF, st[2], st[3]), st[0],
                           lib().svgear_status_string(st[0]).decode())
+
+
+def selftest_wait(arrive, timeout_us, mark_lost=False):
+    """Run the library's bounded device wait on its own (svgear_selftest_wait)
+    and return the device status words (device_status)."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    _check("svgear_selftest_wait", lib().svgear_selftest_wait(
+        _ptr(ws), ws.numel(), int(bool(arrive)), int(timeout_us), int(bool(mark_lost)), _stream()))
+    return device_status(ws)
 
 
 def svgear_cluster(X, C, iters, warm_centroids=None, seed=0, permuted=True, out=None,

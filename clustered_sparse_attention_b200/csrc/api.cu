@@ -5,6 +5,7 @@
 
 #include <atomic>
 
+#include "carve.h"
 #include "common.cuh"
 #include "launchers.h"
 
@@ -16,22 +17,6 @@ void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_rela
 }  // namespace svgear
 
 namespace {
-
-constexpr size_t kAlign = 256;
-
-// Bump allocator over the caller's workspace; with base == nullptr it only
-// measures, so sizing and carving share one description of the layout.
-struct Carve {
-    char* base;
-    size_t off = 0;
-    explicit Carve(void* b) : base(static_cast<char*>(b)) {}
-    template <typename T> T* take(size_t count) {
-        off = (off + kAlign - 1) / kAlign * kAlign;
-        T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
-        off += sizeof(T) * count;
-        return p;
-    }
-};
 
 inline size_t bh_of(const svgear_dims& d) { return (size_t)d.B * (size_t)d.H; }
 
@@ -175,6 +160,9 @@ const char* svgear_status_string(int status) {
         case SVGEAR_ERR_WORKSPACE: return "workspace too small";
         case SVGEAR_ERR_SCRATCH_LIMIT:
             return "sizes exceed the fixed scratch of the allocation-free entry point";
+        case SVGEAR_ERR_TMEM_LOST:
+            return "an earlier tensor-core kernel on this device kept its tensor memory after a "
+                   "timeout; no tensor-core kernel can run in this context";
         default: return "unknown status";
     }
 }
@@ -251,6 +239,7 @@ int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN, dims, C, 0))
         return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
+    if (dims.dtype == SVGEAR_BF16 && tmem_lost_latched()) return SVGEAR_ERR_TMEM_LOST;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
     int* status = cv.take<int>(4);
@@ -305,6 +294,7 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
         return SVGEAR_ERR_INVALID_ARG;
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_CLUSTER, dims, C, 0)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
+    if (dims.dtype == SVGEAR_BF16 && tmem_lost_latched()) return SVGEAR_ERR_TMEM_LOST;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int BH = (int)bh_of(dims);
     Carve cf(ws);
@@ -517,6 +507,7 @@ int svgear_attend_var(const void* Qp, const void* Kp, const void* Vp, svgear_dim
         return SVGEAR_ERR_INVALID_ARG;
     if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_ATTEND, qdims, Cq, Ck)) return SVGEAR_ERR_WORKSPACE;
     if (bh_of(qdims) == 0) return SVGEAR_OK;
+    if (qdims.dtype == SVGEAR_BF16 && tmem_lost_latched()) return SVGEAR_ERR_TMEM_LOST;
     if (lambda == 0.f) kvar = nullptr;   // plain SVG-EAR compensation
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
@@ -580,19 +571,6 @@ int svgear_key_variance(const void* Kp, const int32_t* k_off, int32_t Ck, svgear
     if (!Kp || !k_off || !kvar || !aligned16(Kp)) return SVGEAR_ERR_INVALID_ARG;
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     return launch_segment_var(Kp, k_off, Ck, kdims, kvar, static_cast<cudaStream_t>(stream));
-}
-
-int svgear_device_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
-    if (!ws || !status || ws_bytes < 4 * sizeof(int)) return SVGEAR_ERR_INVALID_ARG;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(status, ws, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
-        return SVGEAR_ERR_CUDA;
-    return SVGEAR_OK;
-}
-
-int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream) {
-    return svgear_device_status(ws, ws_bytes, status, stream);
 }
 
 }  // extern "C"

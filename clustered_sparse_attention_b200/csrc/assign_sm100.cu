@@ -90,8 +90,8 @@ struct Shared {
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
     const uint32_t b = tc::smem_u32(bar);
     const uint64_t t0 = tc::global_timer_ns();
-    while (!tc::mbar_try_wait(b, parity))
-        if (tc::global_timer_ns() - t0 > kDrainNs) return false;
+    for (uint32_t it = 0; !tc::mbar_try_wait(b, parity); ++it)
+        if (tc::global_timer_ns() - t0 > kDrainNs || it >= tc::kMaxSpins) return false;
     return true;
 }
 
@@ -101,10 +101,11 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                     int nB, int resident, int G,
                     const float* __restrict__ cnorm, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
-                    int* __restrict__ err) {
+                    int* __restrict__ err, int* __restrict__ lost) {
     constexpr int KH = D / 64;                   // 64-dim halves of a row
     constexpr uint32_t kABytes = KH * 16384;     // 128 rows x D bf16
-    if (*(volatile int*)err != 0) return;        // an earlier CTA already gave up
+    // an earlier CTA already gave up, or the device's TMEM was lost before
+    if (tc::refuse_start(lost, err)) return;
     const int tiles_per_head = (N + BM - 1) / BM;
     const int nchunk = Cpad / Nc;
     // Work units and plane sets.  Resident: a unit is one token tile, every
@@ -294,7 +295,10 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         // every MMA this warp issued has completed once `drain` flips; if it
         // does not, TMEM stays allocated rather than freed under a running MMA
         tc::commit(tc::smem_u32(&sh.drain));
-        if (!drain_wait(&sh.drain, 0)) sh.keep_tmem = 1;
+        if (!drain_wait(&sh.drain, 0)) {
+            sh.keep_tmem = 1;
+            tc::mark_tmem_lost(lost);
+        }
         }
         __syncwarp();
     } else {
@@ -503,6 +507,9 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
                         const int32_t* done, int32_t* changed) {
     using namespace asg;
     const int BH = dims.B * dims.H, N = dims.N, D = dims.d;
+    if (tmem_lost_latched()) return SVGEAR_ERR_TMEM_LOST;
+    int* lost = nullptr;
+    if (int s = tmem_lost_word(&lost)) return s;
     if ((long long)BH * N >= (1ll << 31)) return SVGEAR_ERR_UNSUPPORTED;   // int32 TMA rows
     int nchunk, Nc;
     chunking(C, &nchunk, &Nc);
@@ -547,7 +554,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
         assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
-                                                               done, changed, err);
+                                                               done, changed, err, lost);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
                                                                                cn, done);
@@ -556,7 +563,7 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
         assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
-                                                              done, changed, err);
+                                                              done, changed, err, lost);
     }
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();

@@ -16,6 +16,11 @@ constexpr int kSortTokens = 1024;
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// guard.cu: the device's tensor-memory-lost word (address in the current
+// context) and whether svgear_device_status has seen it set in this context.
+int tmem_lost_word(int** out);
+bool tmem_lost_latched();
+
 // kmeans.cu
 // k-means++ seeding: one cooperative persistent launch over a shared pool of
 // work (see kpp_pool_kernel); err: device status words (4 ints).

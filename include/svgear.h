@@ -34,8 +34,10 @@
  *
  * Conventions for every call:
  *   - Pointers are DEVICE pointers unless stated; the caller allocates every
- *     buffer (outputs and workspace) and keeps ownership.  The library keeps
- *     no state between calls and never allocates device memory.
+ *     buffer (outputs and workspace) and keeps ownership.  The library never
+ *     allocates device memory and keeps no state between calls, with two
+ *     exceptions: the per-device tensor-memory guard (svgear_device_status)
+ *     and the fixed scratch of svgear_label_sort_noalloc.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
  *     the legacy default stream) and is asynchronous: a return of SVGEAR_OK
  *     means the arguments were valid and the kernels launched.
@@ -69,7 +71,8 @@ typedef enum {
     SVGEAR_ERR_CUDA = -3,
     SVGEAR_ERR_TIMEOUT = -4,
     SVGEAR_ERR_WORKSPACE = -5,
-    SVGEAR_ERR_SCRATCH_LIMIT = -6
+    SVGEAR_ERR_SCRATCH_LIMIT = -6,
+    SVGEAR_ERR_TMEM_LOST = -7
 } svgear_status;
 
 typedef enum { SVGEAR_F32 = 0, SVGEAR_BF16 = 1 } svgear_dtype;
@@ -386,19 +389,49 @@ int svgear_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_di
                        const int32_t* q_perm, float scale, const int32_t* rows, int32_t R,
                        float* recall, float* err2, float* ref2, void* stream);
 
-/* Device status of the last svgear_cluster, svgear_kmeans_assign or
- * svgear_attend that used `ws`: copies 4 int32 to status[0..3] (host memory)
- * and synchronises `stream`.  status[0] is 0 when every wait in the
- * tensor-core kernels completed, SVGEAR_ERR_TIMEOUT when a bounded wait gave
- * up (the kernel drained what it had issued and returned; its outputs are not
- * valid); status[1] and status[2] then say which wait (site * 65536 + index)
- * and which CTA (blockIdx.y * 65536 + blockIdx.x).  The words sit at the start
- * of the workspace and each of those calls clears them first.  The library's
- * own extension, with no counterpart in the method. */
+/* Device status of the last svgear_cluster, svgear_kmeans_assign,
+ * svgear_attend or svgear_selftest_wait that used `ws`: writes 4 int32 to
+ * status[0..3] (host memory) and synchronises `stream`.  status[0] is 0 when
+ * every wait in the tensor-core kernels completed, SVGEAR_ERR_TIMEOUT when a
+ * bounded wait gave up (the kernel drained what it had issued and returned;
+ * its outputs are not valid), SVGEAR_ERR_TMEM_LOST when a kernel refused to
+ * start (below); status[1] and status[2] then say which wait
+ * (site * 65536 + index; site 61 for the refusal) and which CTA
+ * (blockIdx.y * 65536 + blockIdx.x).  These words sit at the start of the
+ * workspace and each of those calls clears them first.
+ * status[3] is 1 when the device's tensor memory is lost: a kernel gave up
+ * while an MMA it had issued might still be running, so it could not free its
+ * tensor memory, and on that SM no later tensor-core kernel could allocate
+ * any.  Every tensor-core kernel checks a device word for this before it
+ * allocates and returns SVGEAR_ERR_TMEM_LOST at once; once this call has seen
+ * the word set, svgear_cluster and svgear_kmeans_assign on bf16 tokens and
+ * svgear_attend(_var) on bf16 return SVGEAR_ERR_TMEM_LOST without launching.
+ * The state lasts as long as the CUDA context (the process, or until a
+ * device reset); nothing clears it.  The library's own extension, with no
+ * counterpart in the method. */
 int svgear_device_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /* The same as svgear_device_status (kept for svgear_attend callers). */
 int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* svgear_selftest_wait -- the bounded device wait that every tensor-core
+ * kernel uses, run on its own so that its give-up path can be checked
+ * without disturbing a real kernel: one thread waits on a shared-memory
+ * mbarrier that expects one arrival.  With arrive = 1 the thread makes that
+ * arrival first and the wait completes; with arrive = 0 nothing arrives and
+ * the wait gives up after timeout_us microseconds, recording
+ * SVGEAR_ERR_TIMEOUT, site 60 and CTA 0 in the status words.  The kernel
+ * allocates no tensor memory and issues no MMA or copy.  With mark_lost = 1 a
+ * wait that gives up also sets the device's tensor-memory-lost word, as a
+ * tensor-core kernel does when its final drain expires; every later
+ * tensor-core call in this CUDA context then refuses to run (see
+ * svgear_device_status), so use it only in a process of its own.
+ *   ws          >= 16 bytes of device memory: the status words that
+ *               svgear_device_status reads (cleared first).
+ *   arrive, mark_lost   0 or 1.  timeout_us  1 .. 10,000,000.
+ * A diagnostic with no counterpart in the method. */
+int svgear_selftest_wait(void* ws, size_t ws_bytes, int32_t arrive, int32_t timeout_us,
+                         int32_t mark_lost, void* stream);
 
 /* --------------------------------------------------------------------------
  * svgear_label_sort_noalloc -- svgear_label_sort for callers that cannot give
@@ -415,9 +448,10 @@ int svgear_attend_status(const void* ws, size_t ws_bytes, int32_t* status, void*
  * that count (the Wan 720p key sort, 40*74*500, fits); larger sizes return
  * SVGEAR_ERR_SCRATCH_LIMIT without launching.  No call allocates or frees
  * device memory.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - The first call in each CUDA context -- on each device, and again after
+ *     a device reset, which destroys the context and the array with it --
+ *     looks up the array's device address (cudaGetSymbolAddress, with that
+ *     device current); make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (every entry a call reads is rewritten by that call first), so
  *     calls that overlap on the GPU -- on different streams, or from several

@@ -108,3 +108,17 @@ def test_empty_batch_is_a_no_op(L):
     assert L.svgear_kmeans_assign(fake, _dims(B=0), fake, 10, fake, fake, ctypes.c_size_t(1 << 20),
                                   None) == 0
     assert L.svgear_centroids(fake, fake, 10, _dims(B=0), fake, None) == 0
+
+
+def test_selftest_wait_validates_before_launch(L):
+    from clustered_sparse_attention_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)
+    ok = ctypes.c_size_t(256)
+    assert L.svgear_selftest_wait(None, ok, 0, 1000, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_selftest_wait(fake, ctypes.c_size_t(8), 0, 1000, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_selftest_wait(fake, ok, 2, 1000, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_selftest_wait(fake, ok, 0, 0, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_selftest_wait(fake, ok, 0, 10_000_001, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_selftest_wait(fake, ok, 0, 1000, 3, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_device_status(None, ok, fake, None) == _lib.ERR_INVALID_ARG
+    assert b"tensor memory" in L.svgear_status_string(_lib.ERR_TMEM_LOST)
