@@ -8,9 +8,8 @@
 // per-block label histograms of the counting sort) lives in the fixed array
 // below, which every GPU that loads the library keeps until the process
 // exits.  Nothing here calls cudaMalloc, cudaFree or an allocating routine.
-#include <mutex>
-
 #include "common.cuh"
+#include "ctx_cache.h"
 #include "launchers.h"
 
 namespace {
@@ -19,24 +18,15 @@ namespace {
 static __device__ __align__(256) int32_t g_sort_scratch[SVGEAR_NOALLOC_SORT_SCRATCH_INTS];
 
 // In host code `g_sort_scratch` names a host-side stand-in, not device memory,
-// so the kernels get the device address looked up once per device.
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-int32_t* g_scratch_addr[kMaxDevices] = {};
+// so the kernels get the device address, looked up once per CUDA context (a
+// device reset makes a new context, whose first call looks it up again).
+svgear::SymbolAddressCache g_scratch_addr;
 
 int scratch_on_current_device(int32_t** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SVGEAR_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SVGEAR_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_sort_scratch) != cudaSuccess || p == nullptr)
-            return SVGEAR_ERR_CUDA;
-        g_scratch_addr[dev] = static_cast<int32_t*>(p);
-    }
-    *out = g_scratch_addr[dev];
-    return SVGEAR_OK;
+    void* p = nullptr;
+    const int s = g_scratch_addr.get(g_sort_scratch, &p);
+    *out = static_cast<int32_t*>(p);
+    return s;
 }
 
 }  // namespace
