@@ -1,9 +1,11 @@
-"""The Wan 720p layer at full size (B=1, H=40, N=75600, d=128, Cq=100, Ck=500,
-40 rounds, density 0.25), run through the C ABI exactly as bench.py times it,
-then checked against the oracle on what the oracle can compute one piece at a
+"""The two 720p layers at full size, run through the C ABI exactly as bench.py
+times them -- Wan 2.1 (B=1, H=40, N=75600) and HunyuanVideo (B=1, H=24,
+N=118800), both d=128, Cq=100, Ck=500, 40 rounds, density 0.25 -- then
+checked against the oracle on what the oracle can compute one piece at a
 time: sampled heads for the sort, means and routing (whole heads), sampled
 tokens for the assignment, sampled query clusters for the probe and sampled
-rows for the attention output; k-means++ is followed seed by seed on one head.
+rows for the attention output (every 128-row tile boundary of four query
+clusters, plus random rows); k-means++ is followed seed by seed on one head.
 """
 import os
 
@@ -18,17 +20,18 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-W = synth.WORKLOADS["wan720p"]
-HEADS = (0, 17, 39)          # sampled heads
+# sampled heads of each shape: first, one inside, last
+SHAPES = {"wan720p": (0, 17, 39), "hunyuan720p": (0, 11, 23)}
 
 
 def _rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-@pytest.fixture(scope="module")
-def run():
+@pytest.fixture(scope="module", params=sorted(SHAPES))
+def run(request):
     import clustered_sparse_attention_b200 as csa
+    W = synth.WORKLOADS[request.param]
     threads = min(16, os.cpu_count() or 1)
     bits = {n: synth.layer_tensor_bits(W, n, threads=threads) for n in ("q", "k", "v")}
     dev = {n: torch.from_numpy(b).view(torch.bfloat16).cuda() for n, b in bits.items()}
@@ -46,13 +49,17 @@ def run():
         b = bits[name][0, h].astype(np.uint32) << 16
         return b.view(np.float32)
 
-    return {"csa": csa, "dev": dev, "host": host, "cq": cq, "ck": ck, "Vp": Vp, "vbar": vbar,
-            "po": po, "pk": pk, "E": E, "O": O}
+    res = {"csa": csa, "W": W, "HEADS": SHAPES[W.name], "dev": dev, "host": host, "cq": cq,
+           "ck": ck, "Vp": Vp, "vbar": vbar, "po": po, "pk": pk, "E": E, "O": O}
+    yield res
+    res.clear()
+    torch.cuda.empty_cache()
 
 
 def test_fullsize_kmeanspp_follows_the_oracle_on_one_head(run):
+    W, HEADS = run["W"], run["HEADS"]
     csa = run["csa"]
-    h = 17
+    h = HEADS[1]
     cent, idx = csa.svgear_kmeanspp_init(run["dev"]["k"], W.Ck, seed=1)
     torch.cuda.synchronize()
     idx = idx.cpu().numpy()[0, h]
@@ -67,8 +74,10 @@ def test_fullsize_kmeanspp_follows_the_oracle_on_one_head(run):
     assert np.array_equal(cent.cpu().numpy()[0, h], X[idx])
 
 
-@pytest.mark.parametrize("name,C", [("q", W.Cq), ("k", W.Ck)])
-def test_fullsize_sort_means_and_permuted_copy(run, name, C):
+@pytest.mark.parametrize("name", ["q", "k"])
+def test_fullsize_sort_means_and_permuted_copy(run, name):
+    W, HEADS = run["W"], run["HEADS"]
+    C = W.Cq if name == "q" else W.Ck
     cl = run["cq"] if name == "q" else run["ck"]
     labels = cl.labels.cpu().numpy()
     perm = cl.perm.cpu().numpy()
@@ -88,6 +97,7 @@ def test_fullsize_sort_means_and_permuted_copy(run, name, C):
 
 
 def test_fullsize_assignment_on_sampled_tokens(run):
+    W, HEADS = run["W"], run["HEADS"]
     csa = run["csa"]
     ck = run["ck"]
     lab = csa.svgear_kmeans_assign(run["dev"]["k"], ck.centroids, check_status=True).cpu().numpy()
@@ -102,6 +112,7 @@ def test_fullsize_assignment_on_sampled_tokens(run):
 
 
 def test_fullsize_probe_on_sampled_query_clusters(run):
+    W, HEADS = run["W"], run["HEADS"]
     cq, ck = run["cq"], run["ck"]
     E = run["E"].cpu().numpy()
     qbar = cq.centroids.cpu().numpy()
@@ -119,6 +130,7 @@ def test_fullsize_probe_on_sampled_query_clusters(run):
 
 
 def test_fullsize_route_bit_exact_given_gpu_errors(run):
+    W, HEADS = run["W"], run["HEADS"]
     cq, ck = run["cq"], run["ck"]
     E = run["E"].cpu().numpy()
     po, pk = run["po"].cpu().numpy(), run["pk"].cpu().numpy()
@@ -130,18 +142,21 @@ def test_fullsize_route_bit_exact_given_gpu_errors(run):
 
 
 def test_fullsize_attention_on_sampled_rows(run):
+    W, HEADS = run["W"], run["HEADS"]
     cq, ck = run["cq"], run["ck"]
     q_off = cq.offsets.cpu().numpy()
     g = np.random.default_rng(7)
     O = run["O"]
     for h in HEADS[:2]:
         qo = q_off[0, h]
-        # rows at both ends of a few query clusters (128-row tile boundaries
-        # and the partial last tile) plus random ones
+        # the first and last row of every 128-row tile of four query clusters
+        # (both halves of each tile pair and the partial last tile) plus
+        # random rows
         rows = set(g.choice(W.N, 32, replace=False).tolist())
         for i in (0, 1, W.Cq // 2, W.Cq - 1):
             a, b = int(qo[i]), int(qo[i + 1])
-            rows.update(r for r in (a, a + 127, a + 128, b - 1) if a <= r < b)
+            for r0 in range(a, b, 128):
+                rows.update((r0, min(r0 + 127, b - 1)))
         rows = np.array(sorted(rows))
         args = (np64(cq.Xp[0, h]), np64(ck.Xp[0, h]), np64(run["Vp"][0, h]), qo,
                 ck.offsets.cpu().numpy()[0, h], run["po"].cpu().numpy()[0, h],
@@ -154,6 +169,7 @@ def test_fullsize_attention_on_sampled_rows(run):
 
 
 def test_fullsize_topp_budget_and_routing(run):
+    W, HEADS = run["W"], run["HEADS"]
     csa = run["csa"]
     cq, ck = run["cq"], run["ck"]
     budget = csa.svgear_topp_budget(cq.centroids, cq.offsets, ck.centroids, ck.offsets, W.N, 0.9,
