@@ -241,6 +241,76 @@ def test_warm_start_is_one_round_from_the_cache():
                      warm.labels.cpu().numpy()[0, h])
 
 
+WARM_SEQ = synth.custom_workload("warm_seq", H=2, frames=2, grid_h=32, grid_w=40, d=128,
+                                  dtype="bf16", Cq=20, Ck=50, iters=5, density=0.25,
+                                  n_centres=32, sigma=0.5, index=55)
+
+
+@pytest.mark.parametrize("density", [0.1, 0.3])
+def test_warm_sequence_stagewise(density):
+    """The centroid cache over a drifting sequence (SVG2 section 3.4, fast
+    k-means with centroid cache): step 0 clusters cold; each later step's
+    inputs drift by 0.05 N(0,1) per element and Q and K are clustered with one
+    round from the previous step's centroids, then routed and attended.  Every
+    stage of every step is checked against the oracle fed that stage's GPU
+    inputs: labels against the cached centroids, the sort, the centroid
+    update, the permuted copies, the value centroids, the pairs given the
+    GPU's errors, and O."""
+    csa = _csa()
+    w = WARM_SEQ
+    warm = {"q": None, "k": None}
+    for step in range(4):
+        host = {n: synth.layer_tensor(w, n, step=step) for n in ("q", "k", "v")}
+        dev = {n: to_torch(a, w.dtype) for n, a in host.items()}
+        cl = {}
+        for name, C, sd in (("q", w.Cq, 0), ("k", w.Ck, 1)):
+            if step == 0:
+                cl[name] = csa.svgear_cluster(dev[name], C, w.iters, seed=sd, check_status=True)
+            else:
+                cl[name] = csa.svgear_cluster(dev[name], C, 1, warm_centroids=warm[name].clone(),
+                                              check_status=True)
+        cq, ck = cl["q"], cl["k"]
+        Vp = csa.svgear_permute(dev["v"], ck.perm)
+        vbar = csa.svgear_centroids(Vp, ck.offsets, w.Ck)
+        po, pk, E = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
+                                     ck.Xp, Vp, density, w.scale, return_errors=True)
+        O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids,
+                              vbar, cq.perm, w.scale, check_status=True)
+        torch.cuda.synchronize()
+        for h in range(w.H):
+            for name, C in (("q", w.Cq), ("k", w.Ck)):
+                c = cl[name]
+                X = host[name][0, h]
+                lab = c.labels.cpu().numpy()[0, h]
+                cents = c.centroids.cpu().numpy()[0, h]
+                if step > 0:   # one round from the cache: argmin against it
+                    check_assign(X, warm[name].cpu().numpy()[0, h], lab)
+                p_o, o_o = oracle.stable_sort(lab, C)
+                assert np.array_equal(c.perm.cpu().numpy()[0, h], p_o)
+                assert np.array_equal(c.offsets.cpu().numpy()[0, h], o_o)
+                prev = warm[name].cpu().numpy()[0, h] if step > 0 else cents
+                ref = oracle.update(X, lab, prev)
+                assert np.all(np.abs(cents - ref) <= update_tolerance(X, lab, C))
+                assert np.array_equal(np64(c.Xp)[0, h], X[p_o].astype(np.float64))
+            k_off = ck.offsets.cpu().numpy()[0, h]
+            V = host["v"][0, h][ck.perm.cpu().numpy()[0, h]]
+            lab_k = np.repeat(np.arange(w.Ck), np.diff(k_off))
+            assert np.all(np.abs(vbar.cpu().numpy()[0, h] - oracle.segment_mean(V, k_off))
+                          <= update_tolerance(V, lab_k, w.Ck))
+            ref_off, ref_kc = oracle.route(E.cpu().numpy()[0, h], cq.offsets.cpu().numpy()[0, h],
+                                           k_off, w.N, density)
+            got_off = po.cpu().numpy()[0, h]
+            assert np.array_equal(got_off, ref_off)
+            assert np.array_equal(pk.cpu().numpy()[0, h][:got_off[-1]], ref_kc)
+            Oo, _ = oracle.attend(np64(cq.Xp)[0, h], np64(ck.Xp)[0, h], np64(Vp)[0, h],
+                                  cq.offsets.cpu().numpy()[0, h], k_off, got_off,
+                                  pk.cpu().numpy()[0, h], ck.centroids.cpu().numpy()[0, h],
+                                  vbar.cpu().numpy()[0, h], cq.perm.cpu().numpy()[0, h], w.scale)
+            Og = np64(O)[0, h]
+            assert _rel_l2(Og, Oo) <= 1e-2 and np.abs(Og - Oo).max() <= 2e-2
+        warm = {"q": cq.centroids, "k": ck.centroids}
+
+
 @pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
 def test_permute_and_value_centroids(w):
     csa = _csa()
