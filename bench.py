@@ -1,18 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of one clustered sparse attention layer call on B200.
 
-A step is one pass of the whole hot path over one layer's synthetic inputs:
-k-means on Q and on K (k-means++ seeding + ``iters`` rounds, the permutation
-and segment offsets), the permuted values and their per-cluster means, the
-compensation-error probe with greedy routing, and the attention pass with
-centroid compensation that writes O in the original token order.
+A step is one pass of the whole hot path over one layer's synthetic inputs,
+one svgear_layer call through the C ABI: k-means on Q and on K (k-means++
+seeding + ``iters`` rounds, the permutation and segment offsets), the
+permuted values and their per-cluster means, the compensation-error probe
+with greedy routing, and the attention pass with centroid compensation that
+writes O in the original token order.  CUDA events recorded by the call at
+its stage boundaries give the per-stage times.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan720p]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own layer call
-(its own batch element, no exchange), so the scaling is weak and
-``value`` = slowest rank's ms per step / N (ms per layer call for the job).
+Multi-GPU (torchrun, one rank per GPU): by default the ranks split the heads
+of one layer call (rank r takes a contiguous head range, no data moves
+between ranks), so the scaling is strong and ``value`` = the slowest rank's
+ms per call; ``--split batch`` instead gives every rank its own batch element
+(weak scaling, ``value`` = slowest rank's ms per step / N).
 """
 from __future__ import annotations
 
@@ -51,9 +55,13 @@ def parse():
     p.add_argument("--iters", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     p.add_argument("--heads", type=int, default=None,
                    help="override the head count (smaller profiling cases)")
+    p.add_argument("--split", choices=["heads", "batch"], default="heads",
+                   help="multi-GPU: split one call's heads (strong) or one batch element per "
+                        "rank (weak)")
+    p.add_argument("--cpu-samples", type=int, default=3,
+                   help="runs of the oracle's sample behind cpu_baseline (the median is kept)")
     return p.parse_args()
 
 
@@ -169,74 +177,102 @@ def attention_work(q_off, k_off, pair_off, pair_kc, d):
 # ---------------------------------------------------------------------------
 # CPU oracle on a bounded sample, extrapolated to one layer call
 # ---------------------------------------------------------------------------
-def oracle_sample_ms(w, seconds=15.0, density=None, iters=None, topp=None):
-    """Time the oracle's steps on one head's data with reduced counts, each
-    scaled by the ratio of full to sampled work, and return (ms per layer
-    call, threads, description).  Setup (inputs, one clustering) is untimed."""
-    import oracle
-    density = w.density if density is None else density
-    iters = w.iters if iters is None else iters
-    frac = max(0.05, min(1.0, seconds / 15.0))
-    Q = synth.head_tensor(w, "q", 0, 0).astype(np.float64)
-    K = synth.head_tensor(w, "k", 0, 0).astype(np.float64)
-    V = synth.head_tensor(w, "v", 0, 0).astype(np.float64)
-    N, d = Q.shape
-    g = np.random.default_rng(0)
-    # untimed setup: clusters from one assignment against sampled tokens
-    cq0 = Q[g.choice(N, w.Cq, replace=False)]
-    ck0 = K[g.choice(N, w.Ck, replace=False)]
-    lq, _, _, _ = oracle.assign(Q, cq0)
-    lk, _, _, _ = oracle.assign(K, ck0)
-    timings = {}
+class OracleSample:
+    """The CPU oracle on head (0, 0) of a workload, from that head's own
+    clustered state, timed on a fixed sample and extrapolated to one layer
+    call.  The same sample serves the bench's cpu_baseline and every step of
+    the reference arm, so the two agree up to timing noise.
 
-    def timed(fn):
-        t = time.perf_counter()
-        r = fn()
-        return time.perf_counter() - t, r
+    Untimed set-up: the head's inputs and its clustering by the oracle itself
+    (k-means++, then Lloyd rounds until no label moves -- the fixed point, at
+    which further rounds repeat the same result -- or ``iters`` rounds), the
+    permuted tensors, value centroids, errors and pairs.
 
-    # k-means++: C sequential passes; time a prefix of the passes
-    npp = max(4, int(24 * frac))
-    t, _ = timed(lambda: oracle.kmeanspp(K, npp, 1, 0))
-    per_pass = t / npp
-    timings["kmeanspp"] = per_pass * (w.Cq + w.Ck) if iters and w.iters else 0.0
-    # assign: cost per (token x centroid); time a token subset against all centroids
-    nt = max(256, int(2048 * frac))
-    t_q, _ = timed(lambda: oracle.assign(Q[:nt], cq0))
-    t_k, _ = timed(lambda: oracle.assign(K[:nt], ck0))
-    timings["assign"] = (t_q + t_k) * (N / nt) * iters
-    t, cent_q = timed(lambda: oracle.update(Q, lq, cq0))
-    t2, cent_k = timed(lambda: oracle.update(K, lk, ck0))
-    timings["update"] = (t + t2) * iters
-    t, (pq, oq) = timed(lambda: oracle.stable_sort(lq, w.Cq))
-    t2, (pk, ok) = timed(lambda: oracle.stable_sort(lk, w.Ck))
-    timings["sort"] = (t + t2) * iters
-    Qp, Kp, Vp = Q[pq], K[pk], V[pk]
-    t, vbar = timed(lambda: oracle.segment_mean(Vp, ok))
-    timings["centroids"] = t
-    npr = max(1, int(4 * frac))
-    t, Es = timed(lambda: oracle.probe(cent_q[:npr], Kp, Vp, cent_k, vbar, ok, w.scale))
-    timings["probe"] = t * w.Cq / npr
-    E = np.concatenate([Es, np.tile(Es, (w.Cq // npr + 1, 1))[:w.Cq - npr]], 0)
-    if topp is None:
-        t, (po, pkc) = timed(lambda: oracle.route(E.astype(np.float32), oq, ok, N, density))
-    else:
-        def topp_route():
-            b, _ = oracle.topp_budget(cent_q, cent_k, oq, ok, topp, w.scale)
-            return oracle.route(E.astype(np.float32), oq, ok, N, 1.0, budgets=b)
-        t, (po, pkc) = timed(topp_route)
-    timings["route"] = t
-    nr = max(32, int(256 * frac))
-    rows = g.choice(N, nr, replace=False)
-    t, _ = timed(lambda: oracle.attend(Qp, Kp, Vp, oq, ok, po, pkc, cent_k, vbar, pq, w.scale,
-                                       rows=rows))
-    timings["attend"] = t * N / nr
-    per_head = sum(timings.values())
-    total_ms = per_head * w.B * w.H * 1e3
-    desc = ("oracle on head (0,0) of %s, extrapolated x%d heads: k-means++ %d of %d passes, "
-            "assign %d of %d tokens x %d iters, probe %d of %d probes, attend %d of %d rows; "
-            "update/sort/centroids/route full" % (w.name, w.B * w.H, npp, w.Cq + w.Ck, nt, N,
-                                                   iters, npr, w.Cq, nr, N))
-    return total_ms, oracle.num_threads(), desc, {k: v * 1e3 for k, v in timings.items()}
+    Timed sample, in the layer's order: k-means++ on Q and on K in full (all
+    Cq + Ck passes); one full round of assign + update + stable sort for Q
+    and for K, counted ``iters`` times (every round does the same work); the
+    value permutation and centroids; the probe for every query cluster and
+    the routing; attention for every ROW_STRIDE-th permuted query row,
+    counted ROW_STRIDE times.  The head's time times B*H is the layer's."""
+
+    ROW_STRIDE = 64
+
+    def __init__(self, w, density=None, iters=None, topp=None, var_lambda=0.0):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        self.density = w.density if density is None else density
+        self.iters = w.iters if iters is None else iters
+        self.topp = topp
+        self.lam = var_lambda
+        f64 = lambda a: np.ascontiguousarray(a, np.float64)  # noqa: E731
+        self.Q, self.K, self.V = (f64(synth.head_tensor(w, t, 0, 0)) for t in ("q", "k", "v"))
+        self.cq = self._cluster(self.Q, w.Cq, 0)
+        self.ck = self._cluster(self.K, w.Ck, 1)
+        self.pq, self.oq = oracle.stable_sort(self.cq[1], w.Cq)
+        self.pk, self.ok = oracle.stable_sort(self.ck[1], w.Ck)
+        self.Qp, self.Kp, self.Vp = self.Q[self.pq], self.K[self.pk], self.V[self.pk]
+        self.vbar = oracle.segment_mean(self.Vp, self.ok)
+        self.rows = np.arange(0, w.N, self.ROW_STRIDE)
+
+    def _cluster(self, X, C, seed):
+        o = self.oracle
+        idx, _ = o.kmeanspp(X, C, seed, 0)
+        cent, labels = X[idx].copy(), None
+        for _ in range(self.iters):
+            lab, _, _, _ = o.assign(X, cent)
+            if labels is not None and np.array_equal(lab, labels):
+                break
+            labels = lab
+            cent = o.update(X, labels, cent)
+        return cent, labels
+
+    def run(self):
+        """(ms per layer call, per-stage ms of the whole call)."""
+        o, w = self.oracle, self.w
+        t = {}
+
+        def timed(name, fn, times=1.0):
+            t0 = time.perf_counter()
+            r = fn()
+            t[name] = t.get(name, 0.0) + (time.perf_counter() - t0) * times
+            return r
+
+        timed("kmeanspp", lambda: o.kmeanspp(self.Q, w.Cq, 0, 0))
+        timed("kmeanspp", lambda: o.kmeanspp(self.K, w.Ck, 1, 0))
+        for X, (cent, lab), C in ((self.Q, self.cq, w.Cq), (self.K, self.ck, w.Ck)):
+            timed("assign", lambda: o.assign(X, cent), self.iters)
+            timed("update", lambda: o.update(X, lab, cent), self.iters)
+            timed("sort", lambda: o.stable_sort(lab, C), self.iters)
+        timed("values", lambda: o.segment_mean(self.V[self.pk], self.ok))
+        E = timed("probe", lambda: o.probe(self.cq[0], self.Kp, self.Vp, self.ck[0], self.vbar,
+                                           self.ok, w.scale))
+        if self.topp is None:
+            po, pkc = timed("route", lambda: o.route(E.astype(np.float32), self.oq, self.ok,
+                                                     w.N, self.density))
+        else:
+            def topp_route():
+                b, _ = o.topp_budget(self.cq[0], self.ck[0], self.oq, self.ok, self.topp,
+                                     w.scale)
+                return o.route(E.astype(np.float32), self.oq, self.ok, w.N, 1.0, budgets=b)
+            po, pkc = timed("route", topp_route)
+        kvar = None
+        if self.lam:
+            kvar = timed("values", lambda: o.segment_var(self.Kp, self.ok))
+        timed("attend", lambda: o.attend(self.Qp, self.Kp, self.Vp, self.oq, self.ok, po, pkc,
+                                         self.ck[0], self.vbar, self.pq, w.scale, rows=self.rows,
+                                         kvar=kvar, lam=self.lam),
+              w.N / len(self.rows))
+        heads = w.B * w.H
+        return sum(t.values()) * heads * 1e3, {k: v * heads * 1e3 for k, v in t.items()}
+
+    def describe(self):
+        w = self.w
+        return ("oracle on head (0,0) of %s from its own clustering, x%d heads: k-means++ in full "
+                "(%d passes), one full assign/update/sort round of Q and K x %d rounds, value "
+                "centroids, probe and routing in full, attention on every %dth permuted row "
+                "(%d of %d) x %d" % (w.name, w.B * w.H, w.Cq + w.Ck, self.iters, self.ROW_STRIDE,
+                                     len(self.rows), w.N, self.ROW_STRIDE))
 
 
 # ---------------------------------------------------------------------------
@@ -267,31 +303,34 @@ def run_reference(args, w):
         return
     import oracle
     oracle.lib()
-    secs = min(args.cpu_sample_seconds, 8.0)
+    sample = OracleSample(w, density=args.density, iters=args.iters, topp=args.topp,
+                          var_lambda=args.var_lambda)
     for _ in range(args.warmup):
-        oracle_sample_ms(w, seconds=secs * 0.3, density=args.density, iters=args.iters,
-                         topp=args.topp)
-    vals = []
-    desc = ""
-    cores = 1
-    for _ in range(args.steps):
-        v, cores, desc, _ = oracle_sample_ms(w, seconds=secs, density=args.density, topp=args.topp,
-                                             iters=args.iters)
-        vals.append(v)
+        sample.run()
+    vals = [sample.run()[0] for _ in range(args.steps)]
     value = float(np.mean(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "ms",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": value,
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w, args),
-        "cpu_baseline": {"value": value, "unit": "ms", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "higher_is_better": False, "scaling": "strong" if args.split == "heads" else "weak",
+        "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, args, ws),
+        "cpu_baseline": {"value": value, "unit": "ms", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample.describe(),
+                         "spread": [float(min(vals)), float(max(vals))]},
         "e2e": {"value": value, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, args):
+def workload_config(w, args, ws=1):
+    if ws > 1 and args.split == "heads":
+        par = ("heads split over %d GPUs (%d-%d heads each), no data exchanged"
+               % (ws, w.H // ws, -(-w.H // ws)))
+    elif ws > 1:
+        par = "one independent layer call per GPU on its own batch element (no exchange)"
+    else:
+        par = "one GPU"
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
             "iters": args.iters or w.iters,
             "compensation": ("variance-corrected, lambda %g" % args.var_lambda if args.var_lambda
@@ -304,21 +343,41 @@ def workload_config(w, args):
                             if w.warm_steps else "k-means++ (cold)"),
             "inputs": "%s, seeded Gaussian mixtures" % w.dtype,
             "l2": "inputs larger than L2 (3 x %.0f MB)" % (w.B * w.H * w.N * w.d * 2 / 1e6),
-            "parallelism": "one independent layer call per GPU (no exchange)"}
+            "parallelism": par}
 
 
-# DRAM bytes (read + write) of one attend_sm100_kernel launch, from the ncu
-# capture of the 8-head Wan 720p case (profiles/attend_sm100_wan720p_h8.md);
-# traffic grows with the heads of a launch (same per-head routing), so other
-# head counts of that shape scale it.  None for shapes not captured, and None
-# while the kernel has changed since the capture.
-ATTEND_TRAFFIC_H8_WAN720P = 561.704960e6 + 139.453696e6
+# ---------------------------------------------------------------------------
+# DRAM traffic of the attention kernel from a committed ncu capture
+# ---------------------------------------------------------------------------
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.json")
+ATTEND_SOURCES = ("attend_sm100.cu", "tc_ptx.cuh", "tc_wait.cuh", "common.cuh", "tma_host.h")
+
+
+def sources_sha256(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "clustered_sparse_attention_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def attend_traffic(w):
-    if (ATTEND_TRAFFIC_H8_WAN720P is not None and w.name.startswith("wan720p") and w.N == 75600
-            and w.d == 128 and w.Ck == 500):
-        return ATTEND_TRAFFIC_H8_WAN720P * (w.B * w.H) / 8.0
+    """DRAM bytes (read + write) of one attention launch of workload w, from
+    the capture record of the same kernel source (sha256 of its files) on the
+    same shape, scaled by the launch's heads (every head has the same routing
+    statistics).  None when no record matches: the kernel changed since its
+    capture, or the shape was never captured."""
+    if not os.path.exists(TRAFFIC_RECORD):
+        return None
+    with open(TRAFFIC_RECORD) as f:
+        records = json.load(f).get("records", [])
+    sha = sources_sha256(ATTEND_SOURCES)
+    for r in records:
+        if (r.get("kernel") == "attend_sm100_kernel" and r.get("sources_sha256") == sha
+                and r.get("N") == w.N and r.get("Cq") == w.Cq and r.get("Ck") == w.Ck
+                and r.get("d") == w.d and abs(r.get("density", -1) - w.density) < 1e-9):
+            return r["dram_bytes_per_launch"] * (w.B * w.H) / r["heads"]
     return None
 
 
@@ -328,6 +387,9 @@ def main():
     if args.heads:
         import dataclasses
         w = dataclasses.replace(w, H=args.heads, name="%s_h%d" % (w.name, args.heads))
+    if args.density:
+        import dataclasses
+        w = dataclasses.replace(w, density=args.density)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -337,39 +399,48 @@ def main():
     from clustered_sparse_attention_b200 import ranks as ranks_mod
     ws, rank, local = dist_setup(args)
     iters = args.iters or w.iters
-    density = args.density or w.density
+    density = w.density
     dev = torch.device("cuda", torch.cuda.current_device())
+    threads = min(16, os.cpu_count() or 1)
 
-    # inputs: this rank's own batch element (weak scaling), resident in HBM
+    # this rank's share: a head range of batch element 0 (head split) or its
+    # own batch element (batch split); the inputs are resident in HBM
+    split = args.split if ws > 1 else "heads"
+    heads = list(range(w.H))
+    batch_offset = 0
+    if split == "heads":
+        lo, hi = ranks_mod.head_range(w.H, ws, rank)
+        heads = list(range(lo, hi))
+    else:
+        batch_offset = ranks_mod.batch_offset(rank)
+    Hl = len(heads)
+
     def host_tensor(name):
-        if w.dtype == "f32":   # the small fp32 workload: every rank draws batch 0
-            return torch.from_numpy(synth.layer_tensor(w, name, threads=min(16, os.cpu_count() or 1)))
-        from clustered_sparse_attention_b200 import ranks
-        bits = synth.layer_tensor_bits(w, name, threads=min(16, os.cpu_count() or 1),
-                                       batch_offset=ranks.batch_offset(rank))
+        if w.dtype == "f32":
+            return torch.from_numpy(synth.layer_tensor(w, name, heads=heads, threads=threads))
+        bits = synth.layer_tensor_bits(w, name, heads=heads, threads=threads,
+                                       batch_offset=batch_offset)
         return torch.from_numpy(bits).view(torch.bfloat16)
 
     host = {n: host_tensor(n).pin_memory() for n in ("q", "k", "v")}
     Q, K, V = (host[n].to(dev) for n in ("q", "k", "v"))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-
     ev_names = ("cluster_q", "cluster_k", "values", "route", "attend")
+    common = dict(scale=w.scale, seed=rank, topp=args.topp, var_lambda=args.var_lambda)
 
-    # Warm-start workload (centroid cache, SVG2 section 3.4): step 0 is a cold
-    # clustering (untimed) that fills the cache; every later step drifts the
-    # inputs by drift * N(0, 1) per element (drawn on the device, before the
-    # timed region) and clusters with one round from the previous centroids.
+    # Warm-start workload (centroid cache, SVG2 section 3.4): a cold call
+    # (untimed) fills the cache; every later step's inputs drift by
+    # drift * N(0, 1) per element (drawn on the device before the timed
+    # region) and each call clusters with one round from the previous
+    # centroids, updating the cache in place.
     warm = {"q": None, "k": None}
+    inputs = None
     if w.warm_steps:
-        cold = csa.svgear_cluster(Q, w.Cq, 40, seed=2 * rank)
-        warm["q"] = cold.centroids
-        cold = csa.svgear_cluster(K, w.Ck, 40, seed=2 * rank + 1)
-        warm["k"] = cold.centroids
+        _, warm["q"], warm["k"] = csa.svgear_layer(Q, K, V, w.Cq, w.Ck, 40, density, **common)
         gen = torch.Generator(device=dev)
-        n_inputs = max(3, args.warmup) + args.steps
         inputs, cur = [], [Q, K, V]
-        for t in range(n_inputs):
+        for t in range(max(3, args.warmup) + args.steps + 1):
             nxt = []
             for i, X in enumerate(cur):
                 gen.manual_seed(1000003 * (t + 1) + 7919 * i + 104729 * rank)
@@ -381,57 +452,39 @@ def main():
         torch.cuda.synchronize()
     step_no = [0]
 
-    def next_inputs(Q, K, V):
-        if not w.warm_steps:
+    def next_inputs():
+        if inputs is None:
             return Q, K, V
         t = step_no[0]
         step_no[0] += 1
         return inputs[t]
 
-    def step(Q, K, V, events=None):
-        def mark(i):
-            if events is not None:
-                events[i].record(stream)
-        mark(0)
-        cq = csa.svgear_cluster(Q, w.Cq, iters, warm_centroids=warm["q"], seed=2 * rank)
-        mark(1)
-        ck = csa.svgear_cluster(K, w.Ck, iters, warm_centroids=warm["k"], seed=2 * rank + 1)
-        mark(2)
-        if w.warm_steps:
-            warm["q"], warm["k"] = cq.centroids, ck.centroids
-        Vp = csa.svgear_permute(V, ck.perm)
-        vbar = csa.svgear_centroids(Vp, ck.offsets, w.Ck)
-        mark(3)
-        if args.topp:
-            po, pk, _ = csa.svgear_route_topp(cq.centroids, cq.offsets, ck.centroids, vbar,
-                                              ck.offsets, ck.Xp, Vp, args.topp, w.scale)
-        else:
-            po, pk = csa.svgear_route(cq.centroids, cq.offsets, ck.centroids, vbar, ck.offsets,
-                                      ck.Xp, Vp, density, w.scale)
-        mark(4)
-        kvar = csa.svgear_key_variance(ck.Xp, ck.offsets, w.Ck) if args.var_lambda else None
-        O = csa.svgear_attend(cq.Xp, ck.Xp, Vp, cq.offsets, ck.offsets, po, pk, ck.centroids,
-                              vbar, cq.perm, w.scale, kvar=kvar, lam=args.var_lambda)
-        mark(5)
-        return O, (cq, ck, po, pk, Vp)
+    O = torch.empty_like(Q)
+
+    def step(Qs, Ks, Vs, events=None):
+        csa.svgear_layer(Qs, Ks, Vs, w.Cq, w.Ck, iters, density, O=O, warm_q=warm["q"],
+                         warm_k=warm["k"], cent_q=warm["q"], cent_k=warm["k"], stage_events=events,
+                         **common)
 
     # the clock sampler starts (and finishes initialising) before the warm-up
     clocks = ClockSampler(local if ws > 1 else torch.cuda.current_device())
     clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for e in (x for row in evs for x in row):
+        e.record(stream)          # each CUDA event exists from its first record
     for _ in range(max(3, args.warmup)):
-        step(*next_inputs(Q, K, V))
+        step(*next_inputs())
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_inputs = [next_inputs(Q, K, V) for _ in range(args.steps)]
+    step_inputs = [next_inputs() for _ in range(args.steps)]
     barrier(ws)
     torch.cuda.synchronize()
     l0 = csa.kernel_launches()
     t_begin = time.time()
     start.record(stream)
     for s in range(args.steps):
-        O, state = step(*step_inputs[s], evs[s])
+        step(*step_inputs[s], evs[s])
     end.record(stream)
     torch.cuda.synchronize()
     t_end = time.time()
@@ -444,9 +497,17 @@ def main():
     stage_ms = {n: float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)]))
                 for i, n in enumerate(ev_names)}
 
-    # algorithmic work of the attention pass (from the last step's routing)
-    cq, ck, po, pk, Vp_last = state
-    BH = w.B * w.H
+    # Work and quality (untimed): the same call run stage by stage on the last
+    # step's inputs returns its intermediates (the kernels are deterministic,
+    # so a cold call repeats the timed one exactly; a warm call is one more
+    # step from the cache).
+    Qs, Ks, Vs = step_inputs[-1]
+    ref = csa.layer(Qs, Ks, Vs, w.Cq, w.Ck, iters, density, w.scale, seed=rank,
+                    warm_q=None if warm["q"] is None else warm["q"].clone(),
+                    warm_k=None if warm["k"] is None else warm["k"].clone(), topp=args.topp,
+                    var_lambda=args.var_lambda)
+    cq, ck, po, pk, Vp_last = ref["q"], ref["k"], ref["pair_off"], ref["pair_kc"], ref["Vp"]
+    BH = w.B * Hl
     q_off = cq.offsets.view(BH, -1).cpu().numpy()
     k_off = ck.offsets.view(BH, -1).cpu().numpy()
     pair_off = po.view(BH, -1).cpu().numpy()
@@ -458,12 +519,14 @@ def main():
     achieved = (f_sel + f_comp) / (attend_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     if w.dtype == "bf16":
+        import dataclasses
+        traffic = attend_traffic(dataclasses.replace(w, H=Hl))
         roofline = {"kernel": "attend_sm100_kernel (svgear_attend, bf16)", "bound": "tensor",
                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak,
                     "peak_kind": "bf16 dense, sustained, %s" % (
                         "of measured" if peaks["source"] == "measured" else "of fallback"),
-                    "traffic": attend_traffic(w), "flops_per_launch": f_sel + f_comp}
+                    "traffic": traffic, "flops_per_launch": f_sel + f_comp}
     else:
         # fp32 SIMT attention: FMA units, 148 SMs x 128 lanes x 2 flops x 1.965 GHz
         alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -473,32 +536,31 @@ def main():
                     "peak_kind": "fp32 FMA, from unit counts and the 1965 MHz clock",
                     "traffic": None, "flops_per_launch": f_sel + f_comp}
 
-    # quality of the timed configuration (not timed): attention recall and the
-    # output error against dense attention on 64 sampled query rows per head
+    # quality of the timed configuration: attention recall and the output
+    # error against dense attention on 64 sampled query rows per head
     g = np.random.default_rng(1234)
     R = min(64, w.N)
     rows = np.stack([np.sort(g.choice(w.N, R, replace=False)) for _ in range(BH)])
     rec, e2, r2 = csa.svgear_diagnostics(
-        cq.Xp, ck.Xp, Vp_last, cq.offsets, ck.offsets, po, pk, O, cq.perm, w.scale,
-        torch.from_numpy(rows.astype(np.int32)).view(w.B, w.H, R).to(dev))
+        cq.Xp, ck.Xp, Vp_last, cq.offsets, ck.offsets, po, pk, ref["O"], cq.perm, w.scale,
+        torch.from_numpy(rows.astype(np.int32)).view(w.B, Hl, R).to(dev))
     rec, e2, r2 = (t.double().cpu().numpy() for t in (rec, e2, r2))
     quality = {"rows_per_head": R, "recall_mean": float(rec.mean()),
                "recall_min": float(rec.min()),
                "relative_mse": float(e2.sum() / max(r2.sum(), 1e-300))}
+    del ref, cq, ck, po, pk, Vp_last
 
-    # end to end through the public host-buffer call: every step copies its
-    # pinned host inputs to the device (overlapped with the stages that do not
-    # read them yet) and reads O back into pinned host memory
+    # end to end through the C ABI's host-buffer call: every step copies this
+    # rank's pinned host inputs to the device inside the call (overlapped with
+    # the stages that do not read them yet) and O back into pinned host memory
     e2e = None
     if not args.no_e2e:
-        Od_host = torch.empty((w.B, w.H, w.N, w.d), dtype=Q.dtype).pin_memory()
+        Od_host = torch.empty(tuple(host["q"].shape), dtype=Q.dtype).pin_memory()
 
         def e2e_step():
-            res = csa.layer_host(host["q"], host["k"], host["v"], w.Cq, w.Ck, iters, density,
-                                 scale=w.scale, seed=rank, warm_q=warm["q"], warm_k=warm["k"],
-                                 topp=args.topp, var_lambda=args.var_lambda, out=Od_host)
-            if w.warm_steps:
-                warm["q"], warm["k"] = res["q"].centroids, res["k"].centroids
+            csa.layer_host(host["q"], host["k"], host["v"], w.Cq, w.Ck, iters, density,
+                           out=Od_host, warm_q=warm["q"], warm_k=warm["k"], cent_q=warm["q"],
+                           cent_k=warm["k"], **common)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -511,26 +573,33 @@ def main():
         torch.cuda.synchronize()
         barrier(ws)
         e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, ws)
-        nbytes = w.B * w.H * w.N * w.d * 2
-        e2e = {"value": ranks_mod.job_ms_per_call(e2e_ms, ws), "unit": "ms",
-               "h2d_bytes_per_step": 3 * nbytes,
-               "d2h_bytes_per_step": nbytes}
+        nbytes = int(host["q"].numel()) * host["q"].element_size()
+        e2e = {"value": ranks_mod.job_ms_per_call(e2e_ms, ws, split), "unit": "ms",
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "call": "svgear_layer_host (C ABI, host buffers)"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        v, cores, desc, parts = oracle_sample_ms(w, seconds=args.cpu_sample_seconds,
-                                                 density=density, iters=iters, topp=args.topp)
-        cpu = {"value": v, "unit": "ms", "cores": cores, "kind": "oracle", "sample": desc,
-               "stages_ms": parts}
+        import oracle
+        sample = OracleSample(w, density=density, iters=iters, topp=args.topp,
+                              var_lambda=args.var_lambda)
+        sample.run()              # warm-up: caches, page faults, CPU clocks
+        runs = [sample.run() for _ in range(max(1, args.cpu_samples))]
+        runs.sort(key=lambda r: r[0])
+        v, parts = runs[len(runs) // 2]
+        cpu = {"value": v, "unit": "ms", "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": sample.describe(), "stages_ms": parts,
+               "spread": [runs[0][0], runs[-1][0]]}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": ranks_mod.job_ms_per_call(ms_step_max, ws), "unit": "ms",
-            "n_gpus": ws,
+            "metric": METRIC, "value": ranks_mod.job_ms_per_call(ms_step_max, ws, split),
+            "unit": "ms", "n_gpus": ws,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step_max,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": False, "scaling": "strong" if split == "heads" else "weak",
+            "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic: seeded patch-coherent Gaussian mixtures at the %s shape" % w.name,
-            "config": {**workload_config(w, args), "density_selected": density_real},
+            "config": {**workload_config(w, args, ws), "density_selected": density_real},
             "effective_tflops": (f_sel + f_comp) / (ms_step * 1e-3) / 1e12,
             "attention_tflops": achieved,
             "stages_ms": stage_ms,

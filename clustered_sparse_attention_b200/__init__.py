@@ -10,11 +10,11 @@ from ._lib import (Clustering, SvgearError, kernel_launches, layer, layer_host, 
                    svgear_kmeanspp_init, svgear_label_sort, svgear_permute, svgear_probe,
                    svgear_route, svgear_route_select, svgear_route_select_budget,
                    svgear_route_topp, svgear_topp_budget, svgear_key_variance,
-                   svgear_probe_value_free, svgear_diagnostics, workspace_bytes)
+                   svgear_probe_value_free, svgear_diagnostics, svgear_layer, workspace_bytes)
 
 __all__ = ["Clustering", "SvgearError", "kernel_launches", "layer", "layer_host", "lib", "svgear_attend", "svgear_centroids",
            "svgear_cluster", "svgear_kmeans_assign", "svgear_kmeans_update",
            "svgear_kmeanspp_init", "svgear_label_sort", "svgear_permute", "svgear_probe",
            "svgear_route", "svgear_route_select", "svgear_route_select_budget",
            "svgear_route_topp", "svgear_topp_budget", "svgear_key_variance",
-           "svgear_probe_value_free", "svgear_diagnostics", "workspace_bytes"]
+           "svgear_probe_value_free", "svgear_diagnostics", "svgear_layer", "workspace_bytes"]

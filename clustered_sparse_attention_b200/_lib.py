@@ -34,12 +34,19 @@ EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
             "svgear_device_status", "svgear_topp_budget", "svgear_route_select_budget",
             "svgear_route_topp", "svgear_key_variance", "svgear_attend_var",
             "svgear_probe_value_free", "svgear_diagnostics",
-            "svgear_label_sort_noalloc", "svgear_selftest_wait")
+            "svgear_label_sort_noalloc", "svgear_selftest_wait", "svgear_layer",
+            "svgear_layer_host", "svgear_layer_workspace_bytes")
 
 
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [("Cq", ctypes.c_int32), ("Ck", ctypes.c_int32), ("iters", ctypes.c_int32),
+                ("density", ctypes.c_float), ("topp", ctypes.c_float), ("scale", ctypes.c_float),
+                ("var_lambda", ctypes.c_float), ("seed", ctypes.c_uint64)]
 
 
 class SvgearError(RuntimeError):
@@ -91,12 +98,17 @@ def lib():
         "svgear_device_status": [P, SZ, P, P],
         "svgear_label_sort_noalloc": [P, Dims, I32, P, P, P],
         "svgear_selftest_wait": [P, SZ, I32, I32, I32, P],
+        "svgear_layer": [P, P, P, Dims, ctypes.POINTER(LayerParams), P, P, P, P, P, P, SZ, P, P],
+        "svgear_layer_host": [P, P, P, Dims, ctypes.POINTER(LayerParams), P, P, P, P, P, P, SZ,
+                              P],
+        "svgear_layer_workspace_bytes": [Dims, ctypes.POINTER(LayerParams), I32],
     }
     for name, args in sig.items():
         f = getattr(L, name)
         f.argtypes = args
         f.restype = ctypes.c_int
     L.svgear_workspace_bytes.restype = SZ
+    L.svgear_layer_workspace_bytes.restype = SZ
     L.svgear_status_string.restype = ctypes.c_char_p
     L.svgear_kernel_launches.restype = ctypes.c_uint64
     _L = L
@@ -483,40 +495,69 @@ def layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm
             "pair_kc": pair_kc, "budget": budget, "kvar": kvar}
 
 
-_copy_streams = {}
+def layer_params(Cq, Ck, iters, density, scale, seed=0, topp=None, var_lambda=0.0):
+    return LayerParams(int(Cq), int(Ck), int(iters), float(density if density else 0.0),
+                       float(topp or 0.0), float(scale), float(var_lambda), int(seed))
+
+
+def svgear_layer(Q, K, V, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None, warm_k=None,
+                 topp=None, var_lambda=0.0, O=None, cent_q=None, cent_k=None, stage_events=None):
+    """The whole layer in one C call on device tensors (svgear_layer).
+    Returns (O, cent_q, cent_k); cent_* are the final centroids (allocated
+    unless given; they may be the warm_* tensors, updated in place).
+    stage_events: None or 6 torch.cuda.Event already recorded once (so that
+    they exist), recorded again at the stage boundaries."""
+    dims = _tokens(Q, "Q")
+    _tokens(K, "K")
+    _tokens(V, "V")
+    B, H, N, d = Q.shape
+    scale = d ** -0.5 if scale is None else scale
+    prm = layer_params(Cq, Ck, iters, density, scale, seed, topp, var_lambda)
+    dev = Q.device
+    O = torch.empty_like(Q) if O is None else O
+    if cent_q is None:
+        cent_q = torch.empty((B, H, Cq, d), dtype=torch.float32, device=dev)
+    if cent_k is None:
+        cent_k = torch.empty((B, H, Ck, d), dtype=torch.float32, device=dev)
+    for t, nm in ((warm_q, "warm_q"), (warm_k, "warm_k"), (cent_q, "cent_q"), (cent_k, "cent_k")):
+        if t is not None:
+            _cuda(t, nm, torch.float32)
+    n = max(int(lib().svgear_layer_workspace_bytes(dims, ctypes.byref(prm), 0)), 256)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
+    _check("svgear_layer", lib().svgear_layer(
+        _ptr(Q), _ptr(K), _ptr(V), dims, ctypes.byref(prm), _ptr(warm_q), _ptr(warm_k), _ptr(O),
+        _ptr(cent_q), _ptr(cent_k), _ptr(ws), n, ev, _stream()))
+    return O, cent_q, cent_k
 
 
 def layer_host(Qh, Kh, Vh, Cq, Ck, iters, density, scale=None, seed=0, warm_q=None,
-               warm_k=None, topp=None, var_lambda=0.0, out=None):
-    """The layer for host tensors (pinned for the copies to overlap): Q, K and
-    V go to the device on a side stream, and each stage of the layer waits
-    only for the input it reads, so clustering Q runs while K and V are still
-    on their way.  O comes back into out (a pinned host tensor like Qh, made if
-    None), ordered after the layer on the current stream.  Returns the layer's
-    dict with "O_host" added; the host tensor is complete once the current
-    stream has passed this call."""
+               warm_k=None, topp=None, var_lambda=0.0, out=None, cent_q=None, cent_k=None):
+    """The layer for host tensors in one C call (svgear_layer_host): the call
+    copies Q, K and V to the device (pinned host tensors let the copies
+    overlap the first stages), runs the layer and copies O back into `out`
+    (a pinned host tensor like Qh, made if None), all on the current stream.
+    Returns {"O_host", "cent_q", "cent_k"}; the host tensor is complete once
+    the current stream has passed this call."""
+    for t, nm in ((Qh, "Q"), (Kh, "K"), (Vh, "V")):
+        if t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous host tensor [B, H, N, d]" % nm)
+    B, H, N, d = Qh.shape
+    dims = Dims(B, H, N, d, _dtype_code(Qh))
+    scale = d ** -0.5 if scale is None else scale
+    prm = layer_params(Cq, Ck, iters, density, scale, seed, topp, var_lambda)
     dev = torch.device("cuda", torch.cuda.current_device())
-    cs = torch.cuda.current_stream(dev)
-    xs = _copy_streams.get(dev.index)
-    if xs is None:
-        xs = _copy_streams[dev.index] = torch.cuda.Stream(dev)
-    ready = {}
-    with torch.cuda.stream(xs):
-        # the device copies belong to the copy stream; record_stream keeps them
-        # from reuse until the layer's stream is done with them
-        Qd, Kd, Vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (Qh, Kh, Vh))
-        for name, d, h in (("q", Qd, Qh), ("k", Kd, Kh), ("v", Vd, Vh)):
-            d.copy_(h, non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(xs)
-            ready[name] = ev
-    for d in (Qd, Kd, Vd):
-        d.record_stream(cs)
-    res = layer(Qd, Kd, Vd, Cq, Ck, iters, density, scale=scale, seed=seed, warm_q=warm_q,
-                warm_k=warm_k, topp=topp, var_lambda=var_lambda, ready=ready)
     if out is None:
-        out = torch.empty(res["O"].shape, dtype=res["O"].dtype, pin_memory=True)
-    out.copy_(res["O"], non_blocking=True)
-    res["O_host"] = out
-    return res
-
+        out = torch.empty(Qh.shape, dtype=Qh.dtype, pin_memory=True)
+    if cent_q is None:
+        cent_q = torch.empty((B, H, Cq, d), dtype=torch.float32, device=dev)
+    if cent_k is None:
+        cent_k = torch.empty((B, H, Ck, d), dtype=torch.float32, device=dev)
+    n = max(int(lib().svgear_layer_workspace_bytes(dims, ctypes.byref(prm), 1)), 256)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    _check("svgear_layer_host", lib().svgear_layer_host(
+        _ptr(Qh), _ptr(Kh), _ptr(Vh), dims, ctypes.byref(prm), _ptr(warm_q), _ptr(warm_k),
+        _ptr(out), _ptr(cent_q), _ptr(cent_k), _ptr(ws), n, _stream()))
+    return {"O_host": out, "cent_q": cent_q, "cent_k": cent_k}

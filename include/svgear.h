@@ -461,6 +461,66 @@ int svgear_selftest_wait(void* ws, size_t ws_bytes, int32_t arrive, int32_t time
 int svgear_label_sort_noalloc(const int32_t* labels, svgear_dims dims, int32_t C,
                               int32_t* perm, int32_t* offsets, void* stream);
 
+/* --------------------------------------------------------------------------
+ * svgear_layer -- one whole layer call ([TASK] the layer and its three
+ * routines, agent steps 1-3; [SVG2] section 3.4): svgear_cluster on Q (seed
+ * 2*seed) and on K (seed 2*seed+1), svgear_permute of V by the key
+ * permutation and svgear_centroids of the result, the probe and greedy
+ * routing (svgear_route, or svgear_route_topp when topp > 0), the key
+ * variance when var_lambda != 0, and svgear_attend(_var), which writes O in
+ * the original token order.  Each stage's result is the one its own entry
+ * point gives; every intermediate lives in the workspace.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t Cq, Ck;     /* query / key clusters per head */
+    int32_t iters;      /* Lloyd rounds of each clustering, >= 1 */
+    float density;      /* floor(density * N) keys per query cluster, in (0, 1]
+                           (unused when topp > 0) */
+    float topp;         /* 0: fixed density; in (0, 1]: the budget of the key
+                           clusters holding topp of the estimated weight */
+    float scale;        /* softmax scale, finite (1/sqrt(d) for the method) */
+    float var_lambda;   /* variance-corrected compensation strength; 0: plain */
+    uint64_t seed;      /* k-means++ draws of a cold call */
+} svgear_layer_params;
+
+/* Workspace bytes of svgear_layer (host_buffers = 0) or svgear_layer_host
+ * (host_buffers = 1); 0 for arguments the call would reject. */
+size_t svgear_layer_workspace_bytes(svgear_dims dims, const svgear_layer_params* params,
+                                    int32_t host_buffers);
+
+/* The layer on device buffers.
+ *   Q, K, V         [B][H][N][d] (dims.dtype), the same shape (self-attention).
+ *   warm_q, warm_k  float [B][H][Cq][d] / [B][H][Ck][d] cached centroids of
+ *                   the previous step, or NULL for a cold start (k-means++).
+ *   O               out [B][H][N][d] (dims.dtype), original token order.
+ *   cent_q, cent_k  out final centroids (the cache of the next step), or NULL;
+ *                   each may alias its warm_ buffer.
+ *   ws, ws_bytes    svgear_layer_workspace_bytes(dims, params, 0).
+ *   stage_events    NULL, or 6 cudaEvent_t (NULL entries skipped) recorded on
+ *                   `stream` before clustering Q, after clustering Q, after
+ *                   clustering K, after the value centroids, after routing
+ *                   and after attention: per-stage timing.
+ * Status, validation and asynchrony as for the stage entry points; a stage's
+ * error status ends the call with that status. */
+int svgear_layer(const void* Q, const void* K, const void* V, svgear_dims dims,
+                 const svgear_layer_params* params, const float* warm_q, const float* warm_k,
+                 void* O, float* cent_q, float* cent_k, void* ws, size_t ws_bytes,
+                 void* const* stage_events, void* stream);
+
+/* The layer on HOST buffers: Q_host, K_host, V_host and O_host are host
+ * memory of the shapes above (page-locked, for the copies to run
+ * asynchronously and overlap the stages).  The call copies Q, K and V to the
+ * workspace on a stream of its own, which first waits for all work already
+ * on `stream`; each stage waits only for the input it reads, so clustering Q
+ * runs while K and V are still arriving.  O is copied back into O_host on
+ * `stream` after attention: O_host is complete once `stream` has passed this
+ * call.  warm_q, warm_k, cent_q, cent_k are device pointers as for
+ * svgear_layer; ws is svgear_layer_workspace_bytes(dims, params, 1). */
+int svgear_layer_host(const void* Q_host, const void* K_host, const void* V_host,
+                      svgear_dims dims, const svgear_layer_params* params, const float* warm_q,
+                      const float* warm_k, void* O_host, float* cent_q, float* cent_k, void* ws,
+                      size_t ws_bytes, void* stream);
+
 /* Workspace bytes for `op` at shape `dims` (N = tokens of the clustered
  * tensor; for SVGEAR_OP_ROUTE and SVGEAR_OP_ATTEND, dims.N = Nq and C2 = Ck),
  * with C1 = C (or Cq).  Returns 0 for arguments the op would reject. */

@@ -122,3 +122,30 @@ def test_selftest_wait_validates_before_launch(L):
     assert L.svgear_selftest_wait(fake, ok, 0, 1000, 3, None) == _lib.ERR_INVALID_ARG
     assert L.svgear_device_status(None, ok, fake, None) == _lib.ERR_INVALID_ARG
     assert b"tensor memory" in L.svgear_status_string(_lib.ERR_TMEM_LOST)
+
+
+def test_layer_entry_points_validate_before_launch(L):
+    from clustered_sparse_attention_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)
+    big = ctypes.c_size_t(1 << 40)
+    good = _lib.layer_params(100, 500, 40, 0.25, 128 ** -0.5)
+    d = _dims(H=40, N=75600)
+    n0 = L.svgear_layer_workspace_bytes(d, ctypes.byref(good), 0)
+    n1 = L.svgear_layer_workspace_bytes(d, ctypes.byref(good), 1)
+    assert n1 - n0 >= 3 * 40 * 75600 * 128 * 2            # the three device input copies
+    for bad in (_lib.layer_params(0, 500, 40, 0.25, 0.1), _lib.layer_params(100, 500, 0, 0.25, 0.1),
+                _lib.layer_params(100, 500, 40, 0.0, 0.1), _lib.layer_params(100, 500, 40, 0.3, 0.1,
+                                                                             topp=1.5),
+                _lib.layer_params(100, 500, 40, 0.3, float("nan")),
+                _lib.layer_params(100, 80000, 40, 0.3, 0.1)):
+        assert L.svgear_layer_workspace_bytes(d, ctypes.byref(bad), 0) == 0
+        assert L.svgear_layer(fake, fake, fake, d, ctypes.byref(bad), None, None, fake, None, None,
+                              fake, big, None, None) != _lib.OK
+    # null output, small workspace
+    assert L.svgear_layer(fake, fake, fake, d, ctypes.byref(good), None, None, None, None, None,
+                          fake, big, None, None) == _lib.ERR_INVALID_ARG
+    assert L.svgear_layer_host(fake, fake, fake, d, ctypes.byref(good), None, None, fake, None,
+                               None, fake, ctypes.c_size_t(n0), None) == _lib.ERR_WORKSPACE
+    # top-p replaces the density: density 0 is then allowed
+    tp = _lib.layer_params(100, 500, 40, 0.0, 0.1, topp=0.9)
+    assert L.svgear_layer_workspace_bytes(d, ctypes.byref(tp), 0) > 0
