@@ -1,6 +1,8 @@
-"""The multi-rank host path (one process per GPU, weak scaling) on the CPU:
-two gloo ranks join, each draws its own batch element, and the job's time is
-the slowest rank's; no data-path collective exists."""
+"""The multi-rank host path (one process per GPU) on the CPU with gloo ranks:
+the head split of one layer call (each rank owns a contiguous head range,
+every head exactly once; O reassembles at the right offsets), the batch split
+(each rank draws its own batch element), and the job's time as the slowest
+rank's.  No data-path collective exists inside the layer."""
 import os
 import socket
 
@@ -28,7 +30,7 @@ def _worker(rank, ws, port, out):
     step_ms = 10.0 + 5.0 * rank                       # rank 1 is the slower one
     ranks.barrier(got_ws)
     worst = ranks.max_over_ranks(step_ms, got_ws)
-    out[rank] = (got_ws, got_rank, worst, ranks.job_ms_per_call(worst, got_ws),
+    out[rank] = (got_ws, got_rank, worst, ranks.job_ms_per_call(worst, got_ws, split="batch"),
                  int(bits.astype(np.int64).sum()))
     ranks.teardown(got_ws)
 
@@ -64,7 +66,66 @@ def test_single_process_needs_no_process_group():
         assert ranks.setup() == (1, 0, 0)
         assert ranks.max_over_ranks(3.5, 1) == 3.5
         assert ranks.job_ms_per_call(8.0, 1) == 8.0
+        assert ranks.head_range(40, 1, 0) == (0, 40)
         ranks.barrier(1)
         ranks.teardown(1)
     finally:
         os.environ.update(env)
+
+
+def test_head_ranges_cover_every_head_exactly_once():
+    for H in (1, 5, 24, 40, 41):
+        for ws in (1, 2, 3, 4, 7, 8, 16, 48):
+            seen = []
+            prev_hi = 0
+            for r in range(ws):
+                lo, hi = ranks.head_range(H, ws, r)
+                assert lo == prev_hi and lo <= hi           # contiguous, in rank order
+                prev_hi = hi
+                seen.extend(range(lo, hi))
+            assert seen == list(range(H))
+            sizes = [ranks.head_range(H, ws, r)[1] - ranks.head_range(H, ws, r)[0]
+                     for r in range(ws)]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        ranks.head_range(8, 2, 2)
+
+
+def _o_value(B, heads, N, d):
+    """A host 'output' whose every element names its batch, head, row and
+    column, so a misplaced slice cannot go unnoticed."""
+    import torch
+    b = torch.arange(B, dtype=torch.float64).view(B, 1, 1, 1)
+    h = torch.tensor(list(heads), dtype=torch.float64).view(1, -1, 1, 1)
+    n = torch.arange(N, dtype=torch.float64).view(1, 1, N, 1)
+    k = torch.arange(d, dtype=torch.float64).view(1, 1, 1, d)
+    return (b * 1e7 + h * 1e5 + n * 1e2 + k).expand(B, len(list(heads)), N, d).contiguous()
+
+
+def _head_worker(rank, ws, port, H, out):
+    os.environ.update({"WORLD_SIZE": str(ws), "RANK": str(rank), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    got_ws, got_rank, _ = ranks.setup("gloo", timeout_s=60)
+    lo, hi = ranks.head_range(H, got_ws, got_rank)
+    B, N, d = 2, 6, 4
+    full = ranks.gather_heads(_o_value(B, range(lo, hi), N, d), H, got_ws, got_rank)
+    out[rank] = (lo, hi, bool((full == _o_value(B, range(H), N, d)).all()))
+    ranks.teardown(got_ws)
+
+
+@pytest.mark.parametrize("ws,H", [(2, 5), (3, 40)])
+def test_head_split_reassembles_o_at_the_right_offsets(ws, H):
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_head_worker, args=(r, ws, port, H, out)) for r in range(ws)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        res = dict(out)
+    covered = sorted(h for r in range(ws) for h in range(res[r][0], res[r][1]))
+    assert covered == list(range(H))
+    assert all(res[r][2] for r in range(ws))
