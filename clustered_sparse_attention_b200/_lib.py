@@ -24,6 +24,7 @@ F32, BF16 = 0, 1
 OP_CLUSTER, OP_KMEANSPP, OP_LABEL_SORT, OP_KMEANS_UPDATE, OP_ROUTE, OP_ATTEND = range(6)
 OP_KMEANS_ASSIGN = 6
 OP_ROUTE_TOPP = 7
+OP_CENTROIDS = 8
 MAX_CLUSTERS = 4096
 
 EXPORTED = ("svgear_cluster", "svgear_kmeanspp_init", "svgear_kmeans_assign",
@@ -76,7 +77,7 @@ def lib():
         "svgear_label_sort": [P, Dims, I32, P, P, P, SZ, P],
         "svgear_kmeans_update": [P, Dims, P, I32, P, P, SZ, P],
         "svgear_permute": [P, P, Dims, P, P],
-        "svgear_centroids": [P, P, I32, Dims, P, P],
+        "svgear_centroids": [P, P, I32, Dims, P, P, SZ, P],
         "svgear_probe": [P, I32, P, P, P, P, P, I32, Dims, F, P, P, SZ, P],
         "svgear_route_select": [P, P, I32, P, I32, I32, I32, I32, F, P, P, P, SZ, P],
         "svgear_route": [P, P, I32, P, P, P, I32, P, P, Dims, F, F, P, P, P, P, SZ, P],
@@ -292,8 +293,9 @@ def svgear_centroids(Xp, offsets, C=None):
     C = offsets.shape[-1] - 1 if C is None else C
     B, H, N, d = Xp.shape
     out = torch.empty((B, H, C, d), dtype=torch.float32, device=Xp.device)
+    ws, n = _workspace(OP_CENTROIDS, dims, C, 0, Xp.device)
     _check("svgear_centroids", lib().svgear_centroids(
-        _ptr(Xp), _ptr(offsets), C, dims, _ptr(out), _stream()))
+        _ptr(Xp), _ptr(offsets), C, dims, _ptr(out), _ptr(ws), n, _stream()))
     return out
 
 

@@ -62,16 +62,21 @@ int32_t* carve_sort(Carve& cv, const svgear_dims& d, int C) {
 void* carve_assign(Carve& cv, const svgear_dims& d, int C) {
     return cv.take<char>(assign_scratch_bytes((int)bh_of(d), C, d.d, d.dtype));
 }
+void* carve_segmean(Carve& cv, const svgear_dims& d) {
+    return cv.take<char>(segmean_scratch_bytes((int)bh_of(d), d.N, d.d));
+}
 struct UpdWs {
     int32_t* perm;
     int32_t* offsets;
     int32_t* hist;
+    void* segmean;
 };
 UpdWs carve_update(Carve& cv, const svgear_dims& d, int C) {
     UpdWs w;
     w.perm = cv.take<int32_t>(bh_of(d) * d.N);
     w.offsets = cv.take<int32_t>(bh_of(d) * (C + 1));
     w.hist = carve_sort(cv, d, C);
+    w.segmean = carve_segmean(cv, d);
     return w;
 }
 struct SelWs {
@@ -139,6 +144,7 @@ size_t ws_cluster(const svgear_dims& d, int C) {
     carve_kpp(a, d, C);
     carve_sort(b, d, C);
     carve_assign(b, d, C);
+    carve_segmean(b, d);
     return (a.off > b.off ? a.off : b.off) + kAlign;
 }
 
@@ -192,6 +198,10 @@ size_t svgear_workspace_bytes(int32_t op, svgear_dims dims, int32_t C1, int32_t 
             cv.take<int>(4);
             carve_assign(cv, dims, C1);
             break;
+        case SVGEAR_OP_CENTROIDS:
+            if (check_C(C1, dims.N)) return 0;
+            carve_segmean(cv, dims);
+            break;
         case SVGEAR_OP_ROUTE:
             if (C1 < 1 || C2 < 1 || C1 > SVGEAR_MAX_CLUSTERS || C2 > SVGEAR_MAX_CLUSTERS) return 0;
             carve_route(cv, bh_of(dims), C1, C2, dims.d);
@@ -225,7 +235,8 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
     int* status = cv.take<int>(4);
     if (cudaMemsetAsync(status, 0, 4 * sizeof(int), st) != cudaSuccess) return SVGEAR_ERR_CUDA;
     KppWs w = carve_kpp(cv, dims, C);
-    return launch_kmeanspp(X, dims, C, seed, centroids, seed_index ? seed_index : w.chosen, w.D2,
+    return launch_kmeanspp(X, dims, C, seed, 0, centroids,
+                           seed_index ? seed_index : w.chosen, w.D2,
                            w.nearest, w.cc2, w.blocksum, w.counter, w.gen, status, st);
 }
 
@@ -278,13 +289,27 @@ int svgear_kmeans_update(const void* X, svgear_dims dims, const int32_t* labels,
     UpdWs w = carve_update(cv, dims, C);
     if ((s = launch_label_sort(labels, (int)bh_of(dims), dims.N, C, w.perm, w.offsets, w.hist, st)))
         return s;
-    return launch_segment_mean(X, w.perm, w.offsets, C, dims, centroids, false, st);
+    return launch_segment_mean(X, w.perm, w.offsets, C, dims, centroids, false, w.segmean, st);
 }
 
 int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
                    const float* warm_centroids, uint64_t seed, int32_t* labels, int32_t* perm,
                    int32_t* offsets, float* centroids, void* Xp, void* ws, size_t ws_bytes,
                    void* stream) {
+    return svgear::cluster_heads(X, dims, C, iters, warm_centroids, seed, 0, labels, perm,
+                                 offsets, centroids, Xp, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+// svgear_cluster on a range of heads of a larger call: head bh of these dims
+// draws its k-means++ numbers from Philox stream sbase + bh, so clustering
+// the heads [h0, h1) with sbase = h0 repeats what a call on all heads gives
+// them (every head's k-means is independent of the others').
+int svgear::cluster_heads(const void* X, svgear_dims dims, int32_t C, int32_t iters,
+                          const float* warm_centroids, uint64_t seed, uint64_t sbase,
+                          int32_t* labels, int32_t* perm, int32_t* offsets, float* centroids,
+                          void* Xp, void* ws, size_t ws_bytes, void* stream) {
     int s = check_dims(dims);
     if (s) return s;
     if ((s = check_C(C, dims.N))) return s;
@@ -310,7 +335,9 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
         Carve cv(ws);
         carve_flags(cv, dims);
         KppWs w = carve_kpp(cv, dims, C);
-        if ((s = launch_kmeanspp(X, dims, C, seed, centroids, w.chosen, w.D2, w.nearest, w.cc2,
+        if ((s = launch_kmeanspp(X, dims, C, seed, sbase, centroids, w.chosen, w.D2,
+                                 w.nearest,
+                                 w.cc2,
                                  w.blocksum, w.counter, w.gen, fl.status, st)))
             return s;
     }
@@ -318,6 +345,7 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
     carve_flags(cv, dims);
     int32_t* hist = carve_sort(cv, dims, C);
     void* ascratch = carve_assign(cv, dims, C);
+    void* mscratch = carve_segmean(cv, dims);
     // Lloyd rounds.  From the second round on, a head whose assignment moved
     // no label has reached the fixed point (the sort and the deterministic
     // update would reproduce the current perm, offsets and centroids), so its
@@ -330,12 +358,15 @@ int svgear_cluster(const void* X, svgear_dims dims, int32_t C, int32_t iters,
         if (track && (s = launch_fixed_point(fl.changed, fl.done, BH, st))) return s;
         if ((s = launch_label_sort(labels, BH, dims.N, C, perm, offsets, hist, st, fl.done)))
             return s;
-        if ((s = launch_segment_mean(X, perm, offsets, C, dims, centroids, false, st, fl.done)))
+        if ((s = launch_segment_mean(X, perm, offsets, C, dims, centroids, false, mscratch, st,
+                                     fl.done)))
             return s;
     }
     if (Xp) return launch_permute(X, perm, dims, Xp, st);
     return SVGEAR_OK;
 }
+
+extern "C" {
 
 int svgear_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp, void* stream) {
     int s = check_dims(dims);
@@ -346,14 +377,17 @@ int svgear_permute(const void* X, const int32_t* perm, svgear_dims dims, void* X
 }
 
 int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C, svgear_dims dims,
-                     float* centroids, void* stream) {
+                     float* centroids, void* ws, size_t ws_bytes, void* stream) {
     int s = check_dims(dims);
     if (s) return s;
     if ((s = check_C(C, dims.N))) return s;
-    if (!Xp || !offsets || !centroids || !aligned16(Xp)) return SVGEAR_ERR_INVALID_ARG;
+    if (!Xp || !offsets || !centroids || !ws || !aligned16(Xp)) return SVGEAR_ERR_INVALID_ARG;
+    if (ws_bytes < svgear_workspace_bytes(SVGEAR_OP_CENTROIDS, dims, C, 0))
+        return SVGEAR_ERR_WORKSPACE;
     if (bh_of(dims) == 0) return SVGEAR_OK;
+    Carve cv(ws);
     return launch_segment_mean(Xp, nullptr, offsets, C, dims, centroids, true,
-                               static_cast<cudaStream_t>(stream));
+                               carve_segmean(cv, dims), static_cast<cudaStream_t>(stream));
 }
 
 static int check_route_common(int Cq, int Ck, int Nk, float density) {

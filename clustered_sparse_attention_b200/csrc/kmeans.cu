@@ -54,9 +54,9 @@ __device__ inline void kpp_block_scan(const float* d2s, double* warp_tot,
 
 template <typename T>
 __global__ void kpp_first_kernel(const T* __restrict__ X, int N, int D, int C,
-                                 uint64_t seed, int32_t* chosen, float* centroids) {
+                                 uint64_t seed, uint64_t sbase, int32_t* chosen, float* centroids) {
     const int bh = blockIdx.x;
-    double u = philox_uniform(seed, (uint64_t)bh, 0);
+    double u = philox_uniform(seed, sbase + (uint64_t)bh, 0);
     long long t = (long long)floor(u * (double)N);
     if (t >= N) t = N - 1;
     if (threadIdx.x == 0) chosen[(size_t)bh * C] = (int32_t)t;
@@ -73,6 +73,7 @@ __global__ void kpp_first_kernel(const T* __restrict__ X, int N, int D, int C,
 template <typename T, int D>
 __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32_t* chosen, int C,
                          int j, const float* D2, const double* blocksum, uint64_t seed,
+                         uint64_t sbase,
                          float* centroids, float* cc2, float* d2s, double* warp_tot, float* cnew) {
     __shared__ int s_blk, s_pick, s_last;
     __shared__ double s_base, s_target;
@@ -108,7 +109,7 @@ __device__ void kpp_pick(const T* __restrict__ X, int N, int nblk, int bh, int32
         int hit = -3;               // every D^2 is zero
         double base = 0.0, target = 0.0;
         if (total > 0.0) {
-            target = philox_uniform(seed, (uint64_t)bh, (uint64_t)j) * total;
+            target = philox_uniform(seed, sbase + (uint64_t)bh, (uint64_t)j) * total;
             const unsigned m = __ballot_sync(0xffffffffu, b1 > b0 && endv > target);
             hit = -2;               // rounding left no block above the target
             if (m) {
@@ -283,8 +284,9 @@ __device__ void kpp_block_update(const T* __restrict__ X, int N, int nblk, int b
         if (need) sm.todo[base + __popc(m & ((1u << wl) - 1u))] = r;
     }
     __syncthreads();
-    // recompute the survivors
+    const int32_t* list = sm.todo;
     const int n = sm.ntodo;
+    // recompute the survivors
     const int lane = tid % L, grp = tid / L;
     for (int b0 = 0; b0 < n; b0 += RP * U) {
         int rr[U];
@@ -292,7 +294,7 @@ __device__ void kpp_block_update(const T* __restrict__ X, int N, int nblk, int b
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = b0 + grp + u * RP;
-            rr[u] = i < n ? sm.todo[i] : -1;
+            rr[u] = i < n ? list[i] : -1;
             raw[u] = make_uint4(0u, 0u, 0u, 0u);
             if (rr[u] >= 0)
                 raw[u] = Elem<T>::load_raw(Xh + (size_t)(blk * kKppTokens + rr[u]) * D + lane * EPC);
@@ -354,7 +356,7 @@ __global__ void __launch_bounds__(kKppThreads, 6)
 kpp_pool_kernel(const T* __restrict__ X, int N, int nblk, int BH, int C, int32_t* chosen,
                 float* D2, int32_t* nearest, float* cc2, double* blocksum,
                 unsigned long long* claim, int32_t* arrive, int32_t* heads_done, uint64_t seed,
-                float* centroids, int* err) {
+                uint64_t sbase, float* centroids, int* err) {
     __shared__ KppSmem<D> sm;
     extern __shared__ float ccs[];             // |c_s - c_a|^2, a < s (dynamic: C floats)
     __shared__ int s_bh, s_pass, s_blk, s_last;
@@ -449,7 +451,7 @@ kpp_pool_kernel(const T* __restrict__ X, int N, int nblk, int BH, int C, int32_t
         __syncthreads();
         if (s_last) {
             __threadfence();
-            kpp_pick<T, D>(X, N, nblk, bh, chosen, C, pass, D2, blocksum, seed, centroids, cc2,
+            kpp_pick<T, D>(X, N, nblk, bh, chosen, C, pass, D2, blocksum, seed, sbase, centroids, cc2,
                            sm.d2s, sm.warp_tot, sm.cen);
             __syncthreads();
             if (tid == 0) {
@@ -475,7 +477,8 @@ __global__ void kpp_init_kernel(unsigned long long* claim, int32_t* arrive, int3
 }
 
 template <typename T, int D>
-static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, uint64_t sbase,
+                         float* cent,
                          int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
                          double* blocksum, int32_t* counter, int32_t* gen, int* err,
                          cudaStream_t st) {
@@ -488,7 +491,7 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
     int32_t* heads_done = gen + BH;
     kpp_init_kernel<<<ceil_div(BH, 128), 128, 0, st>>>(claim, arrive, heads_done, BH);
     count_launches(1);
-    kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, chosen, cent);
+    kpp_first_kernel<T><<<BH, 128, 0, st>>>(X, N, D, C, seed, sbase, chosen, cent);
     count_launches(1);
     SVGEAR_LAUNCH_CHECK();
     if (C < 2) return SVGEAR_OK;
@@ -505,10 +508,10 @@ static int kmeanspp_impl(const T* X, svgear_dims dims, int C, uint64_t seed, flo
     long long grid = (long long)per_sm * sms;
     if (grid > (long long)BH * nblk) grid = (long long)BH * nblk;
     int n_ = N, nblk_ = nblk, BH_ = BH, C_ = C;
-    uint64_t seed_ = seed;
+    uint64_t seed_ = seed, sbase_ = sbase;
     const T* X_ = X;
     void* args[] = {&X_, &n_, &nblk_, &BH_, &C_, &chosen, &D2, &nearest, &cc2, &blocksum,
-                    &claim, &arrive, &heads_done, &seed_, &cent, &err};
+                    &claim, &arrive, &heads_done, &seed_, &sbase_, &cent, &err};
     if (cudaLaunchCooperativeKernel((const void*)kpp_pool_kernel<T, D>, dim3((unsigned)grid),
                                     dim3(kKppThreads), args, ccs_bytes, st) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
@@ -703,71 +706,159 @@ size_t assign_scratch_bytes(int BH, int C, int D, int dtype) {
 }
 
 // ---------------------------------------------------------------------------
-// Segment mean: one block per (cluster, head); a group of lanes per row moves
-// 16-byte chunks; fp32 partial sums are combined in a fixed order.
+// Segment mean (the k-means update and the per-cluster value means).
+//
+// Work is split by position, not by segment, so every CTA moves the same
+// bytes whatever the cluster sizes: CTA (j, bh) takes the permuted positions
+// [jP, (j+1)P) of head bh.  The segments crossing that range are summed one
+// piece at a time (a piece = a segment's positions inside the chunk): lane
+// group g of the CTA adds the rows r0+g, r0+g+R, ... of the piece in order
+// (fp32), and the R group sums are added in group order.  A segment inside
+// one chunk is finished there; a longer one leaves its first piece as the
+// chunk's "trail" partial and the others as "lead" partials of the following
+// chunks, and segment_join_kernel adds trail(j0) + lead(j0+1) + ... +
+// lead(j1) in that order.  The summation order is a function of the
+// positions alone, so results are identical from run to run and for any
+// grid.  An empty segment writes zeros (empty_zero) or keeps its row.
+// Gather mode reads row perm[p] at position p; the chunk's perm entries are
+// staged in shared memory first, so no row load waits on an index load.
 // ---------------------------------------------------------------------------
 constexpr int kSmThreads = 256;
+constexpr int kSmChunk = 512;   // positions per CTA (128 KB of bf16 d = 128 rows)
+constexpr int kSmUnroll = 8;    // rows in flight per lane group
+
+size_t segmean_scratch_bytes(int BH, int N, int D) {
+    const size_t nch = (size_t)ceil_div(N, kSmChunk);
+    return (size_t)BH * nch * (2 * (size_t)D * sizeof(float) + sizeof(int32_t)) + 3 * 256;
+}
+
+// Segment containing position p (offsets non-decreasing, offsets[0] = 0,
+// offsets[C] = N, p < N): the last c with offsets[c] <= p, skipping empties
+// (their offsets[c] == offsets[c + 1] <= p).
+__device__ __forceinline__ int segment_of(const int32_t* off, int C, int p) {
+    int lo = 0, hi = C - 1;   // invariant: off[lo] <= p < off[hi + 1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= p) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
 
 template <typename T, int D, bool GATHER>
 __global__ void __launch_bounds__(kSmThreads)
-segment_mean_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
-                    const int32_t* __restrict__ offsets, int N, int C, float* out,
-                    bool empty_zero, const int32_t* __restrict__ done) {
+segment_piece_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm,
+                     const int32_t* __restrict__ offsets, int N, int C, float* __restrict__ out,
+                     bool empty_zero, const int32_t* __restrict__ done, float* __restrict__ lead,
+                     float* __restrict__ trail, int32_t* __restrict__ trail_seg) {
     constexpr int EPC = Elem<T>::kPerChunk;
-    constexpr int L = D / EPC;
-    constexpr int R = kSmThreads / L;
+    constexpr int L = D / EPC;          // lanes per row
+    constexpr int R = kSmThreads / L;   // lane groups
+    constexpr int U = kSmUnroll;
     __shared__ float part[R][D];
-    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    __shared__ int32_t rows_s[GATHER ? kSmChunk : 1];
+    const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int nch = gridDim.x;
     if (done && done[bh]) return;
     const int32_t* off = offsets + (size_t)bh * (C + 1);
-    const int a = off[c], b = off[c + 1];
-    float* o = out + ((size_t)bh * C + c) * D;
-    if (b <= a || a < 0 || b > N) {   // empty (or malformed) segment
-        if (empty_zero)
-            for (int k = tid; k < D; k += kSmThreads) o[k] = 0.f;
-        return;
-    }
+    const int c0 = j * kSmChunk, c1 = min(c0 + kSmChunk, N);
     const T* Xh = X + (size_t)bh * N * D;
-    const int lane = tid % L, grp = tid / L;
-    float acc[EPC];
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    // Four rows in flight per lane group (index loads first, then the rows);
-    // each lane still adds its rows in increasing p, one at a time.
-    constexpr int U = 4;
-    int p = a + grp;
-    for (; p + (U - 1) * R < b; p += U * R) {
-        int row[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) row[u] = GATHER ? perm[(size_t)bh * N + p + u * R] : p + u * R;
-        float v[U][EPC];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-            if ((unsigned)row[u] < (unsigned)N) Elem<T>::load(Xh + (size_t)row[u] * D + lane * EPC, v[u]);
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-            if ((unsigned)row[u] < (unsigned)N)
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) acc[e] += v[u][e];
+    float* lead_j = lead + ((size_t)bh * nch + j) * D;
+    float* trail_j = trail + ((size_t)bh * nch + j) * D;
+    if (GATHER) {
+        for (int p = c0 + tid; p < c1; p += kSmThreads) rows_s[p - c0] = perm[(size_t)bh * N + p];
     }
-    for (; p < b; p += R) {
-        const int row = GATHER ? perm[(size_t)bh * N + p] : p;
-        if ((unsigned)row >= (unsigned)N) continue;
-        float v[EPC];
-        Elem<T>::load(Xh + (size_t)row * D + lane * EPC, v);
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) acc[e] += v[e];
+    int seg = segment_of(off, C, c0);
+    const bool last_chunk = j == nch - 1;
+    // empty segments: those c with off[c] == off[c+1] in [c0, c1) (or == N on
+    // the last chunk) belong to this chunk
+    if (empty_zero) {
+        int e_lo = 0, hi = C;   // the first c whose offset is >= c0
+        while (e_lo < hi) {
+            const int mid = (e_lo + hi) >> 1;
+            if (off[mid] < c0) e_lo = mid + 1;
+            else hi = mid;
+        }
+        for (int c = e_lo; c < C; ++c) {
+            const int a = off[c];
+            if (a >= c1 && !(last_chunk && a == N)) break;
+            if (off[c + 1] == a)
+                for (int k = tid; k < D; k += kSmThreads) out[((size_t)bh * C + c) * D + k] = 0.f;
+        }
     }
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) part[grp][lane * EPC + e] = acc[e];
+    if (tid == 0) trail_seg[(size_t)bh * nch + j] = -1;
     __syncthreads();
-    const float n = (float)(b - a);
-    for (int k = tid; k < D; k += kSmThreads) {
-        float s = 0.f;
+    const int lane = tid % L, grp = tid / L;
+    for (int p0 = c0; p0 < c1;) {
+        const int a = off[seg], b = off[seg + 1];
+        if (b <= p0 || a > p0) break;          // malformed offsets: stop rather than spin
+        const int r0 = p0, r1 = min(b, c1);   // this piece
+        float acc[EPC];
 #pragma unroll
-        for (int g = 0; g < R; ++g) s += part[g][k];
-        o[k] = s / n;
+        for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+        // U rows in flight per lane group, all loads before the first add;
+        // a slot past the piece reloads the piece's first row and is not
+        // added (nor is a gathered row outside the head: malformed perm)
+        for (int p = r0 + grp; p < r1; p += U * R) {
+            int row[U];
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int q = p + u * R;
+                const int at = q < r1 ? q : r0;
+                const int rr = GATHER ? rows_s[at - c0] : at;
+                row[u] = q < r1 ? rr : -1;
+                const int rc = GATHER ? min(max(rr, 0), N - 1) : rr;
+                v[u] = Elem<T>::load_raw(Xh + (size_t)rc * D + lane * EPC);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if ((unsigned)row[u] >= (unsigned)N) continue;
+                float f[EPC];
+                Elem<T>::unpack(v[u], f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) part[grp][lane * EPC + e] = acc[e];
+        __syncthreads();
+        for (int k = tid; k < D; k += kSmThreads) {
+            float s = 0.f;
+#pragma unroll
+            for (int g = 0; g < R; ++g) s += part[g][k];
+            if (a < c0) lead_j[k] = s;                 // started in an earlier chunk
+            else if (b > c1) trail_j[k] = s;           // continues in later chunks
+            else out[((size_t)bh * C + seg) * D + k] = s / (float)(b - a);
+        }
+        if (tid == 0 && a >= c0 && b > c1) trail_seg[(size_t)bh * nch + j] = seg;
+        __syncthreads();
+        p0 = r1;
+        if (p0 < c1) {   // next non-empty segment
+            if (++seg >= C) break;
+            while (seg < C - 1 && off[seg + 1] <= p0) ++seg;
+        }
     }
+}
+
+// Segments longer than one chunk: trail(j0) + lead(j0+1) + ... + lead(j1).
+template <int D>
+__global__ void segment_join_kernel(const int32_t* __restrict__ offsets, int N, int C,
+                                    float* __restrict__ out, const int32_t* __restrict__ done,
+                                    const float* __restrict__ lead,
+                                    const float* __restrict__ trail,
+                                    const int32_t* __restrict__ trail_seg) {
+    const int j = blockIdx.x, bh = blockIdx.y, k = threadIdx.x;
+    const int nch = gridDim.x;
+    if (done && done[bh]) return;
+    const int c = trail_seg[(size_t)bh * nch + j];
+    if (c < 0 || c >= C) return;
+    const int32_t* off = offsets + (size_t)bh * (C + 1);
+    const int a = off[c], b = off[c + 1];
+    const int j1 = min((b - 1) / kSmChunk, nch - 1);
+    float s = trail[((size_t)bh * nch + j) * D + k];
+    for (int jj = j + 1; jj <= j1; ++jj) s += lead[((size_t)bh * nch + jj) * D + k];
+    out[((size_t)bh * C + c) * D + k] = s / (float)(b - a);
 }
 
 // ---------------------------------------------------------------------------
@@ -872,16 +963,19 @@ __global__ void permute_kernel(const T* __restrict__ X, const int32_t* __restric
     } while (0)
 
 template <typename T, int D>
-static int kmeanspp_disp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+static int kmeanspp_disp(const void* X, svgear_dims dims, int C, uint64_t seed, uint64_t sbase,
+                         float* cent,
                          int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
                          int32_t* counter, int32_t* gen, int* err, cudaStream_t st) {
-    return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, cent, chosen, D2, nearest,
+    return kmeanspp_impl<T, D>(static_cast<const T*>(X), dims, C, seed, sbase, cent, chosen, D2,
+                               nearest,
                                cc2, bs, counter, gen, err, st);
 }
-int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, float* cent,
+int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, uint64_t sbase,
+                    float* cent,
                     int32_t* chosen, float* D2, int32_t* nearest, float* cc2, double* bs,
                     int32_t* counter, int32_t* gen, int* err, cudaStream_t st) {
-    SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, cent, chosen, D2, nearest, cc2, bs,
+    SVGEAR_DISPATCH(dims, kmeanspp_disp, X, dims, C, seed, sbase, cent, chosen, D2, nearest, cc2, bs,
                     counter, gen, err, st);
 }
 
@@ -924,22 +1018,32 @@ int launch_fixed_point(int32_t* changed, int32_t* done, int BH, cudaStream_t st)
 template <typename T, int D>
 static int segmean_disp(const void* X, const int32_t* perm, const int32_t* offsets, int C,
                         svgear_dims dims, float* out, bool empty_zero, const int32_t* done,
-                        cudaStream_t st) {
+                        void* scratch, cudaStream_t st) {
     const int BH = dims.B * dims.H;
+    const int nch = ceil_div(dims.N, kSmChunk);
+    const size_t parts = (size_t)BH * nch * D;
+    float* lead = static_cast<float*>(scratch);
+    float* trail = lead + parts;
+    int32_t* tseg = reinterpret_cast<int32_t*>(trail + parts);
     if (perm)
-        segment_mean_kernel<T, D, true><<<dim3(C, BH), kSmThreads, 0, st>>>(
-            static_cast<const T*>(X), perm, offsets, dims.N, C, out, empty_zero, done);
+        segment_piece_kernel<T, D, true><<<dim3(nch, BH), kSmThreads, 0, st>>>(
+            static_cast<const T*>(X), perm, offsets, dims.N, C, out, empty_zero, done, lead,
+            trail, tseg);
     else
-        segment_mean_kernel<T, D, false><<<dim3(C, BH), kSmThreads, 0, st>>>(
-            static_cast<const T*>(X), nullptr, offsets, dims.N, C, out, empty_zero, done);
-    count_launches(1);
+        segment_piece_kernel<T, D, false><<<dim3(nch, BH), kSmThreads, 0, st>>>(
+            static_cast<const T*>(X), nullptr, offsets, dims.N, C, out, empty_zero, done, lead,
+            trail, tseg);
+    segment_join_kernel<D><<<dim3(nch, BH), D, 0, st>>>(offsets, dims.N, C, out, done, lead, trail,
+                                                       tseg);
+    count_launches(2);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
 }
 int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets, int C,
-                        svgear_dims dims, float* out, bool empty_zero, cudaStream_t st,
-                        const int32_t* done) {
-    SVGEAR_DISPATCH(dims, segmean_disp, X, perm, offsets, C, dims, out, empty_zero, done, st);
+                        svgear_dims dims, float* out, bool empty_zero, void* scratch,
+                        cudaStream_t st, const int32_t* done) {
+    SVGEAR_DISPATCH(dims, segmean_disp, X, perm, offsets, C, dims, out, empty_zero, done, scratch,
+                    st);
 }
 
 template <typename T, int D>

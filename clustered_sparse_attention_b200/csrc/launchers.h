@@ -16,6 +16,13 @@ constexpr int kSortTokens = 1024;
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// api.cu: svgear_cluster on a range of heads of a larger call, drawing the
+// k-means++ numbers of head bh from Philox stream sbase + bh.
+int cluster_heads(const void* X, svgear_dims dims, int32_t C, int32_t iters,
+                  const float* warm_centroids, uint64_t seed, uint64_t sbase, int32_t* labels,
+                  int32_t* perm, int32_t* offsets, float* centroids, void* Xp, void* ws,
+                  size_t ws_bytes, void* stream);
+
 // guard.cu: the device's tensor-memory-lost word (address in the current
 // context) and whether svgear_device_status has seen it set in this context.
 int tmem_lost_word(int** out);
@@ -23,8 +30,10 @@ bool tmem_lost_latched();
 
 // kmeans.cu
 // k-means++ seeding: one cooperative persistent launch over a shared pool of
-// work (see kpp_pool_kernel); err: device status words (4 ints).
-int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed,
+// work (see kpp_pool_kernel); err: device status words (4 ints).  Head bh of
+// the launch draws from Philox stream sbase + bh (sbase = 0 for a whole call;
+// a call on a range of heads passes the range's first flattened head).
+int launch_kmeanspp(const void* X, svgear_dims dims, int C, uint64_t seed, uint64_t sbase,
                     float* centroids, int32_t* chosen, float* D2, int32_t* nearest, float* cc2,
                     double* blocksum, int32_t* counter /* 2 BH words */,
                     int32_t* gen /* BH + 1 words */, int* err,
@@ -55,9 +64,12 @@ int launch_segment_var(const void* X, const int32_t* offsets, int C, svgear_dims
                        float* out, cudaStream_t st);
 // Mean of every segment; rows are perm[p] when perm != NULL (gather) else p.
 // empty_zero: an empty segment writes zeros (else leaves the row untouched).
+// scratch: segmean_scratch_bytes(B*H, N, d) bytes (partial sums of segments
+// that cross position chunks).
 int launch_segment_mean(const void* X, const int32_t* perm, const int32_t* offsets,
-                        int C, svgear_dims dims, float* out, bool empty_zero,
+                        int C, svgear_dims dims, float* out, bool empty_zero, void* scratch,
                         cudaStream_t st, const int32_t* done = nullptr);
+size_t segmean_scratch_bytes(int BH, int N, int D);
 int launch_permute(const void* X, const int32_t* perm, svgear_dims dims, void* Xp,
                    cudaStream_t st);
 

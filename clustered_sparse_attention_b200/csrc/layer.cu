@@ -63,6 +63,8 @@ size_t scratch_need(const svgear_dims& d, const svgear_layer_params* p) {
     if (t > s) s = t;
     t = svgear_workspace_bytes(SVGEAR_OP_ATTEND, d, p->Cq, p->Ck);
     if (t > s) s = t;
+    t = svgear_workspace_bytes(SVGEAR_OP_CENTROIDS, d, p->Ck, 0);
+    if (t > s) s = t;
     return s;
 }
 
@@ -130,7 +132,9 @@ int run_layer(const void* Q, const void* K, const void* V, svgear_dims dims,
     if ((s = record(ev, 2, st))) return s;
     if (ready && (s = wait_on(ready[2], st))) return s;
     if ((s = svgear_permute(V, w.perm_k, dims, w.Vp, vst))) return s;
-    if ((s = svgear_centroids(w.Vp, w.off_k, p->Ck, dims, w.vbar, vst))) return s;
+    if ((s = svgear_centroids(w.Vp, w.off_k, p->Ck, dims, w.vbar, w.scratch, w.scratch_bytes,
+                              vst)))
+        return s;
     if ((s = record(ev, 3, st))) return s;
     if (p->topp > 0.f)
         s = svgear_route_topp(cent_q, w.off_q, p->Cq, cent_k, w.vbar, w.off_k, p->Ck, w.Xp_k, w.Vp,
@@ -149,6 +153,159 @@ int run_layer(const void* Q, const void* K, const void* V, svgear_dims dims,
         return s;
     return record(ev, 5, st);
 }
+
+// The host-buffer layer as a pipeline over head groups (flattened b*H + h):
+// the inputs go up on a copy stream, Q in kQGroups parts, then K and V; Q is
+// clustered part by part as it arrives (each part's k-means++ draws from the
+// Philox streams of its own heads, so the result is the whole call's), K, V,
+// the value centroids and routing run whole, and attention runs in kOGroups
+// parts whose O goes back to the host on a third stream while the next part
+// is computed.  So only the first part of Q and the last part of O cross the
+// host link with nothing to overlap.  The copy stream first waits for all
+// work already on `st` (an earlier call may still read this workspace); the
+// call's streams and events are released once their work is done.
+struct HostPipeline {
+    static constexpr int kQGroups = 2, kOGroups = 4;
+    static constexpr int kMinHeadsPerGroup = 8;
+    cudaStream_t xs = nullptr, ds = nullptr;
+    cudaEvent_t entry = nullptr, done_d2h = nullptr, k_ready = nullptr, v_ready = nullptr;
+    cudaEvent_t q_ready[kQGroups] = {}, o_ready[kOGroups] = {};
+
+    static int groups(int BH, int want) {
+        int g = BH / kMinHeadsPerGroup;
+        return g < 1 ? 1 : (g > want ? want : g);
+    }
+    // heads [lo, hi) of group g of G over BH (contiguous, sizes within one)
+    static void range(int BH, int G, int g, int* lo, int* hi) {
+        const int base = BH / G, extra = BH % G;
+        *lo = g * base + (g < extra ? g : extra);
+        *hi = *lo + base + (g < extra ? 1 : 0);
+    }
+    bool create() {
+        auto ev = [](cudaEvent_t* e) {
+            return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+        };
+        bool ok = cudaStreamCreateWithFlags(&xs, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&ds, cudaStreamNonBlocking) == cudaSuccess &&
+                  ev(&entry) && ev(&done_d2h) && ev(&k_ready) && ev(&v_ready);
+        for (cudaEvent_t& e : q_ready) ok = ok && ev(&e);
+        for (cudaEvent_t& e : o_ready) ok = ok && ev(&e);
+        return ok;
+    }
+    void release() {
+        cudaEvent_t all[] = {entry, done_d2h, k_ready, v_ready};
+        for (cudaEvent_t e : all)
+            if (e) cudaEventDestroy(e);
+        for (cudaEvent_t e : q_ready)
+            if (e) cudaEventDestroy(e);
+        for (cudaEvent_t e : o_ready)
+            if (e) cudaEventDestroy(e);
+        if (xs) cudaStreamDestroy(xs);
+        if (ds) cudaStreamDestroy(ds);
+    }
+
+    int run(const void* Qh, const void* Kh, const void* Vh, svgear_dims dims,
+            const svgear_layer_params* p, const float* warm_q, const float* warm_k, void* Oh,
+            float* cq_out, float* ck_out, const LayerWs& w, cudaStream_t st) {
+        if (!create()) return SVGEAR_ERR_CUDA;
+        int s;
+        void* vst = static_cast<void*>(st);
+        const int BH = (int)bh_of(dims), N = dims.N, D = dims.d;
+        const size_t esz = dims.dtype == SVGEAR_BF16 ? 2 : 4;
+        const size_t head_bytes = (size_t)N * D * esz, tb = tensor_bytes(dims);
+        float* cent_q = cq_out ? cq_out : w.cent_q;
+        float* cent_k = ck_out ? ck_out : w.cent_k;
+        const int GQ = groups(BH, kQGroups), GO = groups(BH, kOGroups);
+        auto sub = [&](int lo, int hi) {   // dims of the flattened heads [lo, hi)
+            svgear_dims d = dims;
+            d.B = 1;
+            d.H = hi - lo;
+            return d;
+        };
+        auto at = [](const void* base, size_t off) {
+            return static_cast<void*>(static_cast<char*>(const_cast<void*>(base)) + off);
+        };
+        // inputs
+        if (cudaEventRecord(entry, st) != cudaSuccess || cudaStreamWaitEvent(xs, entry, 0) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        for (int g = 0; g < GQ; ++g) {
+            int lo, hi;
+            range(BH, GQ, g, &lo, &hi);
+            if (cudaMemcpyAsync(at(w.Qd, lo * head_bytes), at(Qh, lo * head_bytes),
+                                (hi - lo) * head_bytes, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+                cudaEventRecord(q_ready[g], xs) != cudaSuccess)
+                return SVGEAR_ERR_CUDA;
+        }
+        if (cudaMemcpyAsync(w.Kd, Kh, tb, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+            cudaEventRecord(k_ready, xs) != cudaSuccess ||
+            cudaMemcpyAsync(w.Vd, Vh, tb, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+            cudaEventRecord(v_ready, xs) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        // Q, part by part as it arrives
+        const size_t cq_row = (size_t)p->Cq * D;
+        for (int g = 0; g < GQ; ++g) {
+            int lo, hi;
+            range(BH, GQ, g, &lo, &hi);
+            if (cudaStreamWaitEvent(st, q_ready[g], 0) != cudaSuccess) return SVGEAR_ERR_CUDA;
+            if ((s = cluster_heads(at(w.Qd, lo * head_bytes), sub(lo, hi), p->Cq, p->iters,
+                                   warm_q ? warm_q + lo * cq_row : nullptr, 2 * p->seed,
+                                   (uint64_t)lo, w.labels_q + (size_t)lo * N,
+                                   w.perm_q + (size_t)lo * N, w.off_q + (size_t)lo * (p->Cq + 1),
+                                   cent_q + lo * cq_row, at(w.Xp_q, lo * head_bytes), w.scratch,
+                                   w.scratch_bytes, vst)))
+                return s;
+        }
+        // K, V, value centroids, routing: whole
+        if (cudaStreamWaitEvent(st, k_ready, 0) != cudaSuccess) return SVGEAR_ERR_CUDA;
+        if ((s = svgear_cluster(w.Kd, dims, p->Ck, p->iters, warm_k, 2 * p->seed + 1, w.labels_k,
+                                w.perm_k, w.off_k, cent_k, w.Xp_k, w.scratch, w.scratch_bytes, vst)))
+            return s;
+        if (cudaStreamWaitEvent(st, v_ready, 0) != cudaSuccess) return SVGEAR_ERR_CUDA;
+        if ((s = svgear_permute(w.Vd, w.perm_k, dims, w.Vp, vst))) return s;
+        if ((s = svgear_centroids(w.Vp, w.off_k, p->Ck, dims, w.vbar, w.scratch, w.scratch_bytes,
+                                  vst)))
+            return s;
+        if (p->topp > 0.f)
+            s = svgear_route_topp(cent_q, w.off_q, p->Cq, cent_k, w.vbar, w.off_k, p->Ck, w.Xp_k,
+                                  w.Vp, dims, p->topp, p->scale, w.pair_off, w.pair_kc, nullptr,
+                                  nullptr, w.scratch, w.scratch_bytes, vst);
+        else
+            s = svgear_route(cent_q, w.off_q, p->Cq, cent_k, w.vbar, w.off_k, p->Ck, w.Xp_k, w.Vp,
+                             dims, p->density, p->scale, w.pair_off, w.pair_kc, nullptr, w.scratch,
+                             w.scratch_bytes, vst);
+        if (s) return s;
+        if (w.kvar && (s = svgear_key_variance(w.Xp_k, w.off_k, p->Ck, dims, w.kvar, vst)))
+            return s;
+        // attention part by part; O of each part goes back while the next runs
+        // (O lands in Q's device copy: clustering Q was its last reader)
+        const size_t ck_row = (size_t)p->Ck * D;
+        for (int g = 0; g < GO; ++g) {
+            int lo, hi;
+            range(BH, GO, g, &lo, &hi);
+            const svgear_dims dg = sub(lo, hi);
+            if ((s = svgear_attend_var(
+                     at(w.Xp_q, lo * head_bytes), at(w.Xp_k, lo * head_bytes),
+                     at(w.Vp, lo * head_bytes), dg, N, w.off_q + (size_t)lo * (p->Cq + 1), p->Cq,
+                     w.off_k + (size_t)lo * (p->Ck + 1), p->Ck,
+                     w.pair_off + (size_t)lo * (p->Cq + 1),
+                     w.pair_kc + (size_t)lo * p->Cq * p->Ck, cent_k + lo * ck_row,
+                     w.vbar + lo * ck_row, w.kvar ? w.kvar + lo * ck_row : nullptr, p->var_lambda,
+                     w.perm_q + (size_t)lo * N, p->scale, at(w.Qd, lo * head_bytes), w.scratch,
+                     w.scratch_bytes, vst)))
+                return s;
+            if (cudaEventRecord(o_ready[g], st) != cudaSuccess ||
+                cudaStreamWaitEvent(ds, o_ready[g], 0) != cudaSuccess ||
+                cudaMemcpyAsync(at(Oh, lo * head_bytes), at(w.Qd, lo * head_bytes),
+                                (hi - lo) * head_bytes, cudaMemcpyDeviceToHost, ds) != cudaSuccess)
+                return SVGEAR_ERR_CUDA;
+        }
+        // the call ends on `st` once O is on the host
+        if (cudaEventRecord(done_d2h, ds) != cudaSuccess ||
+            cudaStreamWaitEvent(st, done_d2h, 0) != cudaSuccess)
+            return SVGEAR_ERR_CUDA;
+        return SVGEAR_OK;
+    }
+};
 
 }  // namespace
 
@@ -189,48 +346,10 @@ int svgear_layer_host(const void* Q_host, const void* K_host, const void* V_host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Carve cv(ws);
     LayerWs w = carve_layer(cv, dims, params, true);
-    const size_t tb = tensor_bytes(dims);
-    // The copies run on a stream of this call that first waits for all work
-    // already on `st` (an earlier call may still read this workspace); each
-    // stage then waits only for the input it reads, so clustering Q overlaps
-    // the copies of K and V.  The stream and events are released once their
-    // work is done (destruction is deferred by the runtime).
-    cudaStream_t xs = nullptr;
-    cudaEvent_t entry = nullptr, ready[3] = {nullptr, nullptr, nullptr};
-    auto cleanup = [&]() {
-        for (cudaEvent_t e : ready)
-            if (e) cudaEventDestroy(e);
-        if (entry) cudaEventDestroy(entry);
-        if (xs) cudaStreamDestroy(xs);
-    };
-    if (cudaStreamCreateWithFlags(&xs, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&entry, cudaEventDisableTiming) != cudaSuccess) {
-        cleanup();
-        return SVGEAR_ERR_CUDA;
-    }
-    for (cudaEvent_t& e : ready)
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
-            cleanup();
-            return SVGEAR_ERR_CUDA;
-        }
-    const void* src[3] = {Q_host, K_host, V_host};
-    void* dst[3] = {w.Qd, w.Kd, w.Vd};
-    bool ok = cudaEventRecord(entry, st) == cudaSuccess && cudaStreamWaitEvent(xs, entry, 0) ==
-                                                               cudaSuccess;
-    for (int i = 0; i < 3 && ok; ++i)
-        ok = cudaMemcpyAsync(dst[i], src[i], tb, cudaMemcpyHostToDevice, xs) == cudaSuccess &&
-             cudaEventRecord(ready[i], xs) == cudaSuccess;
-    if (!ok) {
-        cleanup();
-        return SVGEAR_ERR_CUDA;
-    }
-    // O lands in Q's device copy: clustering Q is its last reader
-    s = run_layer(w.Qd, w.Kd, w.Vd, dims, params, warm_q, warm_k, w.Qd, cent_q, cent_k, w, nullptr,
-                  ready, st);
-    if (s == SVGEAR_OK &&
-        cudaMemcpyAsync(O_host, w.Qd, tb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        s = SVGEAR_ERR_CUDA;
-    cleanup();
+    HostPipeline hp;
+    s = hp.run(Q_host, K_host, V_host, dims, params, warm_q, warm_k, O_host, cent_q, cent_k, w,
+               st);
+    hp.release();
     return s;
 }
 

@@ -92,7 +92,8 @@ typedef enum {
     SVGEAR_OP_ROUTE = 4,
     SVGEAR_OP_ATTEND = 5,
     SVGEAR_OP_KMEANS_ASSIGN = 6,
-    SVGEAR_OP_ROUTE_TOPP = 7
+    SVGEAR_OP_ROUTE_TOPP = 7,
+    SVGEAR_OP_CENTROIDS = 8
 } svgear_op;
 
 /* Largest cluster count any call accepts (shared-memory tables). */
@@ -191,9 +192,16 @@ int svgear_permute(const void* X, const int32_t* perm, svgear_dims dims, void* X
  *   Xp        [B][H][N][d] permuted tokens (dtype).
  *   offsets   int32[B][H][C+1] segments.
  *   centroids out float[B][H][C][d]; an empty segment gives zeros.
+ *   ws        svgear_workspace_bytes(SVGEAR_OP_CENTROIDS, dims, C, 0): the
+ *             partial sums of segments longer than one 512-position chunk.
+ * The work is split by position (every CTA reads the same 512 rows,
+ * whatever the cluster sizes); each segment is summed in fp32 in an order
+ * fixed by the positions alone (rows of a chunk by lane group, groups in
+ * order, chunks in order), so the result is the same from run to run.
  * ------------------------------------------------------------------------ */
 int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
-                     svgear_dims dims, float* centroids, void* stream);
+                     svgear_dims dims, float* centroids, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /* --------------------------------------------------------------------------
  * svgear_probe -- compensation-error probe ([BLOG] probe paragraph; [REVIEW]

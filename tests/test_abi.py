@@ -107,7 +107,8 @@ def test_empty_batch_is_a_no_op(L):
     # B = 0: valid, nothing to launch, no CUDA call
     assert L.svgear_kmeans_assign(fake, _dims(B=0), fake, 10, fake, fake, ctypes.c_size_t(1 << 20),
                                   None) == 0
-    assert L.svgear_centroids(fake, fake, 10, _dims(B=0), fake, None) == 0
+    assert L.svgear_centroids(fake, fake, 10, _dims(B=0), fake, fake, ctypes.c_size_t(1 << 20),
+                              None) == 0
 
 
 def test_selftest_wait_validates_before_launch(L):

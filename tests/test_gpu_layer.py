@@ -18,6 +18,11 @@ SMALL = synth.custom_workload("layer_small", H=3, frames=2, grid_h=24, grid_w=40
                               dtype="bf16", Cq=16, Ck=40, iters=4, density=0.3, n_centres=24,
                               sigma=0.5, index=71)
 TINY = synth.WORKLOADS["tiny"]
+# enough heads for the host-buffer call to pipeline Q and O over head groups
+# (2 groups of 17 heads for Q, 4 of 8-9 heads for attention and O)
+MANY = synth.custom_workload("layer_many_heads", H=34, frames=1, grid_h=24, grid_w=32, d=64,
+                             dtype="bf16", Cq=8, Ck=20, iters=3, density=0.25, n_centres=12,
+                             sigma=0.5, index=72)
 
 
 def _inputs(w):
@@ -26,7 +31,7 @@ def _inputs(w):
 
 
 @pytest.mark.parametrize("topp,lam", [(None, 0.0), (0.9, 0.0), (None, 1.0)])
-@pytest.mark.parametrize("w", [SMALL, TINY], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [SMALL, TINY, MANY], ids=lambda w: w.name)
 def test_layer_call_equals_stagewise_composition(w, topp, lam):
     import clustered_sparse_attention_b200 as csa
     host, dev = _inputs(w)

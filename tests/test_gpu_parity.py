@@ -311,6 +311,79 @@ def test_warm_sequence_stagewise(density):
         warm = {"q": cq.centroids, "k": ck.centroids}
 
 
+def _hand_offsets(N, C, g):
+    """Segment sizes that stress the position split (chunks of 512): long
+    segments over several chunks, ends exactly on chunk edges, empty
+    segments first, in the middle and last, a single segment of one row."""
+    sizes = np.zeros(C, dtype=np.int64)
+    fixed = [0, 1, 511, 1, 1536, 0, 512, 0, 3000, 7]
+    sizes[:len(fixed)] = fixed[:C]
+    rest = N - int(sizes.sum())
+    free = np.arange(len(fixed), C - 1)             # the last segment stays empty
+    cut = np.sort(g.choice(rest + 1, len(free) - 1, replace=True)) if len(free) > 1 else []
+    parts = np.diff(np.concatenate([[0], cut, [rest]]))
+    sizes[free] = parts
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    assert off[-1] == N and sizes[-1] == 0
+    return off
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 128)])
+def test_segment_means_across_position_chunks(dtype, d):
+    """Means of segments that cross the 512-position chunks of the split
+    kernel: the gathered form (k-means update, rows perm[p]) and the
+    contiguous form (value centroids on X[perm]) sum the same values in the
+    same order, so they agree bit for bit; both within the fp32 bound of the
+    oracle's means, and identical from run to run."""
+    csa = _csa()
+    g = np.random.default_rng(17)
+    B, H, N, C = 1, 2, 9000 + 77, 40
+    X = g.standard_normal((B, H, N, d)).astype(np.float32)
+    if dtype == "bf16":
+        X = synth.round_to_bf16(X)
+    offs = np.stack([_hand_offsets(N, C, g) for _ in range(H)])[None]
+    labels = np.zeros((B, H, N), dtype=np.int32)
+    perm = np.zeros((B, H, N), dtype=np.int32)
+    for h in range(H):
+        sizes = np.diff(offs[0, h])
+        lab_sorted = np.repeat(np.arange(C), sizes).astype(np.int32)
+        p = g.permutation(N).astype(np.int32)          # token perm[i] sits at position i
+        perm[0, h] = p
+        labels[0, h, p] = lab_sorted
+    Xd = to_torch(X, dtype)
+    prev = g.standard_normal((B, H, C, d)).astype(np.float32)
+    upd = csa.svgear_kmeans_update(Xd, torch.from_numpy(labels).cuda(),
+                                   torch.from_numpy(prev).cuda())
+    upd2 = csa.svgear_kmeans_update(Xd, torch.from_numpy(labels).cuda(),
+                                    torch.from_numpy(prev).cuda())
+    Xp = csa.svgear_permute(Xd, torch.from_numpy(perm).cuda())
+    cen = csa.svgear_centroids(Xp, torch.from_numpy(offs).cuda(), C)
+    torch.cuda.synchronize()
+    assert torch.equal(upd, upd2)
+    u, c = upd.cpu().numpy(), cen.cpu().numpy()
+    for h in range(H):
+        sizes = np.diff(offs[0, h])
+        full = sizes > 0
+        # the update's sort is stable, so its perm lists tokens of a cluster in
+        # increasing index; compare with the contiguous form on that order
+        ref = oracle.segment_mean(X[0, h][perm[0, h]], offs[0, h])
+        lab_sorted = np.repeat(np.arange(C), sizes)
+        tol = update_tolerance(X[0, h][perm[0, h]], lab_sorted, C)
+        assert np.all(np.abs(c[0, h] - ref) <= tol)
+        assert np.all(np.abs(u[0, h][full] - ref[full]) <= tol[full])
+        assert np.all(c[0, h][~full] == 0)                       # empty: zeros
+        assert np.array_equal(u[0, h][~full], prev[0, h][~full])  # empty: previous row
+        p_o, o_o = oracle.stable_sort(labels[0, h], C)
+        assert np.array_equal(o_o, offs[0, h])
+    # the gathered form in the sort's own order equals the contiguous form
+    # on the same order, bit for bit
+    ps, _ = csa.svgear_label_sort(torch.from_numpy(labels).cuda(), C)
+    cen_s = csa.svgear_centroids(csa.svgear_permute(Xd, ps), torch.from_numpy(offs).cuda(), C)
+    torch.cuda.synchronize()
+    full = np.diff(offs[0], axis=-1) > 0
+    assert np.array_equal(cen_s.cpu().numpy()[0][full], u[0][full])
+
+
 @pytest.mark.parametrize("w", [TINY, SMALL_BF16, RAGGED_BF16_64], ids=lambda w: w.name)
 def test_permute_and_value_centroids(w):
     csa = _csa()
