@@ -91,14 +91,14 @@ SelWs carve_select(Carve& cv, size_t BH, int Cq, int Ck) {
 }
 struct RouteWs {
     float* E;
-    uint32_t* rowmax;
+    float* cmax;   // the probe's maximum score per (probe, key cluster)
     float* qT;   // probes transposed in blocks of 128: [BH][ceil(Cq/128)][d][128]
     SelWs sel;
 };
 RouteWs carve_route(Carve& cv, size_t BH, int Cq, int Ck, int d) {
     RouteWs w;
     w.E = cv.take<float>(BH * Cq * (size_t)Ck);
-    w.rowmax = cv.take<uint32_t>(BH * Cq);
+    w.cmax = cv.take<float>(BH * Cq * (size_t)Ck);
     w.qT = cv.take<float>(BH * (size_t)ceil_div(Cq, 128) * 128 * (size_t)d);
     w.sel = carve_select(cv, BH, Cq, Ck);
     return w;
@@ -410,7 +410,7 @@ int svgear_probe(const float* qbar, int32_t Cq, const void* Kp, const void* Vp, 
     if (bh_of(kdims) == 0) return SVGEAR_OK;
     Carve cv(ws);
     RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
-    return launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT,
+    return launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.cmax, w.qT,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -452,7 +452,7 @@ int svgear_route(const float* qbar, const int32_t* q_off, int32_t Cq, const floa
     Carve cv(ws);
     RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
     float* E = E_out ? E_out : w.E;
-    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT, st)))
+    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.cmax, w.qT, st)))
         return s;
     const long long budget = (long long)floor((double)density * (double)kdims.N);
     return launch_route_select(E, q_off, Cq, k_off, Ck, (int)bh_of(kdims), budget, nullptr,
@@ -515,7 +515,7 @@ int svgear_route_topp(const float* qbar, const int32_t* q_off, int32_t Cq, const
     int32_t* bud = cv.take<int32_t>(bh_of(kdims) * Cq);
     if (budget_out) bud = budget_out;
     float* E = E_out ? E_out : w.E;
-    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.rowmax, w.qT, st)))
+    if ((s = launch_probe(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kdims, scale, E, w.cmax, w.qT, st)))
         return s;
     if ((s = launch_topp_budget(qbar, q_off, Cq, kbar, k_off, Ck, (int)bh_of(kdims), kdims.d,
                                 (double)p, (double)scale, bud, st)))
@@ -576,7 +576,7 @@ int svgear_probe_value_free(const float* qbar, int32_t Cq, const void* Kp, const
     Carve cv(ws);
     RouteWs w = carve_route(cv, bh_of(kdims), Cq, Ck, kdims.d);
     return launch_probe(qbar, Cq, Kp, nullptr, kbar, nullptr, k_off, Ck, kdims, scale, E,
-                        w.rowmax, w.qT, static_cast<cudaStream_t>(stream), true);
+                        w.cmax, w.qT, static_cast<cudaStream_t>(stream), true);
 }
 
 int svgear_diagnostics(const void* Qp, const void* Kp, const void* Vp, svgear_dims qdims,

@@ -81,7 +81,7 @@ int launch_label_sort(const int32_t* labels, int BH, int N, int C, int32_t* perm
 // route.cu
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp,
                  const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
-                 svgear_dims kdims, float scale, float* E, uint32_t* rowmax, float* qT,
+                 svgear_dims kdims, float scale, float* E, float* cmax, float* qT,
                  cudaStream_t st, bool value_free = false);
 int launch_route_select(const float* E, const int32_t* q_off, int Cq, const int32_t* k_off,
                         int Ck, int BH, long long budget, const int32_t* budgets, int32_t* lists,

@@ -10,12 +10,13 @@
 // the probe costs O(Cq * Nk * d).
 //
 // Kernels (fp32 throughout):
-//   probe_rowmax  m_i = max_t scale*qbar_i.k_t, by an order-independent
-//                 atomicMax on order-preserving integer keys (deterministic);
 //   probe_error   one block per (key cluster, 128 probes, head): every probe
 //                 against every key of the cluster, the error expanded around
 //                 the key's residual from its cluster's value mean (see the
-//                 register-tiled section below), summed in a fixed order;
+//                 register-tiled section below), shifted by the cluster's own
+//                 maximum score m_ic and summed in a fixed order;
+//   probe_rescale one warp per probe row: m_i = max_c m_ic (the maximum over
+//                 every key of the head) and E_ic <- E_ic e^{2 (m_ic - m_i)};
 //   route_select  one block per (query cluster, head): r_c = E/n_c, a bitonic
 //                 sort on (r desc, c asc), the greedy take-if-fits scan, and
 //                 an ascending list of the taken clusters;
@@ -102,50 +103,6 @@ __device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int 
 __device__ __forceinline__ int pb_probe(int pi, int i) { return pi * 4 + (i & 3) + (i >> 2) * 64; }
 __device__ __forceinline__ int pb_key(int ki, int j) { return ki * 4 + (j & 3) + (j >> 2) * 32; }
 
-// m_i = max over keys [t_begin, t_end) of scale * qbar_i . k_t, merged into
-// rowmax by an order-independent atomicMax on order-preserving integers.
-template <typename T, int D>
-__global__ void __launch_bounds__(kPbThreads, 2)
-probe_rowmax_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __restrict__ Kp,
-                       int Nk, float scale, int keys_per_cta, uint32_t* __restrict__ rowmax) {
-    extern __shared__ __align__(16) float pbs[];
-    float* Qs = pbs;                 // [D][128]
-    float* Ks = Qs + D * kPbP;       // [D][64]
-    float* red = Ks + D * kPbK;      // [4][128]
-    const int part = blockIdx.x, blk = blockIdx.y, bh = blockIdx.z, tid = threadIdx.x;
-    const int pi = tid & 15, ki = tid >> 4, lane = tid & 31, warp = tid >> 5;
-    const int t_begin = part * keys_per_cta, t_end = min(Nk, t_begin + keys_per_cta);
-    pb_load_q<D>(qT + ((size_t)bh * nPB + blk) * D * kPbP, Qs);
-    const T* Kh = Kp + (size_t)bh * Nk * D;
-    float mx[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-    for (int t0 = t_begin; t0 < t_end; t0 += kPbK) {
-        __syncthreads();
-        pb_load_k<T, D>(Kh, t0, t_end, Ks);
-        __syncthreads();
-        float acc[8][8];
-        pb_scores<D>(Qs, Ks, pi, ki, acc);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (t0 + pb_key(ki, j) < t_end)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], scale * acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 16));
-    __syncthreads();
-    if (lane < 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp * kPbP + pb_probe(pi, i)] = mx[i];
-    __syncthreads();
-    const int p = blk * kPbP + tid;
-    if (p < Cq) {
-        const float m = fmaxf(fmaxf(red[tid], red[kPbP + tid]), fmaxf(red[2 * kPbP + tid], red[3 * kPbP + tid]));
-        atomicMax(rowmax + (size_t)bh * Cq + p, float_to_ordered(m));
-    }
-}
-
 // E[bh][i][c] for the block's probes, one CTA per (key cluster c, probe
 // block, head).  VF: the value-free error sum_t (a - b)^2.
 template <typename T, int D, bool VF>
@@ -153,7 +110,7 @@ __global__ void __launch_bounds__(kPbThreads, 2)
 probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __restrict__ Kp,
                       const T* __restrict__ Vp, const float* __restrict__ kbar,
                       const float* __restrict__ vbar, const int32_t* __restrict__ k_off, int Ck,
-                      int Nk, float scale, const uint32_t* __restrict__ rowmax,
+                      int Nk, float scale, float* __restrict__ mloc,
                       float* __restrict__ E) {
     extern __shared__ __align__(16) float pbs[];
     float* Qs = pbs;                 // [D][128]
@@ -169,7 +126,10 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
     const int a0 = off[c], a1 = off[c + 1];
     if (a1 <= a0 || a0 < 0 || a1 > Nk) {   // empty (or malformed) key cluster: no error
         const int p = blk * kPbP + tid;
-        if (p < Cq) E[((size_t)bh * Cq + p) * Ck + c] = 0.f;
+        if (p < Cq) {
+            E[((size_t)bh * Cq + p) * Ck + c] = 0.f;
+            mloc[((size_t)bh * Cq + p) * Ck + c] = -INFINITY;
+        }
         return;
     }
     pb_load_q<D>(qT + ((size_t)bh * nPB + blk) * D * kPbP, Qs);
@@ -178,15 +138,20 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
         if (!VF) vb[k] = vbar[((size_t)bh * Ck + c) * D + k];
     }
     __syncthreads();
-    // a_i = exp(scale * qbar_i . kbar_c - m_i) for this thread's probes
-    float ai[8], mi[8];
+    // Every thread shifts its own keys' terms by its running maximum m_i of
+    // the probe's scores (a rescale of its partial sum whenever a tile
+    // raises it); the partial sums are brought to the cluster's maximum m_ic
+    // before they are added, and a last kernel brings E to the row maximum
+    // m_i = max_c m_ic: E(m) = e^{2 (m' - m)} E(m'), every term being
+    // quadratic in (e^{sbar - m}, e^{s - m}).
+    float ai[8], mi[8], sbar[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int p = blk * kPbP + pb_probe(pi, i);
-        mi[i] = p < Cq ? ordered_to_float(rowmax[(size_t)bh * Cq + p]) : 0.f;
         float dotk = 0.f;
         for (int k = 0; k < D; ++k) dotk = fmaf(Qs[k * kPbP + pb_probe(pi, i)], kb[k], dotk);
-        ai[i] = expf(scale * dotk - mi[i]);
+        sbar[i] = scale * dotk;
+        mi[i] = sbar[i];   // the centroid's score (the mean of the members' scores) starts it
+        ai[i] = 1.f;
     }
     float gamma = 0.f;
     if (!VF)
@@ -230,6 +195,18 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
         float acc[8][8];
         pb_scores<D>(Qs, Ks, pi, ki, acc);
 #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float tmx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (t0 + pb_key(ki, j) < a1) tmx = fmaxf(tmx, scale * acc[i][j]);
+            if (tmx > mi[i]) {   // the shift grows: rescale what is summed so far
+                err[i] *= expf(2.f * (mi[i] - tmx));
+                mi[i] = tmx;
+                ai[i] = expf(sbar[i] - tmx);
+            }
+        }
+#pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int tj = pb_key(ki, j);
             if (t0 + tj >= a1) continue;
@@ -251,81 +228,100 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
             }
         }
     }
+    // the cluster's maximum m_ic per probe: over the 8 threads of each probe
 #pragma unroll
-    for (int i = 0; i < 8; ++i) err[i] += __shfl_xor_sync(0xffffffffu, err[i], 16);
+    for (int i = 0; i < 8; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, mi[i], 16);
+        const float eo = __shfl_xor_sync(0xffffffffu, err[i], 16);
+        const float m2 = fmaxf(mi[i], o);
+        err[i] = err[i] * expf(2.f * (mi[i] - m2)) + eo * expf(2.f * (o - m2));
+        mi[i] = m2;
+    }
+    __syncthreads();
+    float* redm = kb;   // kbar_c is no longer needed: the warps' maxima
+    if (lane < 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp * kPbP + pb_probe(pi, i)] = mi[i];
+    __syncthreads();
+    float mw[4];
+    if (tid < kPbP) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mw[w] = red[w * kPbP + tid];
+    }
     __syncthreads();
     if (lane < 16)
 #pragma unroll
         for (int i = 0; i < 8; ++i) red[warp * kPbP + pb_probe(pi, i)] = err[i];
     __syncthreads();
+    (void)redm;
     const int p = blk * kPbP + tid;
-    if (p < Cq)
-        E[((size_t)bh * Cq + p) * Ck + c] =
-            ((red[tid] + red[kPbP + tid]) + red[2 * kPbP + tid]) + red[3 * kPbP + tid];
+    if (p < Cq) {
+        const float m = fmaxf(fmaxf(mw[0], mw[1]), fmaxf(mw[2], mw[3]));
+        float e = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            e += red[w * kPbP + tid] * expf(2.f * (mw[w] - m));
+        E[((size_t)bh * Cq + p) * Ck + c] = e;
+        mloc[((size_t)bh * Cq + p) * Ck + c] = m;
+    }
 }
 
-__global__ void fill_u32_kernel(uint32_t* p, size_t n, uint32_t v) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (size_t)gridDim.x * blockDim.x)
-        p[i] = v;
+// E_ic <- E_ic e^{2 (m_ic - m_i)} with m_i = max_c m_ic (the maximum over
+// every key of the head: each m_ic is the maximum over cluster c's keys),
+// one warp per probe row; empty clusters (E = 0, m = -inf) stay 0.
+__global__ void probe_rescale_kernel(float* __restrict__ E, const float* __restrict__ mloc, int Ck,
+                                     long long rows) {
+    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float* ml = mloc + row * Ck;
+    float* er = E + row * Ck;
+    float m = -INFINITY;
+    for (int c = lane; c < Ck; c += 32) m = fmaxf(m, ml[c]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int c = lane; c < Ck; c += 32) {
+        const float mc = ml[c];
+        er[c] = mc > -INFINITY ? er[c] * expf(2.f * (mc - m)) : 0.f;
+    }
 }
 
 template <typename T, int D>
 static int probe_impl(const float* qbar, int Cq, const void* Kp, const void* Vp,
                       const float* kbar, const float* vbar, const int32_t* k_off, int Ck,
-                      svgear_dims kd, float scale, float* E, uint32_t* rowmax, float* qT,
+                      svgear_dims kd, float scale, float* E, float* cmax, float* qT,
                       bool value_free, cudaStream_t st) {
     const int BH = kd.B * kd.H, Nk = kd.N;
     const int nPB = ceil_div(Cq, kPbP);
     const size_t nrow = (size_t)BH * Cq;
     probe_qT_kernel<D><<<dim3(nPB, BH), 256, 0, st>>>(qbar, Cq, nPB, qT);
     count_launches(1);
-    fill_u32_kernel<<<ceil_div((long long)nrow, 256) < 1024 ? ceil_div((long long)nrow, 256) : 1024,
-                      256, 0, st>>>(rowmax, nrow, 0x007FFFFFu);  // ordered(-inf)
-    count_launches(1);
-    // row maxima: about four CTAs per SM over all (part, probe block, head)
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return SVGEAR_ERR_CUDA;
-    const long long want = 4LL * sms;
-    int parts = (int)((want + (long long)nPB * BH - 1) / ((long long)nPB * BH));
-    const int max_parts = ceil_div(Nk, kPbK);
-    if (parts > max_parts) parts = max_parts;
-    if (parts < 1) parts = 1;
-    const int keys_per_cta = ceil_div(ceil_div(Nk, parts), kPbK) * kPbK;
-    parts = ceil_div(Nk, keys_per_cta);
     const size_t sm1 = sizeof(float) * ((size_t)D * (kPbP + kPbK) + 4 * kPbP);
-    if (cudaFuncSetAttribute(probe_rowmax_v2_kernel<T, D>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1) != cudaSuccess)
-        return SVGEAR_ERR_CUDA;
-    if (Nk > 0) {
-        probe_rowmax_v2_kernel<T, D><<<dim3(parts, nPB, BH), kPbThreads, sm1, st>>>(
-            qT, Cq, nPB, static_cast<const T*>(Kp), Nk, scale, keys_per_cta, rowmax);
-        count_launches(1);
-    }
     const size_t sm2 = sm1 + sizeof(float) * (2 * D + 2 * kPbK);
     auto kern = value_free ? probe_error_v2_kernel<T, D, true> : probe_error_v2_kernel<T, D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2) !=
         cudaSuccess)
         return SVGEAR_ERR_CUDA;
+    float* mloc = cmax;   // [BH][Cq][Ck]: m_ic, the maximum score of probe i over cluster c
     kern<<<dim3(Ck, nPB, BH), kPbThreads, sm2, st>>>(
         qT, Cq, nPB, static_cast<const T*>(Kp), static_cast<const T*>(Vp), kbar, vbar, k_off, Ck,
-        Nk, scale, rowmax, E);
-    count_launches(1);
+        Nk, scale, mloc, E);
+    probe_rescale_kernel<<<(unsigned)ceil_div((long long)nrow, 8), 256, 0, st>>>(E, mloc, Ck,
+                                                                                (long long)nrow);
+    count_launches(2);
     SVGEAR_LAUNCH_CHECK();
     return SVGEAR_OK;
 }
 
 int launch_probe(const float* qbar, int Cq, const void* Kp, const void* Vp, const float* kbar,
                  const float* vbar, const int32_t* k_off, int Ck, svgear_dims kd, float scale,
-                 float* E, uint32_t* rowmax, float* qT, cudaStream_t st, bool value_free) {
+                 float* E, float* cmax, float* qT, cudaStream_t st, bool value_free) {
     if (kd.dtype == SVGEAR_BF16) {
-        if (kd.d == 128) return probe_impl<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
-        if (kd.d == 64) return probe_impl<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
+        if (kd.d == 128) return probe_impl<__nv_bfloat16, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, cmax, qT, value_free, st);
+        if (kd.d == 64) return probe_impl<__nv_bfloat16, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, cmax, qT, value_free, st);
     } else if (kd.dtype == SVGEAR_F32) {
-        if (kd.d == 128) return probe_impl<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
-        if (kd.d == 64) return probe_impl<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, rowmax, qT, value_free, st);
+        if (kd.d == 128) return probe_impl<float, 128>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, cmax, qT, value_free, st);
+        if (kd.d == 64) return probe_impl<float, 64>(qbar, Cq, Kp, Vp, kbar, vbar, k_off, Ck, kd, scale, E, cmax, qT, value_free, st);
     }
     return SVGEAR_ERR_UNSUPPORTED;
 }

@@ -212,7 +212,10 @@ int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
  * ranking within a row unchanged.  E is 0 for an empty key cluster.  Each
  * term is evaluated expanded around the key's residual w_t = v_t - vbar_c,
  * (a-b)^2 |vbar_c|^2 - 2 (a-b) b vbar_c.w_t + b^2 |w_t|^2 with a = e^{sbar-m},
- * b = e^{s-m} (the same quantity), summed in a fixed order.
+ * b = e^{s-m} (the same quantity), summed in a fixed order.  One pass over
+ * the keys: each cluster's sum is first taken with its own maximum score
+ * m_ic as the shift, and then multiplied by e^{2 (m_ic - m_i)} with
+ * m_i = max_c m_ic (every term is quadratic in e^{-m}).
  *   qbar      float[B][H][Cq][d] query centroids (the probes).
  *   Kp, Vp    [B][H][Nk][d] permuted keys and values (kdims.dtype).
  *   kbar,vbar float[B][H][Ck][d] key and value centroids.
@@ -220,7 +223,8 @@ int svgear_centroids(const void* Xp, const int32_t* offsets, int32_t C,
  *   kdims     shape of Kp (N = Nk).
  *   E         out float[B][H][Cq][Ck].
  *   ws        svgear_workspace_bytes(SVGEAR_OP_ROUTE, kdims, Cq, Ck) (holds the
- *             row maxima and the probes transposed in blocks of 128).
+ *             per-cluster maxima m_ic and the probes transposed in blocks of
+ *             128).
  * ------------------------------------------------------------------------ */
 int svgear_probe(const float* qbar, int32_t Cq, const void* Kp, const void* Vp,
                  const float* kbar, const float* vbar, const int32_t* k_off,
