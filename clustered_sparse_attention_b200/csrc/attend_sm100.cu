@@ -92,6 +92,9 @@ struct Shared {
     uint32_t tmem_base;
     int abort_flag;
     int keep_tmem;
+    // split tiles: each half's running max and row sum, for the merge
+    float xm[kHalves][BM];
+    float xl[kHalves][BM];
 };
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -172,6 +175,13 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     // variance term (the upper 64 columns of S_h then hold q^2 of the half)
     const int CW = use_var ? BN / 2 : BN;
     const int T = T_real + (ncomp + CW - 1) / CW;
+    // Split tile: a tile pair with one 128-row half of query rows would leave
+    // the other half's softmax and MMAs idle, so both halves take the same
+    // rows, half h the key tiles j = h, h+2, h+4, ... (tile j sits in ring
+    // stage j % 2 = h), each with its own online softmax; the epilogue merges
+    // the two.  (Not with the variance term, whose q^2 shares S's columns.)
+    const bool split = nh == 1 && T >= 2 && !use_var;
+    const int hq = split ? 2 : nh;                 // halves that run
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ Shared sh;
@@ -219,8 +229,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
     tc::regs_dec<kIssueRegs>();   // one call site for the whole warpgroup
     if (warp == kKWarp || warp == kVWarp) {
         // ------------------------------------------------------------ producers
-        // Warp 8 fills the K ring (freed once both halves' QK are done), warp 9
-        // the V ring (freed once both halves' PV are done); lane 0 issues TMA.
+        // Warp 8 fills the K ring (a slot is freed once the QK of every half
+        // that reads it is done), warp 9 the V ring (likewise with PV); lane 0
+        // issues TMA.  Tile j goes to slot j % 2 in either mode.
         // A key tile is the next 128 entries of the query cluster's list of
         // selected keys, a concatenation of contiguous key-cluster segments:
         // every run [g, g+n) of rows that falls in the tile is copied with 2-D
@@ -342,7 +353,48 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         constexpr uint32_t kIdescPV = tc::idesc_bf16(BM, D, true);
         if (lane == 0) {
         bool ok_run = wait_bar(&sh.q_full, 0, abort_flag, err, (5 << 16));
-        for (int j = 0; ok_run && j <= T; ++j) {
+        // split tile: step s issues, per half h, PV_h of tile 2(s-1)+h and QK_h
+        // of tile 2s+h (the query tile is half 0's); each tile has one consumer,
+        // so its K and V ring slots are released right after its MMAs
+        for (int s = 0; split && ok_run && 2 * s - 1 <= T; ++s) {
+            for (int h = 0; h < 2; ++h) {
+                const int jp = 2 * (s - 1) + h, jc = 2 * s + h;
+                if (s > 0 && jp < T) {
+                    if (!wait_bar(&sh.v_full[h], (s - 1) & 1, abort_flag, err, (11 << 16) + jp) ||
+                        !wait_bar(&sh.p_full[h], (s - 1) & 1, abort_flag, err, (8 << 16) + (h << 12) + jp)) {
+                        ok_run = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    // every tile is 128 keys deep here (no variance term)
+                    tc::mma_bf16_ts_k128(tmem + kHalves * BN + h * D, tmem + h * BN,
+                                         tc::sw128_desc(sV0 + h * kTileBytes, 16384, 1024), kIdescPV,
+                                         s > 1 ? 1u : 0u);
+                    tc::commit(tc::smem_u32(&sh.v_empty[h]));
+                }
+                if (jc < T) {
+                    if (!wait_bar(&sh.k_full[h], s & 1, abort_flag, err, (6 << 16) + jc)) {
+                        ok_run = false;
+                        break;
+                    }
+                    const uint32_t tK = sK0 + h * kTileBytes;
+                    if (D == 128) {
+                        tc::mma_bf16_k128(tmem + h * BN, tc::sw128_desc(sQ0, 16, 1024),
+                                          tc::sw128_desc(tK, 16, 1024), kIdescQK, 0u);
+                    } else {
+#pragma unroll 1
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            tc::mma_bf16(tmem + h * BN, tc::sw128_desc(sQ0 + off, 16, 1024),
+                                         tc::sw128_desc(tK + off, 16, 1024), kIdescQK, ks > 0);
+                        }
+                    }
+                    tc::commit(tc::smem_u32(&sh.s_full[h]));
+                    tc::commit(tc::smem_u32(&sh.k_empty[h]));
+                }
+            }
+        }
+        for (int j = 0; !split && ok_run && j <= T; ++j) {
             const int st = j % KSTAGES, pst = (j + VSTAGES - 1) % VSTAGES;
             for (int h = 0; h < nh; ++h) {
                 if (j > 0) {
@@ -435,7 +487,8 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
         const uint32_t sO = lane_base + kHalves * BN + h * D;
         const float* cb = comp_bias + row_meta;
         float m_use = -INFINITY, l = 0.f;
-        bool ok_run = h < nh;
+        bool ok_run = h < hq;
+        const int Th = split ? (T - h + 1) / 2 : T;      // this half's tiles
         const bool need_q2 = use_var && ncomp > 0;
         if (ok_run && need_q2) {
             // the Q tile is read from shared memory below: wait for its copy
@@ -448,8 +501,9 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             }
         }
         uint32_t v[BN];
-        for (int j = 0; j < T && ok_run; ++j) {
-            if (!warp_wait_bar(&sh.s_full[h], j & 1, abort_flag, err, (2 << 16) + j)) {
+        for (int jl = 0; jl < Th && ok_run; ++jl) {
+            const int j = split ? 2 * jl + h : jl;       // key tile
+            if (!warp_wait_bar(&sh.s_full[h], jl & 1, abort_flag, err, (2 << 16) + j)) {
                 ok_run = false;
                 break;
             }
@@ -523,10 +577,10 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             // rescales together when any row must (the others with alpha = 1).
             // O_h is final up to PV_h(j-1) here: that MMA was issued before
             // QK_h(j), whose commit completed s_full.
-            const bool need = j > 0 && m_new > m_use + kRescaleThreshold;
+            const bool need = jl > 0 && m_new > m_use + kRescaleThreshold;
             const bool any = __any_sync(0xffffffffu, need);
             float alpha = 1.f;
-            if (j == 0) {
+            if (jl == 0) {
                 m_use = m_new;
             } else if (need) {
                 alpha = tc::ex2(m_use - m_new);
@@ -570,8 +624,50 @@ attend_sm100_kernel(const __grid_constant__ TmaMaps maps, int Nq, int Nk, int Cq
             tc::fence_before_sync();
             tc::mbar_arrive(tc::smem_u32(&sh.p_full[h]));
         }
-        // epilogue: O / l back to the original token order
-        if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
+        if (split) {
+            // Split tile: O = (a0 O_0 + a1 O_1) / (a0 l_0 + a1 l_1), a_h = 2^(m_h - m),
+            // m = max(m_0, m_1).  Both halves trade (m, l) through shared memory
+            // (the named barrier is reached on every path) and each writes half
+            // of the row's columns, reading both partial O from its TMEM lanes.
+            const bool ok = ok_run && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16) + h);
+            sh.xm[h][r] = m_use;
+            sh.xl[h][r] = l;
+            asm volatile("bar.sync 1, %0;" ::"n"(2 * kSoftmaxThreads) : "memory");
+            if (ok && !*abort_flag) {
+                tc::fence_after_sync();
+                const float m0 = sh.xm[0][r], m1 = sh.xm[1][r];
+                const float mm = fmaxf(m0, m1);
+                const float a0 = tc::ex2(m0 - mm), a1 = tc::ex2(m1 - mm);
+                const float inv = 1.f / (a0 * sh.xl[0][r] + a1 * sh.xl[1][r]);
+                const float c0 = a0 * inv, c1 = a1 * inv;
+                const int p = q0 + r;
+                const int dst = p < q_end ? q_perm[(size_t)bh * Nq + p] : -1;
+                bf16* orow = O + head + (size_t)max(dst, 0) * D;
+                const uint32_t sO0 = lane_base + kHalves * BN;
+                uint32_t o0[32], o1[32];
+#pragma unroll
+                for (int c4 = h * D / 64; c4 < (h + 1) * D / 64; ++c4) {
+                    tc::tmem_ld32(sO0 + c4 * 32, o0);
+                    tc::tmem_ld32(sO0 + D + c4 * 32, o1);
+                    tc::tmem_ld_wait();
+                    if ((unsigned)dst < (unsigned)Nq) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            __nv_bfloat162 hp = __floats2bfloat162_rn(
+                                fmaf(__uint_as_float(o0[e]), c0, __uint_as_float(o1[e]) * c1),
+                                fmaf(__uint_as_float(o0[e + 1]), c0, __uint_as_float(o1[e + 1]) * c1));
+                            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&hp);
+                        }
+                        uint4* o4 = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            o4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    }
+                }
+            }
+        } else if (ok_run && T > 0 && warp_wait_bar(&sh.o_full, 0, abort_flag, err, (4 << 16))) {
+            // epilogue: O / l back to the original token order
             tc::fence_after_sync();
             const int p = q0 + h * BM + r;
             const float inv = 1.f / l;

@@ -1,6 +1,7 @@
 """The two 720p layers at full size, run through the C ABI exactly as bench.py
 times them -- Wan 2.1 (B=1, H=40, N=75600) and HunyuanVideo (B=1, H=24,
-N=118800), both d=128, Cq=100, Ck=500, 40 rounds, density 0.25 -- then
+N=118800), both d=128, Cq=100, Ck=500, 40 rounds, density 0.25, and the Wan
+shape at the SVG-EAR paper's cluster counts (Cq=300, Ck=1000) -- then
 checked against the oracle on what the oracle can compute one piece at a
 time: sampled heads for the sort, means and routing (whole heads), sampled
 tokens for the assignment, sampled query clusters for the probe and sampled
@@ -20,8 +21,10 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-# sampled heads of each shape: first, one inside, last
-SHAPES = {"wan720p": (0, 17, 39), "hunyuan720p": (0, 11, 23)}
+# sampled heads of each workload: first, one inside, last.  The third is the
+# Wan shape at the SVG-EAR paper's cluster counts (300 query, 1000 key
+# clusters): query clusters of ~250 rows, 1000 k-means++ seeds.
+SHAPES = {"wan720p": (0, 17, 39), "hunyuan720p": (0, 11, 23), "wan720p_q300_k1000": (0, 23, 39)}
 
 
 def _rel_l2(a, b):
@@ -70,7 +73,7 @@ def test_fullsize_kmeanspp_follows_the_oracle_on_one_head(run):
     diff = np.nonzero(own != idx)[0]
     for j in diff:
         assert margin[j] < band, (j, idx[j], own[j], margin[j])
-    assert len(diff) <= 3
+    assert len(diff) <= max(3, W.Ck // 200)   # every flip is inside the band (above)
     assert np.array_equal(cent.cpu().numpy()[0, h], X[idx])
 
 
@@ -108,7 +111,7 @@ def test_fullsize_assignment_on_sampled_tokens(run):
         tok = np.sort(g.choice(W.N, 6000, replace=False))
         X = run["host"]("k", h)
         flips += check_assign(X[tok], cents[0, h], lab[0, h][tok])
-    assert flips <= 6
+    assert flips <= 12   # 0.07 % of the sampled tokens; each one inside the band (check_assign)
 
 
 def test_fullsize_probe_on_sampled_query_clusters(run):
