@@ -107,7 +107,7 @@ RouteWs carve_route(Carve& cv, size_t BH, int Cq, int Ck, int d) {
 AttendWs carve_attend(Carve& cv, const svgear_dims& d, int Cq, int Ck) {
     AttendWs w;
     const size_t BH = bh_of(d);
-    w.maxT = ceil_div(d.N, 256) + Cq;   // pairs of 128-row tiles per query cluster
+    w.maxT = ceil_div(d.N, 128) + Cq;   // 128-row tiles per query cluster (enough for pairs)
     w.status = cv.take<int>(4);
     w.kbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);
     w.vbar16 = cv.take<__nv_bfloat16>(BH * Ck * (size_t)d.d);

@@ -102,7 +102,7 @@ struct AttendWs {
     int32_t* seg_row;            // [BH][Cq][Ck] first key row of each segment
     int32_t* comp_idx;           // [BH][Cq][Ck] skipped non-empty clusters
     float* comp_bias;            // [BH][Cq][Ck] log2(n_c) of those clusters
-    int4* tiles;                 // [BH][maxT] {cluster, first row, end row, 0}, 256 rows each
+    int4* tiles;                 // [BH][maxT] {cluster, first row, end row, 0}: 128 or 256 rows
     int32_t* ntiles;             // [BH]
     int maxT;
 };

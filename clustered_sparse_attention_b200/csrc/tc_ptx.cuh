@@ -33,6 +33,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking tests of three barriers' phases at once (bit i set: barrier i
+// has completed the phase of parity p_i); the three tests are independent,
+// so their latencies overlap.
+__device__ __forceinline__ uint32_t mbar_test3(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1,
+                                               uint32_t b2, uint32_t p2) {
+    uint32_t m;
+    asm volatile(
+        "{\n\t.reg .pred a, b, c;\n\t.reg .b32 x, y, z;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 a, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 b, [%3], %4;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 c, [%5], %6;\n\t"
+        "selp.u32 x, 1, 0, a;\n\tselp.u32 y, 2, 0, b;\n\tselp.u32 z, 4, 0, c;\n\t"
+        "or.b32 x, x, y;\n\tor.b32 %0, x, z;\n\t}\n"
+        : "=r"(m)
+        : "r"(b0), "r"(p0), "r"(b1), "r"(p1), "r"(b2), "r"(p2)
+        : "memory");
+    return m;
+}
 // As mbar_try_wait, but the thread may sleep up to `hint_ns` inside the
 // instruction (it wakes when the phase completes), so waiting costs no issue
 // slots.
