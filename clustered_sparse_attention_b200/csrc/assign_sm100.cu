@@ -15,14 +15,22 @@
 // depth 2d sums x.h + x.m, whose products are exact; for d = 128 split and
 // accumulation together bound the error by the same 1.5 * 2^-16 sum_k
 // |x_k c_k| as an exact three-plane split accumulated over depth 3d, for a
-// third fewer MMAs and plane bytes.  |c|^2 is taken from the fp32 centroid.
+// third fewer MMAs and plane bytes.
+//
+// The norm is folded into the contraction: one more K=16 step multiplies a
+// tile of ones by the centroid's -|c|^2/2 (from the fp32 centroid, split into
+// three bf16 parts, which hold it to 2^-24), so the accumulator holds
+// x.c - |c|^2/2 and the token's label is the column of its maximum.  The
+// step adds three exact products to the fp32 chain; with the planes, the
+// distance -2(x.c - |c|^2/2) errs by at most 2 (2^-17 + (2d+3) u) sum_k
+// |x_k c_k| + (3d+5) u |c|^2 against |x - c|^2 - |x|^2.
 //
 // B200 design: persistent CTAs, one per SM, walk the 128-token tiles of all
 // heads (tiles of heads at their fixed point are skipped).  Centroid planes
 // stay in shared memory: all of a head's when they fit (each tile then runs
 // every chunk), else one chunk's at a time, run against a group of up to
 // kGroupTiles token tiles of the head before the next chunk's planes replace
-// them (each token's running minimum is carried from chunk to chunk).
+// them (each token's running maximum is carried from chunk to chunk).
 //   warp 0     TMA producer: the token tile (2 to 4 stages, as shared memory
 //              allows) and, when the plane set changes, its boxes of Nc rows
 //              x 64 dims (128B-swizzled);
@@ -30,10 +38,10 @@
 //              of two TMEM accumulators, each centroid chunk a chain of
 //              2 planes x d/16 steps;
 //   warps 2-9  epilogue, two warps per TMEM lane quarter (TMEM lane = token
-//              row), each scanning half of every chunk's columns:
-//              dist = |c|^2 - 2 s, running (dist, index) minimum; the upper
-//              half hands its minimum to the lower through shared memory,
-//              which merges (ties to the lower index) and writes the label.
+//              row), each scanning half of every chunk's columns for the
+//              running (x.c - |c|^2/2, index) maximum; the upper half hands
+//              its maximum to the lower through shared memory, which merges
+//              (ties to the lower index) and writes the label.
 // Every wait is bounded (tc_wait.cuh); on expiry the status word records
 // SVGEAR_ERR_TIMEOUT, copies and MMAs in flight are drained and the CTA
 // returns.
@@ -61,11 +69,14 @@ constexpr int kEpiThreads = 256;
 constexpr uint32_t kTmemCols = 512;      // two accumulators of up to 256 columns
 constexpr uint32_t kAccCols = 256;
 constexpr int kMaxAStages = 4;           // token-tile stages: as many as shared memory holds
+constexpr int kNormK = 16;               // the norm step's K: -|c|^2/2 in 3 bf16 parts, then zeros
+constexpr uint32_t kOnesBytes = BM * kNormK * 2;   // the norm step's A: 128 x 16 bf16 ones
 constexpr uint64_t kDrainNs = 200000000ull;    // 0.2 s to let issued work land
 
 struct Maps {
     CUtensorMap x;   // tokens [B*H*N][D], boxes of 128 rows x 64
     CUtensorMap b;   // centroid planes [B*H][2][Cpad][D], boxes of Nc rows x 64
+    CUtensorMap n;   // norm steps [B*H][Cpad][16], boxes of Nc rows x 16 (32-byte swizzle)
 };
 
 struct Shared {
@@ -78,7 +89,7 @@ struct Shared {
     uint64_t drain;
     uint64_t pair_full[4][2];    // per lane quarter and slot: the upper half's minimum is stored
     uint64_t pair_empty[4][2];   // the lower half has read it
-    float pair_d[2][BM];         // the upper half's running minimum, double-buffered by tile
+    float pair_d[2][BM];         // the upper half's running maximum, double-buffered by tile
     uint16_t pair_i[2][BM];      // and its centroid index (C <= SVGEAR_MAX_CLUSTERS)
     uint32_t tmem_base;
     int abort_flag;
@@ -98,8 +109,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, int Nc, int nA,
-                    int nB, int resident, int G,
-                    const float* __restrict__ cnorm, int32_t* __restrict__ labels,
+                    int nB, int resident, int G, int32_t* __restrict__ labels,
                     const int32_t* __restrict__ done, int32_t* __restrict__ changed,
                     int* __restrict__ err, int* __restrict__ lost) {
     constexpr int KH = D / 64;                   // 64-dim halves of a row
@@ -112,7 +122,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     // chunk's planes form one set per head, and each tile runs all chunks.
     // Grouped: a unit is up to G tiles of one head, a set is one chunk's
     // planes, and the unit's tiles run chunk by chunk (one phase per chunk),
-    // carrying each token's running minimum from phase to phase.
+    // carrying each token's running maximum from phase to phase.
     if (resident || G < 1) G = 1;
     if (G > kMaxGroup) G = kMaxGroup;
     const int units_per_head = (tiles_per_head + G - 1) / G;
@@ -126,8 +136,16 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     const uint32_t sA0 = base;
     const uint32_t sB0 = base + nA * kABytes;
     const uint32_t kBStageBytes = (uint32_t)Nc * 128u;   // Nc rows x 64 bf16 (multiple of 2 KB)
+    const uint32_t kNStageBytes = (uint32_t)Nc * 32u;    // Nc rows x 16 bf16 (multiple of 512 B)
+    const uint32_t sN0 = sB0 + nB * kBStageBytes;        // norm steps of the set's chunks
+    const uint32_t sOnes = sN0 + chunks_per_step * kNStageBytes;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the norm step's A operand: bf16 ones in every element (so in any layout)
+    for (uint32_t o = (uint32_t)tid * 16u; o < kOnesBytes; o += kThreads * 16u)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sOnes + o), "r"(0x3F803F80u)
+                     : "memory");
+    tc::fence_async_smem();   // visible to the tensor core
     if (tid == 0) {
         for (int s = 0; s < kMaxAStages; ++s) {
             tc::mbar_init(tc::smem_u32(&sh.a_full[s]), 1);
@@ -164,6 +182,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         if (lane == 0) {
             tc::prefetch_tmap(&maps.x);
             tc::prefetch_tmap(&maps.b);
+            tc::prefetch_tmap(&maps.n);
         }
         int ia = 0;
         int loaded = -1, hc = 0;   // plane set in the slots, plane-set changes
@@ -203,15 +222,19 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                         }
                         if (lane == 0) {
                             const uint32_t bar = tc::smem_u32(&sh.b_full);
-                            tc::mbar_arrive_expect_tx(bar, (uint32_t)(nB * Nc * 128));
+                            tc::mbar_arrive_expect_tx(
+                                bar, (uint32_t)(nB * Nc * 128 + chunks_per_step * Nc * kNormK * 2));
                             const int c0 = resident ? 0 : ph;
-                            for (int c = 0; c < chunks_per_step; ++c)
+                            for (int c = 0; c < chunks_per_step; ++c) {
                                 for (int p = 0; p < kPlanes; ++p)
 #pragma unroll
                                     for (int kh = 0; kh < KH; ++kh)
                                         tc::tma_load_2d(sB0 + ((c * kPlanes + p) * KH + kh) * kBStageBytes,
                                                         &maps.b, kh * 64,
                                                         (bh * kPlanes + p) * Cpad + (c0 + c) * Nc, bar);
+                                tc::tma_load_2d(sN0 + c * kNStageBytes, &maps.n, 0, bh * Cpad + (c0 + c) * Nc,
+                                                bar);
+                            }
                         }
                         __syncwarp();
                         loaded = set;
@@ -235,6 +258,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         // operations; the warp meets again after the drain), so no warp
         // barrier makes it wait for the tensor core to take its queued MMAs.
         const uint32_t idesc = tc::idesc_bf16(BM, Nc, false);
+        const uint64_t ones_desc = tc::sw32_desc(sOnes, 256);
         if (lane == 0) {
         int ia = 0, ic = 0;
         int cur = -1, hc = 0;   // plane set in use, plane-set changes
@@ -283,6 +307,9 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                                     tc::mma_bf16(tmem + buf * kAccCols, ad0 + 2 * ks, bd0 + 2 * ks, idesc,
                                                  (p | kh | ks) != 0 ? 1u : 0u);
                             }
+                        // + ones . (-|c|^2/2 parts)
+                        tc::mma_bf16(tmem + buf * kAccCols, ones_desc,
+                                     tc::sw32_desc(sN0 + c * kNStageBytes, 256), idesc, 1u);
                         tc::commit(tc::smem_u32(&sh.acc_full[buf]));
                         ++ic;
                     }
@@ -314,7 +341,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
         const int s_lo = upper ? (nsteps + 1) / 2 : 0;
         const int s_hi = upper ? nsteps : (nsteps + 1) / 2;
         int it = 0;   // tiles handed over, for the slot and its phase
-        // running minimum of this thread's token in each tile of a unit,
+        // running maximum of this thread's token in each tile of a unit,
         // carried from one phase to the next (grouped units)
         float carry_d[kMaxGroup];
         int carry_i[kMaxGroup];
@@ -325,7 +352,6 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
             if (done && done[bh]) continue;
             const int tlo = (u - bh * units_per_head) * G;
             const int thi = min(tlo + G, tiles_per_head);
-            const float* cn = cnorm + (size_t)bh * Cpad;
             for (int ph = 0; ok && ph < phases; ++ph) {
                 const bool last = ph == phases - 1;
                 for (int ti = tlo; ok && ti < thi; ++ti) {
@@ -333,26 +359,25 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                     int32_t* lp = labels + (size_t)bh * N + t;
                     // the previous label, loaded now and compared once the tile is done
                     const int old = (last && changed && !upper && t < N) ? *lp : -1;
-                    // four interleaved running minima (columns e mod 4), merged with
-                    // ties to the lower index: the first minimum of the sequential scan
+                    // four interleaved running maxima of x.c - |c|^2/2 (columns e mod
+                    // 4), merged with ties to the lower index: the first maximum of the
+                    // sequential scan
                     float best[4];
                     int bi[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        best[e] = __int_as_float(0x7f800000);
+                        best[e] = __int_as_float(0xff800000);
                         bi[e] = 0;
                     }
-                    auto scan = [&](const uint32_t* v, int nq, int base, const float* cnc) {
+                    auto scan = [&](const uint32_t* v, int nq, int base) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             if (q < nq) {
-                                const float4 n4 = __ldg(reinterpret_cast<const float4*>(cnc) + q);
-                                const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    const float dist = fmaf(-2.f, __uint_as_float(v[4 * q + e]), nn[e]);
-                                    if (dist < best[e]) {
-                                        best[e] = dist;
+                                    const float sc = __uint_as_float(v[4 * q + e]);
+                                    if (sc > best[e]) {
+                                        best[e] = sc;
                                         bi[e] = base + 4 * q + e;
                                     }
                                 }
@@ -376,18 +401,18 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                         for (int k = s_lo; k < hi_full; k += 2) {
                             tc::tmem_ld_wait();
                             if (k + 1 < hi_full) tc::tmem_ld32(tb + (k + 1) * 32, vb);
-                            scan(va, 8, cb + k * 32, cn + cb + k * 32);
+                            scan(va, 8, cb + k * 32);
                             if (k + 1 < hi_full) {
                                 tc::tmem_ld_wait();
                                 if (k + 2 < hi_full) tc::tmem_ld32(tb + (k + 2) * 32, va);
-                                scan(vb, 8, cb + (k + 1) * 32, cn + cb + (k + 1) * 32);
+                                scan(vb, 8, cb + (k + 1) * 32);
                             }
                         }
                         if ((Nc & 16) && s_hi == nsteps && s_lo <= nfull) {   // the 16-column step
                             uint32_t v16[16];
                             tc::tmem_ld16(tb + nfull * 32, v16);
                             tc::tmem_ld_wait();
-                            scan(v16, 4, cb + nfull * 32, cn + cb + nfull * 32);
+                            scan(v16, 4, cb + nfull * 32);
                         }
                         // the accumulator is in registers: the MMA may refill it
                         tc::fence_before_sync();
@@ -399,11 +424,11 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                     int bx = bi[0];
 #pragma unroll
                     for (int e = 1; e < 4; ++e)
-                        if (best[e] < bb || (best[e] == bb && bi[e] < bx)) {
+                        if (best[e] > bb || (best[e] == bb && bi[e] < bx)) {
                             bb = best[e];
                             bx = bi[e];
                         }
-                    // the upper half hands its minimum to the lower half of the same rows
+                    // the upper half hands its maximum to the lower half of the same rows
                     const int slot = it & 1;
                     const uint32_t use = (uint32_t)(it >> 1);
                     ++it;
@@ -427,7 +452,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                         const float ud = sh.pair_d[slot][r];
                         const int ux = sh.pair_i[slot][r];
                         tc::mbar_arrive(tc::smem_u32(&sh.pair_empty[quarter][slot]));
-                        if (ud < bb || (ud == bb && ux < bx)) {
+                        if (ud > bb || (ud == bb && ux < bx)) {
                             bb = ud;
                             bx = ux;
                         }
@@ -435,7 +460,7 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
                     if (ph > 0) {
                         // earlier phases hold lower indices: they keep ties
                         const int g = ti - tlo;
-                        if (!(bb < carry_d[g])) {
+                        if (!(bb > carry_d[g])) {
                             bb = carry_d[g];
                             bx = carry_i[g];
                         }
@@ -457,12 +482,14 @@ assign_sm100_kernel(const __grid_constant__ Maps maps, int N, int BH, int Cpad, 
     if (warp == kMmaWarp && !sh.keep_tmem) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Centroid planes and norms, one warp per centroid: planes[bh][p][c][k] for
-// p = hi, lo; padding rows (c >= C) are zero with norm +inf, so they
-// never win the minimum.
+// Centroid planes and norm steps, one warp per centroid: planes[bh][p][c][k]
+// for p = hi, lo, and nstep[bh][c][0..2] = -|c|^2/2 as three bf16 parts (each
+// the rounding of what the previous ones leave, exact in fp32), zeros after;
+// padding rows (c >= C) have zero planes and -1e30 in the norm step, so they
+// never win the maximum.
 template <int D>
 __global__ void centroid_planes_kernel(const float* __restrict__ cent, int C, int Cpad,
-                                       bf16* __restrict__ planes, float* __restrict__ cnorm,
+                                       bf16* __restrict__ planes, bf16* __restrict__ nstep,
                                        const int32_t* __restrict__ done) {
     const int bh = blockIdx.y;
     if (done && done[bh]) return;
@@ -482,7 +509,15 @@ __global__ void centroid_planes_kernel(const float* __restrict__ cent, int C, in
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) cnorm[(size_t)bh * Cpad + c] = c < C ? s : __int_as_float(0x7f800000);
+    if (lane < kNormK) {
+        const float n = c < C ? -0.5f * s : -1e30f;
+        const bf16 p0 = __float2bfloat16_rn(n);
+        const float n1 = n - __bfloat162float(p0);
+        const bf16 p1 = __float2bfloat16_rn(n1);
+        const bf16 p2 = __float2bfloat16_rn(n1 - __bfloat162float(p1));
+        const bf16 z = __float2bfloat16_rn(0.f);
+        nstep[((size_t)bh * Cpad + c) * kNormK + lane] = lane == 0 ? p0 : lane == 1 ? p1 : lane == 2 ? p2 : z;
+    }
 }
 
 // Centroid chunking: as few chunks as possible of at most 256 columns, each a
@@ -499,7 +534,7 @@ size_t assign_sm100_scratch_bytes(int BH, int C, int D) {
     int nchunk, Nc;
     asg::chunking(C, &nchunk, &Nc);
     const size_t Cpad = (size_t)nchunk * Nc;
-    return (size_t)BH * Cpad * (asg::kPlanes * D * sizeof(__nv_bfloat16) + sizeof(float));
+    return (size_t)BH * Cpad * (asg::kPlanes * D + asg::kNormK) * sizeof(__nv_bfloat16);
 }
 
 int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int C,
@@ -515,10 +550,11 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
     chunking(C, &nchunk, &Nc);
     const int Cpad = nchunk * Nc;
     bf16* planes = static_cast<bf16*>(scratch);
-    float* cn = reinterpret_cast<float*>(planes + (size_t)BH * kPlanes * Cpad * D);
+    bf16* nstep = planes + (size_t)BH * kPlanes * Cpad * D;
     Maps maps;
     if (!make_rows_map(&maps.x, X, (uint64_t)BH * N, D, BM) ||
-        !make_rows_map(&maps.b, planes, (uint64_t)BH * kPlanes * Cpad, D, (uint32_t)Nc))
+        !make_rows_map(&maps.b, planes, (uint64_t)BH * kPlanes * Cpad, D, (uint32_t)Nc) ||
+        !make_k16_map(&maps.n, nstep, (uint64_t)BH * Cpad, (uint32_t)Nc))
         return SVGEAR_ERR_CUDA;
     static int num_sms[64] = {};
     int dev = 0;
@@ -527,42 +563,45 @@ int launch_assign_sm100(const void* X, svgear_dims dims, const float* cent, int 
         cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SVGEAR_ERR_CUDA;
     const int tiles = BH * ceil_div(N, BM);
-    // Shared memory: the plane slots, then as many token-tile stages as fit
-    // (2 to kMaxAStages).  All of a head's planes stay resident when they fit
-    // beside two token stages; otherwise one chunk's planes are resident per
-    // phase of a group of kGroupTiles tiles.
+    // Shared memory: the plane slots (with each chunk's norm step) and the
+    // ones tile, then as many token-tile stages as fit (2 to kMaxAStages).
+    // All of a head's planes stay resident when they fit beside two token
+    // stages; otherwise one chunk's planes are resident per phase of a group
+    // of kGroupTiles tiles.
     const size_t a_bytes = (size_t)(D / 64) * 16384, b_stage = (size_t)Nc * 128;
+    const size_t n_stage = (size_t)Nc * kNormK * 2;
     // the static Shared block is placed before the 1024-aligned dynamic block
     const size_t static_bytes = (sizeof(Shared) + 1023) / 1024 * 1024;
     const size_t budget = 227 * 1024 - static_bytes - 1024;
     const int boxes_head = nchunk * kPlanes * (D / 64);
-    const int resident = budget >= 2 * a_bytes + (size_t)boxes_head * b_stage ? 1 : 0;
+    const int resident =
+        budget >= 2 * a_bytes + (size_t)boxes_head * b_stage + nchunk * n_stage + kOnesBytes ? 1 : 0;
     const int nB = resident ? boxes_head : kPlanes * (D / 64);
-    if (budget < 2 * a_bytes + (size_t)nB * b_stage) return SVGEAR_ERR_UNSUPPORTED;
+    const size_t b_bytes = (size_t)nB * b_stage + (resident ? nchunk : 1) * n_stage + kOnesBytes;
+    if (budget < 2 * a_bytes + b_bytes) return SVGEAR_ERR_UNSUPPORTED;
     const int G = resident ? 1 : (kGroupTiles < kMaxGroup ? kGroupTiles : kMaxGroup);
     const int units = resident ? tiles : BH * ceil_div(ceil_div(N, BM), G);
     const int grid = units < num_sms[dev] ? units : num_sms[dev];
-    const size_t b_bytes = (size_t)nB * b_stage;
     int nA = (int)((budget - b_bytes) / a_bytes);
     if (nA > kMaxAStages) nA = kMaxAStages;
     const size_t smem = (size_t)nA * a_bytes + b_bytes + 1024;
     if (D == 128) {
         centroid_planes_kernel<128><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
-                                                                                cn, done);
+                                                                                nstep, done);
         count_launches(1);
         if (cudaFuncSetAttribute(assign_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
+        assign_sm100_kernel<128><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, labels,
                                                                done, changed, err, lost);
     } else {
         centroid_planes_kernel<64><<<dim3(ceil_div(Cpad, 8), BH), 256, 0, st>>>(cent, C, Cpad, planes,
-                                                                               cn, done);
+                                                                               nstep, done);
         count_launches(1);
         if (cudaFuncSetAttribute(assign_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SVGEAR_ERR_CUDA;
-        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, cn, labels,
+        assign_sm100_kernel<64><<<grid, kThreads, smem, st>>>(maps, N, BH, Cpad, Nc, nA, nB, resident, G, labels,
                                                               done, changed, err, lost);
     }
     count_launches(1);

@@ -314,6 +314,16 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
     d |= (uint64_t)2 << 61;
     return d;
 }
+// The same for an operand laid out by TMA with the 32-byte swizzle: rows of
+// 32 bytes (K = 16 bf16), K-major, 8-row groups sbo_bytes (256) apart.
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr, uint32_t sbo_bytes) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;   // leading byte offset: unused for a swizzled K-major operand
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)6 << 61;
+    return d;
+}
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A
 // K-major, B K-major or MN-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
