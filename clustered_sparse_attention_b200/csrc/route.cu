@@ -40,6 +40,7 @@ namespace svgear {
 constexpr int kPbP = 128;        // probes per block
 constexpr int kPbK = 64;         // keys per tile
 constexpr int kPbThreads = 128;
+static_assert(kPbThreads == kPbP, "one thread per probe of a block (the centroid scores)");
 
 // qT[bh][blk][k][p] = qbar[bh][blk * 128 + p][k] (0 past Cq)
 template <int D>
@@ -144,12 +145,19 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
     // before they are added, and a last kernel brings E to the row maximum
     // m_i = max_c m_ic: E(m) = e^{2 (m' - m)} E(m'), every term being
     // quadratic in (e^{sbar - m}, e^{s - m}).
+    // the centroid's score of every probe, once per probe (thread p takes
+    // probe p; the same sequential sum as the plain form), read back by the
+    // eight threads that share each probe
+    {
+        float dotk = 0.f;
+        for (int k = 0; k < D; ++k) dotk = fmaf(Qs[k * kPbP + tid], kb[k], dotk);
+        red[tid] = scale * dotk;
+    }
+    __syncthreads();
     float ai[8], mi[8], sbar[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        float dotk = 0.f;
-        for (int k = 0; k < D; ++k) dotk = fmaf(Qs[k * kPbP + pb_probe(pi, i)], kb[k], dotk);
-        sbar[i] = scale * dotk;
+        sbar[i] = red[pb_probe(pi, i)];
         mi[i] = sbar[i];   // the centroid's score (the mean of the members' scores) starts it
         ai[i] = 1.f;
     }
