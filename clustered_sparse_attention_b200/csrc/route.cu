@@ -80,7 +80,9 @@ __device__ __forceinline__ void pb_load_k(const T* __restrict__ Kh, int t0, int 
     }
 }
 
-template <int D>
+// NJ = 8: all of the thread's keys; NJ = 4: only keys 4ki..4ki+3 (a tile with
+// at most 32 keys, whose upper half is padding; acc[][4..7] stay zero)
+template <int D, int NJ>
 __device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int pi, int ki,
                                           float (&acc)[8][8]) {
 #pragma unroll
@@ -92,13 +94,14 @@ __device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int 
         const float4 qa = *reinterpret_cast<const float4*>(Qs + k * kPbP + pi * 4);
         const float4 qb = *reinterpret_cast<const float4*>(Qs + k * kPbP + 64 + pi * 4);
         const float4 ka = *reinterpret_cast<const float4*>(Ks + k * kPbK + ki * 4);
-        const float4 kb = *reinterpret_cast<const float4*>(Ks + k * kPbK + 32 + ki * 4);
+        float4 kb = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (NJ == 8) kb = *reinterpret_cast<const float4*>(Ks + k * kPbK + 32 + ki * 4);
         const float q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(q[i], kk[j], acc[i][j]);
+            for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(q[i], kk[j], acc[i][j]);
     }
 }
 __device__ __forceinline__ int pb_probe(int pi, int i) { return pi * 4 + (i & 3) + (i >> 2) * 64; }
@@ -201,7 +204,10 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
         }
         __syncthreads();
         float acc[8][8];
-        pb_scores<D>(Qs, Ks, pi, ki, acc);
+        if (a1 - t0 <= kPbK / 2)
+            pb_scores<D, 4>(Qs, Ks, pi, ki, acc);   // a tail of at most 32 keys
+        else
+            pb_scores<D, 8>(Qs, Ks, pi, ki, acc);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float tmx = -INFINITY;
