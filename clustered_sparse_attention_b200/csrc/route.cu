@@ -81,8 +81,10 @@ __device__ __forceinline__ void pb_load_k(const T* __restrict__ Kh, int t0, int 
 }
 
 // NJ = 8: all of the thread's keys; NJ = 4: only keys 4ki..4ki+3 (a tile with
-// at most 32 keys, whose upper half is padding; acc[][4..7] stay zero)
-template <int D, int NJ>
+// at most 32 keys, whose upper half is padding).  NI likewise for the probes:
+// NI = 4 takes only probes 4pi..4pi+3 (a probe block with at most 64 probes).
+// Skipped entries stay zero.
+template <int D, int NI, int NJ>
 __device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int pi, int ki,
                                           float (&acc)[8][8]) {
 #pragma unroll
@@ -92,14 +94,15 @@ __device__ __forceinline__ void pb_scores(const float* Qs, const float* Ks, int 
 #pragma unroll 2
     for (int k = 0; k < D; ++k) {
         const float4 qa = *reinterpret_cast<const float4*>(Qs + k * kPbP + pi * 4);
-        const float4 qb = *reinterpret_cast<const float4*>(Qs + k * kPbP + 64 + pi * 4);
+        float4 qb = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (NI == 8) qb = *reinterpret_cast<const float4*>(Qs + k * kPbP + 64 + pi * 4);
         const float4 ka = *reinterpret_cast<const float4*>(Ks + k * kPbK + ki * 4);
         float4 kb = make_float4(0.f, 0.f, 0.f, 0.f);
         if (NJ == 8) kb = *reinterpret_cast<const float4*>(Ks + k * kPbK + 32 + ki * 4);
         const float q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < NI; ++i)
 #pragma unroll
             for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(q[i], kk[j], acc[i][j]);
     }
@@ -126,6 +129,9 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
     float* be = al + kPbK;           // [64] |w_t|^2
     const int c = blockIdx.x, blk = blockIdx.y, bh = blockIdx.z, tid = threadIdx.x;
     const int pi = tid & 15, ki = tid >> 4, lane = tid & 31, warp = tid >> 5;
+    // the last probe block holds at most 64 probes: probes 64.. of the block
+    // (the upper four of each thread's eight) are padding
+    const bool half = Cq - blk * kPbP <= kPbP / 2;
     const int32_t* off = k_off + (size_t)bh * (Ck + 1);
     const int a0 = off[c], a1 = off[c + 1];
     if (a1 <= a0 || a0 < 0 || a1 > Nk) {   // empty (or malformed) key cluster: no error
@@ -204,10 +210,11 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
         }
         __syncthreads();
         float acc[8][8];
-        if (a1 - t0 <= kPbK / 2)
-            pb_scores<D, 4>(Qs, Ks, pi, ki, acc);   // a tail of at most 32 keys
+        const bool tail = a1 - t0 <= kPbK / 2;   // a tail of at most 32 keys
+        if (half)
+            tail ? pb_scores<D, 4, 4>(Qs, Ks, pi, ki, acc) : pb_scores<D, 4, 8>(Qs, Ks, pi, ki, acc);
         else
-            pb_scores<D, 8>(Qs, Ks, pi, ki, acc);
+            tail ? pb_scores<D, 8, 4>(Qs, Ks, pi, ki, acc) : pb_scores<D, 8, 8>(Qs, Ks, pi, ki, acc);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float tmx = -INFINITY;
@@ -231,6 +238,7 @@ probe_error_v2_kernel(const float* __restrict__ qT, int Cq, int nPB, const T* __
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
+                if (half && i >= 4) continue;   // padding probes of a half block
                 const float b = expf(scale * acc[i][j] - mi[i]);
                 const float dab = ai[i] - b;
                 if (VF) {
