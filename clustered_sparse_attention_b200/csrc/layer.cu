@@ -165,14 +165,17 @@ int run_layer(const void* Q, const void* K, const void* V, svgear_dims dims,
 // work already on `st` (an earlier call may still read this workspace); the
 // call's streams and events are released once their work is done.
 struct HostPipeline {
-    static constexpr int kQGroups = 2, kOGroups = 4;
-    static constexpr int kMinHeadsPerGroup = 8;
+    // Q parts: each clusters at least 8 heads (k-means++ of fewer heads is
+    // bound by its per-seed latency); O parts: the smaller the last one, the
+    // less of O crosses the host link with nothing to overlap
+    static constexpr int kQGroups = 2, kOGroups = 8;
+    static constexpr int kMinHeadsQ = 8, kMinHeadsO = 4;
     cudaStream_t xs = nullptr, ds = nullptr;
     cudaEvent_t entry = nullptr, done_d2h = nullptr, k_ready = nullptr, v_ready = nullptr;
     cudaEvent_t q_ready[kQGroups] = {}, o_ready[kOGroups] = {};
 
-    static int groups(int BH, int want) {
-        int g = BH / kMinHeadsPerGroup;
+    static int groups(int BH, int want, int min_heads) {
+        int g = BH / min_heads;
         return g < 1 ? 1 : (g > want ? want : g);
     }
     // heads [lo, hi) of group g of G over BH (contiguous, sizes within one)
@@ -215,7 +218,7 @@ struct HostPipeline {
         const size_t head_bytes = (size_t)N * D * esz, tb = tensor_bytes(dims);
         float* cent_q = cq_out ? cq_out : w.cent_q;
         float* cent_k = ck_out ? ck_out : w.cent_k;
-        const int GQ = groups(BH, kQGroups), GO = groups(BH, kOGroups);
+        const int GQ = groups(BH, kQGroups, kMinHeadsQ), GO = groups(BH, kOGroups, kMinHeadsO);
         auto sub = [&](int lo, int hi) {   // dims of the flattened heads [lo, hi)
             svgear_dims d = dims;
             d.B = 1;
