@@ -153,8 +153,7 @@ def test_fullsize_attention_on_sampled_rows(run):
     for h in HEADS[:2]:
         qo = q_off[0, h]
         # the first and last row of every 128-row tile of four query clusters
-        # (both halves of each tile pair and the partial last tile) plus
-        # random rows
+        # (every CTA's tile, the partial last one included) plus random rows
         rows = set(g.choice(W.N, 32, replace=False).tolist())
         for i in (0, 1, W.Cq // 2, W.Cq - 1):
             a, b = int(qo[i]), int(qo[i + 1])

@@ -585,6 +585,14 @@ def test_invalid_arguments_are_rejected_before_launch():
     ([64, 64], [5] * 300, [list(range(0, 300, 2)), []]),   # 3 compensation tiles
     ([128], [128, 128, 128], [[0, 1, 2]], "spiky"),    # half the rows rescale O mid-row
     ([256], [100, 60, 200], [[2], [0]], "spiky"),
+    # one key tile of 60 keys, no compensation: the upper 64-key half of the
+    # tile never holds a key (its softmax state stays empty and merges as zero)
+    ([100], [10, 50], [[0, 1]]),
+    # 20 keys and one compensated cluster: both tiles only in the lower half
+    ([130], [20, 30], [[0]]),
+    # 40 keys, then 100 compensated singletons: the upper half meets its first
+    # valid column in the second tile, with nothing summed before it
+    ([128], [40] + [1] * 100, [[0]]),
 ])
 def test_attend_kernel_on_handmade_layouts(D, case):
     """The attention kernel alone on hand-built segments and pair lists,
