@@ -149,14 +149,16 @@ int svgear_kmeanspp_init(const void* X, svgear_dims dims, int32_t C, uint64_t se
                          size_t ws_bytes, void* stream);
 
 /* k-means assignment: labels[t] = argmin_c |x_t - c|^2, lowest c on exact
- * ties, evaluated as |c|^2 - 2 x.c with fp32-grade dot products: f32 tokens
- * by fp32 FMAs; bf16 tokens on the tensor cores, the fp32 centroid split into
- * two bf16 planes (hi, lo) whose products with the bf16 token are exact and
- * accumulate in fp32 (what the planes leave out is at most 2^-17 |c_k| per
- * element: the worst-case rounding of an fp32 dot product of length 128).
+ * ties, evaluated with fp32-grade dot products: f32 tokens as |c|^2 - 2 x.c
+ * by fp32 FMAs; bf16 tokens on the tensor cores as the argmax of
+ * x.c - |c|^2/2, the fp32 centroid split into two bf16 planes (hi, lo) whose
+ * products with the bf16 token are exact and accumulate in fp32 (what the
+ * planes leave out is at most 2^-17 |c_k| per element: the worst-case
+ * rounding of an fp32 dot product of length 128), and -|c|^2/2 added in the
+ * same accumulation as three bf16 parts (held to 2^-24).
  *   ws  svgear_workspace_bytes(SVGEAR_OP_KMEANS_ASSIGN): the device status
  *       words (svgear_device_status), then the centroids re-laid for the
- *       kernel and their norms. */
+ *       kernel (planes and the norm parts). */
 int svgear_kmeans_assign(const void* X, svgear_dims dims, const float* centroids,
                          int32_t C, int32_t* labels, void* ws, size_t ws_bytes,
                          void* stream);
